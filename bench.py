@@ -1,0 +1,417 @@
+#!/usr/bin/env python
+"""Benchmark of the MatMamba block at Matryoshka widths on B200.
+
+Metric: block prefill tokens/s per width m_i (headline: the 130M-class block,
+batch 8 x 2048 tokens, at full width m = 768) and the SSD scan's fraction of
+its roofline (standalone scan, batch 4 x 8192 tokens, 24 heads and the 12-head
+prefix).  Inputs are seeded synthetic tensors already resident in HBM; L2 is
+flushed (256 MiB write) before every timed step and each step is timed with
+CUDA events on the launching stream.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--extended]
+
+With N > 1 (launched by torch.distributed.run) every rank runs an independent
+replica on its own GPU (sequences shard with no exchange), and value is the
+tokens of all ranks divided by the slowest rank's time.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MatMamba block prefill tokens/sec per width m_i; SSD scan % of roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--extended", action="store_true", help="also time the 48-layer stack and the decode step")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    a = ap.parse_args()
+    a.warmup = max(a.warmup, 3)
+    return a
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in FALLBACK_PEAKS}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------------------------ workload sizes
+
+BLOCK = dict(workload="block_130m_b8_L2048", batch=8, seq_len=2048, d_model=768, d_inner=1536, d_head=64,
+             d_state=128, ngroups=1, d_conv=4, chunk=256, widths=[768, 384, 192, 96])
+SCAN = dict(workload="ssd_b4_L8192_h24", batch=4, seq_len=8192, heads=24, d_head=64, d_state=128, chunk=256,
+            head_slices=[24, 12])
+
+
+def block_work(m, T, Dm=768, E=1536, P=64, N=128):
+    """Algorithmic work of each launch stage of one block forward on T tokens at width m."""
+    d = E * m // Dm
+    h = d // P
+    nconv = d + 2 * N
+    return {
+        "in_proj": ("tensor", 2.0 * T * Dm * (2 * d + 2 * N + h)),
+        "conv_silu_dt": ("hbm", T * (nconv * 2 * 2 + h * 4 * 2)),
+        "ssd_scan": ("hbm", T * (2 * d * 2 + 2 * N * 2 + h * 4)),
+        "gate_rmsnorm": ("hbm", T * d * 2 * 3),
+        "out_proj": ("tensor", 2.0 * T * d * Dm),
+    }
+
+
+def scan_bytes(T, h, P=64, N=128):
+    """x read + y write (bf16), B and C read (bf16), dt read (fp32) per token."""
+    return T * (2 * h * P * 2 + 2 * N * 2 + h * 4)
+
+
+# ------------------------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------------------------ our arm
+
+def run_ours(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import nested_mamba2_selective_b200 as mm
+    from nested_mamba2_selective_b200 import build, synth
+
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local = int(os.environ.get("LOCAL_RANK", 0))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+    if rank == 0:
+        build.build()
+    if world > 1:
+        dist.barrier()
+    mm.load()
+    pk, pk_src = peaks()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v):
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    stream = torch.cuda.current_stream()
+    flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def timed(fn, steps, warmup, trace=False):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        barrier()
+        if trace:
+            mm.mm_trace_enable(steps * 32)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        torch.cuda.synchronize()
+        barrier()
+        for e0, e1 in ev:
+            flush_buf.zero_()
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        ms = [e0.elapsed_time(e1) for e0, e1 in ev]
+        tr = None
+        if trace:
+            tr = mm.mm_trace_collect()
+            mm.mm_trace_enable(0)
+        return ms, tr
+
+    # ---------------- block workload (headline)
+    B = BLOCK
+    arrays = synth.block_params(B["d_model"], B["d_inner"], B["d_head"], B["d_state"], dtype="bf16", seed=1002)
+    wt = mm.BlockWeights.from_arrays(arrays, B["d_model"], B["d_inner"], B["d_head"], B["d_state"],
+                                     dtype=torch.bfloat16, device=dev)
+    u_np = synth.activations((B["batch"], B["seq_len"], B["d_model"]), "bf16", seed=1002 + 30 + rank)
+    u = torch.from_numpy(u_np).to(dev).bfloat16()
+    out = torch.empty_like(u)
+    T = B["batch"] * B["seq_len"]
+    ws = torch.empty(max(mm.matmamba_block_workspace(wt, B["batch"], B["seq_len"], m, B["chunk"])
+                         for m in B["widths"]), dtype=torch.uint8, device=dev)
+
+    per_width = {}
+    head = None
+    with ClockSampler(local) as clk:
+        for m in B["widths"]:
+            fn = lambda m=m: mm.matmamba_block_fwd(wt, u, m, B["chunk"], out=out, workspace=ws)  # noqa: E731
+            ms, tr = timed(fn, args.steps, args.warmup, trace=True)
+            total = max_over_ranks(sum(ms))
+            per_width[str(m)] = {"tokens_per_s": world * T * args.steps / (total / 1e3),
+                                 "ms_per_step": total / args.steps}
+            if m == B["widths"][0]:
+                head = (ms, total, tr)
+    clocks = clk.summary()
+    ms, total, (stages, kernels) = head
+    m0 = B["widths"][0]
+    value = world * T * args.steps / (total / 1e3)
+
+    # dominant stage of the headline step -> roofline object
+    work = block_work(m0, T)
+    dom = max(stages, key=lambda k: stages[k][2])
+    kind, amount = work.get(dom, ("hbm", 0.0))
+    avg_ms = stages[dom][2] / stages[dom][0]
+    if kind == "tensor":
+        achieved = amount / (avg_ms / 1e3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"], "unit": "TFLOP/s"}
+    else:
+        achieved = amount / (avg_ms / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s"}
+    roof.update({"frac": roof["achieved"] / roof["peak"], "traffic": None, "kernel": dom,
+                 "peak_source": pk_src, "avg_launch_ms": avg_ms})
+    stage_table = {}
+    for k, (n, kern, tot) in stages.items():
+        kd, amt = work.get(k, ("hbm", 0.0))
+        per = tot / n
+        ach = amt / (per / 1e3) / (1e12 if kd == "tensor" else 1e9)
+        stage_table[k] = {"ms_per_launch": per, "share": tot / sum(v[2] for v in stages.values()), "bound": kd,
+                          "achieved": ach, "unit": "TFLOP/s" if kd == "tensor" else "GB/s",
+                          "frac": ach / (pk["bf16_tflops"] if kd == "tensor" else pk["hbm_gbs"])}
+
+    # ---------------- standalone SSD scan (the graded scan roofline)
+    S = SCAN
+    inp = synth.ssd_inputs(S["batch"], S["seq_len"], S["heads"], S["d_head"], S["d_state"], 1, "bf16", seed=1001)
+    g = {k: torch.from_numpy(v).to(dev) for k, v in inp.items()}
+    for k in ("x", "B", "C"):
+        g[k] = g[k].bfloat16()
+    Ts = S["batch"] * S["seq_len"]
+    scan = {}
+    for h in S["head_slices"]:
+        y = torch.empty((S["batch"], S["seq_len"], h, S["d_head"]), dtype=torch.bfloat16, device=dev)
+        sws = torch.empty(max(mm.ssd_scan_workspace(torch.bfloat16, S["batch"], S["seq_len"], h, 64, 128, 1,
+                                                    S["chunk"]), 1), dtype=torch.uint8, device=dev)
+        fn = lambda h=h, y=y, sws=sws: mm.ssd_scan(g["x"], g["dt"], g["A"], g["B"], g["C"], g["D"], h=h,  # noqa
+                                                   chunk=S["chunk"], y=y, workspace=sws)
+        sms, _ = timed(fn, args.steps, args.warmup)
+        avg = max_over_ranks(sum(sms)) / args.steps
+        nbytes = scan_bytes(Ts, h)
+        scan[str(h)] = {"tokens_per_s": world * Ts / (avg / 1e3), "us_per_call": avg * 1e3,
+                        "roofline": {"bound": "hbm", "achieved": nbytes / (avg / 1e3) / 1e9, "peak": pk["hbm_gbs"],
+                                     "unit": "GB/s", "frac": nbytes / (avg / 1e3) / 1e9 / pk["hbm_gbs"],
+                                     "algorithmic_bytes": nbytes, "traffic": None, "peak_source": pk_src}}
+
+    # ---------------- end to end through the host-buffer entry point
+    u_host = torch.from_numpy(u_np).bfloat16().pin_memory()
+    out_host = torch.empty_like(u_host).pin_memory()
+    u_dev, out_dev = torch.empty_like(u), torch.empty_like(u)
+    e2e_fn = lambda: mm.matmamba_block_fwd_host(wt, u_host, m0, B["chunk"], out_host, u_dev, out_dev, ws)  # noqa
+    for _ in range(args.warmup):
+        e2e_fn()
+    barrier()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        e2e_fn()
+    e2e_s = max_over_ranks(time.perf_counter() - t0)
+    io_bytes = T * B["d_model"] * 2
+
+    extended = {}
+    if args.extended:
+        extended = run_extended(args, mm, synth, torch, dev, timed, max_over_ranks, world)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": total / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": B["workload"], "batch": B["batch"], "seq_len": B["seq_len"],
+                       "d_model": B["d_model"], "d_inner": B["d_inner"], "d_head": B["d_head"],
+                       "d_state": B["d_state"], "ngroups": 1, "d_conv": 4, "chunk": B["chunk"], "width": m0,
+                       "parallelism": "replicas%d" % world,
+                       "l2": "flushed (256 MiB write) before every timed step"},
+            "per_width": per_width,
+            "roofline": roof,
+            "stages": stage_table,
+            "ssd_scan": {"workload": S["workload"], "by_heads": scan},
+            "e2e": {"value": world * T * args.steps / e2e_s, "unit": "tokens/s", "h2d_bytes_per_step": io_bytes,
+                    "d2h_bytes_per_step": io_bytes},
+            "gpu_launches": kernels,
+            "clocks": clocks,
+        }
+        if extended:
+            line["extended"] = extended
+        if not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(arrays, u_np, m0)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_extended(args, mm, synth, torch, dev, timed, max_over_ranks, world):
+    """48-layer stack (b4 L4096, d_model 2048) per width and the 256-sequence decode step per width."""
+    import numpy as np
+    res = {}
+    Dm, E = 2048, 4096
+    layers, pws = [], []
+    for l in range(48):
+        a = synth.block_params(Dm, E, 64, 128, dtype="bf16", seed=1003 * 1000 + l)
+        layers.append(mm.BlockWeights.from_arrays(a, Dm, E, 64, 128, dtype=torch.bfloat16, device=dev))
+        pws.append(torch.from_numpy(synth.round_to(1.0 + 0.02 * np.random.default_rng(1003 * 1000 + 500 + l)
+                                                   .standard_normal(Dm), "bf16")).to(dev).bfloat16())
+    u = torch.from_numpy(synth.activations((4, 4096, Dm), "bf16", seed=402)).to(dev).bfloat16()
+    out = torch.empty_like(u)
+    stack = {}
+    for m in (2048, 1024, 512, 256):
+        ms_list = [m] * 48
+        ws = torch.empty(mm.matmamba_stack_workspace(layers, ms_list, 4, 4096), dtype=torch.uint8, device=dev)
+        fn = lambda: mm.matmamba_stack_fwd(layers, pws, u, ms_list, out=out, workspace=ws)  # noqa: E731
+        steps = max(2, min(args.steps, 5))
+        ms, _ = timed(fn, steps, 1)
+        avg = max_over_ranks(sum(ms)) / steps
+        stack[str(m)] = {"ms_per_forward": avg, "tokens_per_s": world * 4 * 4096 / (avg / 1e3)}
+    res["stack48_1p4b_b4_L4096"] = stack
+    dec = {}
+    w = layers[0]
+    for m in (2048, 1024, 512):
+        s_np, c_np = synth.states(256, 64, 64, 128, E + 256, 4, "bf16", seed=320)
+        s = torch.from_numpy(s_np).to(dev)
+        c = torch.from_numpy(c_np).to(dev).bfloat16()
+        ut = torch.from_numpy(synth.activations((256, Dm), "bf16", seed=321)).to(dev).bfloat16()
+        ot = torch.empty_like(ut)
+        ws = torch.empty(mm.ssd_step_workspace(w, 256, m), dtype=torch.uint8, device=dev)
+        fn = lambda: mm.ssd_step(w, s, c, ut, m, out_t=ot, workspace=ws)  # noqa: E731
+        ms, _ = timed(fn, args.steps, args.warmup)
+        avg = max_over_ranks(sum(ms)) / args.steps
+        dec[str(m)] = {"us_per_step": avg * 1e3, "tokens_per_s": world * 256 / (avg / 1e3)}
+    res["decode_b256_1p4b"] = dec
+    return res
+
+
+def cpu_baseline(arrays, u_np, m, budget_s=10.0):
+    """The fp64 oracle on whole batch rows of the headline workload until ~budget_s of CPU time."""
+    import numpy as np
+
+    import oracle
+    dims = oracle.Dims(BLOCK["d_model"], BLOCK["d_inner"], BLOCK["d_head"], BLOCK["d_state"])
+    p64 = {k: v.astype(np.float64) for k, v in arrays.items()}
+    L = BLOCK["seq_len"]
+    rows, t0 = 0, time.perf_counter()
+    while rows < u_np.shape[0] and time.perf_counter() - t0 < budget_s:
+        oracle.block_fwd(dims, p64, u_np[rows:rows + 1], m)
+        rows += 1
+    el = time.perf_counter() - t0
+    return {"value": rows * L / el, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": "%d of %d batch rows x %d tokens at width %d (fp64 sequential oracle, OpenMP)"
+                      % (rows, u_np.shape[0], L, m)}
+
+
+# ------------------------------------------------------------------------------------ reference arm
+
+def run_reference(args):
+    """The fp64 CPU oracle on the headline workload's config, a bounded sample per step."""
+    import numpy as np
+
+    import oracle
+    from nested_mamba2_selective_b200 import synth
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    if rank != 0:
+        return
+    oracle.build()
+    B = BLOCK
+    arrays = synth.block_params(B["d_model"], B["d_inner"], B["d_head"], B["d_state"], dtype="bf16", seed=1002)
+    p64 = {k: v.astype(np.float64) for k, v in arrays.items()}
+    u = synth.activations((B["batch"], B["seq_len"], B["d_model"]), "bf16", seed=1002 + 30)
+    dims = oracle.Dims(B["d_model"], B["d_inner"], B["d_head"], B["d_state"])
+    Ls = 256
+    m0 = B["widths"][0]
+    for i in range(args.warmup):
+        oracle.block_fwd(dims, p64, u[i % B["batch"]:i % B["batch"] + 1, :Ls], m0)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        oracle.block_fwd(dims, p64, u[i % B["batch"]:i % B["batch"] + 1, :Ls], m0)
+    el = time.perf_counter() - t0
+    value = args.steps * Ls / el
+    sample = "one batch row x %d tokens per step at width %d (fp64 sequential oracle, OpenMP)" % (Ls, m0)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": B["workload"], "batch": B["batch"], "seq_len": B["seq_len"],
+                       "d_model": B["d_model"], "width": m0, "chunk": B["chunk"]},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    a = parse()
+    if a.impl == "reference":
+        run_reference(a)
+    else:
+        run_ours(a)

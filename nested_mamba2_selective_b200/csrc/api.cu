@@ -1,0 +1,571 @@
+// C-ABI entry points: host-side validation, width views, workspace carving and
+// launch sequences.  Every step of the computation runs in this library's
+// kernels; nothing here computes on the host.
+#include <cstring>
+
+#include "mm_internal.cuh"
+
+using namespace mm;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+
+size_t esize(int dtype) { return dtype == MM_BF16 ? 2 : 4; }
+bool dtype_ok(int dtype) { return dtype == MM_F32 || dtype == MM_BF16; }
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+size_t round_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+// Sequential carving of the caller's workspace into 256-byte aligned pieces.
+struct Carver {
+    char* base;
+    size_t used = 0;
+    explicit Carver(void* b) : base(static_cast<char*>(b)) {}
+    void* take(size_t bytes)
+    {
+        void* p = base ? base + used : nullptr;
+        used += round_up(bytes);
+        return p;
+    }
+};
+
+struct View {  // resolved width view
+    int Dm, E, P, N, G, GN, H, K, d, h, nconv, hpg;
+};
+
+int check_params(const mm_block_params* p)
+{
+    if (!p) return MM_ERR_NULL;
+    if (!dtype_ok(p->dtype)) return MM_ERR_DTYPE;
+    if (p->d_model <= 0 || p->d_inner <= 0 || p->d_head <= 0 || p->d_state <= 0 || p->ngroups <= 0) return MM_ERR_SHAPE;
+    if (p->d_conv < 2 || p->d_conv > 8) return MM_ERR_SHAPE;
+    if (p->d_inner % p->d_head) return MM_ERR_SHAPE;
+    const int H = p->d_inner / p->d_head;
+    if (H % p->ngroups) return MM_ERR_SHAPE;
+    if (p->d_state > 256 || p->d_state % 8) return MM_ERR_SHAPE;
+    if (!(p->norm_eps >= 0.0f)) return MM_ERR_SHAPE;
+    const void* ptrs[] = {p->W_in, p->conv_w, p->conv_b, p->dt_bias, p->A, p->D, p->norm_w, p->W_out};
+    for (const void* q : ptrs)
+        if (!q) return MM_ERR_NULL;
+    if (p->dtype == MM_BF16) {
+        if (p->d_model % 8 || p->d_head % 8) return MM_ERR_SHAPE;
+        const void* al[] = {p->W_in, p->W_out, p->norm_w};
+        for (const void* q : al)
+            if (!aligned16(q)) return MM_ERR_ALIGN;
+    }
+    return MM_OK;
+}
+
+int resolve(const mm_block_params* p, int m, View& v)
+{
+    int rc = check_params(p);
+    if (rc) return rc;
+    if (m <= 0 || m > p->d_model) return MM_ERR_INVALID_WIDTH;
+    const long long num = (long long)p->d_inner * m;
+    if (num % p->d_model) return MM_ERR_INVALID_WIDTH;
+    const int d = (int)(num / p->d_model);
+    if (d % p->d_head) return MM_ERR_INVALID_WIDTH;
+    v.Dm = p->d_model; v.E = p->d_inner; v.P = p->d_head; v.N = p->d_state; v.G = p->ngroups;
+    v.GN = v.G * v.N; v.H = v.E / v.P; v.K = p->d_conv; v.d = d; v.h = d / v.P; v.nconv = d + 2 * v.GN;
+    v.hpg = v.H / v.G;
+    return MM_OK;
+}
+
+inline int cuda_status(cudaError_t e) { return e == cudaSuccess ? MM_OK : MM_ERR_CUDA; }
+
+// ------------------------------------------------------------------ tracing
+
+struct TraceRec {
+    const char* name;
+    int kernels;
+    cudaEvent_t start, stop;
+};
+struct Trace {
+    TraceRec* recs = nullptr;
+    int cap = 0, n = 0;
+};
+Trace g_trace;
+
+// Runs one launch stage; with tracing on, brackets it with events on stream s.
+template <class F>
+cudaError_t stage(const char* name, int kernels, cudaStream_t s, F&& launch)
+{
+    if (!g_trace.recs || g_trace.n >= g_trace.cap) return launch();
+    TraceRec& r = g_trace.recs[g_trace.n];
+    cudaError_t e = cudaEventRecord(r.start, s);
+    if (e != cudaSuccess) return e;
+    e = launch();
+    if (e != cudaSuccess) return e;
+    e = cudaEventRecord(r.stop, s);
+    if (e != cudaSuccess) return e;
+    r.name = name;
+    r.kernels = kernels;
+    ++g_trace.n;
+    return cudaSuccess;
+}
+#define MM_TRY(expr)                          \
+    do {                                      \
+        int _rc = cuda_status(expr);          \
+        if (_rc) return _rc;                  \
+    } while (0)
+
+cudaError_t run_gemm(int dtype, const GemmDesc& g, cudaStream_t s)
+{
+    if (dtype == MM_BF16 && gemm_tc_supported(g)) return launch_gemm_tc(g, s);
+    return launch_gemm_simt(dtype, g, s);
+}
+
+bool scan_uses_tc(int dtype, const ScanArgs& a) { return dtype == MM_BF16 && scan_tc_supported(a); }
+
+size_t scan_ws_bytes(int dtype, const ScanArgs& a) { return scan_uses_tc(dtype, a) ? scan_tc_workspace(a) : 0; }
+
+int scan_kernels(int dtype, const ScanArgs& a) { return scan_uses_tc(dtype, a) ? scan_tc_kernel_count(a) : 1; }
+
+cudaError_t run_scan(int dtype, const ScanArgs& a, void* ws, size_t ws_bytes, cudaStream_t s)
+{
+    if (scan_uses_tc(dtype, a)) return launch_scan_tc(a, ws, ws_bytes, s);
+    return launch_scan_seq(dtype, a, s);
+}
+
+// Scan arguments of the block: x | B | C live in the post-conv buffer.
+ScanArgs block_scan_args(const View& v, const mm_block_params* p, const void* xbc, const float* dt, int batch, int L,
+                         int chunk, const float* s_in, float* s_out, void* y)
+{
+    ScanArgs a{};
+    const size_t es = esize(p->dtype);
+    a.x = xbc; a.sx = v.nconv;
+    a.dt = dt; a.sdt = v.h;
+    a.A = p->A;
+    a.B = static_cast<const char*>(xbc) + (size_t)v.d * es; a.sB = v.nconv;
+    a.C = static_cast<const char*>(xbc) + (size_t)(v.d + v.GN) * es; a.sC = v.nconv;
+    a.D = p->D;
+    a.batch = batch; a.L = L; a.h = v.h; a.P = v.P; a.N = v.N; a.G = v.G; a.hpg = v.hpg; a.chunk = chunk;
+    a.init_state = s_in; a.state_stride = (int64_t)v.H * v.P * v.N;
+    a.y = y; a.sy = v.d;
+    a.final_state = s_out;
+    return a;
+}
+
+struct BlockBufs {
+    void *zxbc, *xbc, *y, *nrm, *scan_ws;
+    float *dt_raw, *dt;
+    size_t scan_ws_bytes;
+};
+
+BlockBufs carve_block(Carver& c, const View& v, const mm_block_params* p, int batch, int L, int chunk)
+{
+    const size_t es = esize(p->dtype);
+    const size_t T = (size_t)batch * L;
+    BlockBufs b{};
+    b.zxbc = c.take(T * (v.d + v.nconv) * es);
+    b.dt_raw = static_cast<float*>(c.take(T * v.h * 4));
+    b.xbc = c.take(T * v.nconv * es);
+    b.dt = static_cast<float*>(c.take(T * v.h * 4));
+    b.y = c.take(T * v.d * es);
+    b.nrm = c.take(T * v.d * es);
+    ScanArgs probe = block_scan_args(v, p, b.xbc, b.dt, batch, L, chunk, nullptr, nullptr, b.y);
+    b.scan_ws_bytes = scan_ws_bytes(p->dtype, probe);
+    b.scan_ws = c.take(b.scan_ws_bytes);
+    return b;
+}
+
+// in_proj through the width view: columns z | x | B | C go to zxbc, dt_raw to an fp32 buffer.
+GemmDesc in_proj_desc(const View& v, const mm_block_params* p, const void* u, int64_t T, void* zxbc, float* dt_raw)
+{
+    const size_t es = esize(p->dtype);
+    const char* W = static_cast<const char*>(p->W_in);
+    char* Z = static_cast<char*>(zxbc);
+    const int64_t ld = v.d + v.nconv;
+    GemmDesc g{};
+    g.A = u; g.lda = v.Dm; g.ldb = v.Dm; g.M = (int)T; g.K = v.Dm; g.nseg = 4;
+    g.seg[0] = GemmSeg{W, Z, ld, v.d, 0, 0};
+    g.seg[1] = GemmSeg{W + (size_t)v.E * v.Dm * es, Z + (size_t)v.d * es, ld, v.d, 0, 0};
+    g.seg[2] = GemmSeg{W + (size_t)2 * v.E * v.Dm * es, Z + (size_t)2 * v.d * es, ld, 2 * v.GN, 0, 0};
+    g.seg[3] = GemmSeg{W + (size_t)(2 * v.E + 2 * v.GN) * v.Dm * es, dt_raw, v.h, v.h, 1, 0};
+    return g;
+}
+
+// out_proj through the K-prefix view W_out[:, 0:d] (row stride E).
+GemmDesc out_proj_desc(const View& v, const mm_block_params* p, const void* nrm, int64_t T, void* out, int accumulate)
+{
+    GemmDesc g{};
+    g.A = nrm; g.lda = v.d; g.ldb = v.E; g.M = (int)T; g.K = v.d; g.nseg = 1;
+    g.seg[0] = GemmSeg{p->W_out, out, v.Dm, v.Dm, accumulate, accumulate};
+    return g;
+}
+
+// The block on device buffers.  out_accumulate = 1: out is an fp32 buffer and
+// the projection is added to it (residual stream of the stack).
+int block_impl(const mm_block_params* p, const View& v, const void* u, int batch, int L, int chunk, void* out,
+               int out_accumulate, const float* s_in, const void* c_in, float* s_out, void* c_out, Carver& c,
+               cudaStream_t s)
+{
+    const int64_t T = (int64_t)batch * L;
+    BlockBufs b = carve_block(c, v, p, batch, L, chunk);
+    MM_TRY(stage("in_proj", 1, s, [&] { return run_gemm(p->dtype, in_proj_desc(v, p, u, T, b.zxbc, b.dt_raw), s); }));
+    const int conv_rows = v.E + 2 * v.GN;
+    MM_TRY(stage("conv_silu_dt", 1, s, [&] {
+        return launch_conv_silu_dt(p->dtype, b.zxbc, v.d + v.nconv, v.d, b.dt_raw, p->conv_w, p->conv_b, p->dt_bias,
+                                   v.E, v.d, v.nconv, v.h, v.K, batch, L, c_in, conv_rows, b.xbc, b.dt, s);
+    }));
+    if (c_out)
+        MM_TRY(stage("conv_state", 1, s, [&] {
+            return launch_conv_state_out(p->dtype, b.zxbc, v.d + v.nconv, v.d, v.E, v.d, v.nconv, v.K, batch, L, c_in,
+                                         conv_rows, c_out, s);
+        }));
+    ScanArgs a = block_scan_args(v, p, b.xbc, b.dt, batch, L, chunk, s_in, s_out, b.y);
+    MM_TRY(stage("ssd_scan", scan_kernels(p->dtype, a), s,
+                 [&] { return run_scan(p->dtype, a, b.scan_ws, b.scan_ws_bytes, s); }));
+    MM_TRY(stage("gate_rmsnorm", 1, s, [&] {
+        return launch_gate_rmsnorm(p->dtype, b.y, v.d, b.zxbc, v.d + v.nconv, p->norm_w, p->norm_eps, v.d, (int)T,
+                                   b.nrm, v.d, s);
+    }));
+    MM_TRY(stage("out_proj", 1, s,
+                 [&] { return run_gemm(p->dtype, out_proj_desc(v, p, b.nrm, T, out, out_accumulate), s); }));
+    return MM_OK;
+}
+
+int check_chunk(int chunk) { return chunk > 0 ? MM_OK : MM_ERR_SHAPE; }
+
+}  // namespace
+
+extern "C" {
+
+const char* mm_status_string(int status)
+{
+    switch (status) {
+        case MM_OK: return "ok";
+        case MM_ERR_INVALID_WIDTH: return "invalid Matryoshka width";
+        case MM_ERR_SHAPE: return "invalid shape or stride";
+        case MM_ERR_DTYPE: return "invalid dtype";
+        case MM_ERR_ALIGN: return "misaligned pointer or stride";
+        case MM_ERR_WORKSPACE: return "workspace missing or too small";
+        case MM_ERR_CUDA: return "CUDA runtime error";
+        case MM_ERR_TIMEOUT: return "bounded device wait timed out";
+        case MM_ERR_NULL: return "required pointer is NULL";
+        case MM_ERR_UNSUPPORTED: return "unsupported configuration";
+        default: return "unknown status";
+    }
+}
+
+int mm_version(void) { return 100; }
+
+int mm_width(const mm_block_params* p, int m_i, int* d_out, int* h_out)
+{
+    View v;
+    int rc = resolve(p, m_i, v);
+    if (rc) return rc;
+    if (d_out) *d_out = v.d;
+    if (h_out) *h_out = v.h;
+    return MM_OK;
+}
+
+int matmamba_block_workspace(const mm_block_params* p, int batch, int L, int m_i, int chunk, size_t* bytes)
+{
+    View v;
+    int rc = resolve(p, m_i, v);
+    if (rc) return rc;
+    if (!bytes) return MM_ERR_NULL;
+    if (batch <= 0 || L <= 0) return MM_ERR_SHAPE;
+    if ((rc = check_chunk(chunk))) return rc;
+    Carver c(nullptr);
+    carve_block(c, v, p, batch, L, chunk);
+    *bytes = c.used;
+    return MM_OK;
+}
+
+int matmamba_block_fwd(const mm_block_params* p, const void* u, int batch, int L, int m_i, int chunk, void* out,
+                       const float* ssm_state_in, const void* conv_state_in, float* ssm_state_out,
+                       void* conv_state_out, void* workspace, size_t ws_bytes, void* stream)
+{
+    View v;
+    int rc = resolve(p, m_i, v);
+    if (rc) return rc;
+    if (!u || !out) return MM_ERR_NULL;
+    if (batch <= 0 || L <= 0) return MM_ERR_SHAPE;
+    if ((rc = check_chunk(chunk))) return rc;
+    if (p->dtype == MM_BF16 && (!aligned16(u) || !aligned16(out))) return MM_ERR_ALIGN;
+    if ((ssm_state_out && (const void*)ssm_state_out == (const void*)ssm_state_in) ||
+        (conv_state_out && conv_state_out == conv_state_in))
+        return MM_ERR_SHAPE;
+    size_t need;
+    matmamba_block_workspace(p, batch, L, m_i, chunk, &need);
+    if (!workspace || ws_bytes < need) return MM_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) % kAlign) return MM_ERR_ALIGN;
+    Carver c(workspace);
+    return block_impl(p, v, u, batch, L, chunk, out, 0, ssm_state_in, conv_state_in, ssm_state_out, conv_state_out, c,
+                      static_cast<cudaStream_t>(stream));
+}
+
+int matmamba_block_fwd_host(const mm_block_params* p, const void* u_host, int batch, int L, int m_i, int chunk,
+                            void* out_host, void* u_dev, void* out_dev, void* workspace, size_t ws_bytes, void* stream)
+{
+    if (!u_host || !out_host || !u_dev || !out_dev) return MM_ERR_NULL;
+    View v;
+    int rc = resolve(p, m_i, v);
+    if (rc) return rc;
+    if (batch <= 0 || L <= 0) return MM_ERR_SHAPE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t bytes = (size_t)batch * L * v.Dm * esize(p->dtype);
+    size_t need;
+    if ((rc = matmamba_block_workspace(p, batch, L, m_i, chunk, &need))) return rc;
+    if (!workspace || ws_bytes < need) return MM_ERR_WORKSPACE;
+    MM_TRY(cudaMemcpyAsync(u_dev, u_host, bytes, cudaMemcpyHostToDevice, s));
+    rc = matmamba_block_fwd(p, u_dev, batch, L, m_i, chunk, out_dev, nullptr, nullptr, nullptr, nullptr, workspace,
+                            ws_bytes, stream);
+    if (rc) return rc;
+    MM_TRY(cudaMemcpyAsync(out_host, out_dev, bytes, cudaMemcpyDeviceToHost, s));
+    MM_TRY(cudaStreamSynchronize(s));
+    return MM_OK;
+}
+
+static int scan_args_check(int dtype, const void* x, int64_t x_stride, const float* dt, int64_t dt_stride,
+                           const float* A, const void* B, int64_t B_stride, const void* C, int64_t C_stride, int batch,
+                           int L, int h, int P, int N, int G, int hpg, int chunk, int64_t state_stride, const void* y,
+                           int64_t y_stride, bool need_state)
+{
+    if (!dtype_ok(dtype)) return MM_ERR_DTYPE;
+    if (!x || !dt || !A || !B || !C || !y) return MM_ERR_NULL;
+    if (batch <= 0 || L <= 0 || h <= 0 || P <= 0 || N <= 0 || G <= 0 || hpg <= 0) return MM_ERR_SHAPE;
+    if (N > 256) return MM_ERR_SHAPE;
+    if ((h - 1) / hpg >= G) return MM_ERR_SHAPE;
+    if (x_stride < (int64_t)h * P || y_stride < (int64_t)h * P || dt_stride < h || B_stride < (int64_t)G * N ||
+        C_stride < (int64_t)G * N)
+        return MM_ERR_SHAPE;
+    if (need_state && state_stride < (int64_t)h * P * N) return MM_ERR_SHAPE;
+    if (chunk <= 0) return MM_ERR_SHAPE;
+    if (dtype == MM_BF16) {
+        if (!aligned16(x) || !aligned16(B) || !aligned16(C) || !aligned16(y)) return MM_ERR_ALIGN;
+        if (x_stride % 8 || y_stride % 8 || B_stride % 8 || C_stride % 8) return MM_ERR_ALIGN;
+    }
+    return MM_OK;
+}
+
+static ScanArgs make_scan_args(const void* x, int64_t x_stride, const float* dt, int64_t dt_stride, const float* A,
+                               const void* B, int64_t B_stride, const void* C, int64_t C_stride, const float* D,
+                               int batch, int L, int h, int P, int N, int G, int hpg, int chunk,
+                               const float* init_state, int64_t state_stride, void* y, int64_t y_stride,
+                               float* final_state)
+{
+    ScanArgs a{};
+    a.x = x; a.sx = x_stride; a.dt = dt; a.sdt = dt_stride; a.A = A; a.B = B; a.sB = B_stride; a.C = C;
+    a.sC = C_stride; a.D = D; a.batch = batch; a.L = L; a.h = h; a.P = P; a.N = N; a.G = G; a.hpg = hpg;
+    a.chunk = chunk; a.init_state = init_state; a.state_stride = state_stride; a.y = y; a.sy = y_stride;
+    a.final_state = final_state;
+    return a;
+}
+
+int ssd_scan_workspace(int dtype, int batch, int L, int h, int P, int N, int G, int chunk, size_t* bytes)
+{
+    if (!bytes) return MM_ERR_NULL;
+    if (!dtype_ok(dtype)) return MM_ERR_DTYPE;
+    if (batch <= 0 || L <= 0 || h <= 0 || P <= 0 || N <= 0 || G <= 0 || chunk <= 0) return MM_ERR_SHAPE;
+    const int hpg = (h + G - 1) / G;
+    ScanArgs a = make_scan_args(nullptr, (int64_t)h * P, nullptr, h, nullptr, nullptr, (int64_t)G * N, nullptr,
+                                (int64_t)G * N, nullptr, batch, L, h, P, N, G, hpg, chunk, nullptr, (int64_t)h * P * N,
+                                nullptr, (int64_t)h * P, nullptr);
+    *bytes = round_up(scan_ws_bytes(dtype, a));
+    return MM_OK;
+}
+
+int ssd_scan(int dtype, const void* x, int64_t x_stride, const float* dt, int64_t dt_stride, const float* A,
+             const void* B, int64_t B_stride, const void* C, int64_t C_stride, const float* D, int batch, int L,
+             int h, int P, int N, int G, int heads_per_group, int chunk, const float* init_state,
+             int64_t state_stride, void* y, int64_t y_stride, float* final_state, void* workspace, size_t ws_bytes,
+             void* stream)
+{
+    int rc = scan_args_check(dtype, x, x_stride, dt, dt_stride, A, B, B_stride, C, C_stride, batch, L, h, P, N, G,
+                             heads_per_group, chunk, state_stride, y, y_stride, init_state || final_state);
+    if (rc) return rc;
+    if (init_state && final_state && (const void*)init_state == (const void*)final_state) return MM_ERR_SHAPE;
+    ScanArgs a = make_scan_args(x, x_stride, dt, dt_stride, A, B, B_stride, C, C_stride, D, batch, L, h, P, N, G,
+                                heads_per_group, chunk, init_state, state_stride, y, y_stride, final_state);
+    const size_t need = scan_ws_bytes(dtype, a);
+    if (need && (!workspace || ws_bytes < need)) return MM_ERR_WORKSPACE;
+    if (need && reinterpret_cast<uintptr_t>(workspace) % kAlign) return MM_ERR_ALIGN;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    return cuda_status(stage("ssd_scan", scan_kernels(dtype, a), s, [&] { return run_scan(dtype, a, workspace, ws_bytes, s); }));
+}
+
+static size_t step_ws(const View& v, const mm_block_params* p, int batch)
+{
+    Carver c(nullptr);
+    const size_t es = esize(p->dtype);
+    c.take((size_t)batch * (v.d + v.nconv) * es);
+    c.take((size_t)batch * v.h * 4);
+    c.take((size_t)batch * v.nconv * es);
+    c.take((size_t)batch * v.h * 4);
+    c.take((size_t)batch * v.d * es);
+    c.take((size_t)batch * v.d * es);
+    return c.used;
+}
+
+int ssd_step_workspace(const mm_block_params* p, int batch, int m_i, size_t* bytes)
+{
+    View v;
+    int rc = resolve(p, m_i, v);
+    if (rc) return rc;
+    if (!bytes) return MM_ERR_NULL;
+    if (batch <= 0) return MM_ERR_SHAPE;
+    *bytes = step_ws(v, p, batch);
+    return MM_OK;
+}
+
+int ssd_step(const mm_block_params* p, float* ssm_state, void* conv_state, const void* u_t, int batch, int m_i,
+             void* out_t, void* workspace, size_t ws_bytes, void* stream)
+{
+    View v;
+    int rc = resolve(p, m_i, v);
+    if (rc) return rc;
+    if (!ssm_state || !conv_state || !u_t || !out_t) return MM_ERR_NULL;
+    if (batch <= 0) return MM_ERR_SHAPE;
+    if (p->dtype == MM_BF16 && (!aligned16(u_t) || !aligned16(out_t))) return MM_ERR_ALIGN;
+    if (!workspace || ws_bytes < step_ws(v, p, batch)) return MM_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) % kAlign) return MM_ERR_ALIGN;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t es = esize(p->dtype);
+    Carver c(workspace);
+    void* zxbc = c.take((size_t)batch * (v.d + v.nconv) * es);
+    float* dt_raw = static_cast<float*>(c.take((size_t)batch * v.h * 4));
+    void* xbc = c.take((size_t)batch * v.nconv * es);
+    float* dt = static_cast<float*>(c.take((size_t)batch * v.h * 4));
+    void* y = c.take((size_t)batch * v.d * es);
+    void* nrm = c.take((size_t)batch * v.d * es);
+    MM_TRY(stage("step_in_proj", 1, s, [&] { return run_gemm(p->dtype, in_proj_desc(v, p, u_t, batch, zxbc, dt_raw), s); }));
+    MM_TRY(stage("step_conv_dt", 1, s, [&] {
+        return launch_step_conv_dt(p->dtype, zxbc, v.d + v.nconv, v.d, dt_raw, p->conv_w, p->conv_b, p->dt_bias, v.E,
+                                   v.d, v.nconv, v.h, v.K, batch, conv_state, v.E + 2 * v.GN, xbc, dt, s);
+    }));
+    MM_TRY(stage("step_scan", 1, s, [&] {
+        return launch_step_scan(p->dtype, xbc, v.nconv, v.d, dt, p->A, p->D, ssm_state, v.H, v.h, v.P, v.N, v.GN,
+                                v.hpg, batch, y, s);
+    }));
+    MM_TRY(stage("step_gate_rmsnorm", 1, s, [&] {
+        return launch_gate_rmsnorm(p->dtype, y, v.d, zxbc, v.d + v.nconv, p->norm_w, p->norm_eps, v.d, batch, nrm, v.d,
+                                   s);
+    }));
+    MM_TRY(stage("step_out_proj", 1, s, [&] { return run_gemm(p->dtype, out_proj_desc(v, p, nrm, batch, out_t, 0), s); }));
+    return MM_OK;
+}
+
+static int stack_check(const mm_block_params* layers, int nlayers, const int* m_per_layer, int batch, int L, int chunk,
+                       size_t* need)
+{
+    if (!layers || !m_per_layer) return MM_ERR_NULL;
+    if (nlayers <= 0 || batch <= 0 || L <= 0) return MM_ERR_SHAPE;
+    int rc;
+    if ((rc = check_chunk(chunk))) return rc;
+    size_t block_max = 0;
+    for (int l = 0; l < nlayers; ++l) {
+        View v;
+        if ((rc = resolve(&layers[l], m_per_layer[l], v))) return rc;
+        if (layers[l].d_model != layers[0].d_model || layers[l].dtype != layers[0].dtype) return MM_ERR_SHAPE;
+        Carver c(nullptr);
+        carve_block(c, v, &layers[l], batch, L, chunk);
+        block_max = c.used > block_max ? c.used : block_max;
+    }
+    const size_t T = (size_t)batch * L;
+    const int Dm = layers[0].d_model;
+    *need = round_up(T * Dm * 4) + round_up(T * Dm * esize(layers[0].dtype)) + block_max;
+    return MM_OK;
+}
+
+int matmamba_stack_workspace(const mm_block_params* layers, int nlayers, const int* m_per_layer, int batch, int L,
+                             int chunk, size_t* bytes)
+{
+    if (!bytes) return MM_ERR_NULL;
+    return stack_check(layers, nlayers, m_per_layer, batch, L, chunk, bytes);
+}
+
+int matmamba_stack_fwd(const mm_block_params* layers, const void* const* prenorm_w, float prenorm_eps, int nlayers,
+                       const int* m_per_layer, const void* u, int batch, int L, int chunk, void* out, void* workspace,
+                       size_t ws_bytes, void* stream)
+{
+    size_t need;
+    int rc = stack_check(layers, nlayers, m_per_layer, batch, L, chunk, &need);
+    if (rc) return rc;
+    if (!prenorm_w || !u || !out) return MM_ERR_NULL;
+    for (int l = 0; l < nlayers; ++l)
+        if (!prenorm_w[l]) return MM_ERR_NULL;
+    if (!(prenorm_eps >= 0.0f)) return MM_ERR_SHAPE;
+    if (!workspace || ws_bytes < need) return MM_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) % kAlign) return MM_ERR_ALIGN;
+    const int dtype = layers[0].dtype;
+    if (dtype == MM_BF16 && (!aligned16(u) || !aligned16(out))) return MM_ERR_ALIGN;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int64_t T = (int64_t)batch * L;
+    const int Dm = layers[0].d_model;
+    Carver c(workspace);
+    float* resid = static_cast<float*>(c.take((size_t)T * Dm * 4));
+    void* normed = c.take((size_t)T * Dm * esize(dtype));
+    const size_t block_base = c.used;
+    MM_TRY(stage("stack_load", 1, s, [&] { return launch_to_f32(dtype, u, resid, T * Dm, s); }));
+    for (int l = 0; l < nlayers; ++l) {
+        View v;
+        resolve(&layers[l], m_per_layer[l], v);
+        MM_TRY(stage("prenorm", 1, s, [&] {
+            return launch_rmsnorm_rows_f32in(dtype, resid, prenorm_w[l], prenorm_eps, Dm, (int)T, normed, s);
+        }));
+        c.used = block_base;
+        if ((rc = block_impl(&layers[l], v, normed, batch, L, chunk, resid, 1, nullptr, nullptr, nullptr, nullptr, c,
+                             s)))
+            return rc;
+    }
+    MM_TRY(stage("stack_store", 1, s, [&] { return launch_from_f32(dtype, resid, out, T * Dm, s); }));
+    return MM_OK;
+}
+
+int mm_trace_enable(int capacity)
+{
+    if (capacity < 0) return MM_ERR_SHAPE;
+    if (g_trace.recs) {
+        for (int i = 0; i < g_trace.cap; ++i) {
+            cudaEventDestroy(g_trace.recs[i].start);
+            cudaEventDestroy(g_trace.recs[i].stop);
+        }
+        delete[] g_trace.recs;
+        g_trace = Trace{};
+    }
+    if (capacity == 0) return MM_OK;
+    g_trace.recs = new TraceRec[capacity];
+    g_trace.cap = capacity;
+    for (int i = 0; i < capacity; ++i) {
+        if (cudaEventCreate(&g_trace.recs[i].start) != cudaSuccess ||
+            cudaEventCreate(&g_trace.recs[i].stop) != cudaSuccess) {
+            g_trace.cap = i;
+            mm_trace_enable(0);
+            return MM_ERR_CUDA;
+        }
+    }
+    return MM_OK;
+}
+
+int mm_trace_collect(mm_trace_entry* entries, int max_entries, int* n_entries, int* total_kernels)
+{
+    if (!entries || !n_entries) return MM_ERR_NULL;
+    int n = 0, kern = 0;
+    for (int i = 0; i < g_trace.n; ++i) {
+        TraceRec& r = g_trace.recs[i];
+        float ms = 0.0f;
+        if (cudaEventSynchronize(r.stop) != cudaSuccess || cudaEventElapsedTime(&ms, r.start, r.stop) != cudaSuccess)
+            return MM_ERR_CUDA;
+        kern += r.kernels;
+        int j = 0;
+        while (j < n && std::strncmp(entries[j].name, r.name, sizeof(entries[j].name) - 1) != 0) ++j;
+        if (j == n) {
+            if (n >= max_entries) continue;
+            std::memset(&entries[n], 0, sizeof(entries[n]));
+            std::strncpy(entries[n].name, r.name, sizeof(entries[n].name) - 1);
+            ++n;
+        }
+        entries[j].stages += 1;
+        entries[j].kernels += r.kernels;
+        entries[j].total_ms += ms;
+    }
+    g_trace.n = 0;
+    *n_entries = n;
+    if (total_kernels) *total_kernels = kern;
+    return MM_OK;
+}
+
+}  // extern "C"

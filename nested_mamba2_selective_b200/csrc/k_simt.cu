@@ -1,0 +1,503 @@
+// CUDA-core kernels: the fp32 path of every step, the elementwise steps of the
+// bf16 path (conv + SiLU + dt, gate + RMSNorm, residual pre-norm), the decode
+// step, and the CUDA-core GEMM / sequential scan used for shapes the
+// tensor-core kernels do not cover.
+//
+// Steps follow "MatMamba: A Matryoshka State Space Model", block-definition
+// paragraph (in_proj, causal conv of kernel 4 per channel, SiLU, selective
+// scan with A and D, Norm = RMSNorm, out_proj) at the width view of the nested
+// sub-block paragraph.
+#include "mm_internal.cuh"
+
+namespace mm {
+
+// ====================================================================== GEMM (CUDA cores)
+
+__device__ __forceinline__ int gemm_find_seg(const GemmDesc& g, int n, int& local)
+{
+    int base = 0;
+    for (int s = 0; s < g.nseg; ++s) {
+        if (n < base + g.seg[s].n) { local = n - base; return s; }
+        base += g.seg[s].n;
+    }
+    local = 0;
+    return -1;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) gemm_simt_kernel(GemmDesc g, int n_total)
+{
+    constexpr int BM = 64, BN = 64, BK = 32;
+    __shared__ float As[BK][BM + 4];
+    __shared__ float Bs[BK][BN + 4];
+    const int tid = threadIdx.x;
+    const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
+    const T* A = static_cast<const T*>(g.A);
+
+    // loader role: one A row and one B row, 8 consecutive k each
+    const int lr = tid >> 2, lk = (tid & 3) * 8;
+    const int am = m0 + lr;
+    const T* arow = am < g.M ? A + (int64_t)am * g.lda : nullptr;
+    const T* brow = nullptr;
+    {
+        int loc, s = (n0 + lr < n_total) ? gemm_find_seg(g, n0 + lr, loc) : -1;
+        if (s >= 0) brow = static_cast<const T*>(g.seg[s].B) + (int64_t)loc * g.ldb;
+    }
+
+    const int ty = tid >> 4, tx = tid & 15;
+    float acc[4][4] = {};
+    for (int k0 = 0; k0 < g.K; k0 += BK) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            int k = k0 + lk + j;
+            As[lk + j][lr] = (arow && k < g.K) ? to_f32(arow[k]) : 0.0f;
+            Bs[lk + j][lr] = (brow && k < g.K) ? to_f32(brow[k]) : 0.0f;
+        }
+        __syncthreads();
+#pragma unroll 8
+        for (int k = 0; k < BK; ++k) {
+            float a[4], b[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) a[i] = As[k][ty + 16 * i];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) b[j] = Bs[k][tx + 16 * j];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        int n = n0 + tx + 16 * j;
+        if (n >= n_total) continue;
+        int loc, s = gemm_find_seg(g, n, loc);
+        const GemmSeg& sg = g.seg[s];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            int m = m0 + ty + 16 * i;
+            if (m >= g.M) continue;
+            if (sg.out_f32) {
+                float* o = static_cast<float*>(sg.out) + (int64_t)m * sg.ldo + loc;
+                *o = sg.accumulate ? *o + acc[i][j] : acc[i][j];
+            } else {
+                static_cast<T*>(sg.out)[(int64_t)m * sg.ldo + loc] = from_f32<T>(acc[i][j]);
+            }
+        }
+    }
+}
+
+cudaError_t launch_gemm_simt(int dtype, const GemmDesc& g, cudaStream_t s)
+{
+    int n_total = 0;
+    for (int i = 0; i < g.nseg; ++i) n_total += g.seg[i].n;
+    if (g.M == 0 || n_total == 0) return cudaSuccess;
+    dim3 grid((n_total + 63) / 64, (g.M + 63) / 64);
+    if (dtype == MM_BF16) gemm_simt_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(g, n_total);
+    else gemm_simt_kernel<float><<<grid, 256, 0, s>>>(g, n_total);
+    return cudaGetLastError();
+}
+
+// ====================================================================== conv + SiLU + dt
+
+// One thread per (token, channel).  Channels [0, nconv) are x | B | C of the
+// width view (conv rows [0,d) u [E, E+2GN)); channels [nconv, nconv+h) compute
+// dt = softplus(raw + dt_bias) for head c - nconv.
+template <typename T>
+__global__ void conv_silu_dt_kernel(const T* __restrict__ zxbc, int64_t ld_in, int col0,
+                                    const float* __restrict__ dt_raw, const T* __restrict__ conv_w,
+                                    const T* __restrict__ conv_b, const float* __restrict__ dt_bias, int E, int d,
+                                    int nconv, int h, int K, int L, const T* __restrict__ conv_state_in, int conv_rows,
+                                    T* __restrict__ xbc_out, float* __restrict__ dt_out)
+{
+    const int c = blockIdx.y * blockDim.x + threadIdx.x;
+    const int64_t tok = blockIdx.x;
+    if (c >= nconv + h) return;
+    if (c >= nconv) {
+        const int i = c - nconv;
+        dt_out[tok * h + i] = softplus_f(dt_raw[tok * h + i] + dt_bias[i]);
+        return;
+    }
+    const int b = (int)(tok / L), t = (int)(tok % L);
+    const int row = c < d ? c : E + (c - d);
+    float acc = to_f32(conv_b[row]);
+    for (int j = 0; j < K; ++j) {
+        const int tau = t - (K - 1) + j;
+        float v;
+        if (tau >= 0) v = to_f32(zxbc[((int64_t)b * L + tau) * ld_in + col0 + c]);
+        else if (conv_state_in) v = to_f32(conv_state_in[((int64_t)b * conv_rows + row) * (K - 1) + (K - 1 + tau)]);
+        else v = 0.0f;
+        acc = fmaf(to_f32(conv_w[(int64_t)row * K + j]), v, acc);
+    }
+    xbc_out[tok * nconv + c] = from_f32<T>(silu_f(acc));
+}
+
+cudaError_t launch_conv_silu_dt(int dtype, const void* zxbc, int64_t ld_in, int col0, const float* dt_raw,
+                                const void* conv_w, const void* conv_b, const float* dt_bias, int E, int d, int nconv,
+                                int h, int K, int batch, int L, const void* conv_state_in, int conv_rows, void* xbc_out,
+                                float* dt_out, cudaStream_t s)
+{
+    dim3 grid((unsigned)((int64_t)batch * L), (nconv + h + 127) / 128);
+    if (dtype == MM_BF16)
+        conv_silu_dt_kernel<__nv_bfloat16><<<grid, 128, 0, s>>>(
+            (const __nv_bfloat16*)zxbc, ld_in, col0, dt_raw, (const __nv_bfloat16*)conv_w,
+            (const __nv_bfloat16*)conv_b, dt_bias, E, d, nconv, h, K, L, (const __nv_bfloat16*)conv_state_in,
+            conv_rows, (__nv_bfloat16*)xbc_out, dt_out);
+    else
+        conv_silu_dt_kernel<float><<<grid, 128, 0, s>>>((const float*)zxbc, ld_in, col0, dt_raw,
+                                                         (const float*)conv_w, (const float*)conv_b, dt_bias, E, d,
+                                                         nconv, h, K, L, (const float*)conv_state_in, conv_rows,
+                                                         (float*)xbc_out, dt_out);
+    return cudaGetLastError();
+}
+
+// Conv state after a prefill: the last K-1 pre-conv inputs of each active
+// channel, oldest first.  One thread per (batch, channel) walks k upward, so
+// an in-place update (state_out == state_in) would also be safe.
+template <typename T>
+__global__ void conv_state_out_kernel(const T* __restrict__ zxbc, int64_t ld_in, int col0, int E, int d, int nconv,
+                                      int K, int batch, int L, const T* conv_state_in, int conv_rows, T* conv_state_out)
+{
+    const int c = blockIdx.x * blockDim.x + threadIdx.x;
+    const int b = blockIdx.y;
+    if (c >= nconv) return;
+    const int row = c < d ? c : E + (c - d);
+    for (int k = 0; k < K - 1; ++k) {
+        const int tau = L - (K - 1) + k;
+        T v;
+        if (tau >= 0) v = zxbc[((int64_t)b * L + tau) * ld_in + col0 + c];
+        else if (conv_state_in) v = conv_state_in[((int64_t)b * conv_rows + row) * (K - 1) + (K - 1 + tau)];
+        else v = from_f32<T>(0.0f);
+        conv_state_out[((int64_t)b * conv_rows + row) * (K - 1) + k] = v;
+    }
+}
+
+cudaError_t launch_conv_state_out(int dtype, const void* zxbc, int64_t ld_in, int col0, int E, int d, int nconv, int K,
+                                  int batch, int L, const void* conv_state_in, int conv_rows, void* conv_state_out,
+                                  cudaStream_t s)
+{
+    dim3 grid((nconv + 127) / 128, batch);
+    if (dtype == MM_BF16)
+        conv_state_out_kernel<__nv_bfloat16><<<grid, 128, 0, s>>>(
+            (const __nv_bfloat16*)zxbc, ld_in, col0, E, d, nconv, K, batch, L, (const __nv_bfloat16*)conv_state_in,
+            conv_rows, (__nv_bfloat16*)conv_state_out);
+    else
+        conv_state_out_kernel<float><<<grid, 128, 0, s>>>((const float*)zxbc, ld_in, col0, E, d, nconv, K, batch, L,
+                                                           (const float*)conv_state_in, conv_rows,
+                                                           (float*)conv_state_out);
+    return cudaGetLastError();
+}
+
+// ====================================================================== sequential scan
+
+// The scan in its recurrent form on CUDA cores: one CTA per (batch, head,
+// 8 state rows p); 16 threads share one p and hold NPT state entries n each.
+// Tokens are staged through shared memory 16 at a time.
+template <typename T, int NPT>
+__global__ void __launch_bounds__(128) scan_seq_kernel(ScanArgs a)
+{
+    constexpr int PR = 8, TC = 16;
+    extern __shared__ float sm[];
+    const int N = a.N, P = a.P;
+    float* Bs = sm;                  // [TC][N]
+    float* Cs = Bs + TC * N;         // [TC][N]
+    float* xs = Cs + TC * N;         // [TC][PR]
+    float* dts = xs + TC * PR;       // [TC]
+    const int b = blockIdx.z, i = blockIdx.y, p0 = blockIdx.x * PR;
+    const int tid = threadIdx.x, pr = tid >> 4, nq = tid & 15;
+    const int p = p0 + pr;
+    const int g = i / a.hpg;
+    const float Ai = a.A[i];
+    const float Di = a.D ? a.D[i] : 0.0f;
+    const T* X = static_cast<const T*>(a.x);
+    const T* Bm = static_cast<const T*>(a.B);
+    const T* Cm = static_cast<const T*>(a.C);
+    T* Y = static_cast<T*>(a.y);
+
+    float hs[NPT];
+#pragma unroll
+    for (int j = 0; j < NPT; ++j) {
+        const int n = nq + 16 * j;
+        hs[j] = (a.init_state && p < P && n < N) ? a.init_state[(int64_t)b * a.state_stride + ((int64_t)i * P + p) * N + n]
+                                                 : 0.0f;
+    }
+    for (int t0 = 0; t0 < a.L; t0 += TC) {
+        const int tc = min(TC, a.L - t0);
+        __syncthreads();
+        for (int e = tid; e < TC * N; e += 128) {
+            const int tt = e / N, n = e % N;
+            const int64_t tok = (int64_t)b * a.L + t0 + tt;
+            Bs[e] = tt < tc ? to_f32(Bm[tok * a.sB + (int64_t)g * N + n]) : 0.0f;
+            Cs[e] = tt < tc ? to_f32(Cm[tok * a.sC + (int64_t)g * N + n]) : 0.0f;
+        }
+        for (int e = tid; e < TC * PR; e += 128) {
+            const int tt = e / PR, q = p0 + e % PR;
+            const int64_t tok = (int64_t)b * a.L + t0 + tt;
+            xs[e] = (tt < tc && q < P) ? to_f32(X[tok * a.sx + (int64_t)i * P + q]) : 0.0f;
+        }
+        if (tid < TC) dts[tid] = tid < tc ? a.dt[((int64_t)b * a.L + t0 + tid) * a.sdt + i] : 0.0f;
+        __syncthreads();
+        for (int tt = 0; tt < tc; ++tt) {
+            const float dtv = dts[tt];
+            const float av = expf(dtv * Ai);
+            const float xv = xs[tt * PR + pr];
+            const float dx = dtv * xv;
+            float acc = 0.0f;
+#pragma unroll
+            for (int j = 0; j < NPT; ++j) {
+                const int n = nq + 16 * j;
+                if (n < N) {
+                    hs[j] = fmaf(av, hs[j], dx * Bs[tt * N + n]);
+                    acc = fmaf(Cs[tt * N + n], hs[j], acc);
+                }
+            }
+            acc += __shfl_xor_sync(0xffffffffu, acc, 8);
+            acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+            acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+            acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+            if (nq == 0 && p < P) {
+                const int64_t tok = (int64_t)b * a.L + t0 + tt;
+                Y[tok * a.sy + (int64_t)i * P + p] = from_f32<T>(fmaf(Di, xv, acc));
+            }
+        }
+    }
+    if (a.final_state && p < P) {
+#pragma unroll
+        for (int j = 0; j < NPT; ++j) {
+            const int n = nq + 16 * j;
+            if (n < N) a.final_state[(int64_t)b * a.state_stride + ((int64_t)i * P + p) * N + n] = hs[j];
+        }
+    }
+}
+
+template <typename T>
+static cudaError_t scan_seq_dispatch(const ScanArgs& a, cudaStream_t s)
+{
+    dim3 grid((a.P + 7) / 8, a.h, a.batch);
+    const size_t smem = sizeof(float) * (16 * a.N * 2 + 16 * 8 + 16);
+    if (a.N <= 16) scan_seq_kernel<T, 1><<<grid, 128, smem, s>>>(a);
+    else if (a.N <= 32) scan_seq_kernel<T, 2><<<grid, 128, smem, s>>>(a);
+    else if (a.N <= 64) scan_seq_kernel<T, 4><<<grid, 128, smem, s>>>(a);
+    else if (a.N <= 128) scan_seq_kernel<T, 8><<<grid, 128, smem, s>>>(a);
+    else scan_seq_kernel<T, 16><<<grid, 128, smem, s>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_scan_seq(int dtype, const ScanArgs& a, cudaStream_t s)
+{
+    if (a.batch == 0 || a.L == 0) return cudaSuccess;
+    return dtype == MM_BF16 ? scan_seq_dispatch<__nv_bfloat16>(a, s) : scan_seq_dispatch<float>(a, s);
+}
+
+// ====================================================================== gate + RMSNorm
+
+// One warp per token: q = y * SiLU(z); out = q / sqrt(mean(q^2) + eps) * w.
+template <typename T>
+__global__ void gate_rmsnorm_kernel(const T* __restrict__ y, int64_t ldy, const T* __restrict__ z, int64_t ldz,
+                                    const T* __restrict__ w, float eps, int d, int rows, T* __restrict__ out,
+                                    int64_t ldo)
+{
+    const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= rows) return;
+    const T* yr = y + (int64_t)row * ldy;
+    const T* zr = z + (int64_t)row * ldz;
+    float ss = 0.0f;
+    for (int c = lane; c < d; c += 32) {
+        const float q = to_f32(yr[c]) * silu_f(to_f32(zr[c]));
+        ss = fmaf(q, q, ss);
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    const float rstd = rsqrtf(ss / d + eps);
+    T* orow = out + (int64_t)row * ldo;
+    for (int c = lane; c < d; c += 32) {
+        const float q = to_f32(yr[c]) * silu_f(to_f32(zr[c]));
+        orow[c] = from_f32<T>(q * rstd * to_f32(w[c]));
+    }
+}
+
+cudaError_t launch_gate_rmsnorm(int dtype, const void* y, int64_t ldy, const void* z, int64_t ldz, const void* w,
+                                float eps, int d, int rows, void* out, int64_t ldo, cudaStream_t s)
+{
+    if (rows == 0) return cudaSuccess;
+    dim3 grid((rows + 7) / 8);
+    if (dtype == MM_BF16)
+        gate_rmsnorm_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
+            (const __nv_bfloat16*)y, ldy, (const __nv_bfloat16*)z, ldz, (const __nv_bfloat16*)w, eps, d, rows,
+            (__nv_bfloat16*)out, ldo);
+    else
+        gate_rmsnorm_kernel<float><<<grid, 256, 0, s>>>((const float*)y, ldy, (const float*)z, ldz, (const float*)w,
+                                                         eps, d, rows, (float*)out, ldo);
+    return cudaGetLastError();
+}
+
+// ====================================================================== residual pre-norm
+
+// One warp per row of the fp32 residual stream: out = x / sqrt(mean(x^2)+eps) * w.
+template <typename T>
+__global__ void rmsnorm_rows_kernel(const float* __restrict__ x, const T* __restrict__ w, float eps, int cols, int rows,
+                                    T* __restrict__ out)
+{
+    const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= rows) return;
+    const float* xr = x + (int64_t)row * cols;
+    float ss = 0.0f;
+    for (int c = lane; c < cols; c += 32) ss = fmaf(xr[c], xr[c], ss);
+#pragma unroll
+    for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    const float rstd = rsqrtf(ss / cols + eps);
+    for (int c = lane; c < cols; c += 32) out[(int64_t)row * cols + c] = from_f32<T>(xr[c] * rstd * to_f32(w[c]));
+}
+
+cudaError_t launch_rmsnorm_rows_f32in(int dtype, const float* x, const void* w, float eps, int cols, int rows, void* out,
+                                      cudaStream_t s)
+{
+    if (rows == 0) return cudaSuccess;
+    dim3 grid((rows + 7) / 8);
+    if (dtype == MM_BF16)
+        rmsnorm_rows_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(x, (const __nv_bfloat16*)w, eps, cols, rows,
+                                                                  (__nv_bfloat16*)out);
+    else
+        rmsnorm_rows_kernel<float><<<grid, 256, 0, s>>>(x, (const float*)w, eps, cols, rows, (float*)out);
+    return cudaGetLastError();
+}
+
+template <typename T>
+__global__ void to_f32_kernel(const T* __restrict__ in, float* __restrict__ out, int64_t n)
+{
+    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x)
+        out[e] = to_f32(in[e]);
+}
+
+template <typename T>
+__global__ void from_f32_kernel(const float* __restrict__ in, T* __restrict__ out, int64_t n)
+{
+    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x)
+        out[e] = from_f32<T>(in[e]);
+}
+
+cudaError_t launch_to_f32(int dtype, const void* in, float* out, int64_t n, cudaStream_t s)
+{
+    if (n == 0) return cudaSuccess;
+    const int64_t blocks = (n + 255) / 256;
+    const int grid = (int)(blocks < 148 * 16 ? blocks : 148 * 16);
+    if (dtype == MM_BF16) to_f32_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>((const __nv_bfloat16*)in, out, n);
+    else to_f32_kernel<float><<<grid, 256, 0, s>>>((const float*)in, out, n);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_from_f32(int dtype, const float* in, void* out, int64_t n, cudaStream_t s)
+{
+    if (n == 0) return cudaSuccess;
+    const int64_t blocks = (n + 255) / 256;
+    const int grid = (int)(blocks < 148 * 16 ? blocks : 148 * 16);
+    if (dtype == MM_BF16) from_f32_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(in, (__nv_bfloat16*)out, n);
+    else from_f32_kernel<float><<<grid, 256, 0, s>>>(in, (float*)out, n);
+    return cudaGetLastError();
+}
+
+// ====================================================================== decode step
+
+// Conv window roll for one token: each thread owns one (sequence, channel),
+// reads its K-1 stored inputs, appends the new one, writes the shifted window
+// back and emits SiLU(conv).  Threads past nconv compute dt for one head.
+template <typename T>
+__global__ void step_conv_dt_kernel(const T* __restrict__ zxbc, int64_t ld_in, int col0, const float* __restrict__ dt_raw,
+                                    const T* __restrict__ conv_w, const T* __restrict__ conv_b,
+                                    const float* __restrict__ dt_bias, int E, int d, int nconv, int h, int K,
+                                    T* __restrict__ conv_state, int conv_rows, T* __restrict__ xbc_out,
+                                    float* __restrict__ dt_out)
+{
+    const int c = blockIdx.x * blockDim.x + threadIdx.x;
+    const int b = blockIdx.y;
+    if (c >= nconv + h) return;
+    if (c >= nconv) {
+        const int i = c - nconv;
+        dt_out[(int64_t)b * h + i] = softplus_f(dt_raw[(int64_t)b * h + i] + dt_bias[i]);
+        return;
+    }
+    const int row = c < d ? c : E + (c - d);
+    T* st = conv_state + ((int64_t)b * conv_rows + row) * (K - 1);
+    const T vnew = zxbc[(int64_t)b * ld_in + col0 + c];
+    float acc = to_f32(conv_b[row]);
+    for (int j = 0; j < K; ++j) {
+        const float v = j < K - 1 ? to_f32(st[j]) : to_f32(vnew);
+        acc = fmaf(to_f32(conv_w[(int64_t)row * K + j]), v, acc);
+    }
+    for (int k = 0; k < K - 2; ++k) st[k] = st[k + 1];
+    if (K > 1) st[K - 2] = vnew;
+    xbc_out[(int64_t)b * nconv + c] = from_f32<T>(silu_f(acc));
+}
+
+cudaError_t launch_step_conv_dt(int dtype, const void* zxbc, int64_t ld_in, int col0, const float* dt_raw,
+                                const void* conv_w, const void* conv_b, const float* dt_bias, int E, int d, int nconv,
+                                int h, int K, int batch, void* conv_state, int conv_rows, void* xbc_out, float* dt_out,
+                                cudaStream_t s)
+{
+    dim3 grid((nconv + h + 127) / 128, batch);
+    if (dtype == MM_BF16)
+        step_conv_dt_kernel<__nv_bfloat16><<<grid, 128, 0, s>>>(
+            (const __nv_bfloat16*)zxbc, ld_in, col0, dt_raw, (const __nv_bfloat16*)conv_w,
+            (const __nv_bfloat16*)conv_b, dt_bias, E, d, nconv, h, K, (__nv_bfloat16*)conv_state, conv_rows,
+            (__nv_bfloat16*)xbc_out, dt_out);
+    else
+        step_conv_dt_kernel<float><<<grid, 128, 0, s>>>((const float*)zxbc, ld_in, col0, dt_raw, (const float*)conv_w,
+                                                         (const float*)conv_b, dt_bias, E, d, nconv, h, K,
+                                                         (float*)conv_state, conv_rows, (float*)xbc_out, dt_out);
+    return cudaGetLastError();
+}
+
+// State update for one token: one warp per (sequence, head, p) row of N fp32
+// state entries, H <- exp(dt A) H + dt x_p B; y_p = C . H + D x_p.
+template <typename T>
+__global__ void step_scan_kernel(const T* __restrict__ xbc, int nconv, int d, const float* __restrict__ dt,
+                                 const float* __restrict__ A, const float* __restrict__ D, float* __restrict__ ssm_state,
+                                 int H, int h, int P, int N, int GN, int hpg, int batch, T* __restrict__ y)
+{
+    const int64_t wid = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    const int64_t nrows = (int64_t)batch * h * P;
+    if (wid >= nrows) return;
+    const int p = (int)(wid % P);
+    const int i = (int)((wid / P) % h);
+    const int b = (int)(wid / ((int64_t)P * h));
+    const int g = i / hpg;
+    const T* xr = xbc + (int64_t)b * nconv;
+    const float xv = to_f32(xr[i * P + p]);
+    const float dtv = dt[(int64_t)b * h + i];
+    const float av = expf(dtv * A[i]);
+    const float dx = dtv * xv;
+    const T* Bv = xr + d + g * (N);
+    const T* Cv = xr + d + GN + g * (N);
+    float* st = ssm_state + (((int64_t)b * H + i) * P + p) * N;
+    float acc = 0.0f;
+    for (int n = lane; n < N; n += 32) {
+        const float hv = fmaf(av, st[n], dx * to_f32(Bv[n]));
+        st[n] = hv;
+        acc = fmaf(to_f32(Cv[n]), hv, acc);
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) y[(int64_t)b * d + i * P + p] = from_f32<T>(fmaf(D[i], xv, acc));
+}
+
+cudaError_t launch_step_scan(int dtype, const void* xbc, int nconv, int d, const float* dt, const float* A,
+                             const float* D, float* ssm_state, int H, int h, int P, int N, int GN, int hpg, int batch,
+                             void* y, cudaStream_t s)
+{
+    const int64_t rows = (int64_t)batch * h * P;
+    if (rows == 0) return cudaSuccess;
+    dim3 grid((unsigned)((rows + 7) / 8));
+    if (dtype == MM_BF16)
+        step_scan_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>((const __nv_bfloat16*)xbc, nconv, d, dt, A, D, ssm_state, H,
+                                                              h, P, N, GN, hpg, batch, (__nv_bfloat16*)y);
+    else
+        step_scan_kernel<float><<<grid, 256, 0, s>>>((const float*)xbc, nconv, d, dt, A, D, ssm_state, H, h, P, N, GN,
+                                                      hpg, batch, (float*)y);
+    return cudaGetLastError();
+}
+
+}  // namespace mm

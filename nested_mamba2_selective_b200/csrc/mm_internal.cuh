@@ -1,0 +1,101 @@
+// Internal declarations shared by the kernels and the C-ABI layer.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/matmamba.h"
+
+namespace mm {
+
+// ------------------------------------------------------------------ element access
+
+__device__ __forceinline__ float to_f32(float v) { return v; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
+template <typename T> __device__ __forceinline__ T from_f32(float v);
+template <> __device__ __forceinline__ float from_f32<float>(float v) { return v; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float v) { return __float2bfloat16_rn(v); }
+
+// SiLU(a) = a * sigmoid(a) ("MatMamba: A Matryoshka State Space Model": sigma = SiLU).
+__device__ __forceinline__ float silu_f(float a) { return a / (1.0f + expf(-a)); }
+
+// softplus(v) = log(1 + e^v).  Above 20 the identity is within 2.1e-9 relative.
+__device__ __forceinline__ float softplus_f(float v) { return v > 20.0f ? v : log1pf(expf(v)); }
+
+// ------------------------------------------------------------------ segmented GEMM
+//
+// out_s[m, j] (+)= sum_k A[m, k] * Bs[j, k] for j in [0, n_s) of each segment s.
+// A and every Bs are K-major (rows of K contiguous elements).  The segments
+// concatenate along N; they let one launch read a width view of W_in whose
+// rows sit in four separate blocks, and route each block of output columns to
+// its own buffer (and dtype).
+struct GemmSeg {
+    const void* B;   // first row of this segment's weights, row stride ldb
+    void* out;       // output of this segment's first column, row stride ldo
+    int64_t ldo;
+    int n;           // number of columns (rows of B) in this segment
+    int out_f32;     // output stored as fp32 (else in the input dtype)
+    int accumulate;  // fp32 output only: out += result
+};
+
+constexpr int kMaxSeg = 4;
+
+struct GemmDesc {
+    const void* A;
+    int64_t lda;
+    int64_t ldb;
+    int M, K;
+    int nseg;
+    GemmSeg seg[kMaxSeg];
+};
+
+// ------------------------------------------------------------------ scan arguments
+
+struct ScanArgs {
+    const void* x; int64_t sx;
+    const float* dt; int64_t sdt;
+    const float* A;
+    const void* B; int64_t sB;
+    const void* C; int64_t sC;
+    const float* D;
+    int batch, L, h, P, N, G, hpg, chunk;
+    const float* init_state; int64_t state_stride;
+    void* y; int64_t sy;
+    float* final_state;
+};
+
+// ------------------------------------------------------------------ launchers (return cudaError_t)
+
+cudaError_t launch_gemm_simt(int dtype, const GemmDesc& g, cudaStream_t s);
+cudaError_t launch_conv_silu_dt(int dtype, const void* zxbc, int64_t ld_in, int col0, const float* dt_raw,
+                                const void* conv_w, const void* conv_b, const float* dt_bias, int E, int d, int nconv,
+                                int h, int K, int batch, int L, const void* conv_state_in, int conv_rows, void* xbc_out,
+                                float* dt_out, cudaStream_t s);
+cudaError_t launch_conv_state_out(int dtype, const void* zxbc, int64_t ld_in, int col0, int E, int d, int nconv, int K,
+                                  int batch, int L, const void* conv_state_in, int conv_rows, void* conv_state_out,
+                                  cudaStream_t s);
+cudaError_t launch_scan_seq(int dtype, const ScanArgs& a, cudaStream_t s);
+cudaError_t launch_gate_rmsnorm(int dtype, const void* y, int64_t ldy, const void* z, int64_t ldz, const void* w,
+                                float eps, int d, int rows, void* out, int64_t ldo, cudaStream_t s);
+cudaError_t launch_rmsnorm_rows_f32in(int dtype, const float* x, const void* w, float eps, int cols, int rows, void* out,
+                                      cudaStream_t s);
+cudaError_t launch_to_f32(int dtype, const void* in, float* out, int64_t n, cudaStream_t s);
+cudaError_t launch_from_f32(int dtype, const float* in, void* out, int64_t n, cudaStream_t s);
+cudaError_t launch_step_conv_dt(int dtype, const void* zxbc, int64_t ld_in, int col0, const float* dt_raw,
+                                const void* conv_w, const void* conv_b, const float* dt_bias, int E, int d, int nconv,
+                                int h, int K, int batch, void* conv_state, int conv_rows, void* xbc_out, float* dt_out,
+                                cudaStream_t s);
+cudaError_t launch_step_scan(int dtype, const void* xbc, int nconv, int d, const float* dt, const float* A,
+                             const float* D, float* ssm_state, int H, int h, int P, int N, int GN, int hpg, int batch,
+                             void* y, cudaStream_t s);
+
+// Tensor-core paths (bf16 only).
+bool gemm_tc_supported(const GemmDesc& g);
+cudaError_t launch_gemm_tc(const GemmDesc& g, cudaStream_t s);
+bool scan_tc_supported(const ScanArgs& a);
+size_t scan_tc_workspace(const ScanArgs& a);
+int scan_tc_kernel_count(const ScanArgs& a);
+cudaError_t launch_scan_tc(const ScanArgs& a, void* ws, size_t ws_bytes, cudaStream_t s);
+
+}  // namespace mm
