@@ -98,6 +98,15 @@ const char* mm_status_string(int status);
 int mm_version(void);
 
 /*
+ * Device-side status of the current device: synchronizes `stream`, returns
+ * MM_OK, or MM_ERR_TIMEOUT if a kernel's bounded wait (at most about two
+ * seconds on one barrier) gave up since the last call, and clears the word.
+ * Kernels never trap; a timed-out kernel skips its remaining work and exits,
+ * so its outputs are then undefined.
+ */
+int mm_device_status(void* stream);
+
+/*
  * Width rule (nested sub-block paragraph; Mix'n'Match paragraph: any m_i that
  * gives an integer number of heads is valid).  Host only.
  * Valid iff 0 < m_i <= D_m, E*m_i divisible by D_m, and d = E*m_i/D_m
@@ -143,6 +152,17 @@ int matmamba_block_fwd(const mm_block_params* p, const void* u, int batch, int L
 int matmamba_block_fwd_host(const mm_block_params* p, const void* u_host, int batch, int L, int m_i, int chunk,
                             void* out_host, void* u_dev, void* out_dev, void* workspace, size_t ws_bytes,
                             void* stream);
+
+/*
+ * Projection primitive used for in_proj and out_proj: out[m, n] (+)=
+ * sum_k A[m, k] * W[n, k] for m < M, n < N, k < K.  A (M rows, pitch lda)
+ * and W (N rows, pitch ldw) are K-major in `dtype`.  out has pitch ldo and
+ * holds fp32 when out_f32 != 0 (bf16 inputs only; accumulate != 0 then adds
+ * to it), else `dtype`.  bf16 runs on the tensor cores when the operands are
+ * 16-byte aligned with pitches that are multiples of 8 elements.
+ */
+int mm_linear(int dtype, const void* A, int64_t lda, int M, int K, const void* W, int64_t ldw, int N, void* out,
+              int64_t ldo, int out_f32, int accumulate, void* stream);
 
 /* Workspace bytes for ssd_scan.  Host only. */
 int ssd_scan_workspace(int dtype, int batch, int L, int h, int P, int N, int G, int chunk, size_t* bytes);

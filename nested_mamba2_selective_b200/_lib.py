@@ -42,6 +42,7 @@ _pp = ctypes.POINTER(BlockParamsC)
 _SIGS = {
     "mm_status_string": ([_i], ctypes.c_char_p),
     "mm_version": ([], _i),
+    "mm_device_status": ([_vp], _i),
     "mm_width": ([_pp, _i, ctypes.POINTER(_i), ctypes.POINTER(_i)], _i),
     "matmamba_block_workspace": ([_pp, _i, _i, _i, _i, ctypes.POINTER(_sz)], _i),
     "matmamba_block_fwd": ([_pp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp], _i),
@@ -54,6 +55,7 @@ _SIGS = {
     "matmamba_stack_workspace": ([_pp, _i, ctypes.POINTER(_i), _i, _i, _i, ctypes.POINTER(_sz)], _i),
     "matmamba_stack_fwd": ([_pp, ctypes.POINTER(_vp), _f, _i, ctypes.POINTER(_i), _vp, _i, _i, _i, _vp, _vp, _sz,
                             _vp], _i),
+    "mm_linear": ([_i, _vp, _i64, _i, _i, _vp, _i64, _i, _vp, _i64, _i, _i, _vp], _i),
     "mm_trace_enable": ([_i], _i),
     "mm_trace_collect": ([_vp, _i, ctypes.POINTER(_i), ctypes.POINTER(_i)], _i),
 }
@@ -73,6 +75,11 @@ def load() -> ctypes.CDLL:
             fn.argtypes, fn.restype = args, res
         _lib = lib
     return _lib
+
+
+def mm_device_status(stream=None) -> int:
+    """Synchronize the stream and return (then clear) the device status word."""
+    return int(load().mm_device_status(_stream(stream)))
 
 
 def status_string(status: int) -> str:
@@ -195,6 +202,21 @@ def matmamba_block_fwd_host(w: BlockWeights, u_host: torch.Tensor, m_i: int, chu
                                         _ptr(out_dev), _ptr(workspace), workspace.numel(), _stream(stream))
     _check(rc, "matmamba_block_fwd_host")
     return out_host
+
+
+def mm_linear(A: torch.Tensor, W: torch.Tensor, out=None, out_f32: bool = False, accumulate: bool = False,
+              stream=None):
+    """out (M, N) (+)= A (M, K) . W (N, K)^T through the library's projection kernel."""
+    M, K = A.shape
+    N = W.shape[0]
+    if W.shape[1] != K or W.dtype != A.dtype:
+        raise ValueError("W must be (N, K) in A's dtype")
+    if out is None:
+        out = torch.zeros((M, N), dtype=torch.float32 if out_f32 else A.dtype, device=A.device)
+    rc = load().mm_linear(_DTYPES[A.dtype], _ptr(A), K, M, K, _ptr(W), K, N, _ptr(out), out.shape[1],
+                          int(out_f32), int(accumulate), _stream(stream))
+    _check(rc, "mm_linear")
+    return out
 
 
 def ssd_scan_workspace(dtype, batch, L, h, P, N, G=1, chunk=256) -> int:

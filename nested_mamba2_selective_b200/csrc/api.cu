@@ -7,6 +7,24 @@
 
 using namespace mm;
 
+// Status word a kernel writes when a bounded wait gives up (one per device).
+__device__ int g_mm_device_status;
+
+namespace mm {
+int* device_status_ptr()
+{
+    static int* ptrs[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return nullptr;
+    if (!ptrs[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_mm_device_status) != cudaSuccess) return nullptr;
+        ptrs[dev] = static_cast<int*>(p);
+    }
+    return ptrs[dev];
+}
+}  // namespace mm
+
 namespace {
 
 constexpr size_t kAlign = 256;
@@ -250,6 +268,16 @@ const char* mm_status_string(int status)
 
 int mm_version(void) { return 100; }
 
+int mm_device_status(void* stream)
+{
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return MM_ERR_CUDA;
+    int v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_mm_device_status, sizeof(int)) != cudaSuccess) return MM_ERR_CUDA;
+    if (v && cudaMemcpyToSymbol(g_mm_device_status, &zero, sizeof(int)) != cudaSuccess) return MM_ERR_CUDA;
+    return v;
+}
+
 int mm_width(const mm_block_params* p, int m_i, int* d_out, int* h_out)
 {
     View v;
@@ -385,6 +413,24 @@ int ssd_scan(int dtype, const void* x, int64_t x_stride, const float* dt, int64_
     if (need && reinterpret_cast<uintptr_t>(workspace) % kAlign) return MM_ERR_ALIGN;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     return cuda_status(stage("ssd_scan", scan_kernels(dtype, a), s, [&] { return run_scan(dtype, a, workspace, ws_bytes, s); }));
+}
+
+int mm_linear(int dtype, const void* A, int64_t lda, int M, int K, const void* W, int64_t ldw, int N, void* out,
+              int64_t ldo, int out_f32, int accumulate, void* stream)
+{
+    if (!dtype_ok(dtype)) return MM_ERR_DTYPE;
+    if (!A || !W || !out) return MM_ERR_NULL;
+    if (M < 0 || K <= 0 || N <= 0 || lda < K || ldw < K || ldo < N) return MM_ERR_SHAPE;
+    if (accumulate && !out_f32) return MM_ERR_SHAPE;
+    if (dtype == MM_F32 && !out_f32) out_f32 = 0;
+    if (dtype == MM_BF16 && (!aligned16(A) || !aligned16(W) || lda % 8 || ldw % 8)) return MM_ERR_ALIGN;
+    if (M == 0) return MM_OK;
+    GemmDesc g{};
+    g.A = A; g.lda = lda; g.ldb = ldw; g.M = M; g.K = K; g.nseg = 1;
+    g.seg[0] = GemmSeg{W, out, ldo, N, out_f32 ? 1 : 0, accumulate ? 1 : 0};
+    if (dtype == MM_F32) g.seg[0].out_f32 = 1;  // fp32 path: plain or accumulating fp32 stores
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    return cuda_status(stage("linear", 1, s, [&] { return run_gemm(dtype, g, s); }));
 }
 
 static size_t step_ws(const View& v, const mm_block_params* p, int batch)

@@ -1,0 +1,341 @@
+// Tensor-core projection GEMM for sm_100a: out = A . B^T with bf16 operands,
+// fp32 accumulation in TMEM, TMA-fed shared-memory stages, and a persistent
+// tile loop.  Serves in_proj (A = u, B = the four row blocks of the W_in
+// width view, routed to z | x | B | C and an fp32 dt buffer) and out_proj
+// (A = normalised activations, B = W_out with its K-prefix [0, d)); the width
+// view is a set of row offsets and a K extent, never a weight copy
+// ("MatMamba: A Matryoshka State Space Model", nested sub-block paragraph:
+// W_x becomes W_x[0:d_i] by slicing along d_inner).
+//
+// CTA layout (192 threads): warp 0 issues TMA loads, warp 1 owns TMEM and
+// issues tcgen05.mma from one lane, warps 2-5 drain the accumulator (one TMEM
+// lane = one output row per thread) and store.  Two TMEM accumulators let the
+// drain of tile i overlap the MMAs of tile i+1.
+#include <cuda.h>
+
+#include "mm_internal.cuh"
+#include "sm100.cuh"
+
+namespace mm {
+
+using namespace sm100;
+
+namespace {
+
+constexpr int kBM = 128;  // rows of a tile = TMEM lanes
+constexpr int kBK = 64;   // one 128-byte swizzle atom of bf16 along K
+
+struct TcSeg {
+    void* out;
+    int64_t ldo;
+    int b_row0;  // row of the B tensor map holding this segment's column 0
+    int n;       // columns in the segment
+    int ntiles;  // ceil(n / BN)
+    int out_f32;
+    int accumulate;
+    int vec_ok;  // 16-byte vector stores allowed
+};
+
+struct TcParams {
+    int M, K, ktiles, mtiles, ntiles, nseg;
+    TcSeg seg[kMaxSeg];
+    int* status;
+};
+
+template <int BN>
+struct TileInfo {
+    int mt, seg, n0, nvalid, b_row;
+};
+
+template <int BN>
+__device__ __forceinline__ TileInfo<BN> tile_info(const TcParams& p, int tile)
+{
+    TileInfo<BN> t;
+    t.mt = tile / p.ntiles;
+    int j = tile % p.ntiles;
+    int s = 0;
+    while (s < p.nseg - 1 && j >= p.seg[s].ntiles) j -= p.seg[s++].ntiles;
+    t.seg = s;
+    t.n0 = j * BN;
+    t.nvalid = min(BN, p.seg[s].n - t.n0);
+    t.b_row = p.seg[s].b_row0 + t.n0;
+    return t;
+}
+
+__device__ __forceinline__ void store_chunk(const TcSeg& sg, int64_t row, int col, int ncols, const uint32_t (&v)[32])
+{
+    if (sg.out_f32) {
+        float* o = static_cast<float*>(sg.out) + row * sg.ldo + col;
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+            if (i < ncols) o[i] = sg.accumulate ? o[i] + __uint_as_float(v[i]) : __uint_as_float(v[i]);
+        return;
+    }
+    __nv_bfloat16* o = static_cast<__nv_bfloat16*>(sg.out) + row * sg.ldo + col;
+    if (ncols == 32 && sg.vec_ok) {
+        uint4* o4 = reinterpret_cast<uint4*>(o);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            uint4 w;
+            w.x = pack_bf16(__uint_as_float(v[8 * q + 0]), __uint_as_float(v[8 * q + 1]));
+            w.y = pack_bf16(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3]));
+            w.z = pack_bf16(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5]));
+            w.w = pack_bf16(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7]));
+            o4[q] = w;
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+            if (i < ncols) o[i] = __float2bfloat16_rn(__uint_as_float(v[i]));
+    }
+}
+
+template <int BN, int STAGES>
+__global__ void __launch_bounds__(192, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB, const TcParams p)
+{
+    constexpr int A_BYTES = kBM * kBK * 2;
+    constexpr int B_BYTES = BN * kBK * 2;
+    constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    constexpr uint32_t TMEM_COLS = 2 * BN;
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+    uint64_t* empty = full + STAGES;
+    uint64_t* tfull = empty + STAGES;
+    uint64_t* tempty = tfull + 2;
+    uint64_t* done = tempty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+    volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], 4);
+        }
+        mbar_init(done, 1);
+        *abort = 0;
+        fence_mbar_init();
+        prefetch_tmap(&mapA);
+        prefetch_tmap(&mapB);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const int total = p.mtiles * p.ntiles;
+
+    if (warp == 0) {
+        if (lane == 0) {  // ---------------- TMA producer
+            int it = 0;
+            for (int tile = blockIdx.x; tile < total && !*abort; tile += gridDim.x) {
+                const TileInfo<BN> t = tile_info<BN>(p, tile);
+                for (int kt = 0; kt < p.ktiles; ++kt, ++it) {
+                    const int s = it % STAGES;
+                    if (!mbar_wait(&empty[s], ((it / STAGES) & 1) ^ 1, abort)) {
+                        raise_timeout(abort, p.status);
+                        break;
+                    }
+                    uint8_t* sa = smem + s * STAGE_BYTES;
+                    mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
+                    tma_load_2d(sa, &mapA, &full[s], kt * kBK, t.mt * kBM);
+                    tma_load_2d(sa + A_BYTES, &mapB, &full[s], kt * kBK, t.b_row);
+                }
+            }
+            // every issued load lands before the CTA can exit (bounded)
+            for (int j = max(0, it - STAGES); j < it; ++j) mbar_wait(&full[j % STAGES], (j / STAGES) & 1, abort);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {  // ---------------- MMA issuer
+            int it = 0, tc = 0;
+            for (int tile = blockIdx.x; tile < total && !*abort; tile += gridDim.x, ++tc) {
+                const TileInfo<BN> t = tile_info<BN>(p, tile);
+                const int buf = tc & 1;
+                if (!mbar_wait(&tempty[buf], ((tc >> 1) & 1) ^ 1, abort)) {
+                    raise_timeout(abort, p.status);
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem + buf * BN;
+                const int nmma = (t.nvalid + 15) & ~15;
+                const uint32_t idesc = idesc_bf16(kBM, nmma, 0, 0);
+                for (int kt = 0; kt < p.ktiles; ++kt, ++it) {
+                    const int s = it % STAGES;
+                    if (!mbar_wait(&full[s], (it / STAGES) & 1, abort)) {
+                        raise_timeout(abort, p.status);
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a0 = smem_u32(smem + s * STAGE_BYTES);
+                    const uint32_t b0 = a0 + A_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < kBK / 16; ++kk)
+                        mma_ss(d_tmem, desc_sw128(a0 + kk * 32, 16, 1024), desc_sw128(b0 + kk * 32, 16, 1024), idesc,
+                               (kt | kk) != 0);
+                    mma_commit(&empty[s]);
+                }
+                mma_commit(&tfull[buf]);
+            }
+            // every issued MMA has finished before TMEM can be released (bounded)
+            mma_commit(done);
+            mbar_wait(done, 0, nullptr);
+        }
+    } else {  // ---------------- epilogue: warps 2..5
+        const int q = warp & 3;
+        const int row_in_tile = q * 32 + lane;
+        int tc = 0;
+        for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++tc) {
+            const TileInfo<BN> t = tile_info<BN>(p, tile);
+            const int buf = tc & 1;
+            if (!mbar_wait(&tfull[buf], (tc >> 1) & 1, abort)) {
+                raise_timeout(abort, p.status);
+                break;
+            }
+            tc_fence_after();
+            const TcSeg& sg = p.seg[t.seg];
+            const int64_t row = (int64_t)t.mt * kBM + row_in_tile;
+            for (int c0 = 0; c0 < t.nvalid; c0 += 32) {
+                uint32_t v[32];
+                tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + buf * BN + c0, v);
+                tmem_ld_wait();
+                if (row < p.M) store_chunk(sg, row, t.n0 + c0, min(32, t.nvalid - c0), v);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty[buf]);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, TMEM_COLS);
+}
+
+// --------------------------------------------------------------------------- host side
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+}  // namespace
+
+// 2-D bf16 tensor map with a 128-byte swizzle: inner extent `inner` elements,
+// `rows` rows `pitch` bytes apart, box of box_inner x box_rows.
+bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint64_t pitch,
+                    uint32_t box_inner, uint32_t box_rows)
+{
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {inner, rows};
+    cuuint64_t strides[1] = {pitch};
+    cuuint32_t box[2] = {box_inner, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+static bool tc_shape_ok(const GemmDesc& g)
+{
+    auto al16 = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15u) == 0; };
+    if (g.M <= 0 || g.K <= 0 || g.nseg <= 0 || g.nseg > kMaxSeg) return false;
+    if (g.K % 8 || g.lda % 8 || g.ldb % 8 || g.lda < g.K || g.ldb < g.K) return false;
+    if (!al16(g.A)) return false;
+    const char* base = static_cast<const char*>(g.seg[0].B);
+    for (int s = 0; s < g.nseg; ++s) {
+        const char* b = static_cast<const char*>(g.seg[s].B);
+        if (b < base || (b - base) % (g.ldb * 2) || g.seg[s].n <= 0) return false;
+        if (g.seg[s].accumulate && !g.seg[s].out_f32) return false;
+    }
+    if (!al16(base)) return false;
+    return true;
+}
+
+bool gemm_tc_supported(const GemmDesc& g) { return tc_shape_ok(g) && encode_fn() != nullptr; }
+
+template <int BN, int STAGES>
+static cudaError_t launch_bn(const GemmDesc& g, const TcParams& p0, cudaStream_t s, int* status)
+{
+    TcParams p = p0;
+    p.ntiles = 0;
+    for (int i = 0; i < p.nseg; ++i) {
+        p.seg[i].ntiles = (p.seg[i].n + BN - 1) / BN;
+        p.ntiles += p.seg[i].ntiles;
+    }
+    p.status = status;
+    const char* base = static_cast<const char*>(g.seg[0].B);
+    int64_t rows = 0;
+    for (int i = 0; i < p.nseg; ++i) rows = max(rows, (int64_t)p.seg[i].b_row0 + p.seg[i].n);
+    CUtensorMap mapA, mapB;
+    if (!make_tmap_bf16(&mapA, g.A, g.K, g.M, g.lda * 2, kBK, kBM)) return cudaErrorInvalidValue;
+    if (!make_tmap_bf16(&mapB, base, g.ldb, rows, g.ldb * 2, kBK, BN)) return cudaErrorInvalidValue;
+    constexpr int smem = STAGES * (kBM + BN) * kBK * 2 + 1024 + 256;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    static unsigned long long attr_set = 0;  // one bit per device
+    if (dev < 64 && !(attr_set >> dev & 1ull)) {
+        cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             smem);
+        if (e != cudaSuccess) return e;
+        attr_set |= 1ull << dev;
+    }
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int total = p.mtiles * p.ntiles;
+    const int grid = total < sms ? total : sms;
+    gemm_tc_kernel<BN, STAGES><<<grid, 192, smem, s>>>(mapA, mapB, p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gemm_tc(const GemmDesc& g, cudaStream_t s)
+{
+    TcParams p{};
+    p.M = g.M;
+    p.K = g.K;
+    p.ktiles = (g.K + kBK - 1) / kBK;
+    p.mtiles = (g.M + kBM - 1) / kBM;
+    p.nseg = g.nseg;
+    const char* base = static_cast<const char*>(g.seg[0].B);
+    int n_total = 0;
+    for (int i = 0; i < g.nseg; ++i) {
+        const GemmSeg& sg = g.seg[i];
+        TcSeg& t = p.seg[i];
+        t.out = sg.out;
+        t.ldo = sg.ldo;
+        t.b_row0 = (int)((static_cast<const char*>(sg.B) - base) / (g.ldb * 2));
+        t.n = sg.n;
+        t.out_f32 = sg.out_f32;
+        t.accumulate = sg.accumulate;
+        t.vec_ok = !sg.out_f32 && (reinterpret_cast<uintptr_t>(sg.out) & 15u) == 0 && sg.ldo % 8 == 0;
+        n_total += sg.n;
+    }
+    int* status = device_status_ptr();
+    // Wide tiles when they still give every SM work; narrow ones for skinny problems.
+    const int tiles256 = p.mtiles * ((n_total + 255) / 256);
+    if (tiles256 >= 148) return launch_bn<256, 4>(g, p, s, status);
+    return launch_bn<128, 6>(g, p, s, status);
+}
+
+}  // namespace mm

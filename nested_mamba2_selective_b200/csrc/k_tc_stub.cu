@@ -3,8 +3,6 @@
 #include "mm_internal.cuh"
 
 namespace mm {
-bool gemm_tc_supported(const GemmDesc&) { return false; }
-cudaError_t launch_gemm_tc(const GemmDesc&, cudaStream_t) { return cudaErrorNotSupported; }
 bool scan_tc_supported(const ScanArgs&) { return false; }
 size_t scan_tc_workspace(const ScanArgs&) { return 0; }
 int scan_tc_kernel_count(const ScanArgs&) { return 0; }

@@ -1,6 +1,7 @@
 // Internal declarations shared by the kernels and the C-ABI layer.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -89,6 +90,11 @@ cudaError_t launch_step_conv_dt(int dtype, const void* zxbc, int64_t ld_in, int 
 cudaError_t launch_step_scan(int dtype, const void* xbc, int nconv, int d, const float* dt, const float* A,
                              const float* D, float* ssm_state, int H, int h, int P, int N, int GN, int hpg, int batch,
                              void* y, cudaStream_t s);
+
+// Device status word of the current device (MM_OK or a code a kernel recorded).
+int* device_status_ptr();
+bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint64_t pitch,
+                    uint32_t box_inner, uint32_t box_rows);
 
 // Tensor-core paths (bf16 only).
 bool gemm_tc_supported(const GemmDesc& g);

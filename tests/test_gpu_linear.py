@@ -1,0 +1,47 @@
+"""GPU checks of the projection kernel (mm_linear) against an fp64 matmul of the same inputs."""
+import numpy as np
+import pytest
+import torch
+
+from gpu_util import ensure_built, max_abs_rel, to_np
+from nested_mamba2_selective_b200 import mm_device_status, mm_linear, synth
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    ensure_built()
+
+
+@pytest.mark.parametrize("M,K,N", [(1000, 768, 3352), (256, 2048, 8512), (130, 200, 72), (16384, 1536, 768),
+                                   (7, 64, 16), (300, 4096, 2048)])
+def test_linear_bf16(M, K, N):
+    a = synth.activations((M, K), "bf16", seed=M + K)
+    w = synth.activations((N, K), "bf16", seed=N + 7, std=0.05)
+    out = mm_linear(torch.from_numpy(a).cuda().bfloat16(), torch.from_numpy(w).cuda().bfloat16())
+    assert mm_device_status() == 0
+    ref = a.astype(np.float64) @ w.astype(np.float64).T
+    assert max_abs_rel(to_np(out), ref) <= 5e-3
+
+
+@pytest.mark.parametrize("M,K,N", [(333, 768, 24), (512, 512, 256)])
+def test_linear_fp32_out_and_accumulate(M, K, N):
+    a = synth.activations((M, K), "bf16", seed=1)
+    w = synth.activations((N, K), "bf16", seed=2, std=0.05)
+    A, W = torch.from_numpy(a).cuda().bfloat16(), torch.from_numpy(w).cuda().bfloat16()
+    base = torch.from_numpy(synth.activations((M, N), "f32", seed=3)).cuda()
+    out = mm_linear(A, W, out=base.clone(), out_f32=True, accumulate=True)
+    plain = mm_linear(A, W, out_f32=True)
+    torch.cuda.synchronize()
+    ref = a.astype(np.float64) @ w.astype(np.float64).T
+    assert max_abs_rel(to_np(plain), ref) <= 1e-5
+    assert max_abs_rel(to_np(out), ref + base.cpu().numpy()) <= 1e-5
+
+
+def test_linear_fp32():
+    a = synth.activations((100, 96), "f32", seed=4)
+    w = synth.activations((40, 96), "f32", seed=5)
+    out = mm_linear(torch.from_numpy(a).cuda(), torch.from_numpy(w).cuda())
+    torch.cuda.synchronize()
+    assert max_abs_rel(to_np(out), a.astype(np.float64) @ w.astype(np.float64).T) <= 1e-5
