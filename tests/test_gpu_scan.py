@@ -108,3 +108,23 @@ def test_scan_without_skip_term(orc):
     torch.cuda.synchronize()
     ref, _ = orc.ssd_scan(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], None)
     assert max_abs_rel(to_np(y), ref) <= TOL["bf16"]
+
+
+def test_scan_two_groups(orc):
+    """ngroups = 2: heads 0-1 read group 0, heads 2-3 group 1."""
+    inp = synth.long_memory(synth.ssd_inputs(2, 300, 4, 64, 128, 2, "bf16", seed=206))
+    g = upload(inp, "bf16")
+    y = ssd_scan(g["x"], g["dt"], g["A"], g["B"], g["C"], g["D"], chunk=256, heads_per_group=2)
+    torch.cuda.synchronize()
+    ref, _ = orc.ssd_scan(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], inp["D"], heads_per_group=2)
+    assert max_abs_rel(to_np(y), ref) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("chunk", [128, 256, 512])
+def test_scan_chunk_parameter_does_not_change_the_result(orc, chunk):
+    inp = synth.long_memory(synth.ssd_inputs(1, 700, 3, 64, 128, 1, "bf16", seed=207))
+    g = upload(inp, "bf16")
+    y = ssd_scan(g["x"], g["dt"], g["A"], g["B"], g["C"], g["D"], chunk=chunk)
+    torch.cuda.synchronize()
+    ref, _ = oracle_scan(orc, inp, 3)
+    assert max_abs_rel(to_np(y), ref) <= TOL["bf16"]
