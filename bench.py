@@ -38,8 +38,12 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--extended", action="store_true", help="also time the 48-layer stack and the decode step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", choices=["block", "scan"], default=None,
+                    help="profiling aid: run just the headline block or just the standalone scan, print per-stage "
+                         "times and no benchmark line")
     a = ap.parse_args()
-    a.warmup = max(a.warmup, 3)
+    if a.only is None:
+        a.warmup = max(a.warmup, 3)
     return a
 
 
@@ -66,6 +70,9 @@ def block_work(m, T, Dm=768, E=1536, P=64, N=128):
     h = d // P
     nconv = d + 2 * N
     return {
+        "in_proj_conv": ("tensor", 2.0 * T * Dm * (2 * d + 2 * N + h)),
+        "ssd_scan_gate": ("hbm", T * ((d + 2 * N) * 2 + h * 4 + d * 2 + d * 2 + 2 * h * 4)),
+        "out_proj_norm": ("tensor", 2.0 * T * d * Dm),
         "in_proj": ("tensor", 2.0 * T * Dm * (2 * d + 2 * N + h)),
         "conv_silu_dt": ("hbm", T * (nconv * 2 * 2 + h * 4 * 2)),
         "ssd_scan": ("hbm", T * (2 * d * 2 + 2 * N * 2 + h * 4)),
@@ -193,6 +200,9 @@ def run_ours(args):
             mm.mm_trace_enable(0)
         return ms, tr
 
+    if args.only:
+        return run_only(args, mm, synth, torch, dev, timed)
+
     # ---------------- block workload (headline)
     B = BLOCK
     arrays = synth.block_params(B["d_model"], B["d_inner"], B["d_head"], B["d_state"], dtype="bf16", seed=1002)
@@ -310,6 +320,27 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def run_only(args, mm, synth, torch, dev, timed):
+    """One workload piece with few launches, for ncu captures; prints per-stage device times."""
+    if args.only == "block":
+        B = BLOCK
+        arrays = synth.block_params(B["d_model"], B["d_inner"], B["d_head"], B["d_state"], dtype="bf16", seed=1002)
+        wt = mm.BlockWeights.from_arrays(arrays, B["d_model"], B["d_inner"], B["d_head"], B["d_state"],
+                                         dtype=torch.bfloat16, device=dev)
+        u = torch.from_numpy(synth.activations((B["batch"], B["seq_len"], B["d_model"]), "bf16", seed=1032)).to(dev)
+        u = u.bfloat16()
+        fn = lambda: mm.matmamba_block_fwd(wt, u, B["widths"][0], B["chunk"])  # noqa: E731
+    else:
+        S = SCAN
+        inp = synth.ssd_inputs(S["batch"], S["seq_len"], S["heads"], S["d_head"], S["d_state"], 1, "bf16", seed=1001)
+        g = {k: torch.from_numpy(v).to(dev) for k, v in inp.items()}
+        for k in ("x", "B", "C"):
+            g[k] = g[k].bfloat16()
+        fn = lambda: mm.ssd_scan(g["x"], g["dt"], g["A"], g["B"], g["C"], g["D"], chunk=S["chunk"])  # noqa: E731
+    ms, (stages, kernels) = timed(fn, args.steps, args.warmup, trace=True)
+    print(json.dumps({"only": args.only, "ms_per_step": sum(ms) / len(ms), "stages": stages, "kernels": kernels}))
 
 
 def run_extended(args, mm, synth, torch, dev, timed, max_over_ranks, world):

@@ -212,9 +212,101 @@ GemmDesc out_proj_desc(const View& v, const mm_block_params* p, const void* nrm,
     return g;
 }
 
+// ------------------------------------------------------------------ fused bf16 block
+//
+// in_proj applies conv + SiLU and softplus(dt) in its epilogue (pre-conv
+// values stay in fp32 TMEM), the scan applies the SiLU(z) gate and norm_w and
+// accumulates each token's sum of squares, and out_proj scales its rows by the
+// resulting 1/RMS: three stages instead of six, no pre-conv or y round trip.
+
+bool fused_ok(const mm_block_params* p, const View& v, int chunk)
+{
+    return p->dtype == MM_BF16 && v.K == 4 && v.P == 64 && v.N == 128 && chunk % 128 == 0 && v.Dm % 8 == 0 &&
+           (reinterpret_cast<uintptr_t>(p->conv_w) & 7u) == 0 && (reinterpret_cast<uintptr_t>(p->norm_w) & 15u) == 0;
+}
+
+struct FusedBufs {
+    void *z, *xbc, *nrm, *scan_ws;
+    float *dt, *rowsq;
+    size_t scan_ws_bytes;
+};
+
+FusedBufs carve_fused(Carver& c, const View& v, const mm_block_params* p, int batch, int L, int chunk)
+{
+    const size_t T = (size_t)batch * L;
+    FusedBufs b{};
+    b.z = c.take(T * v.d * 2);
+    b.xbc = c.take(T * v.nconv * 2);
+    b.dt = static_cast<float*>(c.take(T * v.h * 4));
+    b.nrm = c.take(T * v.d * 2);
+    b.rowsq = static_cast<float*>(c.take(T * 2 * v.h * 4));
+    ScanArgs probe = block_scan_args(v, p, b.xbc, b.dt, batch, L, chunk, nullptr, nullptr, b.nrm);
+    b.scan_ws_bytes = scan_tc_workspace(probe);
+    b.scan_ws = c.take(b.scan_ws_bytes);
+    return b;
+}
+
+GemmDesc in_proj_fused_desc(const View& v, const mm_block_params* p, const void* u, int batch, int L,
+                            const FusedBufs& b, const void* c_in, void* c_out)
+{
+    const char* W = static_cast<const char*>(p->W_in);
+    const size_t row = (size_t)v.Dm * 2;
+    GemmDesc g{};
+    g.A = u; g.lda = v.Dm; g.ldb = v.Dm; g.M = batch * L; g.K = v.Dm; g.nseg = 4;
+    g.seg[0] = GemmSeg{W, b.z, v.d, v.d, 0, 0, kEpiStore, 0};
+    g.seg[1] = GemmSeg{W + (size_t)v.E * row, b.xbc, v.nconv, v.d, 0, 0, kEpiConv, 0};
+    g.seg[2] = GemmSeg{W + (size_t)2 * v.E * row, static_cast<char*>(b.xbc) + (size_t)v.d * 2, v.nconv, 2 * v.GN, 0, 0,
+                       kEpiConv, v.E};
+    g.seg[3] = GemmSeg{W + (size_t)(2 * v.E + 2 * v.GN) * row, b.dt, v.h, v.h, 1, 0, kEpiSoftplus, 0};
+    g.ex.conv_w = p->conv_w; g.ex.conv_b = p->conv_b; g.ex.dt_bias = p->dt_bias;
+    g.ex.L = L; g.ex.K = v.K; g.ex.conv_rows = v.E + 2 * v.GN;
+    g.ex.conv_state_in = c_in; g.ex.conv_state_out = c_out;
+    return g;
+}
+
+int block_impl_fused(const mm_block_params* p, const View& v, const void* u, int batch, int L, int chunk, void* out,
+                     int out_accumulate, const float* s_in, const void* c_in, float* s_out, void* c_out, Carver& c,
+                     cudaStream_t s)
+{
+    const int64_t T = (int64_t)batch * L;
+    FusedBufs b = carve_fused(c, v, p, batch, L, chunk);
+    const GemmDesc gin = in_proj_fused_desc(v, p, u, batch, L, b, c_in, c_out);
+    MM_TRY(stage("in_proj_conv", 1, s, [&] { return launch_gemm_tc(gin, s); }));
+    ScanArgs a = block_scan_args(v, p, b.xbc, b.dt, batch, L, chunk, s_in, s_out, b.nrm);
+    ScanGate gate{b.z, v.d, p->norm_w, b.rowsq};
+    MM_TRY(stage("ssd_scan_gate", scan_tc_kernel_count(a), s,
+                 [&] { return launch_scan_tc_gated(a, gate, b.scan_ws, b.scan_ws_bytes, s); }));
+    GemmDesc go = out_proj_desc(v, p, b.nrm, T, out, out_accumulate);
+    go.ex.row_parts = b.rowsq;
+    go.ex.nparts = 2 * v.h;
+    go.ex.rs_inv_n = 1.0f / (float)v.d;
+    go.ex.rs_eps = p->norm_eps;
+    MM_TRY(stage("out_proj_norm", 1, s, [&] { return launch_gemm_tc(go, s); }));
+    return MM_OK;
+}
+
+bool fused_supported(const mm_block_params* p, const View& v, int batch, int L, int chunk)
+{
+    if (!fused_ok(p, v, chunk)) return false;
+    Carver c(nullptr);
+    FusedBufs b = carve_fused(c, v, p, batch, L, chunk);
+    // probe with an aligned stand-in for u (the entry points require 16-byte aligned u)
+    const GemmDesc gin = in_proj_fused_desc(v, p, p->W_in, batch, L, b, nullptr, nullptr);
+    ScanArgs a = block_scan_args(v, p, b.xbc, b.dt, batch, L, chunk, nullptr, nullptr, b.nrm);
+    return gemm_tc_supported(gin) && scan_tc_supported(a);
+}
+
+size_t block_ws_bytes(const mm_block_params* p, const View& v, int batch, int L, int chunk)
+{
+    Carver c(nullptr);
+    if (fused_supported(p, v, batch, L, chunk)) carve_fused(c, v, p, batch, L, chunk);
+    else carve_block(c, v, p, batch, L, chunk);
+    return c.used;
+}
+
 // The block on device buffers.  out_accumulate = 1: out is an fp32 buffer and
 // the projection is added to it (residual stream of the stack).
-int block_impl(const mm_block_params* p, const View& v, const void* u, int batch, int L, int chunk, void* out,
+int block_impl_unfused(const mm_block_params* p, const View& v, const void* u, int batch, int L, int chunk, void* out,
                int out_accumulate, const float* s_in, const void* c_in, float* s_out, void* c_out, Carver& c,
                cudaStream_t s)
 {
@@ -241,6 +333,15 @@ int block_impl(const mm_block_params* p, const View& v, const void* u, int batch
     MM_TRY(stage("out_proj", 1, s,
                  [&] { return run_gemm(p->dtype, out_proj_desc(v, p, b.nrm, T, out, out_accumulate), s); }));
     return MM_OK;
+}
+
+int block_impl(const mm_block_params* p, const View& v, const void* u, int batch, int L, int chunk, void* out,
+               int out_accumulate, const float* s_in, const void* c_in, float* s_out, void* c_out, Carver& c,
+               cudaStream_t s)
+{
+    if (fused_supported(p, v, batch, L, chunk))
+        return block_impl_fused(p, v, u, batch, L, chunk, out, out_accumulate, s_in, c_in, s_out, c_out, c, s);
+    return block_impl_unfused(p, v, u, batch, L, chunk, out, out_accumulate, s_in, c_in, s_out, c_out, c, s);
 }
 
 int check_chunk(int chunk) { return chunk > 0 ? MM_OK : MM_ERR_SHAPE; }
@@ -296,9 +397,7 @@ int matmamba_block_workspace(const mm_block_params* p, int batch, int L, int m_i
     if (!bytes) return MM_ERR_NULL;
     if (batch <= 0 || L <= 0) return MM_ERR_SHAPE;
     if ((rc = check_chunk(chunk))) return rc;
-    Carver c(nullptr);
-    carve_block(c, v, p, batch, L, chunk);
-    *bytes = c.used;
+    *bytes = block_ws_bytes(p, v, batch, L, chunk);
     return MM_OK;
 }
 
@@ -506,9 +605,8 @@ static int stack_check(const mm_block_params* layers, int nlayers, const int* m_
         View v;
         if ((rc = resolve(&layers[l], m_per_layer[l], v))) return rc;
         if (layers[l].d_model != layers[0].d_model || layers[l].dtype != layers[0].dtype) return MM_ERR_SHAPE;
-        Carver c(nullptr);
-        carve_block(c, v, &layers[l], batch, L, chunk);
-        block_max = c.used > block_max ? c.used : block_max;
+        const size_t need_l = block_ws_bytes(&layers[l], v, batch, L, chunk);
+        block_max = need_l > block_max ? need_l : block_max;
     }
     const size_t T = (size_t)batch * L;
     const int Dm = layers[0].d_model;

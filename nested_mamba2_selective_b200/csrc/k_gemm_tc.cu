@@ -22,6 +22,9 @@ using namespace sm100;
 
 namespace {
 
+__device__ __forceinline__ float bf_lo_u(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf_hi_u(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
+
 constexpr int kBM = 128;  // rows of a tile = TMEM lanes
 constexpr int kBK = 64;   // one 128-byte swizzle atom of bf16 along K
 
@@ -34,11 +37,16 @@ struct TcSeg {
     int out_f32;
     int accumulate;
     int vec_ok;  // 16-byte vector stores allowed
+    int kind;    // GemmEpi
+    int conv_row0;
 };
 
 struct TcParams {
     int M, K, ktiles, mtiles, ntiles, nseg;
+    int shift;  // halo rows at the top of each tile (K-1 with a conv segment, else 0)
+    int rows;   // output rows per tile = 128 - shift
     TcSeg seg[kMaxSeg];
+    GemmExtra ex;
     int* status;
 };
 
@@ -62,36 +70,25 @@ __device__ __forceinline__ TileInfo<BN> tile_info(const TcParams& p, int tile)
     return t;
 }
 
-__device__ __forceinline__ void store_chunk(const TcSeg& sg, int64_t row, int col, int ncols, const uint32_t (&v)[32])
+__device__ __forceinline__ float silu_fast(float a) { return __fdividef(a, 1.0f + __expf(-a)); }
+
+__device__ __forceinline__ void store_bf16_chunk(__nv_bfloat16* o, int ncols, bool vec, const float (&v)[32])
 {
-    if (sg.out_f32) {
-        float* o = static_cast<float*>(sg.out) + row * sg.ldo + col;
-#pragma unroll
-        for (int i = 0; i < 32; ++i)
-            if (i < ncols) o[i] = sg.accumulate ? o[i] + __uint_as_float(v[i]) : __uint_as_float(v[i]);
-        return;
-    }
-    __nv_bfloat16* o = static_cast<__nv_bfloat16*>(sg.out) + row * sg.ldo + col;
-    if (ncols == 32 && sg.vec_ok) {
+    if (ncols == 32 && vec) {
         uint4* o4 = reinterpret_cast<uint4*>(o);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            uint4 w;
-            w.x = pack_bf16(__uint_as_float(v[8 * q + 0]), __uint_as_float(v[8 * q + 1]));
-            w.y = pack_bf16(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3]));
-            w.z = pack_bf16(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5]));
-            w.w = pack_bf16(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7]));
-            o4[q] = w;
-        }
+        for (int q = 0; q < 4; ++q)
+            o4[q] = make_uint4(pack_bf16(v[8 * q + 0], v[8 * q + 1]), pack_bf16(v[8 * q + 2], v[8 * q + 3]),
+                               pack_bf16(v[8 * q + 4], v[8 * q + 5]), pack_bf16(v[8 * q + 6], v[8 * q + 7]));
     } else {
 #pragma unroll
         for (int i = 0; i < 32; ++i)
-            if (i < ncols) o[i] = __float2bfloat16_rn(__uint_as_float(v[i]));
+            if (i < ncols) o[i] = __float2bfloat16_rn(v[i]);
     }
 }
 
 template <int BN, int STAGES>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB, const TcParams p)
 {
     constexpr int A_BYTES = kBM * kBK * 2;
@@ -101,7 +98,8 @@ __global__ void __launch_bounds__(192, 1)
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+    float* halo = reinterpret_cast<float*>(smem + STAGES * STAGE_BYTES);  // [2 groups][2 bufs][4 quarters][3][32]
+    uint64_t* full = reinterpret_cast<uint64_t*>(halo + 2 * 2 * 4 * 3 * 32);
     uint64_t* empty = full + STAGES;
     uint64_t* tfull = empty + STAGES;
     uint64_t* tempty = tfull + 2;
@@ -117,7 +115,7 @@ __global__ void __launch_bounds__(192, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&tfull[b], 1);
-            mbar_init(&tempty[b], 4);
+            mbar_init(&tempty[b], 8);
         }
         mbar_init(done, 1);
         *abort = 0;
@@ -140,6 +138,7 @@ __global__ void __launch_bounds__(192, 1)
             int it = 0;
             for (int tile = blockIdx.x; tile < total && !*abort; tile += gridDim.x) {
                 const TileInfo<BN> t = tile_info<BN>(p, tile);
+                const int arow = t.mt * p.rows - p.shift;  // may be negative: rows above 0 load as zeros
                 for (int kt = 0; kt < p.ktiles; ++kt, ++it) {
                     const int s = it % STAGES;
                     if (!mbar_wait(&empty[s], ((it / STAGES) & 1) ^ 1, abort)) {
@@ -148,7 +147,7 @@ __global__ void __launch_bounds__(192, 1)
                     }
                     uint8_t* sa = smem + s * STAGE_BYTES;
                     mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
-                    tma_load_2d(sa, &mapA, &full[s], kt * kBK, t.mt * kBM);
+                    tma_load_2d(sa, &mapA, &full[s], kt * kBK, arow);
                     tma_load_2d(sa + A_BYTES, &mapB, &full[s], kt * kBK, t.b_row);
                 }
             }
@@ -190,10 +189,12 @@ __global__ void __launch_bounds__(192, 1)
             mma_commit(done);
             mbar_wait(done, 0, nullptr);
         }
-    } else {  // ---------------- epilogue: warps 2..5
+    } else {  // ---------------- epilogue: warps 2..9, two groups alternating 32-column chunks
         const int q = warp & 3;
-        const int row_in_tile = q * 32 + lane;
-        int tc = 0;
+        const int eg = (warp - 2) >> 2;
+        const int r = q * 32 + lane;  // tile row = TMEM lane
+        const GemmExtra& ex = p.ex;
+        int tc = 0, nchunk_done = 0;
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++tc) {
             const TileInfo<BN> t = tile_info<BN>(p, tile);
             const int buf = tc & 1;
@@ -203,12 +204,116 @@ __global__ void __launch_bounds__(192, 1)
             }
             tc_fence_after();
             const TcSeg& sg = p.seg[t.seg];
-            const int64_t row = (int64_t)t.mt * kBM + row_in_tile;
-            for (int c0 = 0; c0 < t.nvalid; c0 += 32) {
-                uint32_t v[32];
-                tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + buf * BN + c0, v);
-                tmem_ld_wait();
-                if (row < p.M) store_chunk(sg, row, t.n0 + c0, min(32, t.nvalid - c0), v);
+            const int64_t m = (int64_t)t.mt * p.rows - p.shift + r;  // token of this row
+            const bool row_ok = r >= p.shift && m < p.M;
+            float scale = 1.0f;
+            if (ex.row_parts && row_ok) {
+                const float* rp = ex.row_parts + m * ex.nparts;
+                float ss = 0.0f;
+                for (int j = 0; j < ex.nparts; ++j) ss += rp[j];
+                scale = rsqrtf(ss * ex.rs_inv_n + ex.rs_eps);
+            }
+            const int tpos = (sg.kind == kEpiConv && row_ok) ? (int)(m % ex.L) : 0;
+            for (int c0 = 32 * eg; c0 < t.nvalid; c0 += 64, ++nchunk_done) {
+                float v[32];
+                {
+                    uint32_t raw[32];
+                    tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + buf * BN + c0, raw);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(raw[i]) * scale;
+                }
+                const int ncols = min(32, t.nvalid - c0);
+                const int col = t.n0 + c0;
+                if (sg.kind == kEpiConv) {
+                    // predecessors of this row: lanes above in this warp, the previous warp's last rows via smem
+                    float* hb = halo + ((eg * 2 + (nchunk_done & 1)) * 4) * 96;
+                    if (lane >= 29) {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) hb[q * 96 + (lane - 29) * 32 + i] = v[i];
+                    }
+                    asm volatile("bar.sync %0, 128;" ::"r"(2 + eg) : "memory");
+                    float u1[32], u2[32], u3[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        u1[i] = __shfl_up_sync(0xffffffffu, v[i], 1);
+                        u2[i] = __shfl_up_sync(0xffffffffu, v[i], 2);
+                        u3[i] = __shfl_up_sync(0xffffffffu, v[i], 3);
+                    }
+                    if (lane < 3 && q > 0) {
+                        const float* hp = hb + (q - 1) * 96;  // rows 29, 30, 31 of the previous quarter
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) {
+                            if (lane < 1) u1[i] = hp[2 * 32 + i];
+                            if (lane < 2) u2[i] = hp[(lane + 1) * 32 + i];
+                            u3[i] = hp[lane * 32 + i];
+                        }
+                    }
+                    if (row_ok) {
+                        const int64_t b = m / ex.L;
+                        const __nv_bfloat16* cw = static_cast<const __nv_bfloat16*>(ex.conv_w);
+                        const __nv_bfloat16* cb = static_cast<const __nv_bfloat16*>(ex.conv_b);
+                        const __nv_bfloat16* cin = static_cast<const __nv_bfloat16*>(ex.conv_state_in);
+                        float o[32];
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) {
+                            const int crow = sg.conv_row0 + col + i;
+                            float acc = 0.0f;
+                            if (i < ncols) {
+                                const uint2 w4 = *reinterpret_cast<const uint2*>(cw + (int64_t)crow * 4);
+                                const float w0 = bf_lo_u(w4.x), w1 = bf_hi_u(w4.x), w2 = bf_lo_u(w4.y),
+                                            w3 = bf_hi_u(w4.y);
+                                float x3 = u3[i], x2 = u2[i], x1 = u1[i];
+                                if (tpos < 3) {  // taps before the sequence start: given history or zeros
+                                    const __nv_bfloat16* st = cin ? cin + (b * ex.conv_rows + crow) * 3 : nullptr;
+                                    if (tpos < 3) x3 = st ? __bfloat162float(st[tpos]) : 0.0f;
+                                    if (tpos < 2) x2 = st ? __bfloat162float(st[tpos + 1]) : 0.0f;
+                                    if (tpos < 1) x1 = st ? __bfloat162float(st[tpos + 2]) : 0.0f;
+                                }
+                                acc = __bfloat162float(cb[crow]);
+                                acc = fmaf(w0, x3, acc);
+                                acc = fmaf(w1, x2, acc);
+                                acc = fmaf(w2, x1, acc);
+                                acc = fmaf(w3, v[i], acc);
+                            }
+                            o[i] = silu_fast(acc);
+                        }
+                        store_bf16_chunk(static_cast<__nv_bfloat16*>(sg.out) + m * sg.ldo + col, ncols, sg.vec_ok, o);
+                        if (ex.conv_state_out && tpos >= ex.L - 3) {  // last K-1 pre-conv inputs
+                            __nv_bfloat16* so = static_cast<__nv_bfloat16*>(ex.conv_state_out);
+#pragma unroll
+                            for (int i = 0; i < 32; ++i)
+                                if (i < ncols)
+                                    so[(b * ex.conv_rows + sg.conv_row0 + col + i) * 3 + (tpos - (ex.L - 3))] =
+                                        __float2bfloat16_rn(v[i]);
+                        }
+                        if (ex.conv_state_out && tpos == 0 && ex.L < 3) {  // older entries shift in from the history
+                            __nv_bfloat16* so = static_cast<__nv_bfloat16*>(ex.conv_state_out);
+                            for (int i = 0; i < ncols; ++i) {  // no register array indexed here
+                                const int64_t base = (b * ex.conv_rows + sg.conv_row0 + col + i) * 3;
+                                for (int e = 0; e < 3 - ex.L; ++e)
+                                    so[base + e] = cin ? cin[base + e + ex.L] : __float2bfloat16_rn(0.0f);
+                            }
+                        }
+                    }
+                } else if (row_ok) {
+                    if (sg.kind == kEpiSoftplus) {
+                        float* o = static_cast<float*>(sg.out) + m * sg.ldo + col;
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            if (i < ncols) {
+                                const float a = v[i] + ex.dt_bias[col + i];
+                                o[i] = a > 20.0f ? a : log1pf(__expf(a));
+                            }
+                    } else if (sg.out_f32) {
+                        float* o = static_cast<float*>(sg.out) + m * sg.ldo + col;
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            if (i < ncols) o[i] = sg.accumulate ? o[i] + v[i] : v[i];
+                    } else {
+                        store_bf16_chunk(static_cast<__nv_bfloat16*>(sg.out) + m * sg.ldo + col, ncols, sg.vec_ok, v);
+                    }
+                }
             }
             tc_fence_before();
             __syncwarp();
@@ -269,6 +374,10 @@ static bool tc_shape_ok(const GemmDesc& g)
         const char* b = static_cast<const char*>(g.seg[s].B);
         if (b < base || (b - base) % (g.ldb * 2) || g.seg[s].n <= 0) return false;
         if (g.seg[s].accumulate && !g.seg[s].out_f32) return false;
+        if (g.seg[s].kind == kEpiConv &&
+            (g.ex.K != 4 || !g.ex.conv_w || !g.ex.conv_b || g.ex.L <= 0 || (reinterpret_cast<uintptr_t>(g.ex.conv_w) & 7u)))
+            return false;
+        if (g.seg[s].kind == kEpiSoftplus && (!g.ex.dt_bias || !g.seg[s].out_f32)) return false;
     }
     if (!al16(base)) return false;
     return true;
@@ -292,7 +401,7 @@ static cudaError_t launch_bn(const GemmDesc& g, const TcParams& p0, cudaStream_t
     CUtensorMap mapA, mapB;
     if (!make_tmap_bf16(&mapA, g.A, g.K, g.M, g.lda * 2, kBK, kBM)) return cudaErrorInvalidValue;
     if (!make_tmap_bf16(&mapB, base, g.ldb, rows, g.ldb * 2, kBK, BN)) return cudaErrorInvalidValue;
-    constexpr int smem = STAGES * (kBM + BN) * kBK * 2 + 1024 + 256;
+    constexpr int smem = STAGES * (kBM + BN) * kBK * 2 + 1024 + 2 * 2 * 4 * 3 * 32 * 4 + 256;
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     static unsigned long long attr_set = 0;  // one bit per device
@@ -305,7 +414,7 @@ static cudaError_t launch_bn(const GemmDesc& g, const TcParams& p0, cudaStream_t
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int total = p.mtiles * p.ntiles;
     const int grid = total < sms ? total : sms;
-    gemm_tc_kernel<BN, STAGES><<<grid, 192, smem, s>>>(mapA, mapB, p);
+    gemm_tc_kernel<BN, STAGES><<<grid, 320, smem, s>>>(mapA, mapB, p);
     return cudaGetLastError();
 }
 
@@ -315,8 +424,13 @@ cudaError_t launch_gemm_tc(const GemmDesc& g, cudaStream_t s)
     p.M = g.M;
     p.K = g.K;
     p.ktiles = (g.K + kBK - 1) / kBK;
-    p.mtiles = (g.M + kBM - 1) / kBM;
     p.nseg = g.nseg;
+    p.ex = g.ex;
+    p.shift = 0;
+    for (int i = 0; i < g.nseg; ++i)
+        if (g.seg[i].kind == kEpiConv) p.shift = g.ex.K - 1;
+    p.rows = kBM - p.shift;
+    p.mtiles = (g.M + p.rows - 1) / p.rows;
     const char* base = static_cast<const char*>(g.seg[0].B);
     int n_total = 0;
     for (int i = 0; i < g.nseg; ++i) {
@@ -329,6 +443,8 @@ cudaError_t launch_gemm_tc(const GemmDesc& g, cudaStream_t s)
         t.out_f32 = sg.out_f32;
         t.accumulate = sg.accumulate;
         t.vec_ok = !sg.out_f32 && (reinterpret_cast<uintptr_t>(sg.out) & 15u) == 0 && sg.ldo % 8 == 0;
+        t.kind = sg.kind;
+        t.conv_row0 = sg.conv_row0;
         n_total += sg.n;
     }
     int* status = device_status_ptr();

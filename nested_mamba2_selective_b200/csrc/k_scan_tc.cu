@@ -64,6 +64,11 @@ struct ScanTcParams {
     float* final_state;
     int64_t state_stride;
     int* status;
+    // gated output (optional): y -> (y * SiLU(z)) * norm_w, sum of squares of y * SiLU(z) into row_sumsq
+    const __nv_bfloat16* z;
+    int64_t sz;
+    const __nv_bfloat16* norm_w;
+    float* row_parts;
 };
 
 __device__ __forceinline__ void named_sync_compute() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
@@ -328,22 +333,39 @@ __global__ void __launch_bounds__(320, 1)
                 tmem_ld_wait();
                 const float ey = exp2f(c2);
                 if (valid) {
-                    __nv_bfloat16* yo =
-                        static_cast<__nv_bfloat16*>(p.y) + (tok0 + t0 + r) * p.sy + (int64_t)head * kP + 32 * hf;
+                    const int64_t tok = tok0 + t0 + r;
+                    const int col = head * kP + 32 * hf;
+                    __nv_bfloat16* yo = static_cast<__nv_bfloat16*>(p.y) + tok * p.sy + col;
+                    float ssq = 0.0f;
 #pragma unroll
                     for (int c = 0; c < 4; ++c) {
                         const uint32_t xw[4] = {xs[c].x, xs[c].y, xs[c].z, xs[c].w};
+                        uint4 zw4 = make_uint4(0, 0, 0, 0), nw4 = make_uint4(0, 0, 0, 0);
+                        if (p.z) {
+                            zw4 = *reinterpret_cast<const uint4*>(p.z + tok * p.sz + col + 8 * c);
+                            nw4 = *reinterpret_cast<const uint4*>(p.norm_w + col + 8 * c);
+                        }
+                        const uint32_t zw[4] = {zw4.x, zw4.y, zw4.z, zw4.w};
+                        const uint32_t nw[4] = {nw4.x, nw4.y, nw4.z, nw4.w};
                         uint32_t o[4];
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
                             const int j = 8 * c + 2 * e;
-                            const float a0 = __uint_as_float(yv[j]) + ey * __uint_as_float(ov[j]) + Dh * bf_lo(xw[e]);
-                            const float a1 =
-                                __uint_as_float(yv[j + 1]) + ey * __uint_as_float(ov[j + 1]) + Dh * bf_hi(xw[e]);
+                            float a0 = __uint_as_float(yv[j]) + ey * __uint_as_float(ov[j]) + Dh * bf_lo(xw[e]);
+                            float a1 = __uint_as_float(yv[j + 1]) + ey * __uint_as_float(ov[j + 1]) + Dh * bf_hi(xw[e]);
+                            if (p.z) {
+                                const float z0 = bf_lo(zw[e]), z1 = bf_hi(zw[e]);
+                                a0 *= __fdividef(z0, 1.0f + __expf(-z0));
+                                a1 *= __fdividef(z1, 1.0f + __expf(-z1));
+                                ssq = fmaf(a0, a0, fmaf(a1, a1, ssq));
+                                a0 *= bf_lo(nw[e]);
+                                a1 *= bf_hi(nw[e]);
+                            }
                             o[e] = pack_bf16(a0, a1);
                         }
                         reinterpret_cast<uint4*>(yo)[c] = make_uint4(o[0], o[1], o[2], o[3]);
                     }
+                    if (p.z) p.row_parts[tok * 2 * p.h + 2 * head + hf] = ssq;
                 }
             }
             {
@@ -460,7 +482,21 @@ size_t scan_tc_workspace(const ScanArgs& a)
 
 int scan_tc_kernel_count(const ScanArgs& a) { return plan_for(a, num_sms()).nseg > 1 ? 3 : 1; }
 
+static cudaError_t launch_scan_tc_impl(const ScanArgs& a, const ScanGate* gate, void* ws, size_t ws_bytes,
+                                       cudaStream_t s);
+
 cudaError_t launch_scan_tc(const ScanArgs& a, void* ws, size_t ws_bytes, cudaStream_t s)
+{
+    return launch_scan_tc_impl(a, nullptr, ws, ws_bytes, s);
+}
+
+cudaError_t launch_scan_tc_gated(const ScanArgs& a, const ScanGate& g, void* ws, size_t ws_bytes, cudaStream_t s)
+{
+    return launch_scan_tc_impl(a, &g, ws, ws_bytes, s);
+}
+
+static cudaError_t launch_scan_tc_impl(const ScanArgs& a, const ScanGate* gate, void* ws, size_t ws_bytes,
+                                       cudaStream_t s)
 {
     const Plan pl = plan_for(a, num_sms());
     const int64_t rows = (int64_t)a.batch * a.L;
@@ -474,6 +510,12 @@ cudaError_t launch_scan_tc(const ScanArgs& a, void* ws, size_t ws_bytes, cudaStr
     p.dt = a.dt; p.sdt = a.sdt; p.A = a.A; p.D = a.D; p.y = a.y; p.sy = a.sy;
     p.init_state = a.init_state; p.final_state = a.final_state; p.state_stride = a.state_stride;
     p.status = device_status_ptr();
+    if (gate) {
+        p.z = static_cast<const __nv_bfloat16*>(gate->z);
+        p.sz = gate->sz;
+        p.norm_w = static_cast<const __nv_bfloat16*>(gate->norm_w);
+        p.row_parts = gate->row_parts;
+    }
     const size_t bh = (size_t)a.batch * a.h;
     if (pl.nseg > 1) {
         if (!ws || ws_bytes < scan_tc_workspace(a)) return cudaErrorInvalidValue;

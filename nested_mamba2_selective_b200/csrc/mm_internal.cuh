@@ -31,6 +31,8 @@ __device__ __forceinline__ float softplus_f(float v) { return v > 20.0f ? v : lo
 // concatenate along N; they let one launch read a width view of W_in whose
 // rows sit in four separate blocks, and route each block of output columns to
 // its own buffer (and dtype).
+enum GemmEpi { kEpiStore = 0, kEpiConv = 1, kEpiSoftplus = 2 };
+
 struct GemmSeg {
     const void* B;   // first row of this segment's weights, row stride ldb
     void* out;       // output of this segment's first column, row stride ldo
@@ -38,9 +40,32 @@ struct GemmSeg {
     int n;           // number of columns (rows of B) in this segment
     int out_f32;     // output stored as fp32 (else in the input dtype)
     int accumulate;  // fp32 output only: out += result
+    int kind;        // GemmEpi (tensor-core kernel only)
+    int conv_row0;   // kEpiConv: conv row of column 0; kEpiSoftplus: unused
 };
 
 constexpr int kMaxSeg = 4;
+
+// Epilogue extras of the tensor-core kernel.
+//  - kEpiConv segments apply the block's causal depthwise conv (K taps) and
+//    SiLU down the token axis: tiles then overlap by K-1 rows so every output
+//    row sees its K-1 predecessors, taps never cross a sequence start (L
+//    tokens per sequence) and read the given history there instead.
+//  - kEpiSoftplus segments store softplus(acc + dt_bias[col]) in fp32.
+//  - row_parts != null scales every output row m by
+//    rsqrt(sum_j row_parts[m * nparts + j] * rs_inv_n + rs_eps), the parts
+//    added in index order (RMSNorm applied after the GEMM, deterministic).
+struct GemmExtra {
+    const void* conv_w;
+    const void* conv_b;
+    const float* dt_bias;
+    int L, K, conv_rows;
+    const void* conv_state_in;
+    void* conv_state_out;
+    const float* row_parts;
+    int nparts;
+    float rs_inv_n, rs_eps;
+};
 
 struct GemmDesc {
     const void* A;
@@ -49,6 +74,7 @@ struct GemmDesc {
     int M, K;
     int nseg;
     GemmSeg seg[kMaxSeg];
+    GemmExtra ex;
 };
 
 // ------------------------------------------------------------------ scan arguments
@@ -103,5 +129,16 @@ bool scan_tc_supported(const ScanArgs& a);
 size_t scan_tc_workspace(const ScanArgs& a);
 int scan_tc_kernel_count(const ScanArgs& a);
 cudaError_t launch_scan_tc(const ScanArgs& a, void* ws, size_t ws_bytes, cudaStream_t s);
+
+// Gate + RMSNorm fused into the tensor-core scan's output: instead of y the scan
+// stores (y * SiLU(z)) * norm_w in bf16, and the sum of squares of y * SiLU(z)
+// over each (token, head, 32-channel half) into row_parts[tok * 2h + 2 head + half].
+struct ScanGate {
+    const void* z;
+    int64_t sz;
+    const void* norm_w;
+    float* row_parts;
+};
+cudaError_t launch_scan_tc_gated(const ScanArgs& a, const ScanGate& g, void* ws, size_t ws_bytes, cudaStream_t s);
 
 }  // namespace mm

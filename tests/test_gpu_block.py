@@ -153,3 +153,37 @@ def test_single_token_and_tiny_lengths(orc):
         u = synth.activations((3, L, w.d_model), "bf16", seed=40 + L)
         out = run_block(orc, w, wt, p64, u, 192, 256)
         assert max_abs_rel(to_np(out), orc.block_fwd(dims_of(w), p64, u, 192)) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("L", [1, 2, 5])
+def test_short_prefill_with_history_and_state_out(orc, L):
+    """Prefills shorter than the conv window read the given history and shift it into the new state."""
+    w = synth.WORKLOADS["block_130m_b8_L2048"]
+    wt, p64 = make_block(w)
+    dims = dims_of(w)
+    H, P, N, E = dims.nheads, w.d_head, w.d_state, w.d_inner
+    rows = E + 2 * N
+    u = synth.activations((2, L, w.d_model), "bf16", seed=60 + L)
+    s_in_np, c_in_np = synth.states(2, H, P, N, rows, 4, "bf16", seed=61)
+    s_out = torch.zeros((2, H, P, N), device="cuda")
+    c_out = torch.zeros((2, rows, 3), device="cuda", dtype=torch.bfloat16)
+    out = run_block(orc, w, wt, p64, u, 384, 256, ssm_state_in=torch.from_numpy(s_in_np).cuda(),
+                    conv_state_in=to_device(c_in_np, "bf16"), ssm_state_out=s_out, conv_state_out=c_out)
+    s_ref, c_ref = np.zeros((2, H, P, N)), np.zeros((2, rows, 3))
+    ref = orc.block_fwd(dims, p64, u, 384, ssm_state_in=s_in_np, conv_state_in=c_in_np.astype(np.float64),
+                        ssm_state_out=s_ref, conv_state_out=c_ref)
+    d, h = orc.width(dims, 384)
+    assert max_abs_rel(to_np(out), ref) <= TOL["bf16"]
+    assert max_abs_rel(to_np(s_out[:, :h]), s_ref[:, :h]) <= TOL["bf16"]
+    active = list(range(d)) + list(range(E, rows))
+    assert max_abs_rel(to_np(c_out[:, active]), c_ref[:, active]) <= TOL["bf16"]
+
+
+def test_repeated_calls_are_bit_identical():
+    w = synth.WORKLOADS["block_130m_b8_L2048"]
+    wt, _ = make_block(w)
+    u = to_device(synth.activations((4, 700, w.d_model), "bf16", seed=70), "bf16")
+    a = matmamba_block_fwd(wt, u, 768, 256)
+    b = matmamba_block_fwd(wt, u, 768, 256)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
