@@ -198,10 +198,9 @@ __global__ void __launch_bounds__(320, 1)
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++tc) {
             const TileInfo<BN> t = tile_info<BN>(p, tile);
             const int buf = tc & 1;
-            if (!mbar_wait(&tfull[buf], (tc >> 1) & 1, abort)) {
-                raise_timeout(abort, p.status);
-                break;
-            }
+            // a failed wait skips this tile's work but keeps the group's named barriers in step
+            const bool ok = __all_sync(0xffffffffu, mbar_wait(&tfull[buf], (tc >> 1) & 1, abort));
+            if (!ok) raise_timeout(abort, p.status);
             tc_fence_after();
             const TcSeg& sg = p.seg[t.seg];
             const int64_t m = (int64_t)t.mt * p.rows - p.shift + r;  // token of this row
@@ -216,12 +215,15 @@ __global__ void __launch_bounds__(320, 1)
             const int tpos = (sg.kind == kEpiConv && row_ok) ? (int)(m % ex.L) : 0;
             for (int c0 = 32 * eg; c0 < t.nvalid; c0 += 64, ++nchunk_done) {
                 float v[32];
-                {
+                if (ok) {
                     uint32_t raw[32];
                     tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + buf * BN + c0, raw);
                     tmem_ld_wait();
 #pragma unroll
                     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(raw[i]) * scale;
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) v[i] = 0.0f;
                 }
                 const int ncols = min(32, t.nvalid - c0);
                 const int col = t.n0 + c0;
@@ -249,7 +251,7 @@ __global__ void __launch_bounds__(320, 1)
                             u3[i] = hp[lane * 32 + i];
                         }
                     }
-                    if (row_ok) {
+                    if (row_ok && ok) {
                         const int64_t b = m / ex.L;
                         const __nv_bfloat16* cw = static_cast<const __nv_bfloat16*>(ex.conv_w);
                         const __nv_bfloat16* cb = static_cast<const __nv_bfloat16*>(ex.conv_b);
@@ -296,7 +298,7 @@ __global__ void __launch_bounds__(320, 1)
                             }
                         }
                     }
-                } else if (row_ok) {
+                } else if (row_ok && ok) {
                     if (sg.kind == kEpiSoftplus) {
                         float* o = static_cast<float*>(sg.out) + m * sg.ldo + col;
 #pragma unroll

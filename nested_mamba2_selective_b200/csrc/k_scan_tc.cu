@@ -16,12 +16,16 @@
 //                   state across blocks in registers (tcgen05)
 // Only segment boundary states touch HBM.
 //
-// chunk_scan, one head per CTA (320 threads): warp 0 TMA producer, warp 1
-// TMEM owner and tcgen05.mma issuer, warps 2-9 compute.  Compute thread
-// (quarter q, lane l, half hf) owns TMEM lane r = 32q + l, i.e. token r of the
-// block for Y and state row n = r for S, and half hf of the columns.
-// TMEM columns: G = C B^T (128) | M = masked G as the bf16 A operand (64) |
-// Y (64) | Y_off (64) | S = B^T X' (64).
+// A CTA takes two heads of one (batch, segment) so that the B and C blocks and
+// G = C B^T are loaded and computed once per pair (320 threads): warp 0 TMA
+// producer, warp 1 TMEM owner and tcgen05.mma issuer, warps 2-9 compute.
+// Compute thread (quarter q, lane l, half hf) owns TMEM lane r = 32q + l and
+// head hf of the pair: token r for its Y row, state row n = r for S.  For the
+// masked matrices it takes the columns s in [64 hf, 64 hf + 64) of both heads,
+// written as bf16 A operands over the G columns it has just read.
+// Per block: G, then Y_off = C [H_0 | H_1] once the bf16 state copy H is in
+// shared memory (its space then takes X'), then Y_j = M_j X_j and
+// S = B^T [X'_0 | X'_1]; G of the next block overlaps this block's epilogue.
 #include <cuda.h>
 
 #include <cmath>
@@ -38,16 +42,18 @@ namespace {
 constexpr int kQ = 128;                       // tokens per block
 constexpr int kP = 64;                        // head dim
 constexpr int kN = 128;                       // state dim
-constexpr int kTileQN = kQ * kN * 2;          // C or B block: two 64-column panels
-constexpr int kTileQP = kQ * kP * 2;          // x, X' or H block: one panel
-constexpr int kStage = 2 * kTileQN + kTileQP; // C | B | x
+constexpr int kTileQN = kQ * kN * 2;              // C or B block: two 64-column panels
+constexpr int kTileQP = kQ * kP * 2;              // x, X' or H block of one head: one panel
+constexpr int kOffC = 0, kOffB = kTileQN, kOffX = 2 * kTileQN;
+constexpr int kStage = 2 * kTileQN + 2 * kTileQP; // C | B | x of two heads
 constexpr int kNStage = 2;
-constexpr int kOffXP = kNStage * kStage;
-constexpr int kOffH = kOffXP + kTileQP;
-constexpr int kOffSmall = kOffH + kTileQP;
-constexpr int kSmemBytes = kOffSmall + 2048 + 1024;
+constexpr int kOffHX = kNStage * kStage;          // H (then X') of two heads
+constexpr int kOffSmall = kOffHX + 2 * kTileQP;
+constexpr int kSmemBytes = kOffSmall + 2560;
 
-constexpr uint32_t kTG = 0, kTM = 128, kTY = 192, kTYO = 256, kTS = 320, kTCols = 512;
+// TMEM columns: G = C B^T, overwritten in place by the masked M_0 | M_1 (A operands);
+// Y_0 | Y_1; Y_off of both heads; S of both heads.
+constexpr uint32_t kTG = 0, kTY = 128, kTYO = 256, kTS = 384, kTCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct ScanTcParams {
@@ -84,38 +90,45 @@ __global__ void __launch_bounds__(320, 1)
     ssd_tc_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CUtensorMap mapB,
                   const __grid_constant__ CUtensorMap mapC, const ScanTcParams p)
 {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    float* cs2 = reinterpret_cast<float*>(sm + kOffSmall);  // [128] running log2-decay of each token
-    float* dts = cs2 + kQ;                                    // [128] dt of each token (0 past the end)
-    float* wtot = dts + kQ;                                   // [8] per-warp scan totals
+    extern __shared__ __align__(1024) uint8_t sm[];
+    float* cs2 = reinterpret_cast<float*>(sm + kOffSmall);  // [2 heads][128] running log2 decay through token r
+    float* dts = cs2 + 2 * kQ;                                // [2 heads][128] dt (0 past the end)
+    float* wtot = dts + 2 * kQ;                               // [2 heads][4] per-warp scan totals
     uint64_t* full = reinterpret_cast<uint64_t*>(wtot + 8);
     uint64_t* empty = full + kNStage;
-    uint64_t* g_full = empty + kNStage;
-    uint64_t* m_ready = g_full + 1;
+    uint64_t* g_done = empty + kNStage;
+    uint64_t* yo_done = g_done + 1;
+    uint64_t* h_ready = yo_done + 1;
+    uint64_t* m_ready = h_ready + 1;
     uint64_t* ys_full = m_ready + 1;
     uint64_t* done = ys_full + 1;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
     volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
-    const int head = blockIdx.x, seg = blockIdx.y, b = blockIdx.z;
+    const int pair = blockIdx.x, seg = blockIdx.y, b = blockIdx.z;
+    const int head0 = 2 * pair;
     const int c_begin = seg * p.cps;
     const int c_end = min(p.nchunks, c_begin + p.cps);
     const int nch = c_end - c_begin;
-    const int grp = head / p.hpg;
+    const int grp = head0 / p.hpg;  // both heads of a pair share a group (hpg is even or G == 1)
     const int64_t tok0 = (int64_t)b * p.L;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
+        if (smem_u32(sm) & 1023u) {  // tiles need 1024-byte alignment; never observed, but never fault on it
+            raise_timeout(abort, p.status);
+        }
         for (int s = 0; s < kNStage; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
+            mbar_init(&empty[s], 8);
         }
-        mbar_init(g_full, 1);
+        mbar_init(g_done, 1);
+        mbar_init(yo_done, 1);
+        mbar_init(h_ready, 8);
         mbar_init(m_ready, 8);
         mbar_init(ys_full, 1);
         mbar_init(done, 1);
-        *abort = 0;
+        *abort = (smem_u32(sm) & 1023u) ? 1 : 0;
         fence_mbar_init();
         prefetch_tmap(&mapX);
         prefetch_tmap(&mapB);
@@ -129,10 +142,11 @@ __global__ void __launch_bounds__(320, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    uint8_t* sHX = sm + kOffHX;  // [2 heads] x 16 KB: bf16 state copy H, then X' of the current block
 
     if (warp == 0) {
-        if (lane == 0) {  // ------------------------------------------------ TMA producer
-            constexpr uint32_t bytes = FULL ? kStage : (kTileQN + kTileQP);
+        if (lane == 0 && !*abort) {  // ------------------------------------------------ TMA producer
+            constexpr uint32_t bytes = FULL ? kStage : (kTileQN + 2 * kTileQP);
             int k = 0;
             for (; k < nch; ++k) {
                 const int s = k % kNStage;
@@ -144,37 +158,58 @@ __global__ void __launch_bounds__(320, 1)
                 uint8_t* base = sm + s * kStage;
                 mbar_arrive_expect_tx(&full[s], bytes);
                 if (FULL) {
-                    tma_load_2d(base, &mapC, &full[s], grp * kN, row);
-                    tma_load_2d(base + kTileQN / 2, &mapC, &full[s], grp * kN + 64, row);
+                    tma_load_2d(base + kOffC, &mapC, &full[s], grp * kN, row);
+                    tma_load_2d(base + kOffC + kTileQN / 2, &mapC, &full[s], grp * kN + 64, row);
                 }
-                tma_load_2d(base + kTileQN, &mapB, &full[s], grp * kN, row);
-                tma_load_2d(base + kTileQN + kTileQN / 2, &mapB, &full[s], grp * kN + 64, row);
-                tma_load_2d(base + 2 * kTileQN, &mapX, &full[s], head * kP, row);
+                tma_load_2d(base + kOffB, &mapB, &full[s], grp * kN, row);
+                tma_load_2d(base + kOffB + kTileQN / 2, &mapB, &full[s], grp * kN + 64, row);
+                tma_load_2d(base + kOffX, &mapX, &full[s], head0 * kP, row);
+                // a pair's second head past the last head reloads the last head (its dt is zero)
+                tma_load_2d(base + kOffX + kTileQP, &mapX, &full[s], min(head0 + 1, p.h - 1) * kP, row);
             }
             for (int j = max(0, k - kNStage); j < k; ++j) mbar_wait(&full[j % kNStage], (j / kNStage) & 1, abort);
         }
     } else if (warp == 1) {
-        if (lane == 0) {  // ------------------------------------------------ MMA issuer
-            const uint32_t id_g = idesc_bf16(128, 128, 0, 0);     // C (K-major) x B (K-major)
-            const uint32_t id_y = idesc_bf16(128, 64, 0, 1);      // M (TMEM) / C (K-major) x MN-major
-            const uint32_t id_s = idesc_bf16(128, 64, 1, 1);      // B^T (MN-major) x X' (MN-major)
-            const uint32_t aXP = smem_u32(sm + kOffXP), aH = smem_u32(sm + kOffH);
+        if (lane == 0 && !*abort) {  // ------------------------------------------------ MMA issuer
+            const uint32_t id_g = idesc_bf16(128, 128, 0, 0);   // C (K-major) x B (K-major)
+            const uint32_t id_o = idesc_bf16(128, 128, 0, 1);   // C (K-major) x [H_0 | H_1] (MN-major)
+            const uint32_t id_y = idesc_bf16(128, 64, 0, 1);    // M_j (TMEM) x X_j (MN-major)
+            const uint32_t id_s = idesc_bf16(128, 128, 1, 1);   // B^T (MN-major) x [X'_0 | X'_1] (MN-major)
+            const uint32_t aHX = smem_u32(sHX);
             for (int k = 0; k < nch; ++k) {
                 const int s = k % kNStage;
                 if (!mbar_wait(&full[s], (k / kNStage) & 1, abort)) {
                     raise_timeout(abort, p.status);
                     break;
                 }
+                // the previous block's MMAs (which read M from the G columns) are complete
+                if (k > 0 && !mbar_wait(ys_full, (k - 1) & 1, abort)) {
+                    raise_timeout(abort, p.status);
+                    break;
+                }
                 tc_fence_after();
-                const uint32_t aC = smem_u32(sm + s * kStage), aB = aC + kTileQN, aX = aB + kTileQN;
+                const uint32_t aS = smem_u32(sm + s * kStage);
+                const uint32_t aC = aS + kOffC, aB = aS + kOffB, aX = aS + kOffX;
                 if (FULL) {
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
+                    for (int kk = 0; kk < 8; ++kk) {  // G = C . B^T
                         const uint32_t off = (kk & 3) * 32 + (kk >> 2) * (kTileQN / 2);
                         mma_ss(tmem + kTG, desc_sw128(aC + off, 16, 1024), desc_sw128(aB + off, 16, 1024), id_g,
                                kk > 0);
                     }
-                    mma_commit(g_full);
+                    mma_commit(g_done);
+                    if (!mbar_wait(h_ready, k & 1, abort)) {
+                        raise_timeout(abort, p.status);
+                        break;
+                    }
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {  // Y_off = C . [H_0 | H_1] over the state dim
+                        const uint32_t off = (kk & 3) * 32 + (kk >> 2) * (kTileQN / 2);
+                        mma_ss(tmem + kTYO, desc_sw128(aC + off, 16, 1024),
+                               desc_sw128(aHX + kk * 2048, kTileQP, 1024), id_o, kk > 0);
+                    }
+                    mma_commit(yo_done);
                 }
                 if (!mbar_wait(m_ready, k & 1, abort)) {
                     raise_timeout(abort, p.status);
@@ -183,21 +218,17 @@ __global__ void __launch_bounds__(320, 1)
                 tc_fence_after();
                 if (FULL) {
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)  // Y = M . X over the block's tokens
-                        mma_ts(tmem + kTY, tmem + kTM + kk * 8, desc_sw128(aX + kk * 2048, 16384, 1024), id_y, kk > 0);
+                    for (int j = 0; j < 2; ++j)
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {  // Y_off = C . H_prev over the state dim
-                        const uint32_t off = (kk & 3) * 32 + (kk >> 2) * (kTileQN / 2);
-                        mma_ss(tmem + kTYO, desc_sw128(aC + off, 16, 1024), desc_sw128(aH + kk * 2048, 16384, 1024),
-                               id_y, kk > 0);
-                    }
+                        for (int kk = 0; kk < 8; ++kk)  // Y_j = M_j . X_j over the block's tokens
+                            mma_ts(tmem + kTY + 64 * j, tmem + kTG + 64 * (kk >> 2) + 32 * j + 8 * (kk & 3),
+                                   desc_sw128(aX + j * kTileQP + kk * 2048, kTileQP, 1024), id_y, kk > 0);
                 }
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk)  // S = B^T . X' over the block's tokens
+                for (int kk = 0; kk < 8; ++kk)  // S = B^T . [X'_0 | X'_1] over the block's tokens
                     mma_ss(tmem + kTS, desc_sw128(aB + kk * 2048, kTileQN / 2, 1024),
-                           desc_sw128(aXP + kk * 2048, 16384, 1024), id_s, kk > 0);
+                           desc_sw128(aHX + kk * 2048, kTileQP, 1024), id_s, kk > 0);
                 mma_commit(ys_full);
-                mma_commit(&empty[s]);
             }
             mma_commit(done);
             mbar_wait(done, 0, nullptr);
@@ -206,44 +237,64 @@ __global__ void __launch_bounds__(320, 1)
         const int cw = warp - 2, q = warp & 3, hf = cw >> 2;
         const int r = q * 32 + lane;
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
-        const float A2 = p.A[head] * kLog2e;
-        const float Dh = (FULL && p.D) ? p.D[head] : 0.0f;
+        // this thread's head for the scan, X', output and state: head0 + hf
+        const int head = head0 + hf;
+        const bool head_ok = head < p.h;
+        const float A2 = head_ok ? p.A[head] * kLog2e : 0.0f;
+        const float Dh = (FULL && p.D && head_ok) ? p.D[head] : 0.0f;
         const int64_t bh = (int64_t)b * p.h + head;
         const int PN = kP * kN;
+        float* my_cs2 = cs2 + hf * kQ;
+        float* my_dts = dts + hf * kQ;
+        uint8_t* myHX = sHX + hf * kTileQP;
 
-        // start state: row n = r, columns p in [32 hf, 32 hf + 32)
-        float hs[32];
+        // start state of this head: row n = r, all 64 columns p
+        float hs[64];
         {
             const float* src = nullptr;
-            if (FULL) {
+            if (FULL && head_ok) {
                 if (p.nseg > 1) src = p.states + (bh * p.nseg + seg) * PN;
                 else if (p.init_state) src = p.init_state + (int64_t)b * p.state_stride + (int64_t)head * PN;
             }
 #pragma unroll
-            for (int j = 0; j < 32; ++j) hs[j] = src ? src[(32 * hf + j) * kN + r] : 0.0f;
+            for (int j = 0; j < 64; ++j) hs[j] = src ? src[j * kN + r] : 0.0f;
         }
-        uint8_t* sH = sm + kOffH;
-        uint8_t* sXP = sm + kOffXP;
         auto write_h = [&]() {
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 0; c < 8; ++c) {
                 uint4 v;
                 v.x = pack_bf16(hs[8 * c + 0], hs[8 * c + 1]);
                 v.y = pack_bf16(hs[8 * c + 2], hs[8 * c + 3]);
                 v.z = pack_bf16(hs[8 * c + 4], hs[8 * c + 5]);
                 v.w = pack_bf16(hs[8 * c + 6], hs[8 * c + 7]);
-                *reinterpret_cast<uint4*>(sH + sw128(r, 4 * hf + c)) = v;
+                *reinterpret_cast<uint4*>(myHX + sw128(r, c)) = v;
             }
         };
-        if (FULL) write_h();
+        if (FULL) {
+            write_h();
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(h_ready);
+        }
         float seg_log2 = 0.0f;
+        float dt_next = 0.0f;
+        {
+            const int t0 = c_begin * kQ;
+            if (head_ok && nch > 0 && t0 + r < p.L) dt_next = p.dt[(tok0 + t0 + r) * p.sdt + head];
+        }
 
+        // Every compute warp runs every iteration (the block's two named barriers must see all
+        // eight warps); after a failed wait a warp skips the rest of the block's work.
         for (int k = 0; k < nch; ++k) {
             const int s = k % kNStage;
             const int t0 = (c_begin + k) * kQ;
-            const bool valid = t0 + r < p.L;
-            const float dtv = valid ? p.dt[(tok0 + t0 + r) * p.sdt + head] : 0.0f;
-            // inclusive scan of dt*A (log2 units) over the 128 tokens of the block
+            const bool valid = head_ok && t0 + r < p.L;
+            const float dtv = dt_next;
+            if (k + 1 < nch) {  // prefetch the next block's dt
+                const int t1 = t0 + kQ;
+                dt_next = (head_ok && t1 + r < p.L) ? p.dt[(tok0 + t1 + r) * p.sdt + head] : 0.0f;
+            }
+            // inclusive scan of dt*A (log2 units) over the block, for head hf
             float sc = dtv * A2;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
@@ -259,143 +310,170 @@ __global__ void __launch_bounds__(320, 1)
                 pre += j < q ? w : 0.0f;
                 tot += w;
             }
-            const float c2 = sc + pre;  // log2 decay from the block start through token r
-            if (hf == 0) {
-                cs2[r] = c2;
-                dts[r] = dtv;
-            }
+            const float c2 = sc + pre;
+            my_cs2[r] = c2;
+            my_dts[r] = dtv;
             named_sync_compute();
+            seg_log2 += tot;
 
-            if (!mbar_wait(&full[s], (k / kNStage) & 1, abort)) {
-                raise_timeout(abort, p.status);
-                break;
-            }
-            // X' = exp(cs_end - cs_r) dt_r x_r for this thread's 32 columns; keep x for the D term
-            const uint8_t* sX = sm + s * kStage + 2 * kTileQN;
-            uint4 xs[4];
-            const float wgt = exp2f(tot - c2) * dtv;
+            bool ok = __all_sync(0xffffffffu, mbar_wait(&full[s], (k / kNStage) & 1, abort));
+            const uint8_t* sX = sm + s * kStage + kOffX + hf * kTileQP;
+
+            if (FULL && ok) {
+                ok = __all_sync(0xffffffffu, mbar_wait(g_done, k & 1, abort));
+                if (ok) {
+                    tc_fence_after();
+                    // M_j[t=r, s] = G[r, s] exp(cs_j[r] - cs_j[s]) dt_j[s] (s <= r) for both heads j and
+                    // the columns s in [64 hf, 64 hf + 64), written over the G columns just read
+                    const float c2h[2] = {cs2[r], cs2[kQ + r]};
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                xs[c] = *reinterpret_cast<const uint4*>(sX + sw128(r, 4 * hf + c));
-                uint4 o;
-                o.x = pack_bf16(bf_lo(xs[c].x) * wgt, bf_hi(xs[c].x) * wgt);
-                o.y = pack_bf16(bf_lo(xs[c].y) * wgt, bf_hi(xs[c].y) * wgt);
-                o.z = pack_bf16(bf_lo(xs[c].z) * wgt, bf_hi(xs[c].z) * wgt);
-                o.w = pack_bf16(bf_lo(xs[c].w) * wgt, bf_hi(xs[c].w) * wgt);
-                *reinterpret_cast<uint4*>(sXP + sw128(r, 4 * hf + c)) = o;
-            }
-            fence_async_smem();
-
-            if (FULL) {
-                if (!mbar_wait(g_full, k & 1, abort)) {
-                    raise_timeout(abort, p.status);
-                    break;
+                    for (int half = 0; half < 2; ++half) {
+                        const int s0 = 64 * hf + 32 * half;
+                        uint32_t pk0[16], pk1[16];
+                        if (s0 <= q * 32 + 31) {
+                            uint32_t gv[32];
+                            tmem_ld32(tmem + lane_base + kTG + s0, gv);
+                            tmem_ld_wait();
+#pragma unroll
+                            for (int e = 0; e < 32; e += 2) {
+                                const int sa = s0 + e, sb = sa + 1;
+                                const float ga = __uint_as_float(gv[e]), gb = __uint_as_float(gv[e + 1]);
+                                float v0a = 0.0f, v0b = 0.0f, v1a = 0.0f, v1b = 0.0f;
+                                if (sa <= r) {
+                                    v0a = ga * exp2f(c2h[0] - cs2[sa]) * dts[sa];
+                                    v1a = ga * exp2f(c2h[1] - cs2[kQ + sa]) * dts[kQ + sa];
+                                }
+                                if (sb <= r) {
+                                    v0b = gb * exp2f(c2h[0] - cs2[sb]) * dts[sb];
+                                    v1b = gb * exp2f(c2h[1] - cs2[kQ + sb]) * dts[kQ + sb];
+                                }
+                                pk0[e >> 1] = pack_bf16(v0a, v0b);
+                                pk1[e >> 1] = pack_bf16(v1a, v1b);
+                            }
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) pk0[e] = pk1[e] = 0u;
+                        }
+                        // head j's packed columns for s in [s0, s0 + 32) live at 64 hf + 32 j + 16 half
+                        tmem_st16(tmem + lane_base + kTG + 64 * hf + 16 * half, pk0);
+                        tmem_st16(tmem + lane_base + kTG + 64 * hf + 32 + 16 * half, pk1);
+                    }
+                    tmem_st_wait();
+                    ok = __all_sync(0xffffffffu, mbar_wait(yo_done, k & 1, abort));  // H is read: its space takes X'
                 }
-                tc_fence_after();
-                // M[t=r, s] = G[r, s] exp(cs_r - cs_s) dt_s for s <= r, else 0; columns [64 hf, 64 hf + 64)
+            } else if (!FULL && ok && k > 0) {
+                ok = __all_sync(0xffffffffu, mbar_wait(ys_full, (k - 1) & 1, abort));  // previous X' consumed
+            }
+            if (ok) {  // X'_j[s=r, :] = exp(cs_end - cs_r) dt_r x_j[r, :]
+                const float wgt = exp2f(tot - c2) * dtv;
 #pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    const int s0 = 64 * hf + 32 * j;
-                    uint32_t pk[16];
-                    if (s0 <= q * 32 + 31) {  // warp-uniform: some row of this warp reaches column s0
-                        uint32_t gv[32];
-                        tmem_ld32(tmem + lane_base + kTG + s0, gv);
+                for (int c = 0; c < 8; ++c) {
+                    const uint4 xv = *reinterpret_cast<const uint4*>(sX + sw128(r, c));
+                    uint4 o;
+                    o.x = pack_bf16(bf_lo(xv.x) * wgt, bf_hi(xv.x) * wgt);
+                    o.y = pack_bf16(bf_lo(xv.y) * wgt, bf_hi(xv.y) * wgt);
+                    o.z = pack_bf16(bf_lo(xv.z) * wgt, bf_hi(xv.z) * wgt);
+                    o.w = pack_bf16(bf_lo(xv.w) * wgt, bf_hi(xv.w) * wgt);
+                    *reinterpret_cast<uint4*>(myHX + sw128(r, c)) = o;
+                }
+                fence_async_smem();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(m_ready);
+                    if (!FULL) mbar_arrive(&empty[s]);  // x is read
+                }
+                ok = __all_sync(0xffffffffu, mbar_wait(ys_full, k & 1, abort));
+            }
+            if (ok) {
+                tc_fence_after();
+                if (FULL && valid) {
+                    const float ey = exp2f(c2);
+                    const int64_t tok = tok0 + t0 + r;
+                    const int col = head * kP;
+                    __nv_bfloat16* yo = static_cast<__nv_bfloat16*>(p.y) + tok * p.sy + col;
+                    float ssq[2] = {0.0f, 0.0f};
+#pragma unroll
+                    for (int h2 = 0; h2 < 2; ++h2) {  // 32 output columns at a time
+                        uint32_t yv[32], ov[32];
+                        tmem_ld32(tmem + lane_base + kTY + 64 * hf + 32 * h2, yv);
+                        tmem_ld32(tmem + lane_base + kTYO + 64 * hf + 32 * h2, ov);
                         tmem_ld_wait();
 #pragma unroll
-                        for (int e = 0; e < 32; e += 2) {
-                            const int sa = s0 + e, sb = s0 + e + 1;
-                            const float va = sa <= r ? __uint_as_float(gv[e]) * exp2f(c2 - cs2[sa]) * dts[sa] : 0.0f;
-                            const float vb =
-                                sb <= r ? __uint_as_float(gv[e + 1]) * exp2f(c2 - cs2[sb]) * dts[sb] : 0.0f;
-                            pk[e >> 1] = pack_bf16(va, vb);
-                        }
-                    } else {
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) pk[e] = 0u;
-                    }
-                    tmem_st16(tmem + lane_base + kTM + s0 / 2, pk);
-                }
-                tmem_st_wait();
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(m_ready);
-
-            if (!mbar_wait(ys_full, k & 1, abort)) {
-                raise_timeout(abort, p.status);
-                break;
-            }
-            tc_fence_after();
-            if (FULL) {
-                uint32_t yv[32], ov[32];
-                tmem_ld32(tmem + lane_base + kTY + 32 * hf, yv);
-                tmem_ld32(tmem + lane_base + kTYO + 32 * hf, ov);
-                tmem_ld_wait();
-                const float ey = exp2f(c2);
-                if (valid) {
-                    const int64_t tok = tok0 + t0 + r;
-                    const int col = head * kP + 32 * hf;
-                    __nv_bfloat16* yo = static_cast<__nv_bfloat16*>(p.y) + tok * p.sy + col;
-                    float ssq = 0.0f;
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const uint32_t xw[4] = {xs[c].x, xs[c].y, xs[c].z, xs[c].w};
-                        uint4 zw4 = make_uint4(0, 0, 0, 0), nw4 = make_uint4(0, 0, 0, 0);
-                        if (p.z) {
-                            zw4 = *reinterpret_cast<const uint4*>(p.z + tok * p.sz + col + 8 * c);
-                            nw4 = *reinterpret_cast<const uint4*>(p.norm_w + col + 8 * c);
-                        }
-                        const uint32_t zw[4] = {zw4.x, zw4.y, zw4.z, zw4.w};
-                        const uint32_t nw[4] = {nw4.x, nw4.y, nw4.z, nw4.w};
-                        uint32_t o[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int j = 8 * c + 2 * e;
-                            float a0 = __uint_as_float(yv[j]) + ey * __uint_as_float(ov[j]) + Dh * bf_lo(xw[e]);
-                            float a1 = __uint_as_float(yv[j + 1]) + ey * __uint_as_float(ov[j + 1]) + Dh * bf_hi(xw[e]);
+                        for (int c = 0; c < 4; ++c) {
+                            const int cc = 4 * h2 + c;
+                            const uint4 xv = *reinterpret_cast<const uint4*>(sX + sw128(r, cc));
+                            const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+                            uint4 zw4 = make_uint4(0, 0, 0, 0), nw4 = make_uint4(0, 0, 0, 0);
                             if (p.z) {
-                                const float z0 = bf_lo(zw[e]), z1 = bf_hi(zw[e]);
-                                a0 *= __fdividef(z0, 1.0f + __expf(-z0));
-                                a1 *= __fdividef(z1, 1.0f + __expf(-z1));
-                                ssq = fmaf(a0, a0, fmaf(a1, a1, ssq));
-                                a0 *= bf_lo(nw[e]);
-                                a1 *= bf_hi(nw[e]);
+                                zw4 = *reinterpret_cast<const uint4*>(p.z + tok * p.sz + col + 8 * cc);
+                                nw4 = *reinterpret_cast<const uint4*>(p.norm_w + col + 8 * cc);
                             }
-                            o[e] = pack_bf16(a0, a1);
+                            const uint32_t zw[4] = {zw4.x, zw4.y, zw4.z, zw4.w};
+                            const uint32_t nw[4] = {nw4.x, nw4.y, nw4.z, nw4.w};
+                            uint32_t o[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int j = 8 * c + 2 * e;
+                                float a0 = __uint_as_float(yv[j]) + ey * __uint_as_float(ov[j]) + Dh * bf_lo(xw[e]);
+                                float a1 =
+                                    __uint_as_float(yv[j + 1]) + ey * __uint_as_float(ov[j + 1]) + Dh * bf_hi(xw[e]);
+                                if (p.z) {
+                                    const float z0 = bf_lo(zw[e]), z1 = bf_hi(zw[e]);
+                                    a0 *= __fdividef(z0, 1.0f + __expf(-z0));
+                                    a1 *= __fdividef(z1, 1.0f + __expf(-z1));
+                                    ssq[h2] = fmaf(a0, a0, fmaf(a1, a1, ssq[h2]));
+                                    a0 *= bf_lo(nw[e]);
+                                    a1 *= bf_hi(nw[e]);
+                                }
+                                o[e] = pack_bf16(a0, a1);
+                            }
+                            reinterpret_cast<uint4*>(yo)[cc] = make_uint4(o[0], o[1], o[2], o[3]);
                         }
-                        reinterpret_cast<uint4*>(yo)[c] = make_uint4(o[0], o[1], o[2], o[3]);
                     }
-                    if (p.z) p.row_parts[tok * 2 * p.h + 2 * head + hf] = ssq;
+                    if (p.z) {
+                        p.row_parts[tok * 2 * p.h + 2 * head] = ssq[0];
+                        p.row_parts[tok * 2 * p.h + 2 * head + 1] = ssq[1];
+                    }
+                }
+                {  // state: H <- exp(cs_end) H + S
+                    const float dec = exp2f(tot);
+#pragma unroll
+                    for (int h2 = 0; h2 < 2; ++h2) {
+                        uint32_t sv[32];
+                        tmem_ld32(tmem + lane_base + kTS + 64 * hf + 32 * h2, sv);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            hs[32 * h2 + j] = fmaf(dec, hs[32 * h2 + j], __uint_as_float(sv[j]));
+                    }
+                }
+                tc_fence_before();
+                if (FULL) {
+                    write_h();
+                    fence_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        mbar_arrive(h_ready);
+                        mbar_arrive(&empty[s]);  // x is read
+                    }
                 }
             }
-            {
-                uint32_t sv[32];
-                tmem_ld32(tmem + lane_base + kTS + 32 * hf, sv);
-                tmem_ld_wait();
-                const float dec = exp2f(tot);
-#pragma unroll
-                for (int j = 0; j < 32; ++j) hs[j] = fmaf(dec, hs[j], __uint_as_float(sv[j]));
-            }
-            if (FULL) {
-                write_h();
-                fence_async_smem();
-            }
-            tc_fence_before();
-            seg_log2 += tot;
+            if (!ok) raise_timeout(abort, p.status);
         }
 
-        if (!*abort) {
+        if (!*abort && head_ok) {
             if (FULL) {
                 if (seg == p.nseg - 1 && p.final_state) {
                     float* dst = p.final_state + (int64_t)b * p.state_stride + (int64_t)head * PN;
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) dst[(32 * hf + j) * kN + r] = hs[j];
+                    for (int j = 0; j < 64; ++j) dst[j * kN + r] = hs[j];
                 }
             } else {
                 float* dst = p.states + (bh * p.nseg + seg + 1) * PN;
 #pragma unroll
-                for (int j = 0; j < 32; ++j) dst[(32 * hf + j) * kN + r] = hs[j];
-                if (r == 0 && hf == 0) p.seg_decay[bh * p.nseg + seg] = seg_log2;
+                for (int j = 0; j < 64; ++j) dst[j * kN + r] = hs[j];
+                if (r == 0) p.seg_decay[bh * p.nseg + seg] = seg_log2;
             }
         }
     }
@@ -432,9 +510,13 @@ struct Plan {
 
 Plan plan_for(const ScanArgs& a, int sms)
 {
+    // Cost in units of one block (128 tokens) of chunk-scan work per CTA.  A CTA
+    // also pays a fixed start (TMEM, barriers, state load and pipeline fill,
+    // about 1.5 blocks); the segment-state pass costs about 0.35 of a block per
+    // block, and the combine a little per segment.
     Plan pl;
     pl.nchunks = (a.L + kQ - 1) / kQ;
-    const int64_t bh = (int64_t)a.batch * a.h;
+    const int64_t ctas = (int64_t)a.batch * ((a.h + 1) / 2);  // CTAs per segment: head pairs
     double best = 1e30;
     pl.nseg = 1;
     pl.cps = pl.nchunks;
@@ -442,9 +524,8 @@ Plan plan_for(const ScanArgs& a, int sms)
         const int cps = (pl.nchunks + ns - 1) / ns;
         const int nseg = (pl.nchunks + cps - 1) / cps;
         if (nseg != ns) continue;
-        const double waves = std::ceil((double)(bh * nseg) / sms);
-        double cost = waves * cps;
-        if (nseg > 1) cost += 0.4 * std::ceil((double)(bh * (nseg - 1)) / sms) * cps + 1.0;
+        double cost = std::ceil((double)(ctas * nseg) / sms) * (cps + 1.5);
+        if (nseg > 1) cost += 0.35 * std::ceil((double)(ctas * (nseg - 1)) / sms) * (cps + 1.5) + 2.0 + 0.1 * nseg;
         if (cost < best - 1e-9) {
             best = cost;
             pl.nseg = nseg;
@@ -468,8 +549,9 @@ size_t align256(size_t v) { return (v + 255) / 256 * 256; }
 
 bool scan_tc_supported(const ScanArgs& a)
 {
+    // a CTA takes two consecutive heads, which must read the same B and C group
     return a.P == kP && a.N == kN && a.chunk % kQ == 0 && a.batch > 0 && a.L > 0 && a.h > 0 && a.G > 0 &&
-           (int64_t)a.batch * a.L < (1ll << 31);
+           (a.G == 1 || a.hpg % 2 == 0) && (int64_t)a.batch * a.L < (1ll << 31);
 }
 
 size_t scan_tc_workspace(const ScanArgs& a)
@@ -534,7 +616,7 @@ static cudaError_t launch_scan_tc_impl(const ScanArgs& a, const ScanGate* gate, 
         attr_set |= 1ull << dev;
     }
     if (pl.nseg > 1) {
-        ssd_tc_kernel<false><<<dim3(a.h, pl.nseg - 1, a.batch), 320, kSmemBytes, s>>>(mapX, mapB, mapC, p);
+        ssd_tc_kernel<false><<<dim3((a.h + 1) / 2, pl.nseg - 1, a.batch), 320, kSmemBytes, s>>>(mapX, mapB, mapC, p);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
         const int64_t n = (int64_t)bh * kP * kN;
@@ -543,7 +625,7 @@ static cudaError_t launch_scan_tc_impl(const ScanArgs& a, const ScanGate* gate, 
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
-    ssd_tc_kernel<true><<<dim3(a.h, pl.nseg, a.batch), 320, kSmemBytes, s>>>(mapX, mapB, mapC, p);
+    ssd_tc_kernel<true><<<dim3((a.h + 1) / 2, pl.nseg, a.batch), 320, kSmemBytes, s>>>(mapX, mapB, mapC, p);
     return cudaGetLastError();
 }
 

@@ -7,6 +7,13 @@ from gpu_util import TOL, dims_of, ensure_built, make_block, max_abs_rel, to_dev
 from nested_mamba2_selective_b200 import matmamba_block_fwd, ssd_step, synth
 
 pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _no_device_timeouts():
+    yield
+    from nested_mamba2_selective_b200 import mm_device_status
+    assert mm_device_status() == 0, "a kernel's bounded wait gave up"
 W = synth.WORKLOADS["decode_b256_1p4b"]
 
 

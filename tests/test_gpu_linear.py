@@ -9,6 +9,13 @@ from nested_mamba2_selective_b200 import mm_device_status, mm_linear, synth
 pytestmark = pytest.mark.gpu
 
 
+@pytest.fixture(autouse=True)
+def _no_device_timeouts():
+    yield
+    from nested_mamba2_selective_b200 import mm_device_status
+    assert mm_device_status() == 0, "a kernel's bounded wait gave up"
+
+
 @pytest.fixture(scope="module", autouse=True)
 def _built():
     ensure_built()

@@ -4,7 +4,7 @@ import pytest
 import torch
 
 from gpu_util import TOL, ensure_built, max_abs_rel, to_device, to_np
-from nested_mamba2_selective_b200 import ssd_scan, synth
+from nested_mamba2_selective_b200 import mm_device_status, ssd_scan, synth
 
 pytestmark = pytest.mark.gpu
 
@@ -12,6 +12,12 @@ pytestmark = pytest.mark.gpu
 @pytest.fixture(scope="module", autouse=True)
 def _built():
     ensure_built()
+
+
+@pytest.fixture(autouse=True)
+def _no_device_timeouts():
+    yield
+    assert mm_device_status() == 0, "a kernel's bounded wait gave up"
 
 
 def upload(inp, dtype):

@@ -8,6 +8,13 @@ from gpu_util import TOL, ensure_built, max_abs_rel, to_device, to_np
 from nested_mamba2_selective_b200 import BlockWeights, matmamba_stack_fwd, synth
 
 pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _no_device_timeouts():
+    yield
+    from nested_mamba2_selective_b200 import mm_device_status
+    assert mm_device_status() == 0, "a kernel's bounded wait gave up"
 W = synth.WORKLOADS["stack48_1p4b_b4_L4096"]
 DIMS = oracle.Dims(W.d_model, W.d_inner, W.d_head, W.d_state, W.ngroups, W.d_conv, 1e-5)
 
