@@ -86,6 +86,23 @@ def scan_bytes(T, h, P=64, N=128):
     return T * (2 * h * P * 2 + 2 * N * 2 + h * 4)
 
 
+# ------------------------------------------------------------------------------------ multi-rank aggregation
+
+def max_over_ranks(value, world, dist=None, device=None):
+    """Largest value over all ranks (the slowest rank's time); plain value for one rank."""
+    if world == 1:
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank_step, steps, world, slowest_seconds):
+    """Throughput of the whole job: every rank's units over the slowest rank's time."""
+    return world * units_per_rank_step * steps / slowest_seconds
+
+
 # ------------------------------------------------------------------------------------ clocks
 
 class ClockSampler:
@@ -166,12 +183,8 @@ def run_ours(args):
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(v):
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    def slowest(v):
+        return max_over_ranks(v, world, dist, dev)
 
     stream = torch.cuda.current_stream()
     flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
@@ -221,15 +234,15 @@ def run_ours(args):
         for m in B["widths"]:
             fn = lambda m=m: mm.matmamba_block_fwd(wt, u, m, B["chunk"], out=out, workspace=ws)  # noqa: E731
             ms, tr = timed(fn, args.steps, args.warmup, trace=True)
-            total = max_over_ranks(sum(ms))
-            per_width[str(m)] = {"tokens_per_s": world * T * args.steps / (total / 1e3),
+            total = slowest(sum(ms))
+            per_width[str(m)] = {"tokens_per_s": whole_job_rate(T, args.steps, world, total / 1e3),
                                  "ms_per_step": total / args.steps}
             if m == B["widths"][0]:
                 head = (ms, total, tr)
     clocks = clk.summary()
     ms, total, (stages, kernels) = head
     m0 = B["widths"][0]
-    value = world * T * args.steps / (total / 1e3)
+    value = whole_job_rate(T, args.steps, world, total / 1e3)
 
     # dominant stage of the headline step -> roofline object
     work = block_work(m0, T)
@@ -268,7 +281,7 @@ def run_ours(args):
         fn = lambda h=h, y=y, sws=sws: mm.ssd_scan(g["x"], g["dt"], g["A"], g["B"], g["C"], g["D"], h=h,  # noqa
                                                    chunk=S["chunk"], y=y, workspace=sws)
         sms, _ = timed(fn, args.steps, args.warmup)
-        avg = max_over_ranks(sum(sms)) / args.steps
+        avg = slowest(sum(sms)) / args.steps
         nbytes = scan_bytes(Ts, h)
         scan[str(h)] = {"tokens_per_s": world * Ts / (avg / 1e3), "us_per_call": avg * 1e3,
                         "roofline": {"bound": "hbm", "achieved": nbytes / (avg / 1e3) / 1e9, "peak": pk["hbm_gbs"],
@@ -286,12 +299,12 @@ def run_ours(args):
     t0 = time.perf_counter()
     for _ in range(args.steps):
         e2e_fn()
-    e2e_s = max_over_ranks(time.perf_counter() - t0)
+    e2e_s = slowest(time.perf_counter() - t0)
     io_bytes = T * B["d_model"] * 2
 
     extended = {}
     if args.extended:
-        extended = run_extended(args, mm, synth, torch, dev, timed, max_over_ranks, world)
+        extended = run_extended(args, mm, synth, torch, dev, timed, slowest, world)
 
     if rank == 0:
         line = {
@@ -307,7 +320,7 @@ def run_ours(args):
             "roofline": roof,
             "stages": stage_table,
             "ssd_scan": {"workload": S["workload"], "by_heads": scan},
-            "e2e": {"value": world * T * args.steps / e2e_s, "unit": "tokens/s", "h2d_bytes_per_step": io_bytes,
+            "e2e": {"value": whole_job_rate(T, args.steps, world, e2e_s), "unit": "tokens/s", "h2d_bytes_per_step": io_bytes,
                     "d2h_bytes_per_step": io_bytes},
             "gpu_launches": kernels,
             "clocks": clocks,
@@ -343,7 +356,7 @@ def run_only(args, mm, synth, torch, dev, timed):
     print(json.dumps({"only": args.only, "ms_per_step": sum(ms) / len(ms), "stages": stages, "kernels": kernels}))
 
 
-def run_extended(args, mm, synth, torch, dev, timed, max_over_ranks, world):
+def run_extended(args, mm, synth, torch, dev, timed, slowest, world):
     """48-layer stack (b4 L4096, d_model 2048) per width and the 256-sequence decode step per width."""
     import numpy as np
     res = {}
@@ -363,7 +376,7 @@ def run_extended(args, mm, synth, torch, dev, timed, max_over_ranks, world):
         fn = lambda: mm.matmamba_stack_fwd(layers, pws, u, ms_list, out=out, workspace=ws)  # noqa: E731
         steps = max(2, min(args.steps, 5))
         ms, _ = timed(fn, steps, 1)
-        avg = max_over_ranks(sum(ms)) / steps
+        avg = slowest(sum(ms)) / steps
         stack[str(m)] = {"ms_per_forward": avg, "tokens_per_s": world * 4 * 4096 / (avg / 1e3)}
     res["stack48_1p4b_b4_L4096"] = stack
     dec = {}
@@ -377,7 +390,7 @@ def run_extended(args, mm, synth, torch, dev, timed, max_over_ranks, world):
         ws = torch.empty(mm.ssd_step_workspace(w, 256, m), dtype=torch.uint8, device=dev)
         fn = lambda: mm.ssd_step(w, s, c, ut, m, out_t=ot, workspace=ws)  # noqa: E731
         ms, _ = timed(fn, args.steps, args.warmup)
-        avg = max_over_ranks(sum(ms)) / args.steps
+        avg = slowest(sum(ms)) / args.steps
         dec[str(m)] = {"us_per_step": avg * 1e3, "tokens_per_s": world * 256 / (avg / 1e3)}
     res["decode_b256_1p4b"] = dec
     return res

@@ -94,6 +94,9 @@ typedef struct mm_block_params {
 /* Human-readable name of a status code (static string, never NULL). */
 const char* mm_status_string(int status);
 
+/* Name of the most recent CUDA error behind an MM_ERR_CUDA ("cudaSuccess" if none). */
+const char* mm_last_cuda_error(void);
+
 /* Library version: major*10000 + minor*100 + patch. */
 int mm_version(void);
 

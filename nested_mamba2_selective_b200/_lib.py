@@ -25,7 +25,8 @@ _TORCH = {MM_F32: torch.float32, MM_BF16: torch.bfloat16}
 class MatMambaError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
-        super().__init__("%s failed: %s (status %d)" % (where, status_string(status), status))
+        detail = " [%s]" % load().mm_last_cuda_error().decode() if status == 6 else ""
+        super().__init__("%s failed: %s (status %d)%s" % (where, status_string(status), status, detail))
 
 
 class BlockParamsC(ctypes.Structure):
@@ -41,6 +42,7 @@ _vp, _i, _i64, _sz, _f = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c
 _pp = ctypes.POINTER(BlockParamsC)
 _SIGS = {
     "mm_status_string": ([_i], ctypes.c_char_p),
+    "mm_last_cuda_error": ([], ctypes.c_char_p),
     "mm_version": ([], _i),
     "mm_device_status": ([_vp], _i),
     "mm_width": ([_pp, _i, ctypes.POINTER(_i), ctypes.POINTER(_i)], _i),

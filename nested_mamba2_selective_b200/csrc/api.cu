@@ -89,7 +89,14 @@ int resolve(const mm_block_params* p, int m, View& v)
     return MM_OK;
 }
 
-inline int cuda_status(cudaError_t e) { return e == cudaSuccess ? MM_OK : MM_ERR_CUDA; }
+cudaError_t g_last_cuda_error = cudaSuccess;  // most recent CUDA error a call reported
+
+inline int cuda_status(cudaError_t e)
+{
+    if (e == cudaSuccess) return MM_OK;
+    g_last_cuda_error = e;
+    return MM_ERR_CUDA;
+}
 
 // ------------------------------------------------------------------ tracing
 
@@ -368,6 +375,8 @@ const char* mm_status_string(int status)
 }
 
 int mm_version(void) { return 100; }
+
+const char* mm_last_cuda_error(void) { return cudaGetErrorName(g_last_cuda_error); }
 
 int mm_device_status(void* stream)
 {

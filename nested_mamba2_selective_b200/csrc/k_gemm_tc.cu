@@ -26,6 +26,7 @@ __device__ __forceinline__ float bf_lo_u(uint32_t v) { return __uint_as_float(v 
 __device__ __forceinline__ float bf_hi_u(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
 
 constexpr int kBM = 128;  // rows of a tile = TMEM lanes
+constexpr int kStageLd = 36;  // fp32 row pitch of the conv epilogue's staging buffer (32 columns + pad)
 constexpr int kBK = 64;   // one 128-byte swizzle atom of bf16 along K
 
 struct TcSeg {
@@ -87,7 +88,7 @@ __device__ __forceinline__ void store_bf16_chunk(__nv_bfloat16* o, int ncols, bo
     }
 }
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, bool CONV>
 __global__ void __launch_bounds__(320, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB, const TcParams p)
 {
@@ -98,8 +99,9 @@ __global__ void __launch_bounds__(320, 1)
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    float* halo = reinterpret_cast<float*>(smem + STAGES * STAGE_BYTES);  // [2 groups][2 bufs][4 quarters][3][32]
-    uint64_t* full = reinterpret_cast<uint64_t*>(halo + 2 * 2 * 4 * 3 * 32);
+    // [2 epilogue groups][128 rows][kStageLd]: a 32-column chunk of fp32 accumulators for the conv epilogue
+    float* stage = reinterpret_cast<float*>(smem + STAGES * STAGE_BYTES);
+    uint64_t* full = reinterpret_cast<uint64_t*>(stage + (CONV ? 2 * kBM * kStageLd : 0));
     uint64_t* empty = full + STAGES;
     uint64_t* tfull = empty + STAGES;
     uint64_t* tempty = tfull + 2;
@@ -227,77 +229,93 @@ __global__ void __launch_bounds__(320, 1)
                 }
                 const int ncols = min(32, t.nvalid - c0);
                 const int col = t.n0 + c0;
-                if (sg.kind == kEpiConv) {
-                    // predecessors of this row: lanes above in this warp, the previous warp's last rows via smem
-                    float* hb = halo + ((eg * 2 + (nchunk_done & 1)) * 4) * 96;
-                    if (lane >= 29) {
+                if (CONV && sg.kind == kEpiConv) {
+                    // The chunk goes through shared memory so that each thread can walk down the token
+                    // axis: thread (q, lane) takes columns 2 (lane % 16) and +1 over rows
+                    // [16 rb, 16 rb + 16), rb = 2 q + lane / 16, keeping the last three pre-conv values of
+                    // its two columns in registers.  Taps never cross a sequence start: the window
+                    // restarts from the given history (or zeros) at token position 0.
+                    float* st = stage + eg * (kBM * kStageLd);
+                    if (ok) {
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) hb[q * 96 + (lane - 29) * 32 + i] = v[i];
+                        for (int c = 0; c < 8; ++c)
+                            *reinterpret_cast<float4*>(st + r * kStageLd + 4 * c) =
+                                make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
                     }
                     asm volatile("bar.sync %0, 128;" ::"r"(2 + eg) : "memory");
-                    float u1[32], u2[32], u3[32];
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        u1[i] = __shfl_up_sync(0xffffffffu, v[i], 1);
-                        u2[i] = __shfl_up_sync(0xffffffffu, v[i], 2);
-                        u3[i] = __shfl_up_sync(0xffffffffu, v[i], 3);
-                    }
-                    if (lane < 3 && q > 0) {
-                        const float* hp = hb + (q - 1) * 96;  // rows 29, 30, 31 of the previous quarter
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) {
-                            if (lane < 1) u1[i] = hp[2 * 32 + i];
-                            if (lane < 2) u2[i] = hp[(lane + 1) * 32 + i];
-                            u3[i] = hp[lane * 32 + i];
-                        }
-                    }
-                    if (row_ok && ok) {
-                        const int64_t b = m / ex.L;
+                    const int cp = lane & 15, rb = 2 * q + (lane >> 4);
+                    const int lc = 2 * cp;  // local column pair
+                    if (ok && lc < ncols) {
+                        const int crow = sg.conv_row0 + col + lc;
+                        const bool two = lc + 1 < ncols;
                         const __nv_bfloat16* cw = static_cast<const __nv_bfloat16*>(ex.conv_w);
-                        const __nv_bfloat16* cb = static_cast<const __nv_bfloat16*>(ex.conv_b);
+                        const __nv_bfloat16* cbias = static_cast<const __nv_bfloat16*>(ex.conv_b);
                         const __nv_bfloat16* cin = static_cast<const __nv_bfloat16*>(ex.conv_state_in);
-                        float o[32];
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) {
-                            const int crow = sg.conv_row0 + col + i;
-                            float acc = 0.0f;
-                            if (i < ncols) {
-                                const uint2 w4 = *reinterpret_cast<const uint2*>(cw + (int64_t)crow * 4);
-                                const float w0 = bf_lo_u(w4.x), w1 = bf_hi_u(w4.x), w2 = bf_lo_u(w4.y),
-                                            w3 = bf_hi_u(w4.y);
-                                float x3 = u3[i], x2 = u2[i], x1 = u1[i];
-                                if (tpos < 3) {  // taps before the sequence start: given history or zeros
-                                    const __nv_bfloat16* st = cin ? cin + (b * ex.conv_rows + crow) * 3 : nullptr;
-                                    if (tpos < 3) x3 = st ? __bfloat162float(st[tpos]) : 0.0f;
-                                    if (tpos < 2) x2 = st ? __bfloat162float(st[tpos + 1]) : 0.0f;
-                                    if (tpos < 1) x1 = st ? __bfloat162float(st[tpos + 2]) : 0.0f;
+                        __nv_bfloat16* cout = static_cast<__nv_bfloat16*>(ex.conv_state_out);
+                        const uint2 wa = *reinterpret_cast<const uint2*>(cw + (int64_t)crow * 4);
+                        const uint2 wb = two ? *reinterpret_cast<const uint2*>(cw + (int64_t)(crow + 1) * 4) : wa;
+                        const float a0 = bf_lo_u(wa.x), a1 = bf_hi_u(wa.x), a2 = bf_lo_u(wa.y), a3 = bf_hi_u(wa.y);
+                        const float b0 = bf_lo_u(wb.x), b1 = bf_hi_u(wb.x), b2 = bf_lo_u(wb.y), b3 = bf_hi_u(wb.y);
+                        const float biasa = __bfloat162float(cbias[crow]);
+                        const float biasb = two ? __bfloat162float(cbias[crow + 1]) : 0.0f;
+                        // window start: three rows above the block (inside the tile: rows >= 0)
+                        const int r0 = 16 * rb;
+                        float xa3 = 0.f, xa2 = 0.f, xa1 = 0.f, xb3 = 0.f, xb2 = 0.f, xb1 = 0.f;
+                        if (r0 >= 3) {
+                            const float2 p3 = *reinterpret_cast<const float2*>(st + (r0 - 3) * kStageLd + lc);
+                            const float2 p2 = *reinterpret_cast<const float2*>(st + (r0 - 2) * kStageLd + lc);
+                            const float2 p1 = *reinterpret_cast<const float2*>(st + (r0 - 1) * kStageLd + lc);
+                            xa3 = p3.x; xb3 = p3.y; xa2 = p2.x; xb2 = p2.y; xa1 = p1.x; xb1 = p1.y;
+                        }
+                        int64_t m_r = (int64_t)t.mt * p.rows - p.shift + r0;  // token of row r0
+                        int tp = (int)(((m_r % ex.L) + ex.L) % ex.L);          // its position in its sequence
+#pragma unroll 4
+                        for (int i = 0; i < 16; ++i, ++m_r) {
+                            const int rr = r0 + i;
+                            const float2 xv = *reinterpret_cast<const float2*>(st + rr * kStageLd + lc);
+                            if (tp == 0) {  // sequence start: history from the given state, or zeros
+                                const int64_t bq = m_r / ex.L;
+                                if (cin && m_r >= 0 && m_r < p.M) {
+                                    const __nv_bfloat16* ha = cin + (bq * ex.conv_rows + crow) * 3;
+                                    xa3 = __bfloat162float(ha[0]); xa2 = __bfloat162float(ha[1]);
+                                    xa1 = __bfloat162float(ha[2]);
+                                    if (two) {
+                                        xb3 = __bfloat162float(ha[3]); xb2 = __bfloat162float(ha[4]);
+                                        xb1 = __bfloat162float(ha[5]);
+                                    }
+                                } else {
+                                    xa3 = xa2 = xa1 = xb3 = xb2 = xb1 = 0.0f;
                                 }
-                                acc = __bfloat162float(cb[crow]);
-                                acc = fmaf(w0, x3, acc);
-                                acc = fmaf(w1, x2, acc);
-                                acc = fmaf(w2, x1, acc);
-                                acc = fmaf(w3, v[i], acc);
                             }
-                            o[i] = silu_fast(acc);
-                        }
-                        store_bf16_chunk(static_cast<__nv_bfloat16*>(sg.out) + m * sg.ldo + col, ncols, sg.vec_ok, o);
-                        if (ex.conv_state_out && tpos >= ex.L - 3) {  // last K-1 pre-conv inputs
-                            __nv_bfloat16* so = static_cast<__nv_bfloat16*>(ex.conv_state_out);
-#pragma unroll
-                            for (int i = 0; i < 32; ++i)
-                                if (i < ncols)
-                                    so[(b * ex.conv_rows + sg.conv_row0 + col + i) * 3 + (tpos - (ex.L - 3))] =
-                                        __float2bfloat16_rn(v[i]);
-                        }
-                        if (ex.conv_state_out && tpos == 0 && ex.L < 3) {  // older entries shift in from the history
-                            __nv_bfloat16* so = static_cast<__nv_bfloat16*>(ex.conv_state_out);
-                            for (int i = 0; i < ncols; ++i) {  // no register array indexed here
-                                const int64_t base = (b * ex.conv_rows + sg.conv_row0 + col + i) * 3;
-                                for (int e = 0; e < 3 - ex.L; ++e)
-                                    so[base + e] = cin ? cin[base + e + ex.L] : __float2bfloat16_rn(0.0f);
+                            if (rr >= p.shift && m_r < p.M) {
+                                float oa = fmaf(a3, xv.x, fmaf(a2, xa1, fmaf(a1, xa2, fmaf(a0, xa3, biasa))));
+                                float ob = fmaf(b3, xv.y, fmaf(b2, xb1, fmaf(b1, xb2, fmaf(b0, xb3, biasb))));
+                                oa = silu_fast(oa);
+                                ob = silu_fast(ob);
+                                __nv_bfloat16* o = static_cast<__nv_bfloat16*>(sg.out) + m_r * sg.ldo + col + lc;
+                                if (two) *reinterpret_cast<uint32_t*>(o) = pack_bf16(oa, ob);
+                                else *o = __float2bfloat16_rn(oa);
+                                if (cout && tp >= ex.L - 3) {  // last K-1 pre-conv inputs of the sequence
+                                    const int64_t bq = m_r / ex.L;
+                                    const int slot = tp - (ex.L - 3);
+                                    cout[(bq * ex.conv_rows + crow) * 3 + slot] = __float2bfloat16_rn(xv.x);
+                                    if (two) cout[(bq * ex.conv_rows + crow + 1) * 3 + slot] = __float2bfloat16_rn(xv.y);
+                                }
+                                if (cout && tp == 0 && ex.L < 3) {  // older entries shift in from the history
+                                    const int64_t bq = m_r / ex.L;
+                                    for (int e = 0; e < 3 - ex.L; ++e) {
+                                        const int64_t ba = (bq * ex.conv_rows + crow) * 3;
+                                        cout[ba + e] = cin ? cin[ba + e + ex.L] : __float2bfloat16_rn(0.0f);
+                                        if (two) cout[ba + 3 + e] = cin ? cin[ba + 3 + e + ex.L] : __float2bfloat16_rn(0.0f);
+                                    }
+                                }
                             }
+                            xa3 = xa2; xa2 = xa1; xa1 = xv.x;
+                            xb3 = xb2; xb2 = xb1; xb1 = xv.y;
+                            tp = (tp + 1 == ex.L) ? 0 : tp + 1;
                         }
                     }
+                    asm volatile("bar.sync %0, 128;" ::"r"(2 + eg) : "memory");  // the stage buffer is free again
                 } else if (row_ok && ok) {
                     if (sg.kind == kEpiSoftplus) {
                         float* o = static_cast<float*>(sg.out) + m * sg.ldo + col;
@@ -387,7 +405,7 @@ static bool tc_shape_ok(const GemmDesc& g)
 
 bool gemm_tc_supported(const GemmDesc& g) { return tc_shape_ok(g) && encode_fn() != nullptr; }
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, bool CONV>
 static cudaError_t launch_bn(const GemmDesc& g, const TcParams& p0, cudaStream_t s, int* status)
 {
     TcParams p = p0;
@@ -403,20 +421,21 @@ static cudaError_t launch_bn(const GemmDesc& g, const TcParams& p0, cudaStream_t
     CUtensorMap mapA, mapB;
     if (!make_tmap_bf16(&mapA, g.A, g.K, g.M, g.lda * 2, kBK, kBM)) return cudaErrorInvalidValue;
     if (!make_tmap_bf16(&mapB, base, g.ldb, rows, g.ldb * 2, kBK, BN)) return cudaErrorInvalidValue;
-    constexpr int smem = STAGES * (kBM + BN) * kBK * 2 + 1024 + 2 * 2 * 4 * 3 * 32 * 4 + 256;
+    constexpr int smem = STAGES * (kBM + BN) * kBK * 2 + (CONV ? 2 * kBM * kStageLd * 4 : 0) + 1024 + 256;
+    static_assert(smem <= 232448, "GEMM configuration exceeds 227 KB of shared memory");
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     static unsigned long long attr_set = 0;  // one bit per device
     if (dev < 64 && !(attr_set >> dev & 1ull)) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             smem);
+        cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, STAGES, CONV>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
         attr_set |= 1ull << dev;
     }
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int total = p.mtiles * p.ntiles;
     const int grid = total < sms ? total : sms;
-    gemm_tc_kernel<BN, STAGES><<<grid, 320, smem, s>>>(mapA, mapB, p);
+    gemm_tc_kernel<BN, STAGES, CONV><<<grid, 320, smem, s>>>(mapA, mapB, p);
     return cudaGetLastError();
 }
 
@@ -452,8 +471,10 @@ cudaError_t launch_gemm_tc(const GemmDesc& g, cudaStream_t s)
     int* status = device_status_ptr();
     // Wide tiles when they still give every SM work; narrow ones for skinny problems.
     const int tiles256 = p.mtiles * ((n_total + 255) / 256);
-    if (tiles256 >= 148) return launch_bn<256, 4>(g, p, s, status);
-    return launch_bn<128, 6>(g, p, s, status);
+    const bool conv = p.shift > 0;
+    if (tiles256 >= 148)
+        return conv ? launch_bn<256, 3, true>(g, p, s, status) : launch_bn<256, 4, false>(g, p, s, status);
+    return conv ? launch_bn<128, 5, true>(g, p, s, status) : launch_bn<128, 6, false>(g, p, s, status);
 }
 
 }  // namespace mm

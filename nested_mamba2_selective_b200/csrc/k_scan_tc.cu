@@ -21,8 +21,9 @@
 // producer, warp 1 TMEM owner and tcgen05.mma issuer, warps 2-9 compute.
 // Compute thread (quarter q, lane l, half hf) owns TMEM lane r = 32q + l and
 // head hf of the pair: token r for its Y row, state row n = r for S.  For the
-// masked matrices it takes the columns s in [64 hf, 64 hf + 64) of both heads,
-// written as bf16 A operands over the G columns it has just read.
+// masked matrix M of its own head it covers all 128 columns, 32 at a time;
+// each block of 32 G columns is overwritten (after both heads read it) by
+// head 0's then head 1's 16 packed bf16 columns, the A operands of Y.
 // Per block: G, then Y_off = C [H_0 | H_1] once the bf16 state copy H is in
 // shared memory (its space then takes X'), then Y_j = M_j X_j and
 // S = B^T [X'_0 | X'_1]; G of the next block overlaps this block's epilogue.
@@ -49,7 +50,8 @@ constexpr int kStage = 2 * kTileQN + 2 * kTileQP; // C | B | x of two heads
 constexpr int kNStage = 2;
 constexpr int kOffHX = kNStage * kStage;          // H (then X') of two heads
 constexpr int kOffSmall = kOffHX + 2 * kTileQP;
-constexpr int kSmemBytes = kOffSmall + 2560;
+constexpr int kSmemBytes = kOffSmall + 64 + 2 * 192 * 4 + 128;
+static_assert(kSmemBytes <= 232448, "chunk scan exceeds the 227 KB of shared memory a CTA can have");
 
 // TMEM columns: G = C B^T, overwritten in place by the masked M_0 | M_1 (A operands);
 // Y_0 | Y_1; Y_off of both heads; S of both heads.
@@ -82,6 +84,15 @@ __device__ __forceinline__ void named_sync_compute() { asm volatile("bar.sync 1,
 // Byte offset of 16-byte chunk `c` (0..7) of row `r` in a 128-byte-swizzled panel.
 __device__ __forceinline__ uint32_t sw128(int r, int c) { return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)); }
 
+// 2^x on the MUFU unit (PTX ex2.approx.ftz: relative error ~2^-22, results below 2^-126 flush to 0,
+// far below what the bf16 products built from it can hold).
+__device__ __forceinline__ float ex2(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 __device__ __forceinline__ float bf_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
 
@@ -91,10 +102,12 @@ __global__ void __launch_bounds__(320, 1)
                   const __grid_constant__ CUtensorMap mapC, const ScanTcParams p)
 {
     extern __shared__ __align__(1024) uint8_t sm[];
-    float* cs2 = reinterpret_cast<float*>(sm + kOffSmall);  // [2 heads][128] running log2 decay through token r
-    float* dts = cs2 + 2 * kQ;                                // [2 heads][128] dt (0 past the end)
-    float* wtot = dts + 2 * kQ;                               // [2 heads][4] per-warp scan totals
-    uint64_t* full = reinterpret_cast<uint64_t*>(wtot + 8);
+    float* wtot = reinterpret_cast<float*>(sm + kOffSmall);  // [2 heads][4] per-warp scan totals
+    float* anch = wtot + 8;                                   // [2 heads][4] running log2 decay at rows 32 i
+    // [2 heads][192]: 2^(cs(32 i) - cs(s)) dt(s) for s < 32 i, the column factors of row block i,
+    // packed as i = 1 at [0, 32), i = 2 at [32, 96), i = 3 at [96, 192)
+    float* ecol = anch + 8;
+    uint64_t* full = reinterpret_cast<uint64_t*>(ecol + 2 * 192);
     uint64_t* empty = full + kNStage;
     uint64_t* g_done = empty + kNStage;
     uint64_t* yo_done = g_done + 1;
@@ -221,13 +234,13 @@ __global__ void __launch_bounds__(320, 1)
                     for (int j = 0; j < 2; ++j)
 #pragma unroll
                         for (int kk = 0; kk < 8; ++kk)  // Y_j = M_j . X_j over the block's tokens
-                            mma_ts(tmem + kTY + 64 * j, tmem + kTG + 64 * (kk >> 2) + 32 * j + 8 * (kk & 3),
+                            mma_ts(tmem + kTY + 64 * j, tmem + kTG + 32 * (kk >> 1) + 16 * j + 8 * (kk & 1),
                                    desc_sw128(aX + j * kTileQP + kk * 2048, kTileQP, 1024), id_y, kk > 0);
                 }
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk)  // S = B^T . [X'_0 | X'_1] over the block's tokens
+                for (int kk = 0; kk < 8; ++kk)  // H += B^T . [X'_0 | X'_1] over the block's tokens
                     mma_ss(tmem + kTS, desc_sw128(aB + kk * 2048, kTileQN / 2, 1024),
-                           desc_sw128(aHX + kk * 2048, kTileQP, 1024), id_s, kk > 0);
+                           desc_sw128(aHX + kk * 2048, kTileQP, 1024), id_s, FULL ? 1u : (kk > 0));
                 mma_commit(ys_full);
             }
             mma_commit(done);
@@ -244,37 +257,25 @@ __global__ void __launch_bounds__(320, 1)
         const float Dh = (FULL && p.D && head_ok) ? p.D[head] : 0.0f;
         const int64_t bh = (int64_t)b * p.h + head;
         const int PN = kP * kN;
-        float* my_cs2 = cs2 + hf * kQ;
-        float* my_dts = dts + hf * kQ;
         uint8_t* myHX = sHX + hf * kTileQP;
 
-        // start state of this head: row n = r, all 64 columns p
-        float hs[64];
-        {
+        // The fp32 state of this head lives in TMEM columns kTS + 64 hf (row n = lane r): each
+        // block, the compute warps read H_k for its bf16 copy (Y_off's operand), write back
+        // 2^tot H_k, and the S MMA accumulates B^T X' on top, leaving H_{k+1}.
+        if (FULL) {
             const float* src = nullptr;
-            if (FULL && head_ok) {
+            if (head_ok) {
                 if (p.nseg > 1) src = p.states + (bh * p.nseg + seg) * PN;
                 else if (p.init_state) src = p.init_state + (int64_t)b * p.state_stride + (int64_t)head * PN;
             }
 #pragma unroll
-            for (int j = 0; j < 64; ++j) hs[j] = src ? src[j * kN + r] : 0.0f;
-        }
-        auto write_h = [&]() {
+            for (int h2 = 0; h2 < 2; ++h2) {
+                uint32_t v[32];
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                uint4 v;
-                v.x = pack_bf16(hs[8 * c + 0], hs[8 * c + 1]);
-                v.y = pack_bf16(hs[8 * c + 2], hs[8 * c + 3]);
-                v.z = pack_bf16(hs[8 * c + 4], hs[8 * c + 5]);
-                v.w = pack_bf16(hs[8 * c + 6], hs[8 * c + 7]);
-                *reinterpret_cast<uint4*>(myHX + sw128(r, c)) = v;
+                for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(src ? src[(32 * h2 + j) * kN + r] : 0.0f);
+                tmem_st32(tmem + lane_base + kTS + 64 * hf + 32 * h2, v);
             }
-        };
-        if (FULL) {
-            write_h();
-            fence_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(h_ready);
+            tmem_st_wait();
         }
         float seg_log2 = 0.0f;
         float dt_next = 0.0f;
@@ -311,61 +312,103 @@ __global__ void __launch_bounds__(320, 1)
                 tot += w;
             }
             const float c2 = sc + pre;
-            my_cs2[r] = c2;
-            my_dts[r] = dtv;
+            if (lane == 0) anch[hf * 4 + q] = c2;  // running decay at row 32 q
             named_sync_compute();
             seg_log2 += tot;
+            if (FULL) {  // column factors of the anchored row blocks, this thread's head and column r
+#pragma unroll
+                for (int i = 1; i < 4; ++i)
+                    if (r < 32 * i) ecol[hf * 192 + 16 * i * (i - 1) + r] = ex2(anch[hf * 4 + i] - c2) * dtv;
+                named_sync_compute();  // the table is read by the other row blocks' warps
+            }
+
+            if (FULL) {  // H_k: bf16 copy for Y_off, then 2^tot H_k back into TMEM for the S MMA to add onto
+                const float dec = ex2(tot);
+#pragma unroll
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    uint32_t v[32];
+                    tmem_ld32(tmem + lane_base + kTS + 64 * hf + 32 * h2, v);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        uint4 w;
+                        w.x = pack_bf16(__uint_as_float(v[8 * c + 0]), __uint_as_float(v[8 * c + 1]));
+                        w.y = pack_bf16(__uint_as_float(v[8 * c + 2]), __uint_as_float(v[8 * c + 3]));
+                        w.z = pack_bf16(__uint_as_float(v[8 * c + 4]), __uint_as_float(v[8 * c + 5]));
+                        w.w = pack_bf16(__uint_as_float(v[8 * c + 6]), __uint_as_float(v[8 * c + 7]));
+                        *reinterpret_cast<uint4*>(myHX + sw128(r, 4 * h2 + c)) = w;
+                    }
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(dec * __uint_as_float(v[j]));
+                    tmem_st32(tmem + lane_base + kTS + 64 * hf + 32 * h2, v);
+                }
+                tmem_st_wait();
+                fence_async_smem();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(h_ready);
+            }
 
             bool ok = __all_sync(0xffffffffu, mbar_wait(&full[s], (k / kNStage) & 1, abort));
             const uint8_t* sX = sm + s * kStage + kOffX + hf * kTileQP;
 
-            if (FULL && ok) {
-                ok = __all_sync(0xffffffffu, mbar_wait(g_done, k & 1, abort));
-                if (ok) {
-                    tc_fence_after();
-                    // M_j[t=r, s] = G[r, s] exp(cs_j[r] - cs_j[s]) dt_j[s] (s <= r) for both heads j and
-                    // the columns s in [64 hf, 64 hf + 64), written over the G columns just read
-                    const float c2h[2] = {cs2[r], cs2[kQ + r]};
+            if (FULL) {  // the quarter barriers below run whatever ok is, so no partner warp is stranded
+                if (ok) ok = __all_sync(0xffffffffu, mbar_wait(g_done, k & 1, abort));
+                if (ok) tc_fence_after();
+                {
+                    // M_j[t=r, s] = G[r, s] 2^(cs_j[r] - cs_j[s]) dt_j[s] for s <= r, else 0, built by the
+                    // threads of head j = hf over all 128 columns, 32 at a time.  Both heads' threads read
+                    // a row's 32 G columns before either writes them (a barrier per block); those columns
+                    // then take M_0 then M_1 for these s (16 packed columns each).
+                    // Column blocks below the row block q factor the decay through the anchor 32 q:
+                    // 2^(cs_r - cs_s) = 2^(cs_r - cs_32q) 2^(cs_32q - cs_s), both factors <= 1; the diagonal
+                    // block takes direct exponentials with its tokens' values shuffled in from this warp.
+                    const float er = ex2(c2 - __shfl_sync(0xffffffffu, c2, 0));
 #pragma unroll
-                    for (int half = 0; half < 2; ++half) {
-                        const int s0 = 64 * hf + 32 * half;
-                        uint32_t pk0[16], pk1[16];
-                        if (s0 <= q * 32 + 31) {
-                            uint32_t gv[32];
-                            tmem_ld32(tmem + lane_base + kTG + s0, gv);
+                    for (int cb = 0; cb < 4; ++cb) {  // column block s in [32 cb, 32 cb + 32)
+                        uint32_t gv[32];
+                        if (ok && cb <= q) {
+                            tmem_ld32(tmem + lane_base + kTG + 32 * cb, gv);
                             tmem_ld_wait();
+                        }
+                        asm volatile("bar.sync %0, 64;" ::"r"(2 + q) : "memory");  // both heads have read them
+                        if (!ok) continue;
+                        uint32_t pk[16];
+                        if (cb < q) {
+                            const float* ec = ecol + hf * 192 + 16 * q * (q - 1) + 32 * cb;
+#pragma unroll
+                            for (int e = 0; e < 32; e += 4) {
+                                const float4 f = *reinterpret_cast<const float4*>(ec + e);
+                                pk[e >> 1] = pack_bf16(__uint_as_float(gv[e]) * er * f.x, __uint_as_float(gv[e + 1]) * er * f.y);
+                                pk[(e >> 1) + 1] =
+                                    pack_bf16(__uint_as_float(gv[e + 2]) * er * f.z, __uint_as_float(gv[e + 3]) * er * f.w);
+                            }
+                        } else if (cb == q) {
 #pragma unroll
                             for (int e = 0; e < 32; e += 2) {
-                                const int sa = s0 + e, sb = sa + 1;
-                                const float ga = __uint_as_float(gv[e]), gb = __uint_as_float(gv[e + 1]);
-                                float v0a = 0.0f, v0b = 0.0f, v1a = 0.0f, v1b = 0.0f;
-                                if (sa <= r) {
-                                    v0a = ga * exp2f(c2h[0] - cs2[sa]) * dts[sa];
-                                    v1a = ga * exp2f(c2h[1] - cs2[kQ + sa]) * dts[kQ + sa];
-                                }
-                                if (sb <= r) {
-                                    v0b = gb * exp2f(c2h[0] - cs2[sb]) * dts[sb];
-                                    v1b = gb * exp2f(c2h[1] - cs2[kQ + sb]) * dts[kQ + sb];
-                                }
-                                pk0[e >> 1] = pack_bf16(v0a, v0b);
-                                pk1[e >> 1] = pack_bf16(v1a, v1b);
+                                const float ca = __shfl_sync(0xffffffffu, c2, e);
+                                const float cbv = __shfl_sync(0xffffffffu, c2, e + 1);
+                                const float da = __shfl_sync(0xffffffffu, dtv, e);
+                                const float db = __shfl_sync(0xffffffffu, dtv, e + 1);
+                                const float ma = __uint_as_float(gv[e]) * ex2(fminf(c2 - ca, 0.0f)) * da;
+                                const float mb = __uint_as_float(gv[e + 1]) * ex2(fminf(c2 - cbv, 0.0f)) * db;
+                                pk[e >> 1] = pack_bf16(e <= lane ? ma : 0.0f, e + 1 <= lane ? mb : 0.0f);
                             }
                         } else {
 #pragma unroll
-                            for (int e = 0; e < 16; ++e) pk0[e] = pk1[e] = 0u;
+                            for (int e = 0; e < 16; ++e) pk[e] = 0u;
                         }
-                        // head j's packed columns for s in [s0, s0 + 32) live at 64 hf + 32 j + 16 half
-                        tmem_st16(tmem + lane_base + kTG + 64 * hf + 16 * half, pk0);
-                        tmem_st16(tmem + lane_base + kTG + 64 * hf + 32 + 16 * half, pk1);
+                        // the 32 columns just read take head 0's then head 1's 16 packed columns
+                        tmem_st16(tmem + lane_base + kTG + 32 * cb + 16 * hf, pk);
                     }
-                    tmem_st_wait();
-                    ok = __all_sync(0xffffffffu, mbar_wait(yo_done, k & 1, abort));  // H is read: its space takes X'
+                    if (ok) tmem_st_wait();
+                    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(yo_done, k & 1, abort));  // H read: X' may go there
                 }
             } else if (!FULL && ok && k > 0) {
                 ok = __all_sync(0xffffffffu, mbar_wait(ys_full, (k - 1) & 1, abort));  // previous X' consumed
             }
             if (ok) {  // X'_j[s=r, :] = exp(cs_end - cs_r) dt_r x_j[r, :]
-                const float wgt = exp2f(tot - c2) * dtv;
+                const float wgt = ex2(tot - c2) * dtv;
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
                     const uint4 xv = *reinterpret_cast<const uint4*>(sX + sw128(r, c));
@@ -387,21 +430,22 @@ __global__ void __launch_bounds__(320, 1)
             }
             if (ok) {
                 tc_fence_after();
-                if (FULL && valid) {
-                    const float ey = exp2f(c2);
+                if (FULL) {  // TMEM loads are warp-collective: every lane loads, only valid rows store
+                    const float ey = ex2(c2);
                     const int64_t tok = tok0 + t0 + r;
                     const int col = head * kP;
                     __nv_bfloat16* yo = static_cast<__nv_bfloat16*>(p.y) + tok * p.sy + col;
                     float ssq[2] = {0.0f, 0.0f};
 #pragma unroll
-                    for (int h2 = 0; h2 < 2; ++h2) {  // 32 output columns at a time
-                        uint32_t yv[32], ov[32];
-                        tmem_ld32(tmem + lane_base + kTY + 64 * hf + 32 * h2, yv);
-                        tmem_ld32(tmem + lane_base + kTYO + 64 * hf + 32 * h2, ov);
+                    for (int h2 = 0; h2 < 4; ++h2) {  // 16 output columns at a time
+                        uint32_t yv[16], ov[16];
+                        tmem_ld16(tmem + lane_base + kTY + 64 * hf + 16 * h2, yv);
+                        tmem_ld16(tmem + lane_base + kTYO + 64 * hf + 16 * h2, ov);
                         tmem_ld_wait();
+                        if (!valid) continue;
 #pragma unroll
-                        for (int c = 0; c < 4; ++c) {
-                            const int cc = 4 * h2 + c;
+                        for (int c = 0; c < 2; ++c) {
+                            const int cc = 2 * h2 + c;
                             const uint4 xv = *reinterpret_cast<const uint4*>(sX + sw128(r, cc));
                             const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
                             uint4 zw4 = make_uint4(0, 0, 0, 0), nw4 = make_uint4(0, 0, 0, 0);
@@ -422,7 +466,7 @@ __global__ void __launch_bounds__(320, 1)
                                     const float z0 = bf_lo(zw[e]), z1 = bf_hi(zw[e]);
                                     a0 *= __fdividef(z0, 1.0f + __expf(-z0));
                                     a1 *= __fdividef(z1, 1.0f + __expf(-z1));
-                                    ssq[h2] = fmaf(a0, a0, fmaf(a1, a1, ssq[h2]));
+                                    ssq[h2 >> 1] = fmaf(a0, a0, fmaf(a1, a1, ssq[h2 >> 1]));
                                     a0 *= bf_lo(nw[e]);
                                     a1 *= bf_hi(nw[e]);
                                 }
@@ -431,49 +475,34 @@ __global__ void __launch_bounds__(320, 1)
                             reinterpret_cast<uint4*>(yo)[cc] = make_uint4(o[0], o[1], o[2], o[3]);
                         }
                     }
-                    if (p.z) {
+                    if (p.z && valid) {
                         p.row_parts[tok * 2 * p.h + 2 * head] = ssq[0];
                         p.row_parts[tok * 2 * p.h + 2 * head + 1] = ssq[1];
                     }
                 }
-                {  // state: H <- exp(cs_end) H + S
-                    const float dec = exp2f(tot);
-#pragma unroll
-                    for (int h2 = 0; h2 < 2; ++h2) {
-                        uint32_t sv[32];
-                        tmem_ld32(tmem + lane_base + kTS + 64 * hf + 32 * h2, sv);
-                        tmem_ld_wait();
-#pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            hs[32 * h2 + j] = fmaf(dec, hs[32 * h2 + j], __uint_as_float(sv[j]));
-                    }
-                }
                 tc_fence_before();
                 if (FULL) {
-                    write_h();
-                    fence_async_smem();
                     __syncwarp();
-                    if (lane == 0) {
-                        mbar_arrive(h_ready);
-                        mbar_arrive(&empty[s]);  // x is read
-                    }
+                    if (lane == 0) mbar_arrive(&empty[s]);  // x is read
                 }
             }
             if (!ok) raise_timeout(abort, p.status);
         }
 
-        if (!*abort && head_ok) {
-            if (FULL) {
-                if (seg == p.nseg - 1 && p.final_state) {
-                    float* dst = p.final_state + (int64_t)b * p.state_stride + (int64_t)head * PN;
+        if (FULL && seg == p.nseg - 1 && p.final_state) {  // state after the last block
+            const bool ok = __all_sync(0xffffffffu, !*abort);
+            if (ok) {
+                float* dst = p.final_state + (int64_t)b * p.state_stride + (int64_t)head * PN;
 #pragma unroll
-                    for (int j = 0; j < 64; ++j) dst[j * kN + r] = hs[j];
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    uint32_t v[32];
+                    tmem_ld32(tmem + lane_base + kTS + 64 * hf + 32 * h2, v);
+                    tmem_ld_wait();
+                    if (head_ok) {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) dst[(32 * h2 + j) * kN + r] = __uint_as_float(v[j]);
+                    }
                 }
-            } else {
-                float* dst = p.states + (bh * p.nseg + seg + 1) * PN;
-#pragma unroll
-                for (int j = 0; j < 64; ++j) dst[j * kN + r] = hs[j];
-                if (r == 0) p.seg_decay[bh * p.nseg + seg] = seg_log2;
             }
         }
     }
@@ -481,6 +510,194 @@ __global__ void __launch_bounds__(320, 1)
     __syncthreads();
     tc_fence_after();
     if (warp == 1) tmem_dealloc(tmem, kTCols);
+}
+
+// Segment end states from a zero start, for every segment but the last:
+//   S_seg = sum_s 2^(cs_end - cs_s) dt_s B_s x_s^T        (cs in log2 units, over the segment)
+// The segment's blocks are visited last to first.  With D the decay of the
+// blocks already visited (those after the current one), token s of the block
+// gets the weight 2^(D + tot - cs_s) <= 1, and every block's B^T X'' is
+// accumulated into one TMEM accumulator: no per-block state update, and the
+// compute warps wait for the tensor core only to reuse one of two X'' buffers.
+// Two heads per CTA as in the chunk scan; S of head j sits in TMEM columns
+// [64 j, 64 j + 64), row n = state dim.
+constexpr int kSegStage = kTileQN + 2 * kTileQP;          // B | x of two heads
+constexpr int kSegOffXP = kNStage * kSegStage;            // two X'' buffers of two heads
+constexpr int kSegOffSmall = kSegOffXP + 2 * 2 * kTileQP;
+constexpr int kSegSmemBytes = kSegOffSmall + 2 * kQ * 4 + 32 + 256;
+
+__global__ void __launch_bounds__(320, 1)
+    ssd_seg_state_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CUtensorMap mapB,
+                         const ScanTcParams p)
+{
+    extern __shared__ __align__(1024) uint8_t sm[];
+    float* wtot = reinterpret_cast<float*>(sm + kSegOffSmall);  // [2 heads][4]
+    uint64_t* full = reinterpret_cast<uint64_t*>(wtot + 8 + 2 * kQ);
+    uint64_t* empty = full + kNStage;
+    uint64_t* xr = empty + kNStage;   // X'' buffer written (compute -> MMA)
+    uint64_t* xf = xr + 2;            // X'' buffer consumed (MMA -> compute)
+    uint64_t* done = xf + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+    volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int pair = blockIdx.x, seg = blockIdx.y, b = blockIdx.z;
+    const int head0 = 2 * pair;
+    const int c_begin = seg * p.cps;
+    const int c_end = min(p.nchunks, c_begin + p.cps);
+    const int nch = c_end - c_begin;
+    const int grp = head0 / p.hpg;
+    const int64_t tok0 = (int64_t)b * p.L;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kNStage; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], 1);
+            mbar_init(&xr[i], 8);
+            mbar_init(&xf[i], 1);
+        }
+        mbar_init(done, 1);
+        *abort = (smem_u32(sm) & 1023u) ? 1 : 0;
+        if (*abort) raise_timeout(abort, p.status);
+        fence_mbar_init();
+        prefetch_tmap(&mapX);
+        prefetch_tmap(&mapB);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 128);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0 && !*abort) {  // TMA producer, blocks last to first
+            int k = 0;
+            for (; k < nch; ++k) {
+                const int s = k % kNStage;
+                if (!mbar_wait(&empty[s], ((k / kNStage) & 1) ^ 1, abort)) {
+                    raise_timeout(abort, p.status);
+                    break;
+                }
+                const int row = (int)(tok0 + (int64_t)(c_end - 1 - k) * kQ);
+                uint8_t* base = sm + s * kSegStage;
+                mbar_arrive_expect_tx(&full[s], kSegStage);
+                tma_load_2d(base, &mapB, &full[s], grp * kN, row);
+                tma_load_2d(base + kTileQN / 2, &mapB, &full[s], grp * kN + 64, row);
+                tma_load_2d(base + kTileQN, &mapX, &full[s], head0 * kP, row);
+                tma_load_2d(base + kTileQN + kTileQP, &mapX, &full[s], min(head0 + 1, p.h - 1) * kP, row);
+            }
+            for (int j = max(0, k - kNStage); j < k; ++j) mbar_wait(&full[j % kNStage], (j / kNStage) & 1, abort);
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && !*abort) {  // MMA issuer: S += B^T [X''_0 | X''_1]
+            const uint32_t id_s = idesc_bf16(128, 128, 1, 1);
+            for (int k = 0; k < nch; ++k) {
+                const int s = k % kNStage, xb = k & 1;
+                if (!mbar_wait(&full[s], (k / kNStage) & 1, abort) || !mbar_wait(&xr[xb], (k >> 1) & 1, abort)) {
+                    raise_timeout(abort, p.status);
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t aB = smem_u32(sm + s * kSegStage);
+                const uint32_t aXP = smem_u32(sm + kSegOffXP + xb * 2 * kTileQP);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ss(tmem, desc_sw128(aB + kk * 2048, kTileQN / 2, 1024), desc_sw128(aXP + kk * 2048, kTileQP, 1024),
+                           id_s, (k | kk) != 0);
+                mma_commit(&xf[xb]);
+                mma_commit(&empty[s]);
+            }
+            mma_commit(done);
+            mbar_wait(done, 0, nullptr);  // every issued MMA is done before TMEM can be released (bounded)
+        }
+    } else {  // compute warps: thread (quarter q, lane) = token / state row r, head hf of the pair
+        const int cw = warp - 2, q = warp & 3, hf = cw >> 2;
+        const int r = q * 32 + lane;
+        const int head = head0 + hf;
+        const bool head_ok = head < p.h;
+        const float A2 = head_ok ? p.A[head] * kLog2e : 0.0f;
+        float D2 = 0.0f;
+        float dt_next = 0.0f;
+        if (head_ok && nch > 0) {
+            const int t0 = (c_end - 1) * kQ;
+            if (t0 + r < p.L) dt_next = p.dt[(tok0 + t0 + r) * p.sdt + head];
+        }
+        for (int k = 0; k < nch; ++k) {  // every warp runs every iteration (named barriers)
+            const int s = k % kNStage, xb = k & 1;
+            const int t0 = (c_end - 1 - k) * kQ;
+            const float dtv = dt_next;
+            if (k + 1 < nch) {
+                const int t1 = t0 - kQ;
+                dt_next = (head_ok && t1 + r < p.L) ? p.dt[(tok0 + t1 + r) * p.sdt + head] : 0.0f;
+            }
+            float sc = dtv * A2;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float v = __shfl_up_sync(0xffffffffu, sc, o);
+                if (lane >= o) sc += v;
+            }
+            if (lane == 31) wtot[hf * 4 + q] = sc;
+            named_sync_compute();
+            float pre = 0.0f, tot = 0.0f;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float w = wtot[hf * 4 + j];
+                pre += j < q ? w : 0.0f;
+                tot += w;
+            }
+            named_sync_compute();
+            const float c2 = sc + pre;
+            bool ok = __all_sync(0xffffffffu, mbar_wait(&full[s], (k / kNStage) & 1, abort));
+            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&xf[xb], ((k >> 1) & 1) ^ 1, abort));
+            if (ok) {  // X''[r, :] = 2^(D + tot - cs_r) dt_r x[r, :]
+                const float wgt = ex2(D2 + tot - c2) * dtv;
+                const uint8_t* sX = sm + s * kSegStage + kTileQN + hf * kTileQP;
+                uint8_t* dX = sm + kSegOffXP + xb * 2 * kTileQP + hf * kTileQP;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const uint4 xv = *reinterpret_cast<const uint4*>(sX + sw128(r, c));
+                    uint4 o;
+                    o.x = pack_bf16(bf_lo(xv.x) * wgt, bf_hi(xv.x) * wgt);
+                    o.y = pack_bf16(bf_lo(xv.y) * wgt, bf_hi(xv.y) * wgt);
+                    o.z = pack_bf16(bf_lo(xv.z) * wgt, bf_hi(xv.z) * wgt);
+                    o.w = pack_bf16(bf_lo(xv.w) * wgt, bf_hi(xv.w) * wgt);
+                    *reinterpret_cast<uint4*>(dX + sw128(r, c)) = o;
+                }
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&xr[xb]);
+            } else {
+                raise_timeout(abort, p.status);
+            }
+            D2 += tot;
+        }
+        const bool ok = __all_sync(0xffffffffu, mbar_wait(done, 0, abort));
+        if (ok) {
+            tc_fence_after();
+            float* dst = p.states + (((int64_t)b * p.h + head) * p.nseg + seg + 1) * (kP * kN);
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+                uint32_t sv[32];
+                tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + 64 * hf + 32 * h2, sv);
+                tmem_ld_wait();
+                if (head_ok && !*abort) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) dst[(32 * h2 + j) * kN + r] = __uint_as_float(sv[j]);
+                }
+            }
+            if (head_ok && r == 0 && !*abort) p.seg_decay[((int64_t)b * p.h + head) * p.nseg + seg] = D2;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) {
+        __syncwarp();
+        tmem_dealloc(tmem, 128);
+    }
 }
 
 // Segment start states: slot 0 = initial state (or zero); slot k = state after
@@ -611,12 +828,13 @@ static cudaError_t launch_scan_tc_impl(const ScanArgs& a, const ScanGate* gate, 
         cudaError_t e = cudaFuncSetAttribute(ssd_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              kSmemBytes);
         if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(ssd_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+            e = cudaFuncSetAttribute(ssd_seg_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     kSegSmemBytes);
         if (e != cudaSuccess) return e;
         attr_set |= 1ull << dev;
     }
     if (pl.nseg > 1) {
-        ssd_tc_kernel<false><<<dim3((a.h + 1) / 2, pl.nseg - 1, a.batch), 320, kSmemBytes, s>>>(mapX, mapB, mapC, p);
+        ssd_seg_state_kernel<<<dim3((a.h + 1) / 2, pl.nseg - 1, a.batch), 320, kSegSmemBytes, s>>>(mapX, mapB, p);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
         const int64_t n = (int64_t)bh * kP * kN;
