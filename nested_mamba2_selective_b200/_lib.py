@@ -52,6 +52,8 @@ _SIGS = {
     "ssd_scan_workspace": ([_i, _i, _i, _i, _i, _i, _i, _i, ctypes.POINTER(_sz)], _i),
     "ssd_scan": ([_i, _vp, _i64, _vp, _i64, _vp, _vp, _i64, _vp, _i64, _vp, _i, _i, _i, _i, _i, _i, _i, _i,
                   _vp, _i64, _vp, _i64, _vp, _vp, _sz, _vp], _i),
+    "ssd_scan_static": ([_i, _vp, _i64, _vp, _i64, _vp, _vp, _i64, _vp, _i64, _vp, _i, _i, _i, _i, _i, _i, _i, _i,
+                         _vp, _i64, _vp, _i64, _vp, _vp], _i),
     "ssd_step_workspace": ([_pp, _i, _i, ctypes.POINTER(_sz)], _i),
     "ssd_step": ([_pp, _vp, _vp, _vp, _i, _i, _vp, _vp, _sz, _vp], _i),
     "matmamba_stack_workspace": ([_pp, _i, ctypes.POINTER(_i), _i, _i, _i, ctypes.POINTER(_sz)], _i),
@@ -247,6 +249,27 @@ def ssd_scan(x, dt, A, B, C, D=None, h=None, chunk=256, heads_per_group=None, in
                          G * N, _ptr(D), b, L, h, P, N, G, hpg, int(chunk), _ptr(init_state), st_stride, _ptr(y),
                          y.shape[2] * y.shape[3], _ptr(final_state), _ptr(ws), ws.numel(), _stream(stream))
     _check(rc, "ssd_scan")
+    return y
+
+
+def ssd_scan_static(x, dt, A, B, C, D=None, h=None, chunk=256, heads_per_group=None, init_state=None,
+                    final_state=None, y=None, stream=None):
+    """ssd_scan with the library's own fixed scratch array instead of a workspace (no allocation
+    inside the call; calls on one device must not overlap on the GPU)."""
+    b, L, Hx, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    h = Hx if h is None else h
+    hpg = heads_per_group if heads_per_group is not None else -(-h // G)
+    if y is None:
+        y = torch.empty((b, L, h, P), dtype=x.dtype, device=x.device)
+    st_stride = 0
+    for s in (init_state, final_state):
+        if s is not None:
+            st_stride = s.shape[1] * s.shape[2] * s.shape[3]
+    rc = load().ssd_scan_static(_DTYPES[x.dtype], _ptr(x), Hx * P, _ptr(dt), dt.shape[2], _ptr(A), _ptr(B), G * N,
+                                _ptr(C), G * N, _ptr(D), b, L, h, P, N, G, hpg, int(chunk), _ptr(init_state),
+                                st_stride, _ptr(y), y.shape[2] * y.shape[3], _ptr(final_state), _stream(stream))
+    _check(rc, "ssd_scan_static")
     return y
 
 

@@ -1,0 +1,66 @@
+// ssd_scan_static: the selective scan with its scratch space in a fixed
+// device array owned by this library instead of a caller-provided workspace.
+//
+// Some callers cannot allocate device memory for a call: an engine whose
+// allocator reserves all device memory up front and hands out nothing else, a
+// plugin that is given only its input and output buffers, or a latency-
+// critical loop that must not risk the device-wide synchronisation that
+// cudaMalloc / cudaFree can cause.  This entry point needs no workspace: the
+// scan's segment states live in g_scan_scratch below, which every GPU that
+// loads the library holds until the process exits.
+//
+// Rules of use:
+//  - The array holds kScanScratchBytes; a call whose scan would need more is
+//    rejected with MM_ERR_WORKSPACE before anything is launched (the
+//    ssd_scan_workspace query gives the need).
+//  - All calls on a device share the one array and it keeps whatever the last
+//    call left in it.  The scan writes every scratch byte before reading it,
+//    so nothing has to start at zero, but calls that overlap on the GPU (two
+//    streams, or two host threads) race on the array and give wrong results:
+//    serialise them.
+//  - The first call on a device looks up the array's device address
+//    (cudaGetSymbolAddress, with that device current) and caches it; make
+//    that first call before any stream capture.
+#include "mm_internal.cuh"
+
+namespace {
+
+constexpr size_t kScanScratchBytes = size_t(16) << 20;  // 16 MiB per device
+
+// In host code this name is only a stand-in for the device array; kernels are
+// given the address that cudaGetSymbolAddress returns for the current device.
+static __device__ __align__(256) unsigned char g_scan_scratch[kScanScratchBytes];
+
+// Device address of g_scan_scratch on the current device (looked up once per
+// device); nullptr if the runtime cannot resolve it.
+void* scratch_address()
+{
+    static void* addr[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    if (!addr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_scan_scratch) != cudaSuccess) return nullptr;
+        addr[dev] = p;
+    }
+    return addr[dev];
+}
+
+}  // namespace
+
+extern "C" int ssd_scan_static(int dtype, const void* x, int64_t x_stride, const float* dt, int64_t dt_stride,
+                               const float* A, const void* B, int64_t B_stride, const void* C, int64_t C_stride,
+                               const float* D, int batch, int L, int h, int P, int N, int G, int heads_per_group,
+                               int chunk, const float* init_state, int64_t state_stride, void* y, int64_t y_stride,
+                               float* final_state, void* stream)
+{
+    size_t need = 0;
+    int rc = ssd_scan_workspace(dtype, batch, L, h, P, N, G, chunk, &need);
+    if (rc) return rc;
+    if (need > kScanScratchBytes) return MM_ERR_WORKSPACE;
+    void* scratch = scratch_address();
+    if (!scratch) return MM_ERR_CUDA;
+    return ssd_scan(dtype, x, x_stride, dt, dt_stride, A, B, B_stride, C, C_stride, D, batch, L, h, P, N, G,
+                    heads_per_group, chunk, init_state, state_stride, y, y_stride, final_state, scratch,
+                    kScanScratchBytes, stream);
+}

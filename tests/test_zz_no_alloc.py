@@ -1,0 +1,68 @@
+"""ssd_scan_static: the scan entry point that allocates nothing.
+
+It serves callers that cannot allocate device memory around a call (an engine
+whose allocator owns all device memory, a plugin handed only its buffers, a
+latency-critical loop avoiding cudaMalloc's synchronisation).  Its scratch is
+a fixed array inside the library, so its results must match ssd_scan's, call
+after call, with the array reused.  This file is collected last on purpose.
+"""
+import numpy as np
+import pytest
+import torch
+
+from gpu_util import TOL, ensure_built, max_abs_rel, to_device, to_np
+from nested_mamba2_selective_b200 import (MatMambaError, mm_device_status, ssd_scan, ssd_scan_static,
+                                          ssd_scan_workspace, synth)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    ensure_built()
+
+
+def inputs(seed, batch=2, L=1500, h=24):
+    inp = synth.long_memory(synth.ssd_inputs(batch, L, h, 64, 128, 1, "bf16", seed=seed))
+    return dict(x=to_device(inp["x"], "bf16"), B=to_device(inp["B"], "bf16"), C=to_device(inp["C"], "bf16"),
+                dt=torch.from_numpy(inp["dt"]).cuda(), A=torch.from_numpy(inp["A"]).cuda(),
+                D=torch.from_numpy(inp["D"]).cuda())
+
+
+def test_static_scratch_matches_workspace_entry_point_on_consecutive_calls():
+    for seed in (901, 902):  # two calls in a row: the second reuses what the first left in the array
+        g = inputs(seed)
+        fs_ref = torch.zeros((2, 24, 64, 128), device="cuda")
+        fs = torch.zeros_like(fs_ref)
+        ref = ssd_scan(g["x"], g["dt"], g["A"], g["B"], g["C"], g["D"], chunk=256, final_state=fs_ref)
+        out = ssd_scan_static(g["x"], g["dt"], g["A"], g["B"], g["C"], g["D"], chunk=256, final_state=fs)
+        torch.cuda.synchronize()
+        assert mm_device_status() == 0
+        assert max_abs_rel(to_np(out), to_np(ref)) <= TOL["bf16"]
+        assert max_abs_rel(to_np(fs), to_np(fs_ref)) <= TOL["bf16"]
+
+
+CAPACITY = 16 << 20  # bytes of the library's fixed scratch array (include/matmamba.h)
+
+
+def oversized_shape():
+    """A scan whose segment states need more scratch than the fixed array holds."""
+    for L in (65536, 131072, 262144):
+        for h in (64, 128):
+            if ssd_scan_workspace(torch.bfloat16, 1, L, h, 64, 128, 1, 256) > CAPACITY:
+                return L, h
+    raise AssertionError("no oversized shape found")
+
+
+def test_static_scratch_rejects_sizes_beyond_its_capacity():
+    L, h = oversized_shape()
+    x = torch.zeros((1, L, h, 64), dtype=torch.bfloat16, device="cuda")
+    Bm = torch.zeros((1, L, 1, 128), dtype=torch.bfloat16, device="cuda")
+    dt = torch.full((1, L, h), 1e-3, device="cuda")
+    A = torch.full((h,), -1.0, device="cuda")
+    y = torch.full((1, L, h, 64), 3.0, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(MatMambaError) as ei:
+        ssd_scan_static(x, dt, A, Bm, Bm, None, chunk=256, y=y)
+    assert ei.value.status == 5  # MM_ERR_WORKSPACE: nothing launched
+    torch.cuda.synchronize()
+    assert torch.all(y == 3.0)
