@@ -20,7 +20,7 @@ import os
 import statistics
 import subprocess
 import sys
-import tempfile
+import threading
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -41,10 +41,68 @@ def parse():
     ap.add_argument("--only", choices=["block", "scan"], default=None,
                     help="profiling aid: run just the headline block or just the standalone scan, print per-stage "
                          "times and no benchmark line")
+    ap.add_argument("--ncu-summary", metavar="CSV", default=None,
+                    help="print a per-kernel table (launches, device time, share, DRAM bytes per launch) of an "
+                         "ncu --csv log and exit")
     a = ap.parse_args()
     if a.only is None:
         a.warmup = max(a.warmup, 3)
     return a
+
+
+def ncu_summary(path):
+    """Group an `ncu --csv` metrics log by kernel: launches, summed gpu__time_duration, share of the total,
+    and the mean per launch of every other metric (DRAM bytes, for instance)."""
+    import csv
+    scale = {"nsecond": 1e-3, "usecond": 1.0, "msecond": 1e3, "second": 1e6, "ns": 1e-3, "us": 1.0, "ms": 1e3,
+             "s": 1e6}
+    byte_scale = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9, "KB": 1e3, "MB": 1e6, "GB": 1e9}
+    launches, per = {}, {}
+    with open(path) as f:
+        rows = [r for r in csv.reader(line for line in f if line.startswith('"'))]
+    hdr, rows = rows[0], rows[1:]
+    col = {k: hdr.index(k) for k in ("ID", "Kernel Name", "Metric Name", "Metric Unit", "Metric Value")}
+    for r in rows:
+        name = r[col["Kernel Name"]]
+        name = name.replace("(anonymous namespace)::", "").replace("void ", "").split("(")[0]
+        key = (name, r[col["ID"]])
+        unit, val = r[col["Metric Unit"]], float(r[col["Metric Value"]].replace(",", ""))
+        metric = r[col["Metric Name"]]
+        if metric == "gpu__time_duration.sum":
+            val *= scale.get(unit, 1.0)
+        elif unit in byte_scale:
+            val *= byte_scale[unit]
+        launches.setdefault(name, set()).add(key[1])
+        per.setdefault(name, {}).setdefault(metric, []).append(val)
+    total = sum(sum(m.get("gpu__time_duration.sum", [])) for m in per.values())
+    others = sorted({k for m in per.values() for k in m} - {"gpu__time_duration.sum"})
+    print("| kernel | launches | total us | share |" + "".join(" %s per launch |" % o for o in others))
+    print("|---|---|---|---|" + "---|" * len(others))
+    for name, m in sorted(per.items(), key=lambda kv: -sum(kv[1].get("gpu__time_duration.sum", [0]))):
+        t = sum(m.get("gpu__time_duration.sum", [0]))
+        extra = "".join(" %.4g |" % (sum(m[o]) / len(m[o])) if o in m else " |" for o in others)
+        print("| %s | %d | %.1f | %.3f |%s" % (name, len(launches[name]), t, t / total if total else 0, extra))
+
+
+def traffic_for(stage):
+    """DRAM bytes per launch (read + write) of a stage's kernel from profiles/traffic.txt, or None when the
+    kernel's source has changed since the capture (its sha256 prefix no longer matches)."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        for line in f:
+            parts = line.split()
+            if len(parts) >= 4 and not line.startswith("#") and parts[0] == stage:
+                src = os.path.join(ROOT, parts[1])
+                if not os.path.exists(src):
+                    return None
+                with open(src, "rb") as g:
+                    if hashlib.sha256(g.read()).hexdigest()[:16] != parts[2]:
+                        return None
+                return float(parts[3])
+    return None
 
 
 def peaks():
@@ -106,52 +164,100 @@ def whole_job_rate(units_per_rank_step, steps, world, slowest_seconds):
 # ------------------------------------------------------------------------------------ clocks
 
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock and clock-event reasons of this rank's GPU, polled through NVML
+    every few milliseconds while a timed region is open (`active`).  Falls back
+    to one nvidia-smi query per timed region when NVML cannot be loaded."""
 
-    def __init__(self, index):
-        self.index = index
-        self.proc = None
-        self.path = None
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+               ("sw_power_cap", 0x4), ("hw_power_brake_slowdown", 0x80))
+
+    def __init__(self, device):
+        self.device = device
+        self.samples = []  # (sm_mhz, max_mhz, reasons bitmask)
+        self.active = threading.Event()
+        self.stop = threading.Event()
+        self.thread = None
+        self.handle = None
+        self.nvml = None
+
+    def _open(self):
+        import pynvml
+        import torch
+        pynvml.nvmlInit()
+        prop = torch.cuda.get_device_properties(self.device)
+        bus = "%08x:%02x:%02x.0" % (prop.pci_domain_id, prop.pci_bus_id, prop.pci_device_id)
+        self.handle = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        self.nvml = pynvml
+
+    def _sample(self):
+        n = self.nvml
+        sm = n.nvmlDeviceGetClockInfo(self.handle, n.NVML_CLOCK_SM)
+        mx = n.nvmlDeviceGetMaxClockInfo(self.handle, n.NVML_CLOCK_SM)
+        rs = n.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+        self.samples.append((float(sm), float(mx), int(rs)))
+
+    def _loop(self):
+        while not self.stop.is_set():
+            if self.active.wait(0.05):
+                try:
+                    self._sample()
+                except Exception:  # noqa: BLE001 - a failed poll only loses one sample
+                    pass
+                time.sleep(0.002)
 
     def __enter__(self):
         try:
-            fd, self.path = tempfile.mkstemp(suffix=".csv")
-            os.close(fd)
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
-                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
-        except (OSError, FileNotFoundError):
-            self.proc = None
+            self._open()
+            self.thread = threading.Thread(target=self._loop, daemon=True)
+            self.thread.start()
+        except Exception:  # noqa: BLE001 - NVML missing: nvidia-smi fallback in region_end
+            self.nvml = None
         return self
 
     def __exit__(self, *exc):
-        if self.proc is not None:
-            self.proc.terminate()
+        self.stop.set()
+        self.active.set()
+        if self.thread is not None:
+            self.thread.join(timeout=2)
+        if self.nvml is not None:
             try:
-                self.proc.wait(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
+                self.nvml.nvmlShutdown()
+            except Exception:  # noqa: BLE001
+                pass
+
+    def region_begin(self):
+        self.active.set()
+
+    def region_end(self):
+        """Call with work still queued on the GPU (before the closing synchronize)."""
+        if self.nvml is None:
+            self._smi_sample()
+            self.active.clear()
+            return
+        try:
+            self._sample()  # at least one sample per region, taken under load
+        except Exception:  # noqa: BLE001
+            pass
+        self.active.clear()
+
+    def _smi_sample(self):
+        try:
+            import torch
+            idx = torch.cuda.current_device()
+            out = subprocess.run(["nvidia-smi", "-i", str(idx), "--query-gpu=clocks.sm,clocks.max.sm,"
+                                  "clocks_event_reasons.active", "--format=csv,noheader,nounits"],
+                                 capture_output=True, text=True, timeout=10).stdout.strip().split(",")
+            self.samples.append((float(out[0]), float(out[1]), int(out[2].strip(), 16)))
+        except Exception:  # noqa: BLE001
+            pass
 
     def summary(self):
-        if not self.path or not os.path.exists(self.path):
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        rows = []
-        with open(self.path) as f:
-            for line in f:
-                parts = [x.strip() for x in line.split(",")]
-                if len(parts) >= 9:
-                    rows.append(parts)
-        os.unlink(self.path)
-        if not rows:
+        if not self.samples:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows)}
+        reasons = sorted({name for _, _, rs in self.samples for name, bit in self.REASONS if rs & bit})
+        return {"sm_mhz": statistics.median(s[0] for s in self.samples),
+                "sm_max_mhz": max(s[1] for s in self.samples), "reasons": reasons,
+                "samples": len(self.samples), "source": "nvml" if self.nvml is not None else "nvidia-smi"}
 
 
 # ------------------------------------------------------------------------------------ our arm
@@ -188,6 +294,7 @@ def run_ours(args):
 
     stream = torch.cuda.current_stream()
     flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    clk = ClockSampler(dev).__enter__()  # samples only inside timed regions
 
     def timed(fn, steps, warmup, trace=False):
         for _ in range(warmup):
@@ -199,11 +306,13 @@ def run_ours(args):
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
         torch.cuda.synchronize()
         barrier()
+        clk.region_begin()
         for e0, e1 in ev:
             flush_buf.zero_()
             e0.record(stream)
             fn()
             e1.record(stream)
+        clk.region_end()
         torch.cuda.synchronize()
         barrier()
         ms = [e0.elapsed_time(e1) for e0, e1 in ev]
@@ -214,7 +323,9 @@ def run_ours(args):
         return ms, tr
 
     if args.only:
-        return run_only(args, mm, synth, torch, dev, timed)
+        rc = run_only(args, mm, synth, torch, dev, timed)
+        clk.__exit__(None, None, None)
+        return rc
 
     # ---------------- block workload (headline)
     B = BLOCK
@@ -230,16 +341,14 @@ def run_ours(args):
 
     per_width = {}
     head = None
-    with ClockSampler(local) as clk:
-        for m in B["widths"]:
-            fn = lambda m=m: mm.matmamba_block_fwd(wt, u, m, B["chunk"], out=out, workspace=ws)  # noqa: E731
-            ms, tr = timed(fn, args.steps, args.warmup, trace=True)
-            total = slowest(sum(ms))
-            per_width[str(m)] = {"tokens_per_s": whole_job_rate(T, args.steps, world, total / 1e3),
-                                 "ms_per_step": total / args.steps}
-            if m == B["widths"][0]:
-                head = (ms, total, tr)
-    clocks = clk.summary()
+    for m in B["widths"]:
+        fn = lambda m=m: mm.matmamba_block_fwd(wt, u, m, B["chunk"], out=out, workspace=ws)  # noqa: E731
+        ms, tr = timed(fn, args.steps, args.warmup, trace=True)
+        total = slowest(sum(ms))
+        per_width[str(m)] = {"tokens_per_s": whole_job_rate(T, args.steps, world, total / 1e3),
+                             "ms_per_step": total / args.steps}
+        if m == B["widths"][0]:
+            head = (ms, total, tr)
     ms, total, (stages, kernels) = head
     m0 = B["widths"][0]
     value = whole_job_rate(T, args.steps, world, total / 1e3)
@@ -255,7 +364,7 @@ def run_ours(args):
     else:
         achieved = amount / (avg_ms / 1e3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s"}
-    roof.update({"frac": roof["achieved"] / roof["peak"], "traffic": None, "kernel": dom,
+    roof.update({"frac": roof["achieved"] / roof["peak"], "traffic": traffic_for(dom), "kernel": dom,
                  "peak_source": pk_src, "avg_launch_ms": avg_ms})
     stage_table = {}
     for k, (n, kern, tot) in stages.items():
@@ -286,7 +395,8 @@ def run_ours(args):
         scan[str(h)] = {"tokens_per_s": world * Ts / (avg / 1e3), "us_per_call": avg * 1e3,
                         "roofline": {"bound": "hbm", "achieved": nbytes / (avg / 1e3) / 1e9, "peak": pk["hbm_gbs"],
                                      "unit": "GB/s", "frac": nbytes / (avg / 1e3) / 1e9 / pk["hbm_gbs"],
-                                     "algorithmic_bytes": nbytes, "traffic": None, "peak_source": pk_src}}
+                                     "algorithmic_bytes": nbytes, "traffic": traffic_for("ssd_scan_h%d" % h),
+                                     "peak_source": pk_src}}
 
     # ---------------- end to end through the host-buffer entry point
     u_host = torch.from_numpy(u_np).bfloat16().pin_memory()
@@ -305,6 +415,8 @@ def run_ours(args):
     extended = {}
     if args.extended:
         extended = run_extended(args, mm, synth, torch, dev, timed, slowest, world)
+    clk.__exit__(None, None, None)
+    clocks = clk.summary()
 
     if rank == 0:
         line = {
@@ -455,7 +567,9 @@ def run_reference(args):
 
 if __name__ == "__main__":
     a = parse()
-    if a.impl == "reference":
+    if a.ncu_summary:
+        ncu_summary(a.ncu_summary)
+    elif a.impl == "reference":
         run_reference(a)
     else:
         run_ours(a)
