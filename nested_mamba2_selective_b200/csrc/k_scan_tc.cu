@@ -13,20 +13,12 @@
 //   1. seg_state  : each segment's end state from a zero start (tcgen05)
 //   2. state_pass : segment start states by a short sequential combine
 //   3. chunk_scan : every segment from its true start state, carrying the
-//                   state across blocks in registers (tcgen05)
+//                   state across blocks in TMEM (tcgen05)
 // Only segment boundary states touch HBM.
 //
 // A CTA takes two heads of one (batch, segment) so that the B and C blocks and
-// G = C B^T are loaded and computed once per pair (320 threads): warp 0 TMA
-// producer, warp 1 TMEM owner and tcgen05.mma issuer, warps 2-9 compute.
-// Compute thread (quarter q, lane l, half hf) owns TMEM lane r = 32q + l and
-// head hf of the pair: token r for its Y row, state row n = r for S.  For the
-// masked matrix M of its own head it covers all 128 columns, 32 at a time;
-// each block of 32 G columns is overwritten (after both heads read it) by
-// head 0's then head 1's 16 packed bf16 columns, the A operands of Y.
-// Per block: G, then Y_off = C [H_0 | H_1] once the bf16 state copy H is in
-// shared memory (its space then takes X'), then Y_j = M_j X_j and
-// S = B^T [X'_0 | X'_1]; G of the next block overlaps this block's epilogue.
+// G = C B^T are loaded and computed once per pair; the thread roles of the
+// chunk scan are described above ssd_chunk_kernel.
 #include <cuda.h>
 
 #include <cmath>
@@ -49,9 +41,6 @@ constexpr int kOffC = 0, kOffB = kTileQN, kOffX = 2 * kTileQN;
 constexpr int kStage = 2 * kTileQN + 2 * kTileQP; // C | B | x of two heads
 constexpr int kNStage = 2;
 constexpr int kOffHX = kNStage * kStage;          // H (then X') of two heads
-constexpr int kOffSmall = kOffHX + 2 * kTileQP;
-constexpr int kSmemBytes = kOffSmall + 64 + 2 * 192 * 4 + 128;
-static_assert(kSmemBytes <= 232448, "chunk scan exceeds the 227 KB of shared memory a CTA can have");
 
 // TMEM columns: G = C B^T, overwritten in place by the masked M_0 | M_1 (A operands);
 // Y_0 | Y_1; Y_off of both heads; S of both heads.
@@ -96,24 +85,47 @@ __device__ __forceinline__ float ex2(float x)
 __device__ __forceinline__ float bf_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
 
-template <bool FULL>
-__global__ void __launch_bounds__(320, 1)
-    ssd_tc_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CUtensorMap mapB,
-                  const __grid_constant__ CUtensorMap mapC, const ScanTcParams p)
+// Chunk scan.  A CTA takes two heads of one (batch, segment); 448 threads:
+//   warp 0      TMA producer (one lane)
+//   warp 1      TMEM owner and tcgen05.mma issuer (one lane)
+//   warps 2-5   M builders: thread (quarter q = warp % 4, lane) owns TMEM lane and token row
+//               r = 32 q + lane and builds the masked decay matrix M of both heads from one read of
+//               G = C B^T, in place over G's columns
+//   warps 6-13  state warps: thread (q, lane, head hf) owns row r of head hf: decay scan, the
+//               state read-back (bf16 copy for Y_off, decayed fp32 state for the S MMA), X', and
+//               the output epilogue
+// The M builders work on block k while the state warps finish block k-1's epilogue, so the
+// two largest per-block thread phases overlap.  Per block k the tensor core runs
+//   G = C B^T (after Y of block k-1 has consumed M), Y_off = C [H_0 | H_1] (after the
+//   read-back), then Y_j = M_j X_j and S += B^T [X'_0 | X'_1] (after M and X').
+// M factors the decay through the anchor of each 32-token column block cb (a_cb = cs at row
+// 32 cb): 2^(cs_t - cs_s) dt_s = 2^(cs_t - a_cb) * (2^(a_cb - cs_s) dt_s) for s in block cb,
+// s <= t.  The first factor is <= 1; the second, g_s, is a per-token table bounded by the decay
+// across one 32-token block.  A block whose decay exceeds 2^-kDropMax would overflow g and
+// takes direct exponentials instead (g_s = dt_s, M = G 2^min(cs_t - cs_s, 0) g_s).
+constexpr int kChunkThreads = 448;
+constexpr float kDropMax = 100.0f;  // log2 units
+// small tables after the H/X' buffers (floats): state-warp scan totals [2 parity][2 heads][4],
+// M-builder scan totals [2][2][4], g [2 heads][128], cs [2][128], anchors [2][4], fallback flags [2][4]
+constexpr int kTabWtotS = 0, kTabWtotM = 16, kTabG = 32, kTabC = 288, kTabAnch = 544, kTabFlag = 552, kTabFloats = 560;
+constexpr int kOffTab = kOffHX + 2 * kTileQP;
+constexpr int kOffBar = kOffTab + kTabFloats * 4;
+constexpr int kChunkSmem = kOffBar + 10 * 8 + 16;
+static_assert(kChunkSmem <= 232448, "chunk scan exceeds the 227 KB of shared memory a CTA can have");
+
+__global__ void __launch_bounds__(kChunkThreads, 1)
+    ssd_chunk_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CUtensorMap mapB,
+                     const __grid_constant__ CUtensorMap mapC, const ScanTcParams p)
 {
     extern __shared__ __align__(1024) uint8_t sm[];
-    float* wtot = reinterpret_cast<float*>(sm + kOffSmall);  // [2 heads][4] per-warp scan totals
-    float* anch = wtot + 8;                                   // [2 heads][4] running log2 decay at rows 32 i
-    // [2 heads][192]: 2^(cs(32 i) - cs(s)) dt(s) for s < 32 i, the column factors of row block i,
-    // packed as i = 1 at [0, 32), i = 2 at [32, 96), i = 3 at [96, 192)
-    float* ecol = anch + 8;
-    uint64_t* full = reinterpret_cast<uint64_t*>(ecol + 2 * 192);
+    float* tab = reinterpret_cast<float*>(sm + kOffTab);
+    uint64_t* full = reinterpret_cast<uint64_t*>(sm + kOffBar);
     uint64_t* empty = full + kNStage;
     uint64_t* g_done = empty + kNStage;
-    uint64_t* yo_done = g_done + 1;
-    uint64_t* h_ready = yo_done + 1;
-    uint64_t* m_ready = h_ready + 1;
-    uint64_t* ys_full = m_ready + 1;
+    uint64_t* h_ready = g_done + 1;
+    uint64_t* yo_done = h_ready + 1;
+    uint64_t* mx_ready = yo_done + 1;
+    uint64_t* ys_full = mx_ready + 1;
     uint64_t* done = ys_full + 1;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
     volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -128,24 +140,22 @@ __global__ void __launch_bounds__(320, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        if (smem_u32(sm) & 1023u) {  // tiles need 1024-byte alignment; never observed, but never fault on it
-            raise_timeout(abort, p.status);
-        }
         for (int s = 0; s < kNStage; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 8);
         }
         mbar_init(g_done, 1);
-        mbar_init(yo_done, 1);
         mbar_init(h_ready, 8);
-        mbar_init(m_ready, 8);
+        mbar_init(yo_done, 1);
+        mbar_init(mx_ready, 12);
         mbar_init(ys_full, 1);
         mbar_init(done, 1);
-        *abort = (smem_u32(sm) & 1023u) ? 1 : 0;
+        *abort = (smem_u32(sm) & 1023u) ? 1 : 0;  // tiles need 1024-byte alignment; never fault on it
+        if (*abort) raise_timeout(abort, p.status);
         fence_mbar_init();
         prefetch_tmap(&mapX);
         prefetch_tmap(&mapB);
-        if (FULL) prefetch_tmap(&mapC);
+        prefetch_tmap(&mapC);
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, kTCols);
@@ -159,7 +169,6 @@ __global__ void __launch_bounds__(320, 1)
 
     if (warp == 0) {
         if (lane == 0 && !*abort) {  // ------------------------------------------------ TMA producer
-            constexpr uint32_t bytes = FULL ? kStage : (kTileQN + 2 * kTileQP);
             int k = 0;
             for (; k < nch; ++k) {
                 const int s = k % kNStage;
@@ -169,11 +178,9 @@ __global__ void __launch_bounds__(320, 1)
                 }
                 const int row = (int)(tok0 + (int64_t)(c_begin + k) * kQ);
                 uint8_t* base = sm + s * kStage;
-                mbar_arrive_expect_tx(&full[s], bytes);
-                if (FULL) {
-                    tma_load_2d(base + kOffC, &mapC, &full[s], grp * kN, row);
-                    tma_load_2d(base + kOffC + kTileQN / 2, &mapC, &full[s], grp * kN + 64, row);
-                }
+                mbar_arrive_expect_tx(&full[s], kStage);
+                tma_load_2d(base + kOffC, &mapC, &full[s], grp * kN, row);
+                tma_load_2d(base + kOffC + kTileQN / 2, &mapC, &full[s], grp * kN + 64, row);
                 tma_load_2d(base + kOffB, &mapB, &full[s], grp * kN, row);
                 tma_load_2d(base + kOffB + kTileQN / 2, &mapB, &full[s], grp * kN + 64, row);
                 tma_load_2d(base + kOffX, &mapX, &full[s], head0 * kP, row);
@@ -191,78 +198,186 @@ __global__ void __launch_bounds__(320, 1)
             const uint32_t aHX = smem_u32(sHX);
             for (int k = 0; k < nch; ++k) {
                 const int s = k % kNStage;
-                if (!mbar_wait(&full[s], (k / kNStage) & 1, abort)) {
-                    raise_timeout(abort, p.status);
-                    break;
-                }
-                // the previous block's MMAs (which read M from the G columns) are complete
-                if (k > 0 && !mbar_wait(ys_full, (k - 1) & 1, abort)) {
+                // stage k is loaded, and block k-1's MMAs (which read M from the G columns) are done
+                if (!mbar_wait(&full[s], (k / kNStage) & 1, abort) ||
+                    (k > 0 && !mbar_wait(ys_full, (k - 1) & 1, abort))) {
                     raise_timeout(abort, p.status);
                     break;
                 }
                 tc_fence_after();
                 const uint32_t aS = smem_u32(sm + s * kStage);
                 const uint32_t aC = aS + kOffC, aB = aS + kOffB, aX = aS + kOffX;
-                if (FULL) {
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {  // G = C . B^T
-                        const uint32_t off = (kk & 3) * 32 + (kk >> 2) * (kTileQN / 2);
-                        mma_ss(tmem + kTG, desc_sw128(aC + off, 16, 1024), desc_sw128(aB + off, 16, 1024), id_g,
-                               kk > 0);
-                    }
-                    mma_commit(g_done);
-                    if (!mbar_wait(h_ready, k & 1, abort)) {
-                        raise_timeout(abort, p.status);
-                        break;
-                    }
-                    tc_fence_after();
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {  // Y_off = C . [H_0 | H_1] over the state dim
-                        const uint32_t off = (kk & 3) * 32 + (kk >> 2) * (kTileQN / 2);
-                        mma_ss(tmem + kTYO, desc_sw128(aC + off, 16, 1024),
-                               desc_sw128(aHX + kk * 2048, kTileQP, 1024), id_o, kk > 0);
-                    }
-                    mma_commit(yo_done);
+                for (int kk = 0; kk < 8; ++kk) {  // G = C . B^T
+                    const uint32_t off = (kk & 3) * 32 + (kk >> 2) * (kTileQN / 2);
+                    mma_ss(tmem + kTG, desc_sw128(aC + off, 16, 1024), desc_sw128(aB + off, 16, 1024), id_g, kk > 0);
                 }
-                if (!mbar_wait(m_ready, k & 1, abort)) {
+                mma_commit(g_done);
+                if (!mbar_wait(h_ready, k & 1, abort)) {
                     raise_timeout(abort, p.status);
                     break;
                 }
                 tc_fence_after();
-                if (FULL) {
 #pragma unroll
-                    for (int j = 0; j < 2; ++j)
-#pragma unroll
-                        for (int kk = 0; kk < 8; ++kk)  // Y_j = M_j . X_j over the block's tokens
-                            mma_ts(tmem + kTY + 64 * j, tmem + kTG + 32 * (kk >> 1) + 16 * j + 8 * (kk & 1),
-                                   desc_sw128(aX + j * kTileQP + kk * 2048, kTileQP, 1024), id_y, kk > 0);
+                for (int kk = 0; kk < 8; ++kk) {  // Y_off = C . [H_0 | H_1] over the state dim
+                    const uint32_t off = (kk & 3) * 32 + (kk >> 2) * (kTileQN / 2);
+                    mma_ss(tmem + kTYO, desc_sw128(aC + off, 16, 1024), desc_sw128(aHX + kk * 2048, kTileQP, 1024),
+                           id_o, kk > 0);
                 }
+                mma_commit(yo_done);
+                if (!mbar_wait(mx_ready, k & 1, abort)) {
+                    raise_timeout(abort, p.status);
+                    break;
+                }
+                tc_fence_after();
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk)  // H += B^T . [X'_0 | X'_1] over the block's tokens
+                for (int j = 0; j < 2; ++j)
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)  // Y_j = M_j . X_j over the block's tokens
+                        mma_ts(tmem + kTY + 64 * j, tmem + kTG + 32 * (kk >> 1) + 16 * j + 8 * (kk & 1),
+                               desc_sw128(aX + j * kTileQP + kk * 2048, kTileQP, 1024), id_y, kk > 0);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)  // S += B^T . [X'_0 | X'_1] over the block's tokens
                     mma_ss(tmem + kTS, desc_sw128(aB + kk * 2048, kTileQN / 2, 1024),
-                           desc_sw128(aHX + kk * 2048, kTileQP, 1024), id_s, FULL ? 1u : (kk > 0));
+                           desc_sw128(aHX + kk * 2048, kTileQP, 1024), id_s, 1u);
                 mma_commit(ys_full);
             }
             mma_commit(done);
             mbar_wait(done, 0, nullptr);
         }
-    } else {  // ------------------------------------------------------------ compute warps
-        const int cw = warp - 2, q = warp & 3, hf = cw >> 2;
-        const int r = q * 32 + lane;
-        const uint32_t lane_base = (uint32_t)(q * 32) << 16;
-        // this thread's head for the scan, X', output and state: head0 + hf
+    } else if (warp < 6) {  // ------------------------------------------------------ M builders
+        const int q = warp & 3, r = 32 * q + lane;
+        const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+        float A2[2], dn[2] = {0.0f, 0.0f};
+#pragma unroll
+        for (int j = 0; j < 2; ++j) A2[j] = head0 + j < p.h ? p.A[head0 + j] * kLog2e : 0.0f;
+        if (nch > 0 && c_begin * kQ + r < p.L) {
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+                if (head0 + j < p.h) dn[j] = p.dt[(tok0 + c_begin * kQ + r) * p.sdt + head0 + j];
+        }
+        for (int k = 0; k < nch; ++k) {  // every warp runs every iteration (named barrier 1)
+            const float dv[2] = {dn[0], dn[1]};
+            const int t1 = (c_begin + k + 1) * kQ + r;
+            dn[0] = dn[1] = 0.0f;
+            if (k + 1 < nch && t1 < p.L) {  // prefetch the next block's dt
+#pragma unroll
+                for (int j = 0; j < 2; ++j)
+                    if (head0 + j < p.h) dn[j] = p.dt[(tok0 + t1) * p.sdt + head0 + j];
+            }
+            float* wt = tab + kTabWtotM + 8 * (k & 1);
+            float c2[2];
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {  // inclusive scan of dt A (log2 units) within the warp
+                float sc = dv[j] * A2[j];
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const float v = __shfl_up_sync(0xffffffffu, sc, o);
+                    if (lane >= o) sc += v;
+                }
+                if (lane == 31) wt[4 * j + q] = sc;
+                c2[j] = sc;
+            }
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                float pre = 0.0f;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) pre += i < q ? wt[4 * j + i] : 0.0f;
+                c2[j] += pre;
+                // this row block's anchor (cs at its first row) and the decay across it
+                const float a = __shfl_sync(0xffffffffu, c2[j], 0);
+                const float last = __shfl_sync(0xffffffffu, c2[j], 31);
+                const bool fb = a - last > kDropMax;
+                tab[kTabG + 128 * j + r] = fb ? dv[j] : ex2(a - c2[j]) * dv[j];
+                tab[kTabC + 128 * j + r] = c2[j];
+                if (lane == 0) {
+                    tab[kTabAnch + 4 * j + q] = a;
+                    tab[kTabFlag + 4 * j + q] = fb ? 1.0f : 0.0f;
+                }
+            }
+            asm volatile("bar.sync 1, 128;" ::: "memory");  // tables of block k complete
+
+            const bool ok = __all_sync(0xffffffffu, mbar_wait(g_done, k & 1, abort));
+            if (ok) tc_fence_after();
+#pragma unroll
+            for (int cb = 0; cb < 4; ++cb) {  // column block s in [32 cb, 32 cb + 32)
+                if (!ok) break;
+                if (cb > q) {  // above the diagonal: zeros for both heads
+                    uint32_t z[32];
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) z[e] = 0u;
+                    tmem_st32(tmem + lane_base + kTG + 32 * cb, z);
+                    continue;
+                }
+                uint32_t gv[32];
+                tmem_ld32(tmem + lane_base + kTG + 32 * cb, gv);
+                tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    uint32_t pk[16];
+                    const float* gt = tab + kTabG + 128 * j + 32 * cb;
+                    if (tab[kTabFlag + 4 * j + cb] == 0.0f) {
+                        const float er = ex2(c2[j] - tab[kTabAnch + 4 * j + cb]);
+#pragma unroll
+                        for (int e = 0; e < 32; e += 4) {
+                            const float4 g4 = *reinterpret_cast<const float4*>(gt + e);
+                            float m0 = __uint_as_float(gv[e]) * er * g4.x;
+                            float m1 = __uint_as_float(gv[e + 1]) * er * g4.y;
+                            float m2 = __uint_as_float(gv[e + 2]) * er * g4.z;
+                            float m3 = __uint_as_float(gv[e + 3]) * er * g4.w;
+                            if (cb == q) {  // causal mask inside the diagonal block: s <= t
+                                m0 = e <= lane ? m0 : 0.0f;
+                                m1 = e + 1 <= lane ? m1 : 0.0f;
+                                m2 = e + 2 <= lane ? m2 : 0.0f;
+                                m3 = e + 3 <= lane ? m3 : 0.0f;
+                            }
+                            pk[e >> 1] = pack_bf16(m0, m1);
+                            pk[(e >> 1) + 1] = pack_bf16(m2, m3);
+                        }
+                    } else {  // steep block: direct exponentials, g holds dt
+                        const float* ct = tab + kTabC + 128 * j + 32 * cb;
+#pragma unroll
+                        for (int e = 0; e < 32; e += 2) {
+                            float m0 = __uint_as_float(gv[e]) * ex2(fminf(c2[j] - ct[e], 0.0f)) * gt[e];
+                            float m1 = __uint_as_float(gv[e + 1]) * ex2(fminf(c2[j] - ct[e + 1], 0.0f)) * gt[e + 1];
+                            if (cb == q) {
+                                m0 = e <= lane ? m0 : 0.0f;
+                                m1 = e + 1 <= lane ? m1 : 0.0f;
+                            }
+                            pk[e >> 1] = pack_bf16(m0, m1);
+                        }
+                    }
+                    // head j's 16 packed columns of this block (the A operand of Y_j)
+                    tmem_st16(tmem + lane_base + kTG + 32 * cb + 16 * j, pk);
+                }
+            }
+            if (ok) {
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(mx_ready);
+            } else {
+                raise_timeout(abort, p.status);
+            }
+        }
+    } else {  // ------------------------------------------------------------------- state warps
+        const int cw = warp - 6, q = warp & 3, hf = cw >> 2;
+        const int r = 32 * q + lane;
+        const uint32_t lane_base = (uint32_t)(32 * q) << 16;
         const int head = head0 + hf;
         const bool head_ok = head < p.h;
         const float A2 = head_ok ? p.A[head] * kLog2e : 0.0f;
-        const float Dh = (FULL && p.D && head_ok) ? p.D[head] : 0.0f;
+        const float Dh = (p.D && head_ok) ? p.D[head] : 0.0f;
         const int64_t bh = (int64_t)b * p.h + head;
         const int PN = kP * kN;
         uint8_t* myHX = sHX + hf * kTileQP;
+        const uint32_t bar_id = 2 + hf;
 
         // The fp32 state of this head lives in TMEM columns kTS + 64 hf (row n = lane r): each
-        // block, the compute warps read H_k for its bf16 copy (Y_off's operand), write back
-        // 2^tot H_k, and the S MMA accumulates B^T X' on top, leaving H_{k+1}.
-        if (FULL) {
+        // block, it is read for its bf16 copy (Y_off's operand), 2^tot H_k is written back, and
+        // the S MMA accumulates B^T X' on top, leaving H_{k+1}.
+        {
             const float* src = nullptr;
             if (head_ok) {
                 if (p.nseg > 1) src = p.states + (bh * p.nseg + seg) * PN;
@@ -277,162 +392,49 @@ __global__ void __launch_bounds__(320, 1)
             }
             tmem_st_wait();
         }
-        float seg_log2 = 0.0f;
         float dt_next = 0.0f;
-        {
-            const int t0 = c_begin * kQ;
-            if (head_ok && nch > 0 && t0 + r < p.L) dt_next = p.dt[(tok0 + t0 + r) * p.sdt + head];
-        }
+        if (head_ok && nch > 0 && c_begin * kQ + r < p.L) dt_next = p.dt[(tok0 + c_begin * kQ + r) * p.sdt + head];
+        float c2_prev = 0.0f;
+        bool ok = !*abort;
+        ok = __all_sync(0xffffffffu, ok);
 
-        // Every compute warp runs every iteration (the block's two named barriers must see all
-        // eight warps); after a failed wait a warp skips the rest of the block's work.
-        for (int k = 0; k < nch; ++k) {
-            const int s = k % kNStage;
-            const int t0 = (c_begin + k) * kQ;
-            const bool valid = head_ok && t0 + r < p.L;
-            const float dtv = dt_next;
-            if (k + 1 < nch) {  // prefetch the next block's dt
-                const int t1 = t0 + kQ;
-                dt_next = (head_ok && t1 + r < p.L) ? p.dt[(tok0 + t1 + r) * p.sdt + head] : 0.0f;
-            }
-            // inclusive scan of dt*A (log2 units) over the block, for head hf
-            float sc = dtv * A2;
+        // Iteration k: decay scan of block k, epilogue of block k-1, read-back and X' of block k.
+        // Every warp runs every iteration (named barrier 2 + hf); a failed wait skips work only.
+        for (int k = 0; k <= nch; ++k) {
+            float dtv = 0.0f, c2 = 0.0f, tot = 0.0f;
+            if (k < nch) {
+                dtv = dt_next;
+                const int t1 = (c_begin + k + 1) * kQ + r;
+                dt_next = (head_ok && k + 1 < nch && t1 < p.L) ? p.dt[(tok0 + t1) * p.sdt + head] : 0.0f;
+                float sc = dtv * A2;
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const float v = __shfl_up_sync(0xffffffffu, sc, o);
-                if (lane >= o) sc += v;
-            }
-            if (lane == 31) wtot[hf * 4 + q] = sc;
-            named_sync_compute();
-            float pre = 0.0f, tot = 0.0f;
+                for (int o = 1; o < 32; o <<= 1) {
+                    const float v = __shfl_up_sync(0xffffffffu, sc, o);
+                    if (lane >= o) sc += v;
+                }
+                float* wt = tab + kTabWtotS + 8 * (k & 1) + 4 * hf;
+                if (lane == 31) wt[q] = sc;
+                asm volatile("bar.sync %0, 128;" ::"r"(bar_id) : "memory");
+                float pre = 0.0f;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const float w = wtot[hf * 4 + j];
-                pre += j < q ? w : 0.0f;
-                tot += w;
-            }
-            const float c2 = sc + pre;
-            if (lane == 0) anch[hf * 4 + q] = c2;  // running decay at row 32 q
-            named_sync_compute();
-            seg_log2 += tot;
-            if (FULL) {  // column factors of the anchored row blocks, this thread's head and column r
-#pragma unroll
-                for (int i = 1; i < 4; ++i)
-                    if (r < 32 * i) ecol[hf * 192 + 16 * i * (i - 1) + r] = ex2(anch[hf * 4 + i] - c2) * dtv;
-                named_sync_compute();  // the table is read by the other row blocks' warps
+                for (int i = 0; i < 4; ++i) {
+                    const float w = wt[i];
+                    pre += i < q ? w : 0.0f;
+                    tot += w;
+                }
+                c2 = sc + pre;
             }
 
-            if (FULL) {  // H_k: bf16 copy for Y_off, then 2^tot H_k back into TMEM for the S MMA to add onto
-                const float dec = ex2(tot);
-#pragma unroll
-                for (int h2 = 0; h2 < 2; ++h2) {
-                    uint32_t v[32];
-                    tmem_ld32(tmem + lane_base + kTS + 64 * hf + 32 * h2, v);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        uint4 w;
-                        w.x = pack_bf16(__uint_as_float(v[8 * c + 0]), __uint_as_float(v[8 * c + 1]));
-                        w.y = pack_bf16(__uint_as_float(v[8 * c + 2]), __uint_as_float(v[8 * c + 3]));
-                        w.z = pack_bf16(__uint_as_float(v[8 * c + 4]), __uint_as_float(v[8 * c + 5]));
-                        w.w = pack_bf16(__uint_as_float(v[8 * c + 6]), __uint_as_float(v[8 * c + 7]));
-                        *reinterpret_cast<uint4*>(myHX + sw128(r, 4 * h2 + c)) = w;
-                    }
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(dec * __uint_as_float(v[j]));
-                    tmem_st32(tmem + lane_base + kTS + 64 * hf + 32 * h2, v);
-                }
-                tmem_st_wait();
-                fence_async_smem();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(h_ready);
-            }
-
-            bool ok = __all_sync(0xffffffffu, mbar_wait(&full[s], (k / kNStage) & 1, abort));
-            const uint8_t* sX = sm + s * kStage + kOffX + hf * kTileQP;
-
-            if (FULL) {  // the quarter barriers below run whatever ok is, so no partner warp is stranded
-                if (ok) ok = __all_sync(0xffffffffu, mbar_wait(g_done, k & 1, abort));
-                if (ok) tc_fence_after();
-                {
-                    // M_j[t=r, s] = G[r, s] 2^(cs_j[r] - cs_j[s]) dt_j[s] for s <= r, else 0, built by the
-                    // threads of head j = hf over all 128 columns, 32 at a time.  Both heads' threads read
-                    // a row's 32 G columns before either writes them (a barrier per block); those columns
-                    // then take M_0 then M_1 for these s (16 packed columns each).
-                    // Column blocks below the row block q factor the decay through the anchor 32 q:
-                    // 2^(cs_r - cs_s) = 2^(cs_r - cs_32q) 2^(cs_32q - cs_s), both factors <= 1; the diagonal
-                    // block takes direct exponentials with its tokens' values shuffled in from this warp.
-                    const float er = ex2(c2 - __shfl_sync(0xffffffffu, c2, 0));
-#pragma unroll
-                    for (int cb = 0; cb < 4; ++cb) {  // column block s in [32 cb, 32 cb + 32)
-                        uint32_t gv[32];
-                        if (ok && cb <= q) {
-                            tmem_ld32(tmem + lane_base + kTG + 32 * cb, gv);
-                            tmem_ld_wait();
-                        }
-                        asm volatile("bar.sync %0, 64;" ::"r"(2 + q) : "memory");  // both heads have read them
-                        if (!ok) continue;
-                        uint32_t pk[16];
-                        if (cb < q) {
-                            const float* ec = ecol + hf * 192 + 16 * q * (q - 1) + 32 * cb;
-#pragma unroll
-                            for (int e = 0; e < 32; e += 4) {
-                                const float4 f = *reinterpret_cast<const float4*>(ec + e);
-                                pk[e >> 1] = pack_bf16(__uint_as_float(gv[e]) * er * f.x, __uint_as_float(gv[e + 1]) * er * f.y);
-                                pk[(e >> 1) + 1] =
-                                    pack_bf16(__uint_as_float(gv[e + 2]) * er * f.z, __uint_as_float(gv[e + 3]) * er * f.w);
-                            }
-                        } else if (cb == q) {
-#pragma unroll
-                            for (int e = 0; e < 32; e += 2) {
-                                const float ca = __shfl_sync(0xffffffffu, c2, e);
-                                const float cbv = __shfl_sync(0xffffffffu, c2, e + 1);
-                                const float da = __shfl_sync(0xffffffffu, dtv, e);
-                                const float db = __shfl_sync(0xffffffffu, dtv, e + 1);
-                                const float ma = __uint_as_float(gv[e]) * ex2(fminf(c2 - ca, 0.0f)) * da;
-                                const float mb = __uint_as_float(gv[e + 1]) * ex2(fminf(c2 - cbv, 0.0f)) * db;
-                                pk[e >> 1] = pack_bf16(e <= lane ? ma : 0.0f, e + 1 <= lane ? mb : 0.0f);
-                            }
-                        } else {
-#pragma unroll
-                            for (int e = 0; e < 16; ++e) pk[e] = 0u;
-                        }
-                        // the 32 columns just read take head 0's then head 1's 16 packed columns
-                        tmem_st16(tmem + lane_base + kTG + 32 * cb + 16 * hf, pk);
-                    }
-                    if (ok) tmem_st_wait();
-                    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(yo_done, k & 1, abort));  // H read: X' may go there
-                }
-            } else if (!FULL && ok && k > 0) {
-                ok = __all_sync(0xffffffffu, mbar_wait(ys_full, (k - 1) & 1, abort));  // previous X' consumed
-            }
-            if (ok) {  // X'_j[s=r, :] = exp(cs_end - cs_r) dt_r x_j[r, :]
-                const float wgt = ex2(tot - c2) * dtv;
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const uint4 xv = *reinterpret_cast<const uint4*>(sX + sw128(r, c));
-                    uint4 o;
-                    o.x = pack_bf16(bf_lo(xv.x) * wgt, bf_hi(xv.x) * wgt);
-                    o.y = pack_bf16(bf_lo(xv.y) * wgt, bf_hi(xv.y) * wgt);
-                    o.z = pack_bf16(bf_lo(xv.z) * wgt, bf_hi(xv.z) * wgt);
-                    o.w = pack_bf16(bf_lo(xv.w) * wgt, bf_hi(xv.w) * wgt);
-                    *reinterpret_cast<uint4*>(myHX + sw128(r, c)) = o;
-                }
-                fence_async_smem();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(m_ready);
-                    if (!FULL) mbar_arrive(&empty[s]);  // x is read
-                }
-                ok = __all_sync(0xffffffffu, mbar_wait(ys_full, k & 1, abort));
-            }
-            if (ok) {
-                tc_fence_after();
-                if (FULL) {  // TMEM loads are warp-collective: every lane loads, only valid rows store
-                    const float ey = ex2(c2);
-                    const int64_t tok = tok0 + t0 + r;
+            if (k > 0) {  // ---- epilogue of block k-1 (TMEM loads are warp-collective)
+                if (ok) ok = __all_sync(0xffffffffu, mbar_wait(ys_full, (k - 1) & 1, abort));
+                if (ok) {
+                    tc_fence_after();
+                    const int sp = (k - 1) % kNStage;
+                    const int tp0 = (c_begin + k - 1) * kQ;
+                    const bool valid = head_ok && tp0 + r < p.L;
+                    const uint8_t* sX = sm + sp * kStage + kOffX + hf * kTileQP;
+                    const float ey = ex2(c2_prev);
+                    const int64_t tok = tok0 + tp0 + r;
                     const int col = head * kP;
                     __nv_bfloat16* yo = static_cast<__nv_bfloat16*>(p.y) + tok * p.sy + col;
                     float ssq[2] = {0.0f, 0.0f};
@@ -479,18 +481,65 @@ __global__ void __launch_bounds__(320, 1)
                         p.row_parts[tok * 2 * p.h + 2 * head] = ssq[0];
                         p.row_parts[tok * 2 * p.h + 2 * head + 1] = ssq[1];
                     }
-                }
-                tc_fence_before();
-                if (FULL) {
+                    tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&empty[s]);  // x is read
+                    if (lane == 0) mbar_arrive(&empty[sp]);  // x of block k-1 is read
                 }
             }
+            if (k == nch) break;
+
+            const int s = k % kNStage;
+            if (ok) {  // ---- read-back: H_k as bf16 for Y_off, 2^tot H_k back into TMEM
+                const float dec = ex2(tot);
+#pragma unroll
+                for (int h4 = 0; h4 < 4; ++h4) {  // 16 state columns at a time
+                    uint32_t v[16];
+                    tmem_ld16(tmem + lane_base + kTS + 64 * hf + 16 * h4, v);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) {
+                        uint4 w;
+                        w.x = pack_bf16(__uint_as_float(v[8 * c + 0]), __uint_as_float(v[8 * c + 1]));
+                        w.y = pack_bf16(__uint_as_float(v[8 * c + 2]), __uint_as_float(v[8 * c + 3]));
+                        w.z = pack_bf16(__uint_as_float(v[8 * c + 4]), __uint_as_float(v[8 * c + 5]));
+                        w.w = pack_bf16(__uint_as_float(v[8 * c + 6]), __uint_as_float(v[8 * c + 7]));
+                        *reinterpret_cast<uint4*>(myHX + sw128(r, 2 * h4 + c)) = w;
+                    }
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) v[j] = __float_as_uint(dec * __uint_as_float(v[j]));
+                    tmem_st16(tmem + lane_base + kTS + 64 * hf + 16 * h4, v);
+                }
+                tmem_st_wait();
+                fence_async_smem();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(h_ready);
+            }
+            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&full[s], (k / kNStage) & 1, abort));
+            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(yo_done, k & 1, abort));  // H read: X' may go there
+            if (ok) {  // ---- X'_j[s=r, :] = 2^(tot - cs_r) dt_r x_j[r, :]
+                const uint8_t* sX = sm + s * kStage + kOffX + hf * kTileQP;
+                const float wgt = ex2(tot - c2) * dtv;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const uint4 xv = *reinterpret_cast<const uint4*>(sX + sw128(r, c));
+                    uint4 o;
+                    o.x = pack_bf16(bf_lo(xv.x) * wgt, bf_hi(xv.x) * wgt);
+                    o.y = pack_bf16(bf_lo(xv.y) * wgt, bf_hi(xv.y) * wgt);
+                    o.z = pack_bf16(bf_lo(xv.z) * wgt, bf_hi(xv.z) * wgt);
+                    o.w = pack_bf16(bf_lo(xv.w) * wgt, bf_hi(xv.w) * wgt);
+                    *reinterpret_cast<uint4*>(myHX + sw128(r, c)) = o;
+                }
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(mx_ready);
+            }
             if (!ok) raise_timeout(abort, p.status);
+            c2_prev = c2;
         }
 
-        if (FULL && seg == p.nseg - 1 && p.final_state) {  // state after the last block
-            const bool ok = __all_sync(0xffffffffu, !*abort);
+        if (seg == p.nseg - 1 && p.final_state) {  // state after the last block (ys_full waited above)
+            ok = __all_sync(0xffffffffu, ok && !*abort);
             if (ok) {
                 float* dst = p.final_state + (int64_t)b * p.state_stride + (int64_t)head * PN;
 #pragma unroll
@@ -825,8 +874,8 @@ static cudaError_t launch_scan_tc_impl(const ScanArgs& a, const ScanGate* gate, 
     cudaGetDevice(&dev);
     static unsigned long long attr_set = 0;
     if (dev < 64 && !(attr_set >> dev & 1ull)) {
-        cudaError_t e = cudaFuncSetAttribute(ssd_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             kSmemBytes);
+        cudaError_t e = cudaFuncSetAttribute(ssd_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             kChunkSmem);
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(ssd_seg_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      kSegSmemBytes);
@@ -843,7 +892,7 @@ static cudaError_t launch_scan_tc_impl(const ScanArgs& a, const ScanGate* gate, 
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
-    ssd_tc_kernel<true><<<dim3((a.h + 1) / 2, pl.nseg, a.batch), 320, kSmemBytes, s>>>(mapX, mapB, mapC, p);
+    ssd_chunk_kernel<<<dim3((a.h + 1) / 2, pl.nseg, a.batch), kChunkThreads, kChunkSmem, s>>>(mapX, mapB, mapC, p);
     return cudaGetLastError();
 }
 

@@ -134,3 +134,28 @@ def test_scan_chunk_parameter_does_not_change_the_result(orc, chunk):
     torch.cuda.synchronize()
     ref, _ = oracle_scan(orc, inp, 3)
     assert max_abs_rel(to_np(y), ref) <= TOL["bf16"]
+
+
+def test_scan_steep_decay_blocks(orc):
+    """Decay far stronger than 2^-100 across a 32-token block (dt A down to -96 per token) on some
+    heads and token ranges, next to ordinary ones, and a stretch near that threshold: both ways of
+    forming the decay matrix inside one block of 128 tokens, and the carried state across them."""
+    inp = synth.ssd_inputs(2, 600, 6, 64, 128, 1, "bf16", seed=208)
+    A = inp["A"].copy()
+    A[:3] = -16.0
+    A[3:] = -1.0
+    dt = inp["dt"].copy()
+    dt[:, 130:170, 0:3] = 6.0            # steep: about 138 (log2 units) per token on heads 0-2
+    dt[:, 300:364, 3] = 3.2 / np.log2(np.e)  # about 3.2 per token on head 3: ~100 across a block
+    dt[1, 40:41, 5] = 80.0               # one very steep token on head 5 of batch row 1
+    inp = dict(inp, A=A, dt=dt.astype(np.float32))
+    g = upload(inp, "bf16")
+    fs = torch.zeros((2, 6, 64, 128), device="cuda")
+    y = ssd_scan(g["x"], g["dt"], g["A"], g["B"], g["C"], g["D"], chunk=256, final_state=fs)
+    torch.cuda.synchronize()
+    ref, fs_ref = oracle_scan(orc, inp, 6)
+    assert torch.isfinite(y.float()).all()
+    yn, fsn = to_np(y), to_np(fs)
+    for i in range(6):  # per head: the steep token's large output must not hide errors elsewhere
+        assert max_abs_rel(yn[:, :, i], ref[:, :, i]) <= TOL["bf16"], i
+        assert max_abs_rel(fsn[:, i], fs_ref[:, i]) <= TOL["bf16"], i
