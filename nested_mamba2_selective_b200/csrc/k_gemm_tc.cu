@@ -7,10 +7,11 @@
 // ("MatMamba: A Matryoshka State Space Model", nested sub-block paragraph:
 // W_x becomes W_x[0:d_i] by slicing along d_inner).
 //
-// CTA layout (192 threads): warp 0 issues TMA loads, warp 1 owns TMEM and
-// issues tcgen05.mma from one lane, warps 2-5 drain the accumulator (one TMEM
-// lane = one output row per thread) and store.  Two TMEM accumulators let the
-// drain of tile i overlap the MMAs of tile i+1.
+// CTA layout (320 threads): warp 0 issues TMA loads, warp 1 owns TMEM and
+// issues tcgen05.mma from one lane, warps 2-9 drain the accumulator in two
+// groups of four that take alternate 32-column chunks (one TMEM lane = one
+// output row per thread) and store.  Two TMEM accumulators let the drain of
+// tile i overlap the MMAs of tile i+1.
 #include <cuda.h>
 
 #include "mm_internal.cuh"
@@ -200,21 +201,46 @@ __global__ void __launch_bounds__(320, 1)
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++tc) {
             const TileInfo<BN> t = tile_info<BN>(p, tile);
             const int buf = tc & 1;
-            // a failed wait skips this tile's work but keeps the group's named barriers in step
-            const bool ok = __all_sync(0xffffffffu, mbar_wait(&tfull[buf], (tc >> 1) & 1, abort));
-            if (!ok) raise_timeout(abort, p.status);
-            tc_fence_after();
             const TcSeg& sg = p.seg[t.seg];
             const int64_t m = (int64_t)t.mt * p.rows - p.shift + r;  // token of this row
             const bool row_ok = r >= p.shift && m < p.M;
+            // the row scale does not depend on the accumulator: its loads go out before the wait
             float scale = 1.0f;
             if (ex.row_parts && row_ok) {
                 const float* rp = ex.row_parts + m * ex.nparts;
                 float ss = 0.0f;
-                for (int j = 0; j < ex.nparts; ++j) ss += rp[j];
+                if ((ex.nparts & 3) == 0) {  // rows of partials are 16-byte aligned
+                    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                    for (int j = 0; j < ex.nparts; j += 4) {
+                        const float4 v4 = *reinterpret_cast<const float4*>(rp + j);
+                        acc.x += v4.x; acc.y += v4.y; acc.z += v4.z; acc.w += v4.w;
+                    }
+                    ss = (acc.x + acc.y) + (acc.z + acc.w);
+                } else {
+                    for (int j = 0; j < ex.nparts; ++j) ss += rp[j];
+                }
                 scale = rsqrtf(ss * ex.rs_inv_n + ex.rs_eps);
             }
-            const int tpos = (sg.kind == kEpiConv && row_ok) ? (int)(m % ex.L) : 0;
+            // a failed wait skips this tile's work but keeps the group's named barriers in step
+            const bool ok = __all_sync(0xffffffffu, mbar_wait(&tfull[buf], (tc >> 1) & 1, abort));
+            if (!ok) raise_timeout(abort, p.status);
+            tc_fence_after();
+            // Conv walk of this thread (rows [16 rb, 16 rb + 16) of the tile; output rows start at
+            // w_fr, past the tile's halo): the token of its first output row, that token's position
+            // in its sequence, and whether the walk can take the branch-free path: every output row
+            // is a valid token in the same sequence as its three history rows, and none is one of
+            // the last K-1 of its sequence (conv state output).
+            const int wrb = 2 * q + (lane >> 4), wr0 = 16 * wrb;
+            const int w_fr = max(wr0, p.shift), w_n = wr0 + 16 - w_fr;
+            int64_t w_m0 = 0;
+            int w_tp0 = 0;
+            bool w_fast = false;
+            if (CONV && sg.kind == kEpiConv) {
+                w_m0 = (int64_t)t.mt * p.rows - p.shift + w_fr;
+                w_tp0 = (int)(((w_m0 % ex.L) + ex.L) % ex.L);
+                w_fast = sg.vec_ok && p.shift == 3 && w_m0 >= 0 && w_m0 + w_n - 1 < p.M && w_tp0 >= 3 &&
+                         w_tp0 + w_n - 1 + 3 < ex.L;
+            }
             for (int c0 = 32 * eg; c0 < t.nvalid; c0 += 64, ++nchunk_done) {
                 float v[32];
                 if (ok) {
@@ -222,7 +248,11 @@ __global__ void __launch_bounds__(320, 1)
                     tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + buf * BN + c0, raw);
                     tmem_ld_wait();
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(raw[i]) * scale;
+                    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(raw[i]);
+                    if (ex.row_parts) {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) v[i] *= scale;
+                    }
                 } else {
 #pragma unroll
                     for (int i = 0; i < 32; ++i) v[i] = 0.0f;
@@ -243,9 +273,34 @@ __global__ void __launch_bounds__(320, 1)
                                 make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
                     }
                     asm volatile("bar.sync %0, 128;" ::"r"(2 + eg) : "memory");
-                    const int cp = lane & 15, rb = 2 * q + (lane >> 4);
+                    const int cp = lane & 15, rb = wrb;
                     const int lc = 2 * cp;  // local column pair
-                    if (ok && lc < ncols) {
+                    if (ok && lc + 1 < ncols && w_fast) {
+                        // all 16 rows are outputs of one sequence, history in the rows above
+                        const int crow = sg.conv_row0 + col + lc;
+                        const __nv_bfloat16* cw = static_cast<const __nv_bfloat16*>(ex.conv_w);
+                        const __nv_bfloat16* cbias = static_cast<const __nv_bfloat16*>(ex.conv_b);
+                        const uint2 wa = *reinterpret_cast<const uint2*>(cw + (int64_t)crow * 4);
+                        const uint2 wb = *reinterpret_cast<const uint2*>(cw + (int64_t)(crow + 1) * 4);
+                        const float a0 = bf_lo_u(wa.x), a1 = bf_hi_u(wa.x), a2 = bf_lo_u(wa.y), a3 = bf_hi_u(wa.y);
+                        const float b0 = bf_lo_u(wb.x), b1 = bf_hi_u(wb.x), b2 = bf_lo_u(wb.y), b3 = bf_hi_u(wb.y);
+                        const float biasa = __bfloat162float(cbias[crow]), biasb = __bfloat162float(cbias[crow + 1]);
+                        // rows w_fr - 3 .. w_fr + 15 of the staged chunk (all inside the tile; the top
+                        // walk reads three rows past its 13 outputs and ignores them)
+                        const float* sr = st + (w_fr - 3) * kStageLd + lc;
+                        float2 xw[19];
+#pragma unroll
+                        for (int i = 0; i < 19; ++i) xw[i] = *reinterpret_cast<const float2*>(sr + i * kStageLd);
+                        uint32_t* o = reinterpret_cast<uint32_t*>(static_cast<__nv_bfloat16*>(sg.out) + w_m0 * sg.ldo +
+                                                                  col + lc);
+                        const int64_t step = sg.ldo / 2;  // output row pitch in bf16 pairs
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            float oa = fmaf(a3, xw[i + 3].x, fmaf(a2, xw[i + 2].x, fmaf(a1, xw[i + 1].x, fmaf(a0, xw[i].x, biasa))));
+                            float ob = fmaf(b3, xw[i + 3].y, fmaf(b2, xw[i + 2].y, fmaf(b1, xw[i + 1].y, fmaf(b0, xw[i].y, biasb))));
+                            if (i < w_n) o[i * step] = pack_bf16(silu_fast(oa), silu_fast(ob));
+                        }
+                    } else if (ok && lc < ncols) {
                         const int crow = sg.conv_row0 + col + lc;
                         const bool two = lc + 1 < ncols;
                         const __nv_bfloat16* cw = static_cast<const __nv_bfloat16*>(ex.conv_w);
