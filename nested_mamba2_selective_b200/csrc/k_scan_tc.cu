@@ -85,25 +85,27 @@ __device__ __forceinline__ float ex2(float x)
 __device__ __forceinline__ float bf_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
 
-// Chunk scan.  A CTA takes two heads of one (batch, segment); 448 threads:
-//   warp 0      TMA producer (one lane)
-//   warp 1      TMEM owner and tcgen05.mma issuer (one lane)
-//   warps 2-5   M builders: thread (quarter q = warp % 4, lane) owns TMEM lane and token row
-//               r = 32 q + lane and builds the masked decay matrix M of both heads from one read of
-//               G = C B^T, in place over G's columns
-//   warps 6-13  state warps: thread (q, lane, head hf) owns row r of head hf: decay scan, the
-//               state read-back (bf16 copy for Y_off, decayed fp32 state for the S MMA), X', and
-//               the output epilogue
-// The M builders work on block k while the state warps finish block k-1's epilogue, so the
-// two largest per-block thread phases overlap.  Per block k the tensor core runs
-//   G = C B^T (after Y of block k-1 has consumed M), Y_off = C [H_0 | H_1] (after the
-//   read-back), then Y_j = M_j X_j and S += B^T [X'_0 | X'_1] (after M and X').
+// Chunk scan.  A CTA takes two heads of one (batch, segment); 512 threads in roles:
+//   warps 0-7   M builders, except warp 4: thread (quarter q = warp % 4, lane) owns TMEM lane and
+//               token row r = 32 q + lane and builds, for both heads, the masked decay matrix M
+//               over some of its row's 32-token column blocks, in place over G = C B^T.  The two
+//               warps of a quarter split the causal blocks (at most two blocks of both heads per
+//               warp) and one of them writes the zero blocks above the diagonal.
+//   warp 4      control: one lane issues the TMA loads and the tcgen05.mma; the warp owns TMEM
+//   warps 8-15  state warps: thread (q, lane, head hf) owns row r of head hf: decay scan, state
+//               read-back (bf16 copy for Y_off, decayed fp32 state for the S MMA), X', epilogue
+// The M builders work on block k while the state warps finish block k-1's epilogue.  Per block
+// k the tensor core runs G = C B^T (once Y of block k-1 has consumed M), Y_off = C [H_0 | H_1]
+// (after the read-back), then Y_j = M_j X_j and S += B^T [X'_0 | X'_1] (after M and X').
 // M factors the decay through the anchor of each 32-token column block cb (a_cb = cs at row
 // 32 cb): 2^(cs_t - cs_s) dt_s = 2^(cs_t - a_cb) * (2^(a_cb - cs_s) dt_s) for s in block cb,
 // s <= t.  The first factor is <= 1; the second, g_s, is a per-token table bounded by the decay
 // across one 32-token block.  A block whose decay exceeds 2^-kDropMax would overflow g and
 // takes direct exponentials instead (g_s = dt_s, M = G 2^min(cs_t - cs_s, 0) g_s).
-constexpr int kChunkThreads = 448;
+// Element-wise products use the paired fp32 instructions (mul/fma .f32x2, rounded per lane
+// exactly like their scalar forms).
+constexpr int kChunkThreads = 512;
+constexpr int kCtlWarp = 4;
 constexpr float kDropMax = 100.0f;  // log2 units
 // small tables after the H/X' buffers (floats): state-warp scan totals [2 parity][2 heads][4],
 // M-builder scan totals [2][2][4], g [2 heads][128], cs [2][128], anchors [2][4], fallback flags [2][4]
@@ -112,6 +114,11 @@ constexpr int kOffTab = kOffHX + 2 * kTileQP;
 constexpr int kOffBar = kOffTab + kTabFloats * 4;
 constexpr int kChunkSmem = kOffBar + 10 * 8 + 16;
 static_assert(kChunkSmem <= 232448, "chunk scan exceeds the 227 KB of shared memory a CTA can have");
+
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ float2 bf2(uint32_t v) { return make_float2(bf_lo(v), bf_hi(v)); }
+__device__ __forceinline__ uint32_t pack2(float2 v) { return pack_bf16(v.x, v.y); }
 
 __global__ void __launch_bounds__(kChunkThreads, 1)
     ssd_chunk_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CUtensorMap mapB,
@@ -147,7 +154,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
         mbar_init(g_done, 1);
         mbar_init(h_ready, 8);
         mbar_init(yo_done, 1);
-        mbar_init(mx_ready, 12);
+        mbar_init(mx_ready, 15);  // 7 M-builder warps and 8 state warps
         mbar_init(ys_full, 1);
         mbar_init(done, 1);
         *abort = (smem_u32(sm) & 1023u) ? 1 : 0;  // tiles need 1024-byte alignment; never fault on it
@@ -157,7 +164,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
         prefetch_tmap(&mapB);
         prefetch_tmap(&mapC);
     }
-    if (warp == 1) {
+    if (warp == kCtlWarp) {
         tmem_alloc(tmem_slot, kTCols);
         tmem_relinquish();
     }
@@ -167,16 +174,16 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
     const uint32_t tmem = *tmem_slot;
     uint8_t* sHX = sm + kOffHX;  // [2 heads] x 16 KB: bf16 state copy H, then X' of the current block
 
-    if (warp == 0) {
-        if (lane == 0 && !*abort) {  // ------------------------------------------------ TMA producer
-            int k = 0;
-            for (; k < nch; ++k) {
-                const int s = k % kNStage;
-                if (!mbar_wait(&empty[s], ((k / kNStage) & 1) ^ 1, abort)) {
-                    raise_timeout(abort, p.status);
-                    break;
-                }
-                const int row = (int)(tok0 + (int64_t)(c_begin + k) * kQ);
+    if (warp == kCtlWarp) {
+        if (lane == 0 && !*abort) {  // ------------------------------------ TMA loads and tcgen05.mma
+            const uint32_t id_g = idesc_bf16(128, 128, 0, 0);   // C (K-major) x B (K-major)
+            const uint32_t id_o = idesc_bf16(128, 128, 0, 1);   // C (K-major) x [H_0 | H_1] (MN-major)
+            const uint32_t id_y = idesc_bf16(128, 64, 0, 1);    // M_j (TMEM) x X_j (MN-major)
+            const uint32_t id_s = idesc_bf16(128, 128, 1, 1);   // B^T (MN-major) x [X'_0 | X'_1] (MN-major)
+            const uint32_t aHX = smem_u32(sHX);
+            auto load = [&](int c) {  // block c of the segment into stage c % 2
+                const int s = c % kNStage;
+                const int row = (int)(tok0 + (int64_t)(c_begin + c) * kQ);
                 uint8_t* base = sm + s * kStage;
                 mbar_arrive_expect_tx(&full[s], kStage);
                 tma_load_2d(base + kOffC, &mapC, &full[s], grp * kN, row);
@@ -186,16 +193,9 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
                 tma_load_2d(base + kOffX, &mapX, &full[s], head0 * kP, row);
                 // a pair's second head past the last head reloads the last head (its dt is zero)
                 tma_load_2d(base + kOffX + kTileQP, &mapX, &full[s], min(head0 + 1, p.h - 1) * kP, row);
-            }
-            for (int j = max(0, k - kNStage); j < k; ++j) mbar_wait(&full[j % kNStage], (j / kNStage) & 1, abort);
-        }
-    } else if (warp == 1) {
-        if (lane == 0 && !*abort) {  // ------------------------------------------------ MMA issuer
-            const uint32_t id_g = idesc_bf16(128, 128, 0, 0);   // C (K-major) x B (K-major)
-            const uint32_t id_o = idesc_bf16(128, 128, 0, 1);   // C (K-major) x [H_0 | H_1] (MN-major)
-            const uint32_t id_y = idesc_bf16(128, 64, 0, 1);    // M_j (TMEM) x X_j (MN-major)
-            const uint32_t id_s = idesc_bf16(128, 128, 1, 1);   // B^T (MN-major) x [X'_0 | X'_1] (MN-major)
-            const uint32_t aHX = smem_u32(sHX);
+            };
+            int loaded = 0;  // blocks whose loads were issued
+            for (; loaded < nch && loaded < kNStage; ++loaded) load(loaded);
             for (int k = 0; k < nch; ++k) {
                 const int s = k % kNStage;
                 // stage k is loaded, and block k-1's MMAs (which read M from the G columns) are done
@@ -213,6 +213,14 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
                     mma_ss(tmem + kTG, desc_sw128(aC + off, 16, 1024), desc_sw128(aB + off, 16, 1024), id_g, kk > 0);
                 }
                 mma_commit(g_done);
+                // block k+1 goes into the stage block k-1 used, free once its epilogue has read x
+                if (loaded == k + 1 && loaded < nch) {
+                    if (!mbar_wait(&empty[loaded % kNStage], ((loaded / kNStage) & 1) ^ 1, abort)) {
+                        raise_timeout(abort, p.status);
+                        break;
+                    }
+                    load(loaded++);
+                }
                 if (!mbar_wait(h_ready, k & 1, abort)) {
                     raise_timeout(abort, p.status);
                     break;
@@ -231,23 +239,30 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
                 }
                 tc_fence_after();
 #pragma unroll
+                for (int kk = 0; kk < 8; ++kk)  // S += B^T . [X'_0 | X'_1] over the block's tokens
+                    mma_ss(tmem + kTS, desc_sw128(aB + kk * 2048, kTileQN / 2, 1024),
+                           desc_sw128(aHX + kk * 2048, kTileQP, 1024), id_s, 1u);
+#pragma unroll
                 for (int j = 0; j < 2; ++j)
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)  // Y_j = M_j . X_j over the block's tokens
                         mma_ts(tmem + kTY + 64 * j, tmem + kTG + 32 * (kk >> 1) + 16 * j + 8 * (kk & 1),
                                desc_sw128(aX + j * kTileQP + kk * 2048, kTileQP, 1024), id_y, kk > 0);
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)  // S += B^T . [X'_0 | X'_1] over the block's tokens
-                    mma_ss(tmem + kTS, desc_sw128(aB + kk * 2048, kTileQN / 2, 1024),
-                           desc_sw128(aHX + kk * 2048, kTileQP, 1024), id_s, 1u);
                 mma_commit(ys_full);
             }
+            // every issued load lands before the CTA exits (bounded; only the last two can be pending)
+            for (int j = max(0, loaded - kNStage); j < loaded; ++j) mbar_wait(&full[j % kNStage], (j / kNStage) & 1, abort);
             mma_commit(done);
             mbar_wait(done, 0, nullptr);
         }
-    } else if (warp < 6) {  // ------------------------------------------------------ M builders
-        const int q = warp & 3, r = 32 * q + lane;
+    } else if (warp < 8) {  // ------------------------------------------------------ M builders
+        const int q = warp & 3, hb = warp >> 2, r = 32 * q + lane;
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+        // causal column blocks of this warp, and the zero blocks it writes
+        // quarter 0: {0} (its second warp is the control warp); 1: {0} {1}; 2: {0,1} {2}; 3: {0,1} {2,3}
+        const int cb_lo = hb == 0 ? 0 : (q >= 2 ? 2 : 1);
+        const int cb_hi = hb == 0 ? (q >= 2 ? 1 : 0) : q;  // inclusive
+        const bool zero_writer = (q <= 1) ? hb == 0 : hb == 1;
         float A2[2], dn[2] = {0.0f, 0.0f};
 #pragma unroll
         for (int j = 0; j < 2; ++j) A2[j] = head0 + j < p.h ? p.A[head0 + j] * kLog2e : 0.0f;
@@ -275,84 +290,87 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
                     const float v = __shfl_up_sync(0xffffffffu, sc, o);
                     if (lane >= o) sc += v;
                 }
-                if (lane == 31) wt[4 * j + q] = sc;
+                if (lane == 31 && hb == 0) wt[4 * j + q] = sc;
                 c2[j] = sc;
             }
-            asm volatile("bar.sync 1, 128;" ::: "memory");
+            asm volatile("bar.sync 1, 224;" ::: "memory");
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
                 float pre = 0.0f;
 #pragma unroll
                 for (int i = 0; i < 4; ++i) pre += i < q ? wt[4 * j + i] : 0.0f;
                 c2[j] += pre;
-                // this row block's anchor (cs at its first row) and the decay across it
-                const float a = __shfl_sync(0xffffffffu, c2[j], 0);
-                const float last = __shfl_sync(0xffffffffu, c2[j], 31);
-                const bool fb = a - last > kDropMax;
-                tab[kTabG + 128 * j + r] = fb ? dv[j] : ex2(a - c2[j]) * dv[j];
-                tab[kTabC + 128 * j + r] = c2[j];
-                if (lane == 0) {
-                    tab[kTabAnch + 4 * j + q] = a;
-                    tab[kTabFlag + 4 * j + q] = fb ? 1.0f : 0.0f;
+                if (hb == 0) {  // this row block's anchor (cs at its first row) and the decay across it
+                    const float a = __shfl_sync(0xffffffffu, c2[j], 0);
+                    const float last = __shfl_sync(0xffffffffu, c2[j], 31);
+                    const bool fb = a - last > kDropMax;
+                    tab[kTabG + 128 * j + r] = fb ? dv[j] : ex2(a - c2[j]) * dv[j];
+                    tab[kTabC + 128 * j + r] = c2[j];
+                    if (lane == 0) {
+                        tab[kTabAnch + 4 * j + q] = a;
+                        tab[kTabFlag + 4 * j + q] = fb ? 1.0f : 0.0f;
+                    }
                 }
             }
-            asm volatile("bar.sync 1, 128;" ::: "memory");  // tables of block k complete
+            asm volatile("bar.sync 1, 224;" ::: "memory");  // tables of block k complete
 
             const bool ok = __all_sync(0xffffffffu, mbar_wait(g_done, k & 1, abort));
-            if (ok) tc_fence_after();
-#pragma unroll
-            for (int cb = 0; cb < 4; ++cb) {  // column block s in [32 cb, 32 cb + 32)
-                if (!ok) break;
-                if (cb > q) {  // above the diagonal: zeros for both heads
+            if (ok) {
+                tc_fence_after();
+                if (zero_writer) {  // above the diagonal: zeros for both heads
                     uint32_t z[32];
 #pragma unroll
                     for (int e = 0; e < 32; ++e) z[e] = 0u;
-                    tmem_st32(tmem + lane_base + kTG + 32 * cb, z);
-                    continue;
+#pragma unroll
+                    for (int cb = 1; cb < 4; ++cb)
+                        if (cb > q) tmem_st32(tmem + lane_base + kTG + 32 * cb, z);
                 }
-                uint32_t gv[32];
-                tmem_ld32(tmem + lane_base + kTG + 32 * cb, gv);
-                tmem_ld_wait();
+#pragma unroll 1
+                for (int cb = cb_lo; cb <= cb_hi; ++cb) {  // column block s in [32 cb, 32 cb + 32)
+                    uint32_t gv[32];
+                    tmem_ld32(tmem + lane_base + kTG + 32 * cb, gv);
+                    tmem_ld_wait();
+                    const bool diag = cb == q;
 #pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    uint32_t pk[16];
-                    const float* gt = tab + kTabG + 128 * j + 32 * cb;
-                    if (tab[kTabFlag + 4 * j + cb] == 0.0f) {
-                        const float er = ex2(c2[j] - tab[kTabAnch + 4 * j + cb]);
+                    for (int j = 0; j < 2; ++j) {
+                        uint32_t pk[16];
+                        const float* gt = tab + kTabG + 128 * j + 32 * cb;
+                        if (tab[kTabFlag + 4 * j + cb] == 0.0f) {
+                            const float er = ex2(c2[j] - tab[kTabAnch + 4 * j + cb]);
+                            const float2 er2 = make_float2(er, er);
 #pragma unroll
-                        for (int e = 0; e < 32; e += 4) {
-                            const float4 g4 = *reinterpret_cast<const float4*>(gt + e);
-                            float m0 = __uint_as_float(gv[e]) * er * g4.x;
-                            float m1 = __uint_as_float(gv[e + 1]) * er * g4.y;
-                            float m2 = __uint_as_float(gv[e + 2]) * er * g4.z;
-                            float m3 = __uint_as_float(gv[e + 3]) * er * g4.w;
-                            if (cb == q) {  // causal mask inside the diagonal block: s <= t
-                                m0 = e <= lane ? m0 : 0.0f;
-                                m1 = e + 1 <= lane ? m1 : 0.0f;
-                                m2 = e + 2 <= lane ? m2 : 0.0f;
-                                m3 = e + 3 <= lane ? m3 : 0.0f;
+                            for (int e = 0; e < 32; e += 4) {
+                                const float4 g4 = *reinterpret_cast<const float4*>(gt + e);
+                                float2 m01 = mul2(mul2(make_float2(__uint_as_float(gv[e]), __uint_as_float(gv[e + 1])), er2),
+                                                  make_float2(g4.x, g4.y));
+                                float2 m23 = mul2(mul2(make_float2(__uint_as_float(gv[e + 2]), __uint_as_float(gv[e + 3])), er2),
+                                                  make_float2(g4.z, g4.w));
+                                if (diag) {  // causal mask inside the diagonal block: s <= t
+                                    m01.x = e <= lane ? m01.x : 0.0f;
+                                    m01.y = e + 1 <= lane ? m01.y : 0.0f;
+                                    m23.x = e + 2 <= lane ? m23.x : 0.0f;
+                                    m23.y = e + 3 <= lane ? m23.y : 0.0f;
+                                }
+                                pk[e >> 1] = pack2(m01);
+                                pk[(e >> 1) + 1] = pack2(m23);
                             }
-                            pk[e >> 1] = pack_bf16(m0, m1);
-                            pk[(e >> 1) + 1] = pack_bf16(m2, m3);
-                        }
-                    } else {  // steep block: direct exponentials, g holds dt
-                        const float* ct = tab + kTabC + 128 * j + 32 * cb;
+                        } else {  // steep block: direct exponentials, g holds dt
+                            const float* ct = tab + kTabC + 128 * j + 32 * cb;
 #pragma unroll
-                        for (int e = 0; e < 32; e += 2) {
-                            float m0 = __uint_as_float(gv[e]) * ex2(fminf(c2[j] - ct[e], 0.0f)) * gt[e];
-                            float m1 = __uint_as_float(gv[e + 1]) * ex2(fminf(c2[j] - ct[e + 1], 0.0f)) * gt[e + 1];
-                            if (cb == q) {
-                                m0 = e <= lane ? m0 : 0.0f;
-                                m1 = e + 1 <= lane ? m1 : 0.0f;
+                            for (int e = 0; e < 32; e += 2) {
+                                float m0 = __uint_as_float(gv[e]) * ex2(fminf(c2[j] - ct[e], 0.0f)) * gt[e];
+                                float m1 = __uint_as_float(gv[e + 1]) * ex2(fminf(c2[j] - ct[e + 1], 0.0f)) * gt[e + 1];
+                                if (diag) {
+                                    m0 = e <= lane ? m0 : 0.0f;
+                                    m1 = e + 1 <= lane ? m1 : 0.0f;
+                                }
+                                pk[e >> 1] = pack_bf16(m0, m1);
                             }
-                            pk[e >> 1] = pack_bf16(m0, m1);
                         }
+                        // head j's 16 packed columns of this block (the A operand of Y_j)
+                        tmem_st16(tmem + lane_base + kTG + 32 * cb + 16 * j, pk);
                     }
-                    // head j's 16 packed columns of this block (the A operand of Y_j)
-                    tmem_st16(tmem + lane_base + kTG + 32 * cb + 16 * j, pk);
                 }
-            }
-            if (ok) {
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
@@ -362,7 +380,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
             }
         }
     } else {  // ------------------------------------------------------------------- state warps
-        const int cw = warp - 6, q = warp & 3, hf = cw >> 2;
+        const int cw = warp - 8, q = warp & 3, hf = cw >> 2;
         const int r = 32 * q + lane;
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
         const int head = head0 + hf;
@@ -395,8 +413,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
         float dt_next = 0.0f;
         if (head_ok && nch > 0 && c_begin * kQ + r < p.L) dt_next = p.dt[(tok0 + c_begin * kQ + r) * p.sdt + head];
         float c2_prev = 0.0f;
-        bool ok = !*abort;
-        ok = __all_sync(0xffffffffu, ok);
+        bool ok = __all_sync(0xffffffffu, !*abort);
 
         // Iteration k: decay scan of block k, epilogue of block k-1, read-back and X' of block k.
         // Every warp runs every iteration (named barrier 2 + hf); a failed wait skips work only.
@@ -434,6 +451,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
                     const bool valid = head_ok && tp0 + r < p.L;
                     const uint8_t* sX = sm + sp * kStage + kOffX + hf * kTileQP;
                     const float ey = ex2(c2_prev);
+                    const float2 ey2 = make_float2(ey, ey), dh2 = make_float2(Dh, Dh);
                     const int64_t tok = tok0 + tp0 + r;
                     const int col = head * kP;
                     __nv_bfloat16* yo = static_cast<__nv_bfloat16*>(p.y) + tok * p.sy + col;
@@ -461,18 +479,18 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
 #pragma unroll
                             for (int e = 0; e < 4; ++e) {
                                 const int j = 8 * c + 2 * e;
-                                float a0 = __uint_as_float(yv[j]) + ey * __uint_as_float(ov[j]) + Dh * bf_lo(xw[e]);
-                                float a1 =
-                                    __uint_as_float(yv[j + 1]) + ey * __uint_as_float(ov[j + 1]) + Dh * bf_hi(xw[e]);
+                                // y = Y + 2^cs Y_off + D x, two columns at a time
+                                float2 a = fma2(ey2, make_float2(__uint_as_float(ov[j]), __uint_as_float(ov[j + 1])),
+                                                make_float2(__uint_as_float(yv[j]), __uint_as_float(yv[j + 1])));
+                                a = fma2(dh2, bf2(xw[e]), a);
                                 if (p.z) {
                                     const float z0 = bf_lo(zw[e]), z1 = bf_hi(zw[e]);
-                                    a0 *= __fdividef(z0, 1.0f + __expf(-z0));
-                                    a1 *= __fdividef(z1, 1.0f + __expf(-z1));
-                                    ssq[h2 >> 1] = fmaf(a0, a0, fmaf(a1, a1, ssq[h2 >> 1]));
-                                    a0 *= bf_lo(nw[e]);
-                                    a1 *= bf_hi(nw[e]);
+                                    a = mul2(a, make_float2(__fdividef(z0, 1.0f + __expf(-z0)),
+                                                            __fdividef(z1, 1.0f + __expf(-z1))));
+                                    ssq[h2 >> 1] = fmaf(a.x, a.x, fmaf(a.y, a.y, ssq[h2 >> 1]));
+                                    a = mul2(a, bf2(nw[e]));
                                 }
-                                o[e] = pack_bf16(a0, a1);
+                                o[e] = pack2(a);
                             }
                             reinterpret_cast<uint4*>(yo)[cc] = make_uint4(o[0], o[1], o[2], o[3]);
                         }
@@ -491,6 +509,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
             const int s = k % kNStage;
             if (ok) {  // ---- read-back: H_k as bf16 for Y_off, 2^tot H_k back into TMEM
                 const float dec = ex2(tot);
+                const float2 dec2 = make_float2(dec, dec);
 #pragma unroll
                 for (int h4 = 0; h4 < 4; ++h4) {  // 16 state columns at a time
                     uint32_t v[16];
@@ -506,7 +525,11 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
                         *reinterpret_cast<uint4*>(myHX + sw128(r, 2 * h4 + c)) = w;
                     }
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) v[j] = __float_as_uint(dec * __uint_as_float(v[j]));
+                    for (int j = 0; j < 16; j += 2) {
+                        const float2 d = mul2(dec2, make_float2(__uint_as_float(v[j]), __uint_as_float(v[j + 1])));
+                        v[j] = __float_as_uint(d.x);
+                        v[j + 1] = __float_as_uint(d.y);
+                    }
                     tmem_st16(tmem + lane_base + kTS + 64 * hf + 16 * h4, v);
                 }
                 tmem_st_wait();
@@ -520,14 +543,15 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
             if (ok) {  // ---- X'_j[s=r, :] = 2^(tot - cs_r) dt_r x_j[r, :]
                 const uint8_t* sX = sm + s * kStage + kOffX + hf * kTileQP;
                 const float wgt = ex2(tot - c2) * dtv;
+                const float2 w2 = make_float2(wgt, wgt);
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
                     const uint4 xv = *reinterpret_cast<const uint4*>(sX + sw128(r, c));
                     uint4 o;
-                    o.x = pack_bf16(bf_lo(xv.x) * wgt, bf_hi(xv.x) * wgt);
-                    o.y = pack_bf16(bf_lo(xv.y) * wgt, bf_hi(xv.y) * wgt);
-                    o.z = pack_bf16(bf_lo(xv.z) * wgt, bf_hi(xv.z) * wgt);
-                    o.w = pack_bf16(bf_lo(xv.w) * wgt, bf_hi(xv.w) * wgt);
+                    o.x = pack2(mul2(bf2(xv.x), w2));
+                    o.y = pack2(mul2(bf2(xv.y), w2));
+                    o.z = pack2(mul2(bf2(xv.z), w2));
+                    o.w = pack2(mul2(bf2(xv.w), w2));
                     *reinterpret_cast<uint4*>(myHX + sw128(r, c)) = o;
                 }
                 fence_async_smem();
@@ -558,7 +582,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 1) tmem_dealloc(tmem, kTCols);
+    if (warp == kCtlWarp) tmem_dealloc(tmem, kTCols);
 }
 
 // Segment end states from a zero start, for every segment but the last:
