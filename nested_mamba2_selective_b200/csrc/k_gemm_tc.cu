@@ -438,6 +438,24 @@ bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D bf16 tensor map with a 128-byte swizzle: extents {inner, rows, planes}, `pitch` bytes
+// between rows and `plane_pitch` between planes, box of box_inner x box_rows x 1.  Rows past
+// `rows` inside a plane are outside the tensor, so a box that overhangs a plane is clipped there
+// (stores drop those rows) rather than reaching into the next plane.
+bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint64_t planes,
+                       uint64_t pitch, uint64_t plane_pitch, uint32_t box_inner, uint32_t box_rows)
+{
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {inner, rows, planes};
+    cuuint64_t strides[2] = {pitch, plane_pitch};
+    cuuint32_t box[3] = {box_inner, box_rows, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 static bool tc_shape_ok(const GemmDesc& g)
 {
     auto al16 = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15u) == 0; };

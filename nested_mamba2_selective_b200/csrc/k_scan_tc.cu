@@ -22,6 +22,7 @@
 #include <cuda.h>
 
 #include <cmath>
+#include <cstring>
 
 #include "mm_internal.cuh"
 #include "sm100.cuh"
@@ -66,6 +67,7 @@ struct ScanTcParams {
     int64_t sz;
     const __nv_bfloat16* norm_w;
     float* row_parts;
+    int y_tma;  // 1: y tiles leave through bulk tensor stores (mapY), 0: per-thread stores
 };
 
 __device__ __forceinline__ void named_sync_compute() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
@@ -122,7 +124,8 @@ __device__ __forceinline__ uint32_t pack2(float2 v) { return pack_bf16(v.x, v.y)
 
 __global__ void __launch_bounds__(kChunkThreads, 1)
     ssd_chunk_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CUtensorMap mapB,
-                     const __grid_constant__ CUtensorMap mapC, const ScanTcParams p)
+                     const __grid_constant__ CUtensorMap mapC, const __grid_constant__ CUtensorMap mapY,
+                     const ScanTcParams p)
 {
     extern __shared__ __align__(1024) uint8_t sm[];
     float* tab = reinterpret_cast<float*>(sm + kOffTab);
@@ -163,6 +166,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
         prefetch_tmap(&mapX);
         prefetch_tmap(&mapB);
         prefetch_tmap(&mapC);
+        if (p.y_tma) prefetch_tmap(&mapY);
     }
     if (warp == kCtlWarp) {
         tmem_alloc(tmem_slot, kTCols);
@@ -444,12 +448,14 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
 
             if (k > 0) {  // ---- epilogue of block k-1 (TMEM loads are warp-collective)
                 if (ok) ok = __all_sync(0xffffffffu, mbar_wait(ys_full, (k - 1) & 1, abort));
+                const int sp = (k - 1) % kNStage;
+                const int tp0 = (c_begin + k - 1) * kQ;
+                // x of block k-1 (this head); with bulk stores each thread overwrites its own row of
+                // it with its y row, in the same swizzled layout, once that row's x has been read
+                uint8_t* sX = sm + sp * kStage + kOffX + hf * kTileQP;
                 if (ok) {
                     tc_fence_after();
-                    const int sp = (k - 1) % kNStage;
-                    const int tp0 = (c_begin + k - 1) * kQ;
                     const bool valid = head_ok && tp0 + r < p.L;
-                    const uint8_t* sX = sm + sp * kStage + kOffX + hf * kTileQP;
                     const float ey = ex2(c2_prev);
                     const float2 ey2 = make_float2(ey, ey), dh2 = make_float2(Dh, Dh);
                     const int64_t tok = tok0 + tp0 + r;
@@ -462,14 +468,14 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
                         tmem_ld16(tmem + lane_base + kTY + 64 * hf + 16 * h2, yv);
                         tmem_ld16(tmem + lane_base + kTYO + 64 * hf + 16 * h2, ov);
                         tmem_ld_wait();
-                        if (!valid) continue;
+                        if (!valid && !p.y_tma) continue;
 #pragma unroll
                         for (int c = 0; c < 2; ++c) {
                             const int cc = 2 * h2 + c;
                             const uint4 xv = *reinterpret_cast<const uint4*>(sX + sw128(r, cc));
                             const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
                             uint4 zw4 = make_uint4(0, 0, 0, 0), nw4 = make_uint4(0, 0, 0, 0);
-                            if (p.z) {
+                            if (p.z && valid) {
                                 zw4 = *reinterpret_cast<const uint4*>(p.z + tok * p.sz + col + 8 * cc);
                                 nw4 = *reinterpret_cast<const uint4*>(p.norm_w + col + 8 * cc);
                             }
@@ -492,7 +498,8 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
                                 }
                                 o[e] = pack2(a);
                             }
-                            reinterpret_cast<uint4*>(yo)[cc] = make_uint4(o[0], o[1], o[2], o[3]);
+                            if (p.y_tma) *reinterpret_cast<uint4*>(sX + sw128(r, cc)) = make_uint4(o[0], o[1], o[2], o[3]);
+                            else reinterpret_cast<uint4*>(yo)[cc] = make_uint4(o[0], o[1], o[2], o[3]);
                         }
                     }
                     if (p.z && valid) {
@@ -500,8 +507,23 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
                         p.row_parts[tok * 2 * p.h + 2 * head + 1] = ssq[1];
                     }
                     tc_fence_before();
+                }
+                if (p.y_tma) {  // the head's 128 x 64 tile leaves in one bulk store (rows past L clipped)
+                    fence_async_smem();
+                    asm volatile("bar.sync %0, 128;" ::"r"(bar_id) : "memory");
+                    if (q == 0) {
+                        ok = __all_sync(0xffffffffu, ok && !*abort);
+                        if (ok && head_ok && lane == 0) {
+                            tma_store_3d(&mapY, sX, head * kP, tp0, b);
+                            bulk_commit();
+                            bulk_wait_read0();
+                        }
+                        __syncwarp();
+                    }
+                }
+                if (ok) {
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&empty[sp]);  // x of block k-1 is read
+                    if (lane == 0) mbar_arrive(&empty[sp]);  // x of block k-1 is read (and the y tile sent)
                 }
             }
             if (k == nch) break;
@@ -562,6 +584,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
             c2_prev = c2;
         }
 
+        if (p.y_tma && q == 0 && lane == 0) bulk_wait0();  // this head's y tiles are in global memory
         if (seg == p.nseg - 1 && p.final_state) {  // state after the last block (ys_full waited above)
             ok = __all_sync(0xffffffffu, ok && !*abort);
             if (ok) {
@@ -877,8 +900,16 @@ static cudaError_t launch_scan_tc_impl(const ScanArgs& a, const ScanGate* gate, 
     if (!make_tmap_bf16(&mapB, a.B, (uint64_t)a.G * kN, rows, a.sB * 2, 64, kQ)) return cudaErrorInvalidValue;
     if (!make_tmap_bf16(&mapC, a.C, (uint64_t)a.G * kN, rows, a.sC * 2, 64, kQ)) return cudaErrorInvalidValue;
 
+    // y leaves through bulk tensor stores when it is 16-byte aligned with 16-byte row pitches
+    CUtensorMap mapY;
+    std::memset(&mapY, 0, sizeof(mapY));
+    const bool y_tma = (reinterpret_cast<uintptr_t>(a.y) & 15u) == 0 && (a.sy * 2) % 16 == 0 &&
+                       make_tmap_bf16_3d(&mapY, a.y, (uint64_t)a.h * kP, (uint64_t)a.L, (uint64_t)a.batch,
+                                         (uint64_t)a.sy * 2, (uint64_t)a.sy * 2 * a.L, 64, kQ);
+
     ScanTcParams p{};
     p.L = a.L; p.h = a.h; p.nseg = pl.nseg; p.cps = pl.cps; p.nchunks = pl.nchunks; p.hpg = a.hpg;
+    p.y_tma = y_tma ? 1 : 0;
     p.dt = a.dt; p.sdt = a.sdt; p.A = a.A; p.D = a.D; p.y = a.y; p.sy = a.sy;
     p.init_state = a.init_state; p.final_state = a.final_state; p.state_stride = a.state_stride;
     p.status = device_status_ptr();
@@ -916,7 +947,8 @@ static cudaError_t launch_scan_tc_impl(const ScanArgs& a, const ScanGate* gate, 
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
-    ssd_chunk_kernel<<<dim3((a.h + 1) / 2, pl.nseg, a.batch), kChunkThreads, kChunkSmem, s>>>(mapX, mapB, mapC, p);
+    ssd_chunk_kernel<<<dim3((a.h + 1) / 2, pl.nseg, a.batch), kChunkThreads, kChunkSmem, s>>>(mapX, mapB, mapC, mapY,
+                                                                                             p);
     return cudaGetLastError();
 }
 

@@ -450,53 +450,95 @@ cudaError_t launch_step_conv_dt(int dtype, const void* zxbc, int64_t ld_in, int 
     return cudaGetLastError();
 }
 
-// State update for one token: one warp per (sequence, head, p) row of N fp32
-// state entries, H <- exp(dt A) H + dt x_p B; y_p = C . H + D x_p.
+// State update for one token, H <- exp(dt A) H + dt x_p B; y_p = C . H + D x_p.
+// One CTA per (sequence, head): B and C of the head's group are read once into
+// registers and every warp walks state rows p = warp, warp + 8, ...  With
+// N == 128 a lane owns state entries [4 lane, 4 lane + 4) of a row, so a warp
+// moves a whole 512-byte row with one 16-byte load and one 16-byte store per lane.
 template <typename T>
-__global__ void step_scan_kernel(const T* __restrict__ xbc, int nconv, int d, const float* __restrict__ dt,
-                                 const float* __restrict__ A, const float* __restrict__ D, float* __restrict__ ssm_state,
-                                 int H, int h, int P, int N, int GN, int hpg, int batch, T* __restrict__ y)
+__global__ void __launch_bounds__(256) step_scan_kernel(const T* __restrict__ xbc, int nconv, int d,
+                                                        const float* __restrict__ dt, const float* __restrict__ A,
+                                                        const float* __restrict__ D, float* __restrict__ ssm_state,
+                                                        int H, int h, int P, int N, int GN, int hpg, int vec,
+                                                        T* __restrict__ y)
 {
-    const int64_t wid = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
-    const int64_t nrows = (int64_t)batch * h * P;
-    if (wid >= nrows) return;
-    const int p = (int)(wid % P);
-    const int i = (int)((wid / P) % h);
-    const int b = (int)(wid / ((int64_t)P * h));
+    const int b = blockIdx.x / h, i = blockIdx.x % h;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = i / hpg;
     const T* xr = xbc + (int64_t)b * nconv;
-    const float xv = to_f32(xr[i * P + p]);
     const float dtv = dt[(int64_t)b * h + i];
     const float av = expf(dtv * A[i]);
-    const float dx = dtv * xv;
-    const T* Bv = xr + d + g * (N);
-    const T* Cv = xr + d + GN + g * (N);
-    float* st = ssm_state + (((int64_t)b * H + i) * P + p) * N;
-    float acc = 0.0f;
-    for (int n = lane; n < N; n += 32) {
-        const float hv = fmaf(av, st[n], dx * to_f32(Bv[n]));
-        st[n] = hv;
-        acc = fmaf(to_f32(Cv[n]), hv, acc);
-    }
+    const float Di = D[i];
+    const T* Bv = xr + d + g * N;
+    const T* Cv = xr + d + GN + g * N;
+    float* st = ssm_state + ((int64_t)b * H + i) * P * N;
+    if (vec) {  // N == 128, 16-byte aligned state rows
+        float bq[4], cq[4];
 #pragma unroll
-    for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (lane == 0) y[(int64_t)b * d + i * P + p] = from_f32<T>(fmaf(D[i], xv, acc));
+        for (int e = 0; e < 4; ++e) {
+            bq[e] = to_f32(Bv[4 * lane + e]);
+            cq[e] = to_f32(Cv[4 * lane + e]);
+        }
+        for (int p0 = warp; p0 < P; p0 += 16) {  // two rows in flight per warp
+            const int p1 = p0 + 8;
+            const bool two = p1 < P;
+            float4* r0 = reinterpret_cast<float4*>(st + (int64_t)p0 * N) + lane;
+            float4* r1 = reinterpret_cast<float4*>(st + (int64_t)p1 * N) + lane;
+            float4 s0 = *r0, s1 = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (two) s1 = *r1;
+            const float x0 = to_f32(xr[i * P + p0]), x1 = two ? to_f32(xr[i * P + p1]) : 0.0f;
+            const float d0 = dtv * x0, d1 = dtv * x1;
+            s0.x = fmaf(av, s0.x, d0 * bq[0]); s0.y = fmaf(av, s0.y, d0 * bq[1]);
+            s0.z = fmaf(av, s0.z, d0 * bq[2]); s0.w = fmaf(av, s0.w, d0 * bq[3]);
+            s1.x = fmaf(av, s1.x, d1 * bq[0]); s1.y = fmaf(av, s1.y, d1 * bq[1]);
+            s1.z = fmaf(av, s1.z, d1 * bq[2]); s1.w = fmaf(av, s1.w, d1 * bq[3]);
+            *r0 = s0;
+            if (two) *r1 = s1;
+            float a0 = fmaf(cq[3], s0.w, fmaf(cq[2], s0.z, fmaf(cq[1], s0.y, cq[0] * s0.x)));
+            float a1 = fmaf(cq[3], s1.w, fmaf(cq[2], s1.z, fmaf(cq[1], s1.y, cq[0] * s1.x)));
+#pragma unroll
+            for (int o = 16; o; o >>= 1) {
+                a0 += __shfl_xor_sync(0xffffffffu, a0, o);
+                a1 += __shfl_xor_sync(0xffffffffu, a1, o);
+            }
+            if (lane == 0) {
+                y[(int64_t)b * d + i * P + p0] = from_f32<T>(fmaf(Di, x0, a0));
+                if (two) y[(int64_t)b * d + i * P + p1] = from_f32<T>(fmaf(Di, x1, a1));
+            }
+        }
+        return;
+    }
+    for (int p = warp; p < P; p += 8) {  // any N: lanes stride the row
+        const float xv = to_f32(xr[i * P + p]);
+        const float dx = dtv * xv;
+        float* row = st + (int64_t)p * N;
+        float acc = 0.0f;
+        for (int n = lane; n < N; n += 32) {
+            const float hv = fmaf(av, row[n], dx * to_f32(Bv[n]));
+            row[n] = hv;
+            acc = fmaf(to_f32(Cv[n]), hv, acc);
+        }
+#pragma unroll
+        for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (lane == 0) y[(int64_t)b * d + i * P + p] = from_f32<T>(fmaf(Di, xv, acc));
+    }
 }
 
 cudaError_t launch_step_scan(int dtype, const void* xbc, int nconv, int d, const float* dt, const float* A,
                              const float* D, float* ssm_state, int H, int h, int P, int N, int GN, int hpg, int batch,
                              void* y, cudaStream_t s)
 {
-    const int64_t rows = (int64_t)batch * h * P;
-    if (rows == 0) return cudaSuccess;
-    dim3 grid((unsigned)((rows + 7) / 8));
+    const int64_t heads = (int64_t)batch * h;
+    if (heads == 0) return cudaSuccess;
+    if (heads > 0x7fffffff) return cudaErrorInvalidValue;
+    const int vec = N == 128 && (reinterpret_cast<uintptr_t>(ssm_state) & 15u) == 0;
     if (dtype == MM_BF16)
-        step_scan_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>((const __nv_bfloat16*)xbc, nconv, d, dt, A, D, ssm_state, H,
-                                                              h, P, N, GN, hpg, batch, (__nv_bfloat16*)y);
+        step_scan_kernel<__nv_bfloat16><<<(unsigned)heads, 256, 0, s>>>((const __nv_bfloat16*)xbc, nconv, d, dt, A, D,
+                                                                         ssm_state, H, h, P, N, GN, hpg, vec,
+                                                                         (__nv_bfloat16*)y);
     else
-        step_scan_kernel<float><<<grid, 256, 0, s>>>((const float*)xbc, nconv, d, dt, A, D, ssm_state, H, h, P, N, GN,
-                                                      hpg, batch, (float*)y);
+        step_scan_kernel<float><<<(unsigned)heads, 256, 0, s>>>((const float*)xbc, nconv, d, dt, A, D, ssm_state, H, h,
+                                                                 P, N, GN, hpg, vec, (float*)y);
     return cudaGetLastError();
 }
 

@@ -121,6 +121,8 @@ cudaError_t launch_step_scan(int dtype, const void* xbc, int nconv, int d, const
 int* device_status_ptr();
 bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint64_t pitch,
                     uint32_t box_inner, uint32_t box_rows);
+bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint64_t planes,
+                       uint64_t pitch, uint64_t plane_pitch, uint32_t box_inner, uint32_t box_rows);
 
 // Tensor-core paths (bf16 only).
 bool gemm_tc_supported(const GemmDesc& g);
