@@ -14,6 +14,8 @@
 // tile i overlap the MMAs of tile i+1.
 #include <cuda.h>
 
+#include <cstring>
+
 #include "mm_internal.cuh"
 #include "sm100.cuh"
 
@@ -39,8 +41,15 @@ struct TcSeg {
     int out_f32;
     int accumulate;
     int vec_ok;  // 16-byte vector stores allowed
+    int tma;     // bf16 tiles leave through bulk tensor stores (OutMaps::m[segment])
     int kind;    // GemmEpi
     int conv_row0;
+};
+
+// Output tensor maps of the segments whose tiles leave through bulk tensor stores
+// (bf16, 64 x 128 boxes, 128-byte swizzle).
+struct OutMaps {
+    CUtensorMap m[kMaxSeg];
 };
 
 struct TcParams {
@@ -61,6 +70,8 @@ template <int BN>
 __device__ __forceinline__ TileInfo<BN> tile_info(const TcParams& p, int tile)
 {
     TileInfo<BN> t;
+    // row-block major: the N tiles of a row block are consecutive, so CTAs working at the same
+    // time share its A rows in L2, and a CTA's walk (stride = grid) mixes the segments' kinds
     t.mt = tile / p.ntiles;
     int j = tile % p.ntiles;
     int s = 0;
@@ -91,7 +102,8 @@ __device__ __forceinline__ void store_bf16_chunk(__nv_bfloat16* o, int ncols, bo
 
 template <int BN, int STAGES, bool CONV>
 __global__ void __launch_bounds__(320, 1)
-    gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB, const TcParams p)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
+                   const __grid_constant__ OutMaps omaps, const TcParams p)
 {
     constexpr int A_BYTES = kBM * kBK * 2;
     constexpr int B_BYTES = BN * kBK * 2;
@@ -100,9 +112,11 @@ __global__ void __launch_bounds__(320, 1)
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    // [2 epilogue groups][128 rows][kStageLd]: a 32-column chunk of fp32 accumulators for the conv epilogue
+    // [2 epilogue groups][128 rows][kStageLd]: a 32-column chunk of fp32 accumulators for the conv epilogue.
+    // The same bytes (group g at g * kGroupStage) stage 64-column bf16 tiles for the bulk stores.
+    constexpr int kGroupStage = CONV ? kBM * kStageLd * 4 : kBM * 128;  // both multiples of 1024
     float* stage = reinterpret_cast<float*>(smem + STAGES * STAGE_BYTES);
-    uint64_t* full = reinterpret_cast<uint64_t*>(stage + (CONV ? 2 * kBM * kStageLd : 0));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES + 2 * kGroupStage);
     uint64_t* empty = full + STAGES;
     uint64_t* tfull = empty + STAGES;
     uint64_t* tempty = tfull + 2;
@@ -240,6 +254,52 @@ __global__ void __launch_bounds__(320, 1)
                 w_tp0 = (int)(((w_m0 % ex.L) + ex.L) % ex.L);
                 w_fast = sg.vec_ok && p.shift == 3 && w_m0 >= 0 && w_m0 + w_n - 1 < p.M && w_tp0 >= 3 &&
                          w_tp0 + w_n - 1 + 3 < ex.L;
+            }
+            const int64_t tile_row0 = (int64_t)t.mt * p.rows - p.shift;  // token of tile row 0
+            if (sg.tma && tile_row0 >= 0) {
+                // 64-column units (group eg takes units eg, eg + 2, ...): rows staged as bf16 in the
+                // 128-byte-swizzled layout, then one bulk store per unit.  Halo rows above the tile's
+                // outputs rewrite the identical values the previous row block wrote.
+                uint8_t* stg = reinterpret_cast<uint8_t*>(stage) + eg * kGroupStage;
+                for (int u = eg; 64 * u < t.nvalid; u += 2) {
+                    // the previous unit's store has read the staging rows (its issuer waited)
+                    asm volatile("bar.sync %0, 128;" ::"r"(2 + eg) : "memory");
+                    if (ok) {
+#pragma unroll
+                        for (int hh = 0; hh < 2; ++hh) {
+                            uint32_t raw[32];
+                            tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + buf * BN + 64 * u + 32 * hh, raw);
+                            tmem_ld_wait();
+                            float v[32];
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(raw[i]);
+                            if (ex.row_parts) {
+#pragma unroll
+                                for (int i = 0; i < 32; ++i) v[i] *= scale;
+                            }
+#pragma unroll
+                            for (int c = 0; c < 4; ++c) {
+                                const uint4 w = make_uint4(pack_bf16(v[8 * c + 0], v[8 * c + 1]), pack_bf16(v[8 * c + 2], v[8 * c + 3]),
+                                                           pack_bf16(v[8 * c + 4], v[8 * c + 5]), pack_bf16(v[8 * c + 6], v[8 * c + 7]));
+                                const int chunk = 4 * hh + c;
+                                *reinterpret_cast<uint4*>(stg + r * 128 + ((chunk ^ (r & 7)) << 4)) = w;
+                            }
+                        }
+                    }
+                    fence_async_smem();
+                    asm volatile("bar.sync %0, 128;" ::"r"(2 + eg) : "memory");
+                    if (ok && q == 2 && lane == 0) {  // one issuer per group
+                        tma_store_2d(&omaps.m[t.seg], stg, t.n0 + 64 * u, (int)tile_row0);
+                        bulk_commit();
+                        bulk_wait_read0();
+                    }
+                }
+                // the last store has read the staging rows before the group writes them again
+                asm volatile("bar.sync %0, 128;" ::"r"(2 + eg) : "memory");
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&tempty[buf]);
+                continue;
             }
             for (int c0 = 32 * eg; c0 < t.nvalid; c0 += 64, ++nchunk_done) {
                 float v[32];
@@ -395,6 +455,7 @@ __global__ void __launch_bounds__(320, 1)
             if (lane == 0) mbar_arrive(&tempty[buf]);
         }
     }
+    if (warp >= 2 && (warp & 3) == 2 && lane == 0) bulk_wait0();  // this group's bulk stores are complete
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -494,7 +555,15 @@ static cudaError_t launch_bn(const GemmDesc& g, const TcParams& p0, cudaStream_t
     CUtensorMap mapA, mapB;
     if (!make_tmap_bf16(&mapA, g.A, g.K, g.M, g.lda * 2, kBK, kBM)) return cudaErrorInvalidValue;
     if (!make_tmap_bf16(&mapB, base, g.ldb, rows, g.ldb * 2, kBK, BN)) return cudaErrorInvalidValue;
-    constexpr int smem = STAGES * (kBM + BN) * kBK * 2 + (CONV ? 2 * kBM * kStageLd * 4 : 0) + 1024 + 256;
+    OutMaps om;
+    std::memset(&om, 0, sizeof(om));
+    for (int i = 0; i < p.nseg; ++i) {  // plain bf16 outputs leave through bulk stores
+        TcSeg& t = p.seg[i];
+        t.tma = 0;
+        if (t.kind == kEpiStore && !t.out_f32 && !t.accumulate && t.vec_ok)
+            t.tma = make_tmap_bf16(&om.m[i], t.out, (uint64_t)t.n, (uint64_t)g.M, (uint64_t)t.ldo * 2, 64, kBM) ? 1 : 0;
+    }
+    constexpr int smem = STAGES * (kBM + BN) * kBK * 2 + (CONV ? 2 * kBM * kStageLd * 4 : 2 * kBM * 128) + 1024 + 256;
     static_assert(smem <= 232448, "GEMM configuration exceeds 227 KB of shared memory");
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
@@ -508,7 +577,7 @@ static cudaError_t launch_bn(const GemmDesc& g, const TcParams& p0, cudaStream_t
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int total = p.mtiles * p.ntiles;
     const int grid = total < sms ? total : sms;
-    gemm_tc_kernel<BN, STAGES, CONV><<<grid, 320, smem, s>>>(mapA, mapB, p);
+    gemm_tc_kernel<BN, STAGES, CONV><<<grid, 320, smem, s>>>(mapA, mapB, om, p);
     return cudaGetLastError();
 }
 
