@@ -23,6 +23,7 @@
 
 #include <cmath>
 #include <cstring>
+#include <utility>
 
 #include "mm_internal.cuh"
 #include "sm100.cuh"
@@ -50,6 +51,8 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 struct ScanTcParams {
     int L, h, nseg, cps, nchunks, hpg;
+    int c0;         // blocks in segment 0; segments 1.. take cps blocks each (the last may be shorter)
+    int wait_all;   // 1: every chunk-scan CTA waits for the segment-state grid (y overlaps an input)
     const float* dt;
     int64_t sdt;
     const float* A;
@@ -57,7 +60,7 @@ struct ScanTcParams {
     void* y;
     int64_t sy;
     float* states;     // [b*h][nseg][P*N]: slot k = start state of segment k
-    float* seg_decay;  // [b*h][nseg]: log2 of the decay over segment k
+    float* seg_decay;  // [b*h][nseg]: log2 of the decay over segment k (k < nseg - 1)
     const float* init_state;
     float* final_state;
     int64_t state_stride;
@@ -106,6 +109,18 @@ __device__ __forceinline__ float bf_hi(uint32_t v) { return __uint_as_float(v & 
 // takes direct exponentials instead (g_s = dt_s, M = G 2^min(cs_t - cs_s, 0) g_s).
 // Element-wise products use the paired fp32 instructions (mul/fma .f32x2, rounded per lane
 // exactly like their scalar forms).
+// Blocks [c_begin, c_end) of segment `seg`.
+__device__ __forceinline__ void seg_range(const ScanTcParams& p, int seg, int* c_begin, int* c_end)
+{
+    *c_begin = seg == 0 ? 0 : p.c0 + (seg - 1) * p.cps;
+    *c_end = min(p.nchunks, seg == 0 ? p.c0 : *c_begin + p.cps);
+}
+
+// Programmatic dependent launch: let the dependent grid start, and wait for the
+// prerequisite grid's completion (and its memory) before reading what it wrote.
+__device__ __forceinline__ void grid_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 constexpr int kChunkThreads = 512;
 constexpr int kCtlWarp = 4;
 constexpr float kDropMax = 100.0f;  // log2 units
@@ -140,11 +155,13 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
     volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
-    const int pair = blockIdx.x, seg = blockIdx.y, b = blockIdx.z;
+    // segment is the slowest grid dimension: segment 0's CTAs are scheduled first, on the SMs the
+    // segment-state grid leaves free, since they need no carried state
+    const int pair = blockIdx.x, b = blockIdx.y, seg = blockIdx.z;
     const int head0 = 2 * pair;
-    const int c_begin = seg * p.cps;
-    const int c_end = min(p.nchunks, c_begin + p.cps);
-    const int nch = c_end - c_begin;
+    int c_begin, c_end;
+    seg_range(p, seg, &c_begin, &c_end);
+    const int nch = max(c_end - c_begin, 0);
     const int grp = head0 / p.hpg;  // both heads of a pair share a group (hpg is even or G == 1)
     const int64_t tok0 = (int64_t)b * p.L;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -398,19 +415,29 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
 
         // The fp32 state of this head lives in TMEM columns kTS + 64 hf (row n = lane r): each
         // block, it is read for its bf16 copy (Y_off's operand), 2^tot H_k is written back, and
-        // the S MMA accumulates B^T X' on top, leaving H_{k+1}.
+        // the S MMA accumulates B^T X' on top, leaving H_{k+1}.  A segment's start state is the
+        // initial state (or zero) carried over the earlier segments:
+        // H <- 2^decay_j H + S_j, S_j being segment j's end state from a zero start.
         {
-            const float* src = nullptr;
-            if (head_ok) {
-                if (p.nseg > 1) src = p.states + (bh * p.nseg + seg) * PN;
-                else if (p.init_state) src = p.init_state + (int64_t)b * p.state_stride + (int64_t)head * PN;
-            }
+            if (p.nseg > 1 && (seg > 0 || p.wait_all)) grid_dependency_wait();  // segment end states written
+            const float* init = (head_ok && p.init_state)
+                                    ? p.init_state + (int64_t)b * p.state_stride + (int64_t)head * PN
+                                    : nullptr;
 #pragma unroll
             for (int h2 = 0; h2 < 2; ++h2) {
-                uint32_t v[32];
+                float v[32];
 #pragma unroll
-                for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(src ? src[(32 * h2 + j) * kN + r] : 0.0f);
-                tmem_st32(tmem + lane_base + kTS + 64 * hf + 32 * h2, v);
+                for (int j = 0; j < 32; ++j) v[j] = init ? init[(32 * h2 + j) * kN + r] : 0.0f;
+                for (int sj = 0; head_ok && sj < seg; ++sj) {
+                    const float dec = exp2f(p.seg_decay[bh * p.nseg + sj]);
+                    const float* sp = p.states + (bh * p.nseg + sj + 1) * PN;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) v[j] = fmaf(dec, v[j], sp[(32 * h2 + j) * kN + r]);
+                }
+                uint32_t u[32];
+#pragma unroll
+                for (int j = 0; j < 32; ++j) u[j] = __float_as_uint(v[j]);
+                tmem_st32(tmem + lane_base + kTS + 64 * hf + 32 * h2, u);
             }
             tmem_st_wait();
         }
@@ -638,12 +665,13 @@ __global__ void __launch_bounds__(320, 1)
 
     const int pair = blockIdx.x, seg = blockIdx.y, b = blockIdx.z;
     const int head0 = 2 * pair;
-    const int c_begin = seg * p.cps;
-    const int c_end = min(p.nchunks, c_begin + p.cps);
-    const int nch = c_end - c_begin;
+    int c_begin, c_end;
+    seg_range(p, seg, &c_begin, &c_end);
+    const int nch = max(c_end - c_begin, 0);
     const int grp = head0 / p.hpg;
     const int64_t tok0 = (int64_t)b * p.L;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    grid_launch_dependents();  // the chunk scan may start its first segment beside this grid
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kNStage; ++i) {
@@ -796,53 +824,53 @@ __global__ void __launch_bounds__(320, 1)
     }
 }
 
-// Segment start states: slot 0 = initial state (or zero); slot k = state after
-// segment k-1, combined in order from the local end states K_a left in slots
-// 1..nseg-1.  One thread per state element.
-__global__ void ssd_state_pass_kernel(float* states, const float* seg_decay, const float* init, int64_t state_stride,
-                                      int64_t bh_total, int h, int nseg)
-{
-    constexpr int PN = kP * kN;
-    const int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
-    if (idx >= bh_total * PN) return;
-    const int64_t bh = idx / PN;
-    const int e = (int)(idx % PN);
-    const int64_t b = bh / h, i = bh % h;
-    float cur = init ? init[b * state_stride + i * PN + e] : 0.0f;
-    float* base = states + bh * nseg * PN + e;
-    base[0] = cur;
-    for (int k = 1; k < nseg; ++k) {
-        cur = fmaf(exp2f(seg_decay[bh * nseg + k - 1]), cur, base[(int64_t)k * PN]);
-        base[(int64_t)k * PN] = cur;
-    }
-}
-
 struct Plan {
     int nchunks, nseg, cps;
+    int c0;       // blocks of segment 0 (>= cps when it runs beside the segment-state grid)
+    bool overlap;  // segment 0's CTAs fit beside the segment-state grid
 };
 
 Plan plan_for(const ScanArgs& a, int sms)
 {
-    // Cost in units of one block (128 tokens) of chunk-scan work per CTA.  A CTA
-    // also pays a fixed start (TMEM, barriers, state load and pipeline fill,
-    // about 1.5 blocks); the segment-state pass costs about 0.35 of a block per
-    // block, and the combine a little per segment.
+    // Costs in units of one 128-token block of chunk-scan work per CTA.  A CTA also pays a
+    // fixed start (TMEM, barriers, state fold and pipeline fill: about 1.5 blocks).  A block of
+    // the segment-state pass costs about 0.3 of a chunk-scan block.  Segment 0 needs no carried
+    // state: when its CTAs fit on the SMs the segment-state grid leaves free, it starts at once
+    // and may take more blocks than the others, which start after the segment-state grid.
     Plan pl;
     pl.nchunks = (a.L + kQ - 1) / kQ;
     const int64_t ctas = (int64_t)a.batch * ((a.h + 1) / 2);  // CTAs per segment: head pairs
     double best = 1e30;
     pl.nseg = 1;
     pl.cps = pl.nchunks;
+    pl.c0 = pl.nchunks;
+    pl.overlap = false;
     for (int ns = 1; ns <= pl.nchunks && ns <= 64; ++ns) {
-        const int cps = (pl.nchunks + ns - 1) / ns;
-        const int nseg = (pl.nchunks + cps - 1) / cps;
-        if (nseg != ns) continue;
-        double cost = std::ceil((double)(ctas * nseg) / sms) * (cps + 1.5);
-        if (nseg > 1) cost += 0.35 * std::ceil((double)(ctas * (nseg - 1)) / sms) * (cps + 1.5) + 2.0 + 0.1 * nseg;
-        if (cost < best - 1e-9) {
-            best = cost;
-            pl.nseg = nseg;
-            pl.cps = cps;
+        const bool overlap = ns > 1 && ctas * ns <= sms;
+        const int even = (pl.nchunks + ns - 1) / ns;
+        // segment 0 of c0 blocks, the others of c1 blocks each (the last one shorter, never empty);
+        // only an overlapped segment 0 may be longer than the even split
+        for (int c0 = even; c0 <= (overlap ? pl.nchunks - (ns - 1) : even); ++c0) {
+            const int rest = pl.nchunks - c0;
+            int c1 = 0;
+            double cost;
+            if (ns == 1) {
+                cost = std::ceil((double)ctas / sms) * (c0 + 1.5);
+            } else {
+                if (rest < ns - 1) continue;
+                c1 = (rest + ns - 2) / (ns - 1);
+                if (rest - (ns - 2) * c1 <= 0) continue;
+                const double seg_pass = 0.3 * std::ceil((double)(ctas * (ns - 1)) / sms) * (std::max(c0, c1) + 1.5) + 0.4;
+                cost = overlap ? std::max(c0 + 1.5, seg_pass + (c1 + 1.5))
+                               : seg_pass + std::ceil((double)(ctas * ns) / sms) * (std::max(c0, c1) + 1.5);
+            }
+            if (cost < best - 1e-9) {
+                best = cost;
+                pl.nseg = ns;
+                pl.c0 = c0;
+                pl.cps = ns > 1 ? c1 : c0;
+                pl.overlap = overlap;
+            }
         }
     }
     return pl;
@@ -875,7 +903,7 @@ size_t scan_tc_workspace(const ScanArgs& a)
     return align256(bh * pl.nseg * kP * kN * 4) + align256(bh * pl.nseg * 4);
 }
 
-int scan_tc_kernel_count(const ScanArgs& a) { return plan_for(a, num_sms()).nseg > 1 ? 3 : 1; }
+int scan_tc_kernel_count(const ScanArgs& a) { return plan_for(a, num_sms()).nseg > 1 ? 2 : 1; }
 
 static cudaError_t launch_scan_tc_impl(const ScanArgs& a, const ScanGate* gate, void* ws, size_t ws_bytes,
                                        cudaStream_t s);
@@ -909,6 +937,7 @@ static cudaError_t launch_scan_tc_impl(const ScanArgs& a, const ScanGate* gate, 
 
     ScanTcParams p{};
     p.L = a.L; p.h = a.h; p.nseg = pl.nseg; p.cps = pl.cps; p.nchunks = pl.nchunks; p.hpg = a.hpg;
+    p.c0 = pl.c0;
     p.y_tma = y_tma ? 1 : 0;
     p.dt = a.dt; p.sdt = a.sdt; p.A = a.A; p.D = a.D; p.y = a.y; p.sy = a.sy;
     p.init_state = a.init_state; p.final_state = a.final_state; p.state_stride = a.state_stride;
@@ -937,19 +966,41 @@ static cudaError_t launch_scan_tc_impl(const ScanArgs& a, const ScanGate* gate, 
         if (e != cudaSuccess) return e;
         attr_set |= 1ull << dev;
     }
-    if (pl.nseg > 1) {
-        ssd_seg_state_kernel<<<dim3((a.h + 1) / 2, pl.nseg - 1, a.batch), 320, kSegSmemBytes, s>>>(mapX, mapB, p);
-        cudaError_t e = cudaGetLastError();
-        if (e != cudaSuccess) return e;
-        const int64_t n = (int64_t)bh * kP * kN;
-        ssd_state_pass_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(p.states, p.seg_decay, a.init_state,
-                                                                           a.state_stride, (int64_t)bh, a.h, pl.nseg);
-        e = cudaGetLastError();
-        if (e != cudaSuccess) return e;
+    const dim3 cgrid((a.h + 1) / 2, a.batch, pl.nseg);
+    if (pl.nseg == 1) {
+        ssd_chunk_kernel<<<cgrid, kChunkThreads, kChunkSmem, s>>>(mapX, mapB, mapC, mapY, p);
+        return cudaGetLastError();
     }
-    ssd_chunk_kernel<<<dim3((a.h + 1) / 2, pl.nseg, a.batch), kChunkThreads, kChunkSmem, s>>>(mapX, mapB, mapC, mapY,
-                                                                                             p);
-    return cudaGetLastError();
+    // The chunk scan is launched as a programmatic dependent of the segment-state grid: segment
+    // 0's CTAs may run beside it, the others wait for its completion before reading the
+    // segment end states.  If y overlaps an input the segment-state grid still reads, every
+    // CTA waits.
+    {
+        auto span = [](const void* q, int64_t bytes) { return std::make_pair((uintptr_t)q, (uintptr_t)q + bytes); };
+        const int64_t T = (int64_t)a.batch * a.L;
+        const int esz = 2;
+        const auto ys = span(a.y, ((T - 1) * a.sy + (int64_t)a.h * kP) * esz);
+        const std::pair<uintptr_t, uintptr_t> ins[3] = {span(a.x, ((T - 1) * a.sx + (int64_t)a.h * kP) * esz),
+                                                        span(a.B, ((T - 1) * a.sB + (int64_t)a.G * kN) * esz),
+                                                        span(a.dt, ((T - 1) * a.sdt + a.h) * 4)};
+        p.wait_all = (pl.overlap ? 0 : 1);
+        for (const auto& in : ins)
+            if (ys.first < in.second && in.first < ys.second) p.wait_all = 1;
+    }
+    ssd_seg_state_kernel<<<dim3((a.h + 1) / 2, pl.nseg - 1, a.batch), 320, kSegSmemBytes, s>>>(mapX, mapB, p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = cgrid;
+    cfg.blockDim = dim3(kChunkThreads);
+    cfg.dynamicSmemBytes = kChunkSmem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, ssd_chunk_kernel, mapX, mapB, mapC, mapY, p);
 }
 
 }  // namespace mm
