@@ -87,6 +87,15 @@ __device__ __forceinline__ float ex2(float x)
     return y;
 }
 
+// x / (1 + 2^(-x log2 e)) from the MUFU approximations of 2^x and 1/x (relative error of each
+// about 2^-22); -0 for very negative x, where 2^(-x log2 e) overflows to +inf.
+__device__ __forceinline__ float silu_approx(float x)
+{
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(1.0f + ex2(-x * kLog2e)));
+    return x * r;
+}
+
 __device__ __forceinline__ float bf_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
 
@@ -489,6 +498,20 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
                     const int col = head * kP;
                     __nv_bfloat16* yo = static_cast<__nv_bfloat16*>(p.y) + tok * p.sy + col;
                     float ssq[2] = {0.0f, 0.0f};
+                    // z rows of this warp's 32 tokens, loaded four rows per instruction (coalesced) into
+                    // the warp's own 32 rows of the H / X' buffer, which is free until the read-back
+                    uint8_t* zs = myHX + 32 * q * 128;
+                    if (p.z) {
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const int rr = (lane >> 3) + 4 * i, ch = lane & 7;
+                            uint4 zv = make_uint4(0, 0, 0, 0);
+                            if (head_ok && tp0 + 32 * q + rr < p.L)
+                                zv = *reinterpret_cast<const uint4*>(p.z + (tok0 + tp0 + 32 * q + rr) * p.sz + col + 8 * ch);
+                            *reinterpret_cast<uint4*>(zs + rr * 128 + ((ch ^ (rr & 7)) << 4)) = zv;
+                        }
+                        __syncwarp();
+                    }
 #pragma unroll
                     for (int h2 = 0; h2 < 4; ++h2) {  // 16 output columns at a time
                         uint32_t yv[16], ov[16];
@@ -503,7 +526,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
                             const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
                             uint4 zw4 = make_uint4(0, 0, 0, 0), nw4 = make_uint4(0, 0, 0, 0);
                             if (p.z && valid) {
-                                zw4 = *reinterpret_cast<const uint4*>(p.z + tok * p.sz + col + 8 * cc);
+                                zw4 = *reinterpret_cast<const uint4*>(zs + lane * 128 + ((cc ^ (lane & 7)) << 4));
                                 nw4 = *reinterpret_cast<const uint4*>(p.norm_w + col + 8 * cc);
                             }
                             const uint32_t zw[4] = {zw4.x, zw4.y, zw4.z, zw4.w};
@@ -518,8 +541,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
                                 a = fma2(dh2, bf2(xw[e]), a);
                                 if (p.z) {
                                     const float z0 = bf_lo(zw[e]), z1 = bf_hi(zw[e]);
-                                    a = mul2(a, make_float2(__fdividef(z0, 1.0f + __expf(-z0)),
-                                                            __fdividef(z1, 1.0f + __expf(-z1))));
+                                    a = mul2(a, make_float2(silu_approx(z0), silu_approx(z1)));
                                     ssq[h2 >> 1] = fmaf(a.x, a.x, fmaf(a.y, a.y, ssq[h2 >> 1]));
                                     a = mul2(a, bf2(nw[e]));
                                 }
