@@ -214,6 +214,17 @@ int ssd_scan_static(int dtype, const void* x, int64_t x_stride, const float* dt,
                     int L, int h, int P, int N, int G, int heads_per_group, int chunk, const float* init_state,
                     int64_t state_stride, void* y, int64_t y_stride, float* final_state, void* stream);
 
+/*
+ * Failure-path self-test (no counterpart in the paper): launches one CTA that
+ * waits on an mbarrier nothing arrives on, through the same bounded wait the
+ * tensor-core kernels use, with a limit of timeout_us microseconds (1 ..
+ * 1,000,000).  The wait gives up, the kernel records MM_ERR_TIMEOUT in the
+ * device status word and returns; mm_device_status then reports it (and
+ * clears it) and the context stays usable.  Returns MM_ERR_SHAPE for a limit
+ * out of range, MM_ERR_CUDA if the launch fails, else MM_OK.
+ */
+int mm_selftest_wait_timeout(unsigned timeout_us, void* stream);
+
 /* Workspace bytes for ssd_step.  Host only. */
 int ssd_step_workspace(const mm_block_params* p, int batch, int m_i, size_t* bytes);
 

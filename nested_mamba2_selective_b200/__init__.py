@@ -7,5 +7,5 @@ synthetic input recipes shared by tests and benchmarks (synth.py).
 """
 from ._lib import (BlockWeights, MatMambaError, load, matmamba_block_fwd, matmamba_block_fwd_host,  # noqa: F401
                    matmamba_block_workspace, matmamba_stack_fwd, matmamba_stack_workspace, mm_trace_collect,
-                   mm_device_status, mm_linear, mm_trace_enable, mm_width, ssd_scan,
+                   mm_device_status, mm_linear, mm_selftest_wait_timeout, mm_trace_enable, mm_width, ssd_scan,
                    ssd_scan_static, ssd_scan_workspace, ssd_step, ssd_step_workspace, status_string)

@@ -54,6 +54,7 @@ _SIGS = {
                   _vp, _i64, _vp, _i64, _vp, _vp, _sz, _vp], _i),
     "ssd_scan_static": ([_i, _vp, _i64, _vp, _i64, _vp, _vp, _i64, _vp, _i64, _vp, _i, _i, _i, _i, _i, _i, _i, _i,
                          _vp, _i64, _vp, _i64, _vp, _vp], _i),
+    "mm_selftest_wait_timeout": ([ctypes.c_uint, _vp], _i),
     "ssd_step_workspace": ([_pp, _i, _i, ctypes.POINTER(_sz)], _i),
     "ssd_step": ([_pp, _vp, _vp, _vp, _i, _i, _vp, _vp, _sz, _vp], _i),
     "matmamba_stack_workspace": ([_pp, _i, ctypes.POINTER(_i), _i, _i, _i, ctypes.POINTER(_sz)], _i),
@@ -271,6 +272,12 @@ def ssd_scan_static(x, dt, A, B, C, D=None, h=None, chunk=256, heads_per_group=N
                                 st_stride, _ptr(y), y.shape[2] * y.shape[3], _ptr(final_state), _stream(stream))
     _check(rc, "ssd_scan_static")
     return y
+
+
+def mm_selftest_wait_timeout(timeout_us=20000, stream=None):
+    """Run the failure-path self-test: a kernel whose bounded wait gives up after timeout_us and
+    records MM_ERR_TIMEOUT in the device status word (read it with mm_device_status)."""
+    _check(load().mm_selftest_wait_timeout(int(timeout_us), _stream(stream)), "mm_selftest_wait_timeout")
 
 
 def ssd_step_workspace(w: BlockWeights, batch: int, m_i: int) -> int:

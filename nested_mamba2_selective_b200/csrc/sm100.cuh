@@ -77,13 +77,14 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
 // Wait for the phase with the given parity.  Returns false if the wait gave up
 // (time limit, or another thread of the CTA raised *abort).  The thread sleeps
 // inside try_wait and checks the limit and the abort flag only when it wakes.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort)
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          uint64_t limit_ns = kWaitNs)
 {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
     while (!mbar_try_wait_sleep(bar, parity, 50000u)) {
         if (abort && *abort) return false;
-        if (globaltimer() - t0 > kWaitNs) return false;
+        if (globaltimer() - t0 > limit_ns) return false;
     }
     return true;
 }

@@ -94,3 +94,10 @@ def test_status_strings(lib):
     for s in range(10):
         assert lib.mm_status_string(s)
     assert lib.mm_version() >= 100
+
+
+def test_selftest_rejects_limits_out_of_range_on_the_host():
+    from nested_mamba2_selective_b200 import _lib
+    lib = _lib.load()
+    for bad in (0, 2_000_000):
+        assert lib.mm_selftest_wait_timeout(bad, None) == 2  # MM_ERR_SHAPE, before any launch
