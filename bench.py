@@ -502,8 +502,15 @@ def run_extended(args, mm, synth, torch, dev, timed, slowest, world):
         ms, _ = timed(g.replay, steps, 1)
         avg = slowest(sum(ms)) / steps
         del g
+        # one eager forward, traced: the summed device time of each stage over the 48 layers
+        mm.mm_trace_enable(48 * 8 + 16)
+        fn()
+        torch.cuda.synchronize()
+        stg, _ = mm.mm_trace_collect()
+        mm.mm_trace_enable(0)
         stack[str(m)] = {"ms_per_forward": avg, "tokens_per_s": world * 4 * 4096 / (avg / 1e3),
-                         "timing": "CUDA graph replay of the 48-layer forward"}
+                         "timing": "CUDA graph replay of the 48-layer forward",
+                         "stages_eager_ms": {k: round(v[2], 3) for k, v in stg.items()}}
     res["stack48_1p4b_b4_L4096"] = stack
     dec = {}
     w = layers[0]
@@ -519,8 +526,10 @@ def run_extended(args, mm, synth, torch, dev, timed, slowest, world):
         ms, _ = timed(g.replay, args.steps, args.warmup)
         avg = slowest(sum(ms)) / args.steps
         del g
+        _, (stg, _) = timed(fn, 3, 1, trace=True)  # eager, traced: where a step's time goes
         dec[str(m)] = {"us_per_step": avg * 1e3, "tokens_per_s": world * 256 / (avg / 1e3),
-                       "timing": "CUDA graph replay of one step, L2 flushed before each"}
+                       "timing": "CUDA graph replay of one step, L2 flushed before each",
+                       "stages_eager_us": {k: round(v[2] / v[0] * 1e3, 1) for k, v in stg.items()}}
     res["decode_b256_1p4b"] = dec
     return res
 

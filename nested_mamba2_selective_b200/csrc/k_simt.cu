@@ -293,28 +293,53 @@ cudaError_t launch_scan_seq(int dtype, const ScanArgs& a, cudaStream_t s)
 // ====================================================================== gate + RMSNorm
 
 // One warp per token: q = y * SiLU(z); out = q / sqrt(mean(q^2) + eps) * w.
+// n = RMSNorm_d(y (x) SiLU(z)) (x) w, one CTA of 256 threads per row: each thread
+// keeps q = y * SiLU(z) for up to kGateCols / 256 channels in registers between
+// the sum of squares (a block reduction) and the scaled store.
+constexpr int kGateThreads = 256, kGatePer = 16;  // rows up to 4096 channels stay in registers
+
 template <typename T>
-__global__ void gate_rmsnorm_kernel(const T* __restrict__ y, int64_t ldy, const T* __restrict__ z, int64_t ldz,
-                                    const T* __restrict__ w, float eps, int d, int rows, T* __restrict__ out,
-                                    int64_t ldo)
+__global__ void __launch_bounds__(kGateThreads) gate_rmsnorm_kernel(const T* __restrict__ y, int64_t ldy,
+                                                                    const T* __restrict__ z, int64_t ldz,
+                                                                    const T* __restrict__ w, float eps, int d,
+                                                                    T* __restrict__ out, int64_t ldo)
 {
-    const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
-    if (row >= rows) return;
+    __shared__ float wsum[kGateThreads / 32];
+    const int row = blockIdx.x;
     const T* yr = y + (int64_t)row * ldy;
     const T* zr = z + (int64_t)row * ldz;
+    T* orow = out + (int64_t)row * ldo;
+    float q[kGatePer];
     float ss = 0.0f;
-    for (int c = lane; c < d; c += 32) {
-        const float q = to_f32(yr[c]) * silu_f(to_f32(zr[c]));
-        ss = fmaf(q, q, ss);
+#pragma unroll
+    for (int i = 0; i < kGatePer; ++i) {
+        const int c = threadIdx.x + i * kGateThreads;
+        q[i] = 0.0f;
+        if (c < d) {
+            q[i] = to_f32(yr[c]) * silu_f(to_f32(zr[c]));
+            ss = fmaf(q[i], q[i], ss);
+        }
+    }
+    for (int c = threadIdx.x + kGatePer * kGateThreads; c < d; c += kGateThreads) {  // wider rows
+        const float v = to_f32(yr[c]) * silu_f(to_f32(zr[c]));
+        ss = fmaf(v, v, ss);
     }
 #pragma unroll
     for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    const float rstd = rsqrtf(ss / d + eps);
-    T* orow = out + (int64_t)row * ldo;
-    for (int c = lane; c < d; c += 32) {
-        const float q = to_f32(yr[c]) * silu_f(to_f32(zr[c]));
-        orow[c] = from_f32<T>(q * rstd * to_f32(w[c]));
+    if ((threadIdx.x & 31) == 0) wsum[threadIdx.x >> 5] = ss;
+    __syncthreads();
+    float tot = 0.0f;
+#pragma unroll
+    for (int j = 0; j < kGateThreads / 32; ++j) tot += wsum[j];
+    const float rstd = rsqrtf(tot / d + eps);
+#pragma unroll
+    for (int i = 0; i < kGatePer; ++i) {
+        const int c = threadIdx.x + i * kGateThreads;
+        if (c < d) orow[c] = from_f32<T>(q[i] * rstd * to_f32(w[c]));
+    }
+    for (int c = threadIdx.x + kGatePer * kGateThreads; c < d; c += kGateThreads) {
+        const float v = to_f32(yr[c]) * silu_f(to_f32(zr[c]));
+        orow[c] = from_f32<T>(v * rstd * to_f32(w[c]));
     }
 }
 
@@ -322,14 +347,13 @@ cudaError_t launch_gate_rmsnorm(int dtype, const void* y, int64_t ldy, const voi
                                 float eps, int d, int rows, void* out, int64_t ldo, cudaStream_t s)
 {
     if (rows == 0) return cudaSuccess;
-    dim3 grid((rows + 7) / 8);
     if (dtype == MM_BF16)
-        gate_rmsnorm_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
-            (const __nv_bfloat16*)y, ldy, (const __nv_bfloat16*)z, ldz, (const __nv_bfloat16*)w, eps, d, rows,
+        gate_rmsnorm_kernel<__nv_bfloat16><<<rows, kGateThreads, 0, s>>>(
+            (const __nv_bfloat16*)y, ldy, (const __nv_bfloat16*)z, ldz, (const __nv_bfloat16*)w, eps, d,
             (__nv_bfloat16*)out, ldo);
     else
-        gate_rmsnorm_kernel<float><<<grid, 256, 0, s>>>((const float*)y, ldy, (const float*)z, ldz, (const float*)w,
-                                                         eps, d, rows, (float*)out, ldo);
+        gate_rmsnorm_kernel<float><<<rows, kGateThreads, 0, s>>>((const float*)y, ldy, (const float*)z, ldz,
+                                                                  (const float*)w, eps, d, (float*)out, ldo);
     return cudaGetLastError();
 }
 
