@@ -41,7 +41,8 @@ struct TcSeg {
     int out_f32;
     int accumulate;
     int vec_ok;  // 16-byte vector stores allowed
-    int tma;     // bf16 tiles leave through bulk tensor stores (OutMaps::m[segment])
+    int tma;     // tiles leave through bulk tensor operations (OutMaps::m[segment]): 1 bf16 store,
+                 // 2 fp32 store, 3 fp32 add into the output (accumulate)
     int kind;    // GemmEpi
     int conv_row0;
 };
@@ -256,7 +257,45 @@ __global__ void __launch_bounds__(320, 1)
                          w_tp0 + w_n - 1 + 3 < ex.L;
             }
             const int64_t tile_row0 = (int64_t)t.mt * p.rows - p.shift;  // token of tile row 0
-            if (sg.tma && tile_row0 >= 0) {
+            if (sg.tma >= 2 && tile_row0 >= 0) {
+                // fp32 outputs: 32-column units (group eg takes units eg, eg + 2, ...), rows staged in
+                // the 128-byte-swizzled layout, then one bulk store or bulk add per unit.  Each output
+                // element gets exactly one add per launch, the same fp32 add as a read-modify-write.
+                uint8_t* stg = reinterpret_cast<uint8_t*>(stage) + eg * kGroupStage;
+                for (int u = eg; 32 * u < t.nvalid; u += 2) {
+                    asm volatile("bar.sync %0, 128;" ::"r"(2 + eg) : "memory");  // staging rows free
+                    if (ok) {
+                        uint32_t raw[32];
+                        tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + buf * BN + 32 * u, raw);
+                        tmem_ld_wait();
+                        float v[32];
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(raw[i]);
+                        if (ex.row_parts) {
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) v[i] *= scale;
+                        }
+#pragma unroll
+                        for (int c = 0; c < 8; ++c)
+                            *reinterpret_cast<float4*>(stg + r * 128 + ((c ^ (r & 7)) << 4)) =
+                                make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+                    }
+                    fence_async_smem();
+                    asm volatile("bar.sync %0, 128;" ::"r"(2 + eg) : "memory");
+                    if (ok && q == 2 && lane == 0) {  // one issuer per group
+                        if (sg.tma == 3) tma_reduce_add_2d(&omaps.m[t.seg], stg, t.n0 + 32 * u, (int)tile_row0);
+                        else tma_store_2d(&omaps.m[t.seg], stg, t.n0 + 32 * u, (int)tile_row0);
+                        bulk_commit();
+                        bulk_wait_read0();
+                    }
+                }
+                asm volatile("bar.sync %0, 128;" ::"r"(2 + eg) : "memory");  // last unit's rows read
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&tempty[buf]);
+                continue;
+            }
+            if (sg.tma == 1 && tile_row0 >= 0) {
                 // 64-column units (group eg takes units eg, eg + 2, ...): rows staged as bf16 in the
                 // 128-byte-swizzled layout, then one bulk store per unit.  Halo rows above the tile's
                 // outputs rewrite the identical values the previous row block wrote.
@@ -499,6 +538,21 @@ bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2-D fp32 tensor map with a 128-byte swizzle (box_inner * 4 bytes must be 128).
+static bool make_tmap_f32(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint64_t pitch,
+                          uint32_t box_inner, uint32_t box_rows)
+{
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {inner, rows};
+    cuuint64_t strides[1] = {pitch};
+    cuuint32_t box[2] = {box_inner, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // 3-D bf16 tensor map with a 128-byte swizzle: extents {inner, rows, planes}, `pitch` bytes
 // between rows and `plane_pitch` between planes, box of box_inner x box_rows x 1.  Rows past
 // `rows` inside a plane are outside the tensor, so a box that overhangs a plane is clipped there
@@ -557,11 +611,16 @@ static cudaError_t launch_bn(const GemmDesc& g, const TcParams& p0, cudaStream_t
     if (!make_tmap_bf16(&mapB, base, g.ldb, rows, g.ldb * 2, kBK, BN)) return cudaErrorInvalidValue;
     OutMaps om;
     std::memset(&om, 0, sizeof(om));
-    for (int i = 0; i < p.nseg; ++i) {  // plain bf16 outputs leave through bulk stores
+    for (int i = 0; i < p.nseg; ++i) {  // plain outputs leave through bulk stores (fp32: or bulk adds)
         TcSeg& t = p.seg[i];
         t.tma = 0;
-        if (t.kind == kEpiStore && !t.out_f32 && !t.accumulate && t.vec_ok)
+        if (t.kind != kEpiStore) continue;
+        if (!t.out_f32 && !t.accumulate && t.vec_ok)
             t.tma = make_tmap_bf16(&om.m[i], t.out, (uint64_t)t.n, (uint64_t)g.M, (uint64_t)t.ldo * 2, 64, kBM) ? 1 : 0;
+        else if (t.out_f32 && (reinterpret_cast<uintptr_t>(t.out) & 15u) == 0 && t.ldo % 4 == 0 &&
+                 (p.shift == 0 || !t.accumulate))  // halo rows are written twice: never add them twice
+            t.tma = make_tmap_f32(&om.m[i], t.out, (uint64_t)t.n, (uint64_t)g.M, (uint64_t)t.ldo * 4, 32, kBM)
+                        ? (t.accumulate ? 3 : 2) : 0;
     }
     constexpr int smem = STAGES * (kBM + BN) * kBK * 2 + (CONV ? 2 * kBM * kStageLd * 4 : 2 * kBM * 128) + 1024 + 256;
     static_assert(smem <= 232448, "GEMM configuration exceeds 227 KB of shared memory");
