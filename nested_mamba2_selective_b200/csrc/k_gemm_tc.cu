@@ -84,7 +84,14 @@ __device__ __forceinline__ TileInfo<BN> tile_info(const TcParams& p, int tile)
     return t;
 }
 
-__device__ __forceinline__ float silu_fast(float a) { return __fdividef(a, 1.0f + __expf(-a)); }
+// a / (1 + 2^(-a log2 e)) from the MUFU approximations of 2^x and 1/x; -0 for very negative a.
+__device__ __forceinline__ float silu_fast(float a)
+{
+    float e, r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(a * -1.4426950408889634f));
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(1.0f + e));
+    return a * r;
+}
 
 __device__ __forceinline__ void store_bf16_chunk(__nv_bfloat16* o, int ncols, bool vec, const float (&v)[32])
 {
@@ -365,6 +372,22 @@ __global__ void __launch_bounds__(320, 1)
                     // its two columns in registers.  Taps never cross a sequence start: the window
                     // restarts from the given history (or zeros) at token position 0.
                     float* st = stage + eg * (kBM * kStageLd);
+                    const int cp = lane & 15, rb = wrb;
+                    const int lc = 2 * cp;  // local column pair
+                    // this thread's two filters and biases: loaded before the staging so their latency
+                    // hides behind it and the barrier
+                    const bool fast = ok && lc + 1 < ncols && w_fast;
+                    uint2 wa = make_uint2(0, 0), wb = make_uint2(0, 0);
+                    __nv_bfloat16 bia = __float2bfloat16_rn(0.0f), bib = bia;
+                    if (fast) {
+                        const int crow = sg.conv_row0 + col + lc;
+                        const __nv_bfloat16* cw = static_cast<const __nv_bfloat16*>(ex.conv_w);
+                        const __nv_bfloat16* cbias = static_cast<const __nv_bfloat16*>(ex.conv_b);
+                        wa = *reinterpret_cast<const uint2*>(cw + (int64_t)crow * 4);
+                        wb = *reinterpret_cast<const uint2*>(cw + (int64_t)(crow + 1) * 4);
+                        bia = cbias[crow];
+                        bib = cbias[crow + 1];
+                    }
                     if (ok) {
 #pragma unroll
                         for (int c = 0; c < 8; ++c)
@@ -372,18 +395,11 @@ __global__ void __launch_bounds__(320, 1)
                                 make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
                     }
                     asm volatile("bar.sync %0, 128;" ::"r"(2 + eg) : "memory");
-                    const int cp = lane & 15, rb = wrb;
-                    const int lc = 2 * cp;  // local column pair
-                    if (ok && lc + 1 < ncols && w_fast) {
+                    if (fast) {
                         // all 16 rows are outputs of one sequence, history in the rows above
-                        const int crow = sg.conv_row0 + col + lc;
-                        const __nv_bfloat16* cw = static_cast<const __nv_bfloat16*>(ex.conv_w);
-                        const __nv_bfloat16* cbias = static_cast<const __nv_bfloat16*>(ex.conv_b);
-                        const uint2 wa = *reinterpret_cast<const uint2*>(cw + (int64_t)crow * 4);
-                        const uint2 wb = *reinterpret_cast<const uint2*>(cw + (int64_t)(crow + 1) * 4);
                         const float a0 = bf_lo_u(wa.x), a1 = bf_hi_u(wa.x), a2 = bf_lo_u(wa.y), a3 = bf_hi_u(wa.y);
                         const float b0 = bf_lo_u(wb.x), b1 = bf_hi_u(wb.x), b2 = bf_lo_u(wb.y), b3 = bf_hi_u(wb.y);
-                        const float biasa = __bfloat162float(cbias[crow]), biasb = __bfloat162float(cbias[crow + 1]);
+                        const float biasa = __bfloat162float(bia), biasb = __bfloat162float(bib);
                         // rows w_fr - 3 .. w_fr + 15 of the staged chunk (all inside the tile; the top
                         // walk reads three rows past its 13 outputs and ignores them)
                         const float* sr = st + (w_fr - 3) * kStageLd + lc;
