@@ -243,14 +243,6 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
                     mma_ss(tmem + kTG, desc_sw128(aC + off, 16, 1024), desc_sw128(aB + off, 16, 1024), id_g, kk > 0);
                 }
                 mma_commit(g_done);
-                // block k+1 goes into the stage block k-1 used, free once its epilogue has read x
-                if (loaded == k + 1 && loaded < nch) {
-                    if (!mbar_wait(&empty[loaded % kNStage], ((loaded / kNStage) & 1) ^ 1, abort)) {
-                        raise_timeout(abort, p.status);
-                        break;
-                    }
-                    load(loaded++);
-                }
                 if (!mbar_wait(h_ready, k & 1, abort)) {
                     raise_timeout(abort, p.status);
                     break;
@@ -263,6 +255,15 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
                            id_o, kk > 0);
                 }
                 mma_commit(yo_done);
+                // block k+1 goes into the stage block k-1 used, free once its epilogue has read x and
+                // its y tile has left (released after the read-back that h_ready waited for)
+                if (loaded == k + 1 && loaded < nch) {
+                    if (!mbar_wait(&empty[loaded % kNStage], ((loaded / kNStage) & 1) ^ 1, abort)) {
+                        raise_timeout(abort, p.status);
+                        break;
+                    }
+                    load(loaded++);
+                }
                 if (!mbar_wait(mx_ready, k & 1, abort)) {
                     raise_timeout(abort, p.status);
                     break;
@@ -454,6 +455,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
         if (head_ok && nch > 0 && c_begin * kQ + r < p.L) dt_next = p.dt[(tok0 + c_begin * kQ + r) * p.sdt + head];
         float c2_prev = 0.0f;
         bool ok = __all_sync(0xffffffffu, !*abort);
+        bool pending_release = false;  // the storing warp still owes the previous stage's release
 
         // Iteration k: decay scan of block k, epilogue of block k-1, read-back and X' of block k.
         // Every warp runs every iteration (named barrier 2 + hf); a failed wait skips work only.
@@ -565,15 +567,17 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
                         if (ok && head_ok && lane == 0) {
                             tma_store_3d(&mapY, sX, head * kP, tp0, b);
                             bulk_commit();
-                            bulk_wait_read0();
                         }
                         __syncwarp();
                     }
                 }
-                if (ok) {
+                // x of block k-1 is read.  The storing warp releases the stage only after its store
+                // has read the y tile, which it waits for after the read-back below.
+                if (ok && !(p.y_tma && q == 0)) {
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&empty[sp]);  // x of block k-1 is read (and the y tile sent)
+                    if (lane == 0) mbar_arrive(&empty[sp]);
                 }
+                pending_release = ok && p.y_tma && q == 0;
             }
             if (k == nch) break;
 
@@ -608,6 +612,14 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(h_ready);
+            }
+            if (pending_release) {  // the y tile of block k-1 has been read: release its stage
+                if (lane == 0) {
+                    bulk_wait_read0();
+                    mbar_arrive(&empty[(k - 1) % kNStage]);
+                }
+                __syncwarp();
+                pending_release = false;
             }
             if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&full[s], (k / kNStage) & 1, abort));
             if (ok) ok = __all_sync(0xffffffffu, mbar_wait(yo_done, k & 1, abort));  // H read: X' may go there
