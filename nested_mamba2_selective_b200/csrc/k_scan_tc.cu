@@ -138,7 +138,7 @@ constexpr float kDropMax = 100.0f;  // log2 units
 constexpr int kTabWtotS = 0, kTabWtotM = 16, kTabG = 32, kTabC = 288, kTabAnch = 544, kTabFlag = 552, kTabFloats = 560;
 constexpr int kOffTab = kOffHX + 2 * kTileQP;
 constexpr int kOffBar = kOffTab + kTabFloats * 4;
-constexpr int kChunkSmem = kOffBar + 10 * 8 + 16;
+constexpr int kChunkSmem = kOffBar + 11 * 8 + 16;
 static_assert(kChunkSmem <= 232448, "chunk scan exceeds the 227 KB of shared memory a CTA can have");
 
 __device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
@@ -159,8 +159,9 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
     uint64_t* h_ready = g_done + 1;
     uint64_t* yo_done = h_ready + 1;
     uint64_t* mx_ready = yo_done + 1;
-    uint64_t* ys_full = mx_ready + 1;
-    uint64_t* done = ys_full + 1;
+    uint64_t* ys_full = mx_ready + 1;  // all MMAs of the block done (Y, then S)
+    uint64_t* y_done = ys_full + 1;    // Y of the block done (S may still run)
+    uint64_t* done = y_done + 1;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
     volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -185,6 +186,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
         mbar_init(yo_done, 1);
         mbar_init(mx_ready, 15);  // 7 M-builder warps and 8 state warps
         mbar_init(ys_full, 1);
+        mbar_init(y_done, 1);
         mbar_init(done, 1);
         *abort = (smem_u32(sm) & 1023u) ? 1 : 0;  // tiles need 1024-byte alignment; never fault on it
         if (*abort) raise_timeout(abort, p.status);
@@ -269,16 +271,18 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
                     break;
                 }
                 tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)  // S += B^T . [X'_0 | X'_1] over the block's tokens
-                    mma_ss(tmem + kTS, desc_sw128(aB + kk * 2048, kTileQN / 2, 1024),
-                           desc_sw128(aHX + kk * 2048, kTileQP, 1024), id_s, 1u);
+                // Y first, so the epilogue can start while S still runs
 #pragma unroll
                 for (int j = 0; j < 2; ++j)
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)  // Y_j = M_j . X_j over the block's tokens
                         mma_ts(tmem + kTY + 64 * j, tmem + kTG + 32 * (kk >> 1) + 16 * j + 8 * (kk & 1),
                                desc_sw128(aX + j * kTileQP + kk * 2048, kTileQP, 1024), id_y, kk > 0);
+                mma_commit(y_done);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)  // S += B^T . [X'_0 | X'_1] over the block's tokens
+                    mma_ss(tmem + kTS, desc_sw128(aB + kk * 2048, kTileQN / 2, 1024),
+                           desc_sw128(aHX + kk * 2048, kTileQP, 1024), id_s, 1u);
                 mma_commit(ys_full);
             }
             // every issued load lands before the CTA exits (bounded; only the last two can be pending)
@@ -485,7 +489,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
             }
 
             if (k > 0) {  // ---- epilogue of block k-1 (TMEM loads are warp-collective)
-                if (ok) ok = __all_sync(0xffffffffu, mbar_wait(ys_full, (k - 1) & 1, abort));
+                if (ok) ok = __all_sync(0xffffffffu, mbar_wait(y_done, (k - 1) & 1, abort));
                 const int sp = (k - 1) % kNStage;
                 const int tp0 = (c_begin + k - 1) * kQ;
                 // x of block k-1 (this head); with bulk stores each thread overwrites its own row of
@@ -501,8 +505,8 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
                     __nv_bfloat16* yo = static_cast<__nv_bfloat16*>(p.y) + tok * p.sy + col;
                     float ssq[2] = {0.0f, 0.0f};
                     // z rows of this warp's 32 tokens, loaded four rows per instruction (coalesced) into
-                    // the warp's own 32 rows of the H / X' buffer, which is free until the read-back
-                    uint8_t* zs = myHX + 32 * q * 128;
+                    // this warp's 4 KB of block k-1's C tile, which no MMA reads any more
+                    uint8_t* zs = sm + sp * kStage + kOffC + hf * (kTileQN / 2) + 32 * q * 128;
                     if (p.z) {
 #pragma unroll
                         for (int i = 0; i < 8; ++i) {
@@ -571,17 +575,14 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
                         __syncwarp();
                     }
                 }
-                // x of block k-1 is read.  The storing warp releases the stage only after its store
-                // has read the y tile, which it waits for after the read-back below.
-                if (ok && !(p.y_tma && q == 0)) {
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&empty[sp]);
-                }
-                pending_release = ok && p.y_tma && q == 0;
+                // Block k-1's stage is released after the read-back below, which waits for its S MMA
+                // (S reads B there); the storing warp also waits for its store to read the y tile.
+                pending_release = ok;
             }
             if (k == nch) break;
 
             const int s = k % kNStage;
+            if (ok && k > 0) ok = __all_sync(0xffffffffu, mbar_wait(ys_full, (k - 1) & 1, abort));  // S done
             if (ok) {  // ---- read-back: H_k as bf16 for Y_off, 2^tot H_k back into TMEM
                 const float dec = ex2(tot);
                 const float2 dec2 = make_float2(dec, dec);
@@ -613,40 +614,44 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(h_ready);
             }
-            if (pending_release) {  // the y tile of block k-1 has been read: release its stage
+            if (pending_release) {  // block k-1 is done with its stage: release it
                 if (lane == 0) {
-                    bulk_wait_read0();
+                    if (p.y_tma && q == 0) bulk_wait_read0();  // the y tile has been read
                     mbar_arrive(&empty[(k - 1) % kNStage]);
                 }
                 __syncwarp();
                 pending_release = false;
             }
             if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&full[s], (k / kNStage) & 1, abort));
-            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(yo_done, k & 1, abort));  // H read: X' may go there
-            if (ok) {  // ---- X'_j[s=r, :] = 2^(tot - cs_r) dt_r x_j[r, :]
+            if (ok) {  // ---- X'_j[s=r, :] = 2^(tot - cs_r) dt_r x_j[r, :], formed while Y_off runs
                 const uint8_t* sX = sm + s * kStage + kOffX + hf * kTileQP;
                 const float wgt = ex2(tot - c2) * dtv;
                 const float2 w2 = make_float2(wgt, wgt);
+                uint4 xq[8];
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
                     const uint4 xv = *reinterpret_cast<const uint4*>(sX + sw128(r, c));
-                    uint4 o;
-                    o.x = pack2(mul2(bf2(xv.x), w2));
-                    o.y = pack2(mul2(bf2(xv.y), w2));
-                    o.z = pack2(mul2(bf2(xv.z), w2));
-                    o.w = pack2(mul2(bf2(xv.w), w2));
-                    *reinterpret_cast<uint4*>(myHX + sw128(r, c)) = o;
+                    xq[c].x = pack2(mul2(bf2(xv.x), w2));
+                    xq[c].y = pack2(mul2(bf2(xv.y), w2));
+                    xq[c].z = pack2(mul2(bf2(xv.z), w2));
+                    xq[c].w = pack2(mul2(bf2(xv.w), w2));
                 }
-                fence_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(mx_ready);
+                ok = __all_sync(0xffffffffu, mbar_wait(yo_done, k & 1, abort));  // H read: X' may go there
+                if (ok) {
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(myHX + sw128(r, c)) = xq[c];
+                    fence_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(mx_ready);
+                }
             }
             if (!ok) raise_timeout(abort, p.status);
             c2_prev = c2;
         }
 
         if (p.y_tma && q == 0 && lane == 0) bulk_wait0();  // this head's y tiles are in global memory
-        if (seg == p.nseg - 1 && p.final_state) {  // state after the last block (ys_full waited above)
+        if (seg == p.nseg - 1 && p.final_state) {  // state after the last block: its S MMA is done
+            if (ok && nch > 0) ok = __all_sync(0xffffffffu, mbar_wait(ys_full, (nch - 1) & 1, abort));
             ok = __all_sync(0xffffffffu, ok && !*abort);
             if (ok) {
                 float* dst = p.final_state + (int64_t)b * p.state_stride + (int64_t)head * PN;
