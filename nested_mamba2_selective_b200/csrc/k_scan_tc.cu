@@ -230,9 +230,10 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
             for (; loaded < nch && loaded < kNStage; ++loaded) load(loaded);
             for (int k = 0; k < nch; ++k) {
                 const int s = k % kNStage;
-                // stage k is loaded, and block k-1's MMAs (which read M from the G columns) are done
+                // stage k is loaded, and block k-1's Y MMAs (which read M from the G columns) are done;
+                // its S MMAs may still run, ahead of G in the tensor pipe
                 if (!mbar_wait(&full[s], (k / kNStage) & 1, abort) ||
-                    (k > 0 && !mbar_wait(ys_full, (k - 1) & 1, abort))) {
+                    (k > 0 && !mbar_wait(y_done, (k - 1) & 1, abort))) {
                     raise_timeout(abort, p.status);
                     break;
                 }
