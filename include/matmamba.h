@@ -69,8 +69,18 @@ typedef enum { MM_F32 = 0, MM_BF16 = 1 } mm_dtype;
  * paragraph: (d_inner, .) parameters keep their first d_i rows, (n_heads)
  * parameters their first h_i entries; B and C do not depend on d_inner and
  * stay whole).
- * Requirements: E % P == 0, H % G == 0, K == 4, N % 8 == 0, N <= 256;
- * bf16 also needs D_m % 64 == 0, P == 64 and all pointers 16-byte aligned.
+ * Requirements (else MM_ERR_SHAPE / MM_ERR_ALIGN / MM_ERR_NULL before any
+ * launch): E % P == 0, H % G == 0, 2 <= K <= 8, N % 8 == 0, N <= 256,
+ * norm_eps >= 0, no null weight pointer; bf16 also needs D_m % 8 == 0,
+ * P % 8 == 0 and W_in, W_out, norm_w 16-byte aligned.  A valid width m has
+ * 0 < m <= D_m, E*m divisible by D_m and d = E*m/D_m divisible by P
+ * (MM_ERR_INVALID_WIDTH otherwise).
+ * Which kernels run: bf16 blocks with K == 4, P == 64, N == 128, chunk a
+ * multiple of 128, conv_w 8-byte and norm_w 16-byte aligned take the fused
+ * tensor-core path (in_proj + conv + dt in one GEMM, scan + gate, out_proj +
+ * 1/RMS); everything else takes the unfused path: separate conv, gate and
+ * norm kernels on CUDA cores, with the tensor-core GEMM and scan where their
+ * shape rules hold (bf16) and CUDA-core GEMM and scan otherwise.
  */
 typedef struct mm_block_params {
     int d_model;

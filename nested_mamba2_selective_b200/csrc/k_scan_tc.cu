@@ -11,10 +11,12 @@
 // which unrolls the recurrence exactly.  The sequence is cut into segments of
 // whole blocks so that (batch, head, segment) CTAs fill the GPU:
 //   1. seg_state  : each segment's end state from a zero start (tcgen05)
-//   2. state_pass : segment start states by a short sequential combine
-//   3. chunk_scan : every segment from its true start state, carrying the
-//                   state across blocks in TMEM (tcgen05)
-// Only segment boundary states touch HBM.
+//   2. chunk_scan : every segment from its true start state (the initial state
+//                   carried over the earlier segments' end states at the CTA's
+//                   start), carrying the state across blocks in TMEM (tcgen05).
+//                   It is a programmatic dependent of seg_state: segment 0 needs
+//                   no carried state and may run beside it.
+// Only segment end states touch HBM.
 //
 // A CTA takes two heads of one (batch, segment) so that the B and C blocks and
 // G = C B^T are loaded and computed once per pair; the thread roles of the
