@@ -7,11 +7,15 @@
 // ("MatMamba: A Matryoshka State Space Model", nested sub-block paragraph:
 // W_x becomes W_x[0:d_i] by slicing along d_inner).
 //
-// CTA layout (320 threads): warp 0 issues TMA loads, warp 1 owns TMEM and
-// issues tcgen05.mma from one lane, warps 2-9 drain the accumulator in two
-// groups of four that take alternate 32-column chunks (one TMEM lane = one
-// output row per thread) and store.  Two TMEM accumulators let the drain of
-// tile i overlap the MMAs of tile i+1.
+// CTA layout (320 threads): warp 0 schedules tiles and issues TMA loads, warp 1
+// owns TMEM and issues tcgen05.mma from one lane, warps 2-9 drain the
+// accumulator in two groups of four that take alternate 32-column chunks (one
+// TMEM lane = one output row per thread) and store.  Two TMEM accumulators let
+// the drain of tile i overlap the MMAs of tile i+1.
+//
+// Scheduling: the grid has one CTA per tile, but a running CTA keeps taking the
+// tiles of CTAs that have not started yet (cluster launch control), so the SMs
+// that drain their tiles faster take more of them and all finish together.
 #include <cuda.h>
 
 #include <cstring>
@@ -31,6 +35,7 @@ __device__ __forceinline__ float bf_hi_u(uint32_t v) { return __uint_as_float(v 
 constexpr int kBM = 128;  // rows of a tile = TMEM lanes
 constexpr int kStageLd = 36;  // fp32 row pitch of the conv epilogue's staging buffer (32 columns + pad)
 constexpr int kBK = 64;   // one 128-byte swizzle atom of bf16 along K
+constexpr int kTileRing = 6;  // launch-control answers in flight (producer leads the drain by <= 4 tiles)
 
 struct TcSeg {
     void* out;
@@ -72,7 +77,7 @@ __device__ __forceinline__ TileInfo<BN> tile_info(const TcParams& p, int tile)
 {
     TileInfo<BN> t;
     // row-block major: the N tiles of a row block are consecutive, so CTAs working at the same
-    // time share its A rows in L2, and a CTA's walk (stride = grid) mixes the segments' kinds
+    // time share its A rows in L2
     t.mt = tile / p.ntiles;
     int j = tile % p.ntiles;
     int s = 0;
@@ -124,12 +129,16 @@ __global__ void __launch_bounds__(320, 1)
     // The same bytes (group g at g * kGroupStage) stage 64-column bf16 tiles for the bulk stores.
     constexpr int kGroupStage = CONV ? kBM * kStageLd * 4 : kBM * 128;  // both multiples of 1024
     float* stage = reinterpret_cast<float*>(smem + STAGES * STAGE_BYTES);
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES + 2 * kGroupStage);
+    // answers of the launch-control requests (one per tile position, kTileRing in flight at most)
+    uint4* cresp = reinterpret_cast<uint4*>(smem + STAGES * STAGE_BYTES + 2 * kGroupStage);
+    uint64_t* full = reinterpret_cast<uint64_t*>(cresp + kTileRing);
     uint64_t* empty = full + STAGES;
     uint64_t* tfull = empty + STAGES;
     uint64_t* tempty = tfull + 2;
     uint64_t* done = tempty + 2;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+    uint64_t* cfull = done + 1;          // answer j has landed
+    uint64_t* cempty = cfull + kTileRing;  // answer j has been read by the MMA lane and the 8 drain warps
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(cempty + kTileRing);
     volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -141,6 +150,10 @@ __global__ void __launch_bounds__(320, 1)
         for (int b = 0; b < 2; ++b) {
             mbar_init(&tfull[b], 1);
             mbar_init(&tempty[b], 8);
+        }
+        for (int j = 0; j < kTileRing; ++j) {
+            mbar_init(&cfull[j], 1);
+            mbar_init(&cempty[j], 9);
         }
         mbar_init(done, 1);
         *abort = 0;
@@ -157,11 +170,36 @@ __global__ void __launch_bounds__(320, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const int total = p.mtiles * p.ntiles;
+    // The tile of position j + 1 (`total` once the walk is over) from the scheduler's answer j;
+    // each reader then releases the answer's slot (the MMA lane alone, or a drain warp once all
+    // its lanes have read).  The wait ignores the abort flag, so every reader of an answer that
+    // landed follows the same tile sequence and the drain groups' named barriers stay in step.
+    auto next_tile = [&](int j, bool single) -> int {
+        const int cs = j % kTileRing;
+        bool got = mbar_wait(&cfull[cs], (j / kTileRing) & 1, nullptr);
+        if (!single) got = __all_sync(0xffffffffu, got);
+        const int nx = got ? clc_cancelled_x(&cresp[cs]) : -1;
+        if (!single) __syncwarp();
+        if (single || lane == 0) mbar_arrive(&cempty[cs]);
+        return nx < 0 ? total : nx;
+    };
 
     if (warp == 0) {
-        if (lane == 0) {  // ---------------- TMA producer
-            int it = 0;
-            for (int tile = blockIdx.x; tile < total && !*abort; tile += gridDim.x) {
+        if (lane == 0) {  // ---------------- tile scheduler and TMA producer
+            // Tile position 0 is this CTA's own index; the tile of position j + 1 is the index of a
+            // CTA that had not started yet, cancelled by a launch-control request made while tile j
+            // loads.  An answer that cancelled nothing ends the walk (the grid has one CTA per tile).
+            int it = 0, j = 0, tile = blockIdx.x;
+            bool asked = false;  // an answer is in flight
+            while (tile < total && !*abort) {
+                const int cs = j % kTileRing;
+                if (!mbar_wait(&cempty[cs], ((j / kTileRing) & 1) ^ 1, abort)) {
+                    raise_timeout(abort, p.status);
+                    break;
+                }
+                mbar_arrive_expect_tx(&cfull[cs], 16);
+                clc_try_cancel(&cresp[cs], &cfull[cs]);
+                asked = true;
                 const TileInfo<BN> t = tile_info<BN>(p, tile);
                 const int arow = t.mt * p.rows - p.shift;  // may be negative: rows above 0 load as zeros
                 for (int kt = 0; kt < p.ktiles; ++kt, ++it) {
@@ -175,14 +213,23 @@ __global__ void __launch_bounds__(320, 1)
                     tma_load_2d(sa, &mapA, &full[s], kt * kBK, arow);
                     tma_load_2d(sa + A_BYTES, &mapB, &full[s], kt * kBK, t.b_row);
                 }
+                if (!mbar_wait(&cfull[cs], (j / kTileRing) & 1, abort)) {
+                    raise_timeout(abort, p.status);
+                    break;
+                }
+                asked = false;
+                const int nx = clc_cancelled_x(&cresp[cs]);
+                tile = nx < 0 ? total : nx;
+                ++j;
             }
-            // every issued load lands before the CTA can exit (bounded)
-            for (int j = max(0, it - STAGES); j < it; ++j) mbar_wait(&full[j % STAGES], (j / STAGES) & 1, abort);
+            // the last answer and every issued load land before the CTA can exit (bounded)
+            if (asked) mbar_wait(&cfull[j % kTileRing], (j / kTileRing) & 1, nullptr);
+            for (int i = max(0, it - STAGES); i < it; ++i) mbar_wait(&full[i % STAGES], (i / STAGES) & 1, nullptr);
         }
     } else if (warp == 1) {
         if (lane == 0) {  // ---------------- MMA issuer
             int it = 0, tc = 0;
-            for (int tile = blockIdx.x; tile < total && !*abort; tile += gridDim.x, ++tc) {
+            for (int tile = blockIdx.x; tile < total && !*abort; ++tc) {
                 const TileInfo<BN> t = tile_info<BN>(p, tile);
                 const int buf = tc & 1;
                 if (!mbar_wait(&tempty[buf], ((tc >> 1) & 1) ^ 1, abort)) {
@@ -209,6 +256,7 @@ __global__ void __launch_bounds__(320, 1)
                     mma_commit(&empty[s]);
                 }
                 mma_commit(&tfull[buf]);
+                tile = next_tile(tc, true);
             }
             // every issued MMA has finished before TMEM can be released (bounded)
             mma_commit(done);
@@ -219,8 +267,8 @@ __global__ void __launch_bounds__(320, 1)
         const int eg = (warp - 2) >> 2;
         const int r = q * 32 + lane;  // tile row = TMEM lane
         const GemmExtra& ex = p.ex;
-        int tc = 0, nchunk_done = 0;
-        for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++tc) {
+        int tc = 0;
+        for (int tile = blockIdx.x; tile < total; tile = next_tile(tc++, false)) {
             const TileInfo<BN> t = tile_info<BN>(p, tile);
             const int buf = tc & 1;
             const TcSeg& sg = p.seg[t.seg];
@@ -243,25 +291,82 @@ __global__ void __launch_bounds__(320, 1)
                 }
                 scale = rsqrtf(ss * ex.rs_inv_n + ex.rs_eps);
             }
+            // Conv tiles: this thread's walk (rows [16 rb, 16 rb + 16) of the tile, rb = 2 q + lane / 16,
+            // outputs from w_fr on, past the tile's halo), the token of its first output, that token's
+            // position in its sequence, its valid outputs, and its path: 1 = every output's three
+            // history rows are earlier rows of the walk's window in the same sequence (and no output is
+            // one of the last K-1 of its sequence when the conv state is written), 2 = the walk meets a
+            // sequence start or the end of the tokens, 0 = anything else.  The filters and biases of
+            // the thread's column pair in each of its group's chunks are loaded before the accumulator
+            // wait, so that their latency hides behind it.
+            constexpr int kChunks = BN / 64;
+            const int wrb = 2 * q + (lane >> 4), wr0 = 16 * wrb;
+            const int w_fr = max(wr0, p.shift), w_n = wr0 + 16 - w_fr;
+            const int lc = 2 * (lane & 15);  // the walk's column pair within a chunk
+            int64_t w_m0 = 0;
+            int w_tp0 = 0, w_nout = 0, w_path = 0;
+            uint2 fwa[kChunks], fwb[kChunks];
+            uint32_t fbias[kChunks];
+            if (CONV && sg.kind == kEpiConv) {
+                w_m0 = (int64_t)t.mt * p.rows - p.shift + w_fr;
+                w_tp0 = (int)(((w_m0 % ex.L) + ex.L) % ex.L);
+                const int64_t left = (int64_t)p.M - w_m0;  // tokens from the walk's first output on
+                w_nout = left <= 0 ? 0 : (left < w_n ? (int)left : w_n);
+                const bool vec = sg.vec_ok && p.shift == 3 && w_m0 >= 0;
+                const int tail = ex.conv_state_out ? 3 : 0;
+                if (vec && w_nout == w_n && w_tp0 >= 3 && w_tp0 + w_n - 1 + tail < ex.L) w_path = 1;
+                else if (vec && ex.L >= 19 && w_nout > 0) w_path = 2;
+                const __nv_bfloat16* cw = static_cast<const __nv_bfloat16*>(ex.conv_w);
+                const __nv_bfloat16* cb = static_cast<const __nv_bfloat16*>(ex.conv_b);
+#pragma unroll
+                for (int j = 0; j < kChunks; ++j) {
+                    const int cc = 32 * eg + 64 * j + lc;  // tile column of the pair in chunk j
+                    fwa[j] = fwb[j] = make_uint2(0, 0);
+                    fbias[j] = 0;
+                    if (w_path && cc + 1 < t.nvalid) {
+                        const int crow = sg.conv_row0 + t.n0 + cc;
+                        fwa[j] = *reinterpret_cast<const uint2*>(cw + (int64_t)crow * 4);
+                        fwb[j] = *reinterpret_cast<const uint2*>(cw + (int64_t)(crow + 1) * 4);
+                        fbias[j] = (uint32_t)__bfloat16_as_ushort(cb[crow]) |
+                                   ((uint32_t)__bfloat16_as_ushort(cb[crow + 1]) << 16);
+                    }
+                }
+            }
+            // dt biases of the group's first 16-column chunk of a softplus tile, loaded before the wait
+            float dtb[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) dtb[i] = 0.0f;
+            if (sg.kind == kEpiSoftplus) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    if (16 * eg + i < t.nvalid) dtb[i] = ex.dt_bias[t.n0 + 16 * eg + i];
+            }
             // a failed wait skips this tile's work but keeps the group's named barriers in step
             const bool ok = __all_sync(0xffffffffu, mbar_wait(&tfull[buf], (tc >> 1) & 1, abort));
             if (!ok) raise_timeout(abort, p.status);
             tc_fence_after();
-            // Conv walk of this thread (rows [16 rb, 16 rb + 16) of the tile; output rows start at
-            // w_fr, past the tile's halo): the token of its first output row, that token's position
-            // in its sequence, and whether the walk can take the branch-free path: every output row
-            // is a valid token in the same sequence as its three history rows, and none is one of
-            // the last K-1 of its sequence (conv state output).
-            const int wrb = 2 * q + (lane >> 4), wr0 = 16 * wrb;
-            const int w_fr = max(wr0, p.shift), w_n = wr0 + 16 - w_fr;
-            int64_t w_m0 = 0;
-            int w_tp0 = 0;
-            bool w_fast = false;
-            if (CONV && sg.kind == kEpiConv) {
-                w_m0 = (int64_t)t.mt * p.rows - p.shift + w_fr;
-                w_tp0 = (int)(((w_m0 % ex.L) + ex.L) % ex.L);
-                w_fast = sg.vec_ok && p.shift == 3 && w_m0 >= 0 && w_m0 + w_n - 1 < p.M && w_tp0 >= 3 &&
-                         w_tp0 + w_n - 1 + 3 < ex.L;
+            if (sg.kind == kEpiSoftplus) {
+                // dt columns (a few dozen at most): 16-column chunks, group eg takes chunks eg, eg + 2, ...
+                for (int c0 = 16 * eg; c0 < t.nvalid; c0 += 32) {
+                    if (!ok) continue;
+                    uint32_t raw[16];
+                    tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + buf * BN + c0, raw);
+                    tmem_ld_wait();
+                    if (row_ok) {
+                        float* o = static_cast<float*>(sg.out) + m * sg.ldo + t.n0 + c0;
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            if (c0 + i < t.nvalid) {
+                                const float bias = c0 == 16 * eg ? dtb[i] : ex.dt_bias[t.n0 + c0 + i];
+                                const float a = __uint_as_float(raw[i]) + bias;
+                                o[i] = a > 20.0f ? a : log1pf(__expf(a));
+                            }
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&tempty[buf]);
+                continue;
             }
             const int64_t tile_row0 = (int64_t)t.mt * p.rows - p.shift;  // token of tile row 0
             if (sg.tma >= 2 && tile_row0 >= 0) {
@@ -347,7 +452,7 @@ __global__ void __launch_bounds__(320, 1)
                 if (lane == 0) mbar_arrive(&tempty[buf]);
                 continue;
             }
-            for (int c0 = 32 * eg; c0 < t.nvalid; c0 += 64, ++nchunk_done) {
+            for (int c0 = 32 * eg; c0 < t.nvalid; c0 += 64) {
                 float v[32];
                 if (ok) {
                     uint32_t raw[32];
@@ -367,26 +472,18 @@ __global__ void __launch_bounds__(320, 1)
                 const int col = t.n0 + c0;
                 if (CONV && sg.kind == kEpiConv) {
                     // The chunk goes through shared memory so that each thread can walk down the token
-                    // axis: thread (q, lane) takes columns 2 (lane % 16) and +1 over rows
-                    // [16 rb, 16 rb + 16), rb = 2 q + lane / 16, keeping the last three pre-conv values of
-                    // its two columns in registers.  Taps never cross a sequence start: the window
-                    // restarts from the given history (or zeros) at token position 0.
+                    // axis over its column pair, keeping a window of pre-conv values in registers.
+                    // Taps never cross a sequence start: there the window restarts from the given
+                    // history (or zeros).
                     float* st = stage + eg * (kBM * kStageLd);
-                    const int cp = lane & 15, rb = wrb;
-                    const int lc = 2 * cp;  // local column pair
-                    // this thread's two filters and biases: loaded before the staging so their latency
-                    // hides behind it and the barrier
-                    const bool fast = ok && lc + 1 < ncols && w_fast;
-                    uint2 wa = make_uint2(0, 0), wb = make_uint2(0, 0);
-                    __nv_bfloat16 bia = __float2bfloat16_rn(0.0f), bib = bia;
-                    if (fast) {
-                        const int crow = sg.conv_row0 + col + lc;
-                        const __nv_bfloat16* cw = static_cast<const __nv_bfloat16*>(ex.conv_w);
-                        const __nv_bfloat16* cbias = static_cast<const __nv_bfloat16*>(ex.conv_b);
-                        wa = *reinterpret_cast<const uint2*>(cw + (int64_t)crow * 4);
-                        wb = *reinterpret_cast<const uint2*>(cw + (int64_t)(crow + 1) * 4);
-                        bia = cbias[crow];
-                        bib = cbias[crow + 1];
+                    // this chunk's filters and biases; the next chunk's move to the front
+                    const uint2 wa = fwa[0], wb = fwb[0];
+                    const uint32_t bab = fbias[0];
+#pragma unroll
+                    for (int j = 0; j + 1 < kChunks; ++j) {
+                        fwa[j] = fwa[j + 1];
+                        fwb[j] = fwb[j + 1];
+                        fbias[j] = fbias[j + 1];
                     }
                     if (ok) {
 #pragma unroll
@@ -395,11 +492,10 @@ __global__ void __launch_bounds__(320, 1)
                                 make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
                     }
                     asm volatile("bar.sync %0, 128;" ::"r"(2 + eg) : "memory");
-                    if (fast) {
-                        // all 16 rows are outputs of one sequence, history in the rows above
+                    if (ok && lc + 1 < ncols && w_path) {
                         const float a0 = bf_lo_u(wa.x), a1 = bf_hi_u(wa.x), a2 = bf_lo_u(wa.y), a3 = bf_hi_u(wa.y);
                         const float b0 = bf_lo_u(wb.x), b1 = bf_hi_u(wb.x), b2 = bf_lo_u(wb.y), b3 = bf_hi_u(wb.y);
-                        const float biasa = __bfloat162float(bia), biasb = __bfloat162float(bib);
+                        const float biasa = bf_lo_u(bab), biasb = bf_hi_u(bab);
                         // rows w_fr - 3 .. w_fr + 15 of the staged chunk (all inside the tile; the top
                         // walk reads three rows past its 13 outputs and ignores them)
                         const float* sr = st + (w_fr - 3) * kStageLd + lc;
@@ -409,13 +505,69 @@ __global__ void __launch_bounds__(320, 1)
                         uint32_t* o = reinterpret_cast<uint32_t*>(static_cast<__nv_bfloat16*>(sg.out) + w_m0 * sg.ldo +
                                                                   col + lc);
                         const int64_t step = sg.ldo / 2;  // output row pitch in bf16 pairs
+                        if (w_path == 1) {
+                            // every output's taps are rows of the window
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            float oa = fmaf(a3, xw[i + 3].x, fmaf(a2, xw[i + 2].x, fmaf(a1, xw[i + 1].x, fmaf(a0, xw[i].x, biasa))));
-                            float ob = fmaf(b3, xw[i + 3].y, fmaf(b2, xw[i + 2].y, fmaf(b1, xw[i + 1].y, fmaf(b0, xw[i].y, biasb))));
-                            if (i < w_n) o[i * step] = pack_bf16(silu_fast(oa), silu_fast(ob));
+                            for (int i = 0; i < 16; ++i) {
+                                float oa = fmaf(a3, xw[i + 3].x, fmaf(a2, xw[i + 2].x, fmaf(a1, xw[i + 1].x, fmaf(a0, xw[i].x, biasa))));
+                                float ob = fmaf(b3, xw[i + 3].y, fmaf(b2, xw[i + 2].y, fmaf(b1, xw[i + 1].y, fmaf(b0, xw[i].y, biasb))));
+                                if (i < w_n) o[i * step] = pack_bf16(silu_fast(oa), silu_fast(ob));
+                            }
+                        } else {
+                            // A sequence whose first outputs reach into the history starts at output kst:
+                            // 0..2 tokens before the walk (kst = -position of the first output) or inside
+                            // it (one start at most: sequences are at least 19 tokens long).  Its history
+                            // (the K-1 pre-conv values before its first token, oldest first) comes from
+                            // the given conv state or is zero.
+                            const int L = ex.L;
+                            const int kst = w_tp0 < 3 ? -w_tp0 : (L - w_tp0 < w_nout ? L - w_tp0 : 16);
+                            const int crow = sg.conv_row0 + col + lc;
+                            float2 h0 = make_float2(0.f, 0.f), h1 = h0, h2 = h0;
+                            const __nv_bfloat16* cin = static_cast<const __nv_bfloat16*>(ex.conv_state_in);
+                            if (kst < 16 && cin) {
+                                const __nv_bfloat16* ha = cin + (((w_m0 + kst) / L) * ex.conv_rows + crow) * 3;
+                                h0 = make_float2(__bfloat162float(ha[0]), __bfloat162float(ha[3]));
+                                h1 = make_float2(__bfloat162float(ha[1]), __bfloat162float(ha[4]));
+                                h2 = make_float2(__bfloat162float(ha[2]), __bfloat162float(ha[5]));
+                            }
+                            // the three pre-conv values before output 0, oldest first
+                            float2 p3 = xw[0], p2 = xw[1], p1 = xw[2];
+                            if (kst == -1) {
+                                p3 = h1;
+                                p2 = h2;
+                            } else if (kst == -2) {
+                                p3 = h2;
+                            }
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) {
+                                if (i == kst) {
+                                    p3 = h0;
+                                    p2 = h1;
+                                    p1 = h2;
+                                }
+                                const float2 cur = xw[i + 3];
+                                float oa = fmaf(a3, cur.x, fmaf(a2, p1.x, fmaf(a1, p2.x, fmaf(a0, p3.x, biasa))));
+                                float ob = fmaf(b3, cur.y, fmaf(b2, p1.y, fmaf(b1, p2.y, fmaf(b0, p3.y, biasb))));
+                                if (i < w_nout) o[i * step] = pack_bf16(silu_fast(oa), silu_fast(ob));
+                                p3 = p2;
+                                p2 = p1;
+                                p1 = cur;
+                            }
+                            __nv_bfloat16* cout = static_cast<__nv_bfloat16*>(ex.conv_state_out);
+                            if (cout) {  // the last K-1 pre-conv inputs of each sequence ending in the walk
+#pragma unroll
+                                for (int sl = 0; sl < 3; ++sl) {
+                                    const int i = ((L - 3 + sl - w_tp0) % L + L) % L;  // output at position L-3+sl
+                                    if (i < w_nout) {
+                                        const int64_t bq = (w_m0 + i) / L;
+                                        const float2 xv = *reinterpret_cast<const float2*>(st + (w_fr + i) * kStageLd + lc);
+                                        cout[(bq * ex.conv_rows + crow) * 3 + sl] = __float2bfloat16_rn(xv.x);
+                                        cout[(bq * ex.conv_rows + crow + 1) * 3 + sl] = __float2bfloat16_rn(xv.y);
+                                    }
+                                }
+                            }
                         }
-                    } else if (ok && lc < ncols) {
+                    } else if (ok && lc < ncols && w_nout > 0) {
                         const int crow = sg.conv_row0 + col + lc;
                         const bool two = lc + 1 < ncols;
                         const __nv_bfloat16* cw = static_cast<const __nv_bfloat16*>(ex.conv_w);
@@ -429,7 +581,7 @@ __global__ void __launch_bounds__(320, 1)
                         const float biasa = __bfloat162float(cbias[crow]);
                         const float biasb = two ? __bfloat162float(cbias[crow + 1]) : 0.0f;
                         // window start: three rows above the block (inside the tile: rows >= 0)
-                        const int r0 = 16 * rb;
+                        const int r0 = wr0;
                         float xa3 = 0.f, xa2 = 0.f, xa1 = 0.f, xb3 = 0.f, xb2 = 0.f, xb1 = 0.f;
                         if (r0 >= 3) {
                             const float2 p3 = *reinterpret_cast<const float2*>(st + (r0 - 3) * kStageLd + lc);
@@ -487,15 +639,7 @@ __global__ void __launch_bounds__(320, 1)
                     }
                     asm volatile("bar.sync %0, 128;" ::"r"(2 + eg) : "memory");  // the stage buffer is free again
                 } else if (row_ok && ok) {
-                    if (sg.kind == kEpiSoftplus) {
-                        float* o = static_cast<float*>(sg.out) + m * sg.ldo + col;
-#pragma unroll
-                        for (int i = 0; i < 32; ++i)
-                            if (i < ncols) {
-                                const float a = v[i] + ex.dt_bias[col + i];
-                                o[i] = a > 20.0f ? a : log1pf(__expf(a));
-                            }
-                    } else if (sg.out_f32) {
+                    if (sg.out_f32) {
                         float* o = static_cast<float*>(sg.out) + m * sg.ldo + col;
 #pragma unroll
                         for (int i = 0; i < 32; ++i)
@@ -638,9 +782,9 @@ static cudaError_t launch_bn(const GemmDesc& g, const TcParams& p0, cudaStream_t
             t.tma = make_tmap_f32(&om.m[i], t.out, (uint64_t)t.n, (uint64_t)g.M, (uint64_t)t.ldo * 4, 32, kBM)
                         ? (t.accumulate ? 3 : 2) : 0;
     }
-    constexpr int smem = STAGES * (kBM + BN) * kBK * 2 + (CONV ? 2 * kBM * kStageLd * 4 : 2 * kBM * 128) + 1024 + 256;
+    constexpr int smem = STAGES * (kBM + BN) * kBK * 2 + (CONV ? 2 * kBM * kStageLd * 4 : 2 * kBM * 128) + 1024 + 512;
     static_assert(smem <= 232448, "GEMM configuration exceeds 227 KB of shared memory");
-    int dev = 0, sms = 148;
+    int dev = 0;
     cudaGetDevice(&dev);
     static unsigned long long attr_set = 0;  // one bit per device
     if (dev < 64 && !(attr_set >> dev & 1ull)) {
@@ -649,10 +793,8 @@ static cudaError_t launch_bn(const GemmDesc& g, const TcParams& p0, cudaStream_t
         if (e != cudaSuccess) return e;
         attr_set |= 1ull << dev;
     }
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int total = p.mtiles * p.ntiles;
-    const int grid = total < sms ? total : sms;
-    gemm_tc_kernel<BN, STAGES, CONV><<<grid, 320, smem, s>>>(mapA, mapB, om, p);
+    // one CTA per tile: the CTAs that start first take over the others' tiles as they go
+    gemm_tc_kernel<BN, STAGES, CONV><<<p.mtiles * p.ntiles, 320, smem, s>>>(mapA, mapB, om, p);
     return cudaGetLastError();
 }
 

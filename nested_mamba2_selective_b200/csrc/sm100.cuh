@@ -1,6 +1,7 @@
 // Thin wrappers over the sm_100a instructions used by the tensor-core kernels:
-// mbarriers (with time-bounded waits), TMA tile loads, and the tcgen05 family
-// (TMEM allocation, MMA issue/commit, TMEM loads and stores).  Descriptor bit
+// mbarriers (with time-bounded waits), TMA tile loads, the tcgen05 family
+// (TMEM allocation, MMA issue/commit, TMEM loads and stores), and cluster
+// launch control for dynamic tile scheduling.  Descriptor bit
 // layouts follow the PTX ISA's shared-memory descriptor and kind::f16
 // instruction descriptor tables.
 #pragma once
@@ -268,6 +269,36 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)
 
 // Order generic-proxy shared-memory writes before async-proxy (tcgen05/TMA) reads.
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// ------------------------------------------------------------------ cluster launch control
+
+// Ask the hardware to cancel one CTA of this grid that has not started yet, so that the
+// caller takes over its work.  The 16-byte answer is written to `resp` (shared, 16-byte
+// aligned) and completes 16 bytes of `bar`'s transaction count.  After an answer that
+// cancelled nothing, no further request may be made.
+__device__ __forceinline__ void clc_try_cancel(void* resp, uint64_t* bar)
+{
+    asm volatile("clusterlaunchcontrol.try_cancel.async.shared::cta.mbarrier::complete_tx::bytes.b128 [%0], [%1];" ::"r"(
+                     smem_u32(resp)),
+                 "r"(smem_u32(bar))
+                 : "memory");
+}
+
+// Decode an answer: the x index of the CTA it cancelled, or -1 if it cancelled none.
+__device__ __forceinline__ int clc_cancelled_x(const void* resp)
+{
+    int x;
+    asm volatile(
+        "{\n\t.reg .b128 r;\n\t.reg .pred p;\n\t"
+        "ld.shared.b128 r, [%1];\n\t"
+        "clusterlaunchcontrol.query_cancel.is_canceled.pred.b128 p, r;\n\t"
+        "mov.s32 %0, -1;\n\t"
+        "@p clusterlaunchcontrol.query_cancel.get_first_ctaid::x.b32.b128 %0, r;\n\t}"
+        : "=r"(x)
+        : "r"(smem_u32(resp))
+        : "memory");
+    return x;
+}
 
 }  // namespace sm100
 }  // namespace mm

@@ -52,3 +52,19 @@ def test_linear_fp32():
     out = mm_linear(torch.from_numpy(a).cuda(), torch.from_numpy(w).cuda())
     torch.cuda.synchronize()
     assert max_abs_rel(to_np(out), a.astype(np.float64) @ w.astype(np.float64).T) <= 1e-5
+
+
+@pytest.mark.parametrize("out_f32", [False, True])
+def test_linear_many_tiles_writes_every_tile_once(out_f32):
+    """Twelve times more tiles than SMs: running CTAs take over the tiles of CTAs that have not
+    started, and each tile must still be written (the output starts as NaN) with the plain value."""
+    M, K, N = 8192, 768, 3352
+    a = synth.activations((M, K), "bf16", seed=11)
+    w = synth.activations((N, K), "bf16", seed=12, std=0.05)
+    A, W = torch.from_numpy(a).cuda().bfloat16(), torch.from_numpy(w).cuda().bfloat16()
+    out = torch.full((M, N), float("nan"), dtype=torch.float32 if out_f32 else torch.bfloat16, device="cuda")
+    mm_linear(A, W, out=out, out_f32=out_f32)
+    torch.cuda.synchronize()
+    assert not torch.isnan(out).any()
+    ref = a.astype(np.float64) @ w.astype(np.float64).T
+    assert max_abs_rel(to_np(out), ref) <= (1e-5 if out_f32 else 5e-3)
