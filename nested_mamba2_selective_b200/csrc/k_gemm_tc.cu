@@ -1,6 +1,6 @@
 // Tensor-core projection GEMM for sm_100a: out = A . B^T with bf16 operands,
-// fp32 accumulation in TMEM, TMA-fed shared-memory stages, and a persistent
-// tile loop.  Serves in_proj (A = u, B = the four row blocks of the W_in
+// fp32 accumulation in TMEM, TMA-fed shared-memory stages, and a tile loop
+// per CTA.  Serves in_proj (A = u, B = the four row blocks of the W_in
 // width view, routed to z | x | B | C and an fp32 dt buffer) and out_proj
 // (A = normalised activations, B = W_out with its K-prefix [0, d)); the width
 // view is a set of row offsets and a K extent, never a weight copy
@@ -33,8 +33,8 @@ __device__ __forceinline__ float bf_lo_u(uint32_t v) { return __uint_as_float(v 
 __device__ __forceinline__ float bf_hi_u(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
 
 constexpr int kBM = 128;  // rows of a tile = TMEM lanes
-constexpr int kStageLd = 36;  // fp32 row pitch of the conv epilogue's staging buffer (32 columns + pad)
 constexpr int kBK = 64;   // one 128-byte swizzle atom of bf16 along K
+constexpr int kStageLd = 36;  // fp32 row pitch of the conv walks' staging rows (32 columns + pad)
 constexpr int kTileRing = 6;  // launch-control answers in flight (producer leads the drain by <= 4 tiles)
 
 struct TcSeg {
@@ -62,6 +62,11 @@ struct TcParams {
     int M, K, ktiles, mtiles, ntiles, nseg;
     int shift;  // halo rows at the top of each tile (K-1 with a conv segment, else 0)
     int rows;   // output rows per tile = 128 - shift
+    // Paired tiles (the first pair_tiles tiles of a row block): columns [n0, n0 + BN/2) of segment
+    // pair_a (a plain bf16 store) in accumulator columns [0, BN/2) and the same columns of segment
+    // pair_b (conv) in [BN/2, BN), so that every tile's drain mixes cheap stores and conv walks.
+    // Both segments then have ntiles = 0 in the walk over the rest.
+    int pair_tiles, pair_a, pair_b;
     TcSeg seg[kMaxSeg];
     GemmExtra ex;
     int* status;
@@ -70,6 +75,7 @@ struct TcParams {
 template <int BN>
 struct TileInfo {
     int mt, seg, n0, nvalid, b_row;
+    int seg2, b_row2;  // paired tile: the conv segment and its B row (else seg2 = -1)
 };
 
 template <int BN>
@@ -80,6 +86,18 @@ __device__ __forceinline__ TileInfo<BN> tile_info(const TcParams& p, int tile)
     // time share its A rows in L2
     t.mt = tile / p.ntiles;
     int j = tile % p.ntiles;
+    t.seg2 = -1;
+    t.b_row2 = 0;
+    if (j < p.pair_tiles) {
+        t.seg = p.pair_a;
+        t.seg2 = p.pair_b;
+        t.n0 = j * (BN / 2);
+        t.nvalid = min(BN / 2, p.seg[t.seg].n - t.n0);
+        t.b_row = p.seg[t.seg].b_row0 + t.n0;
+        t.b_row2 = p.seg[t.seg2].b_row0 + t.n0;
+        return t;
+    }
+    j -= p.pair_tiles;
     int s = 0;
     while (s < p.nseg - 1 && j >= p.seg[s].ntiles) j -= p.seg[s++].ntiles;
     t.seg = s;
@@ -116,7 +134,7 @@ __device__ __forceinline__ void store_bf16_chunk(__nv_bfloat16* o, int ncols, bo
 template <int BN, int STAGES, bool CONV>
 __global__ void __launch_bounds__(320, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
-                   const __grid_constant__ OutMaps omaps, const TcParams p)
+                   const __grid_constant__ CUtensorMap mapB2, const __grid_constant__ OutMaps omaps, const TcParams p)
 {
     constexpr int A_BYTES = kBM * kBK * 2;
     constexpr int B_BYTES = BN * kBK * 2;
@@ -125,8 +143,9 @@ __global__ void __launch_bounds__(320, 1)
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    // [2 epilogue groups][128 rows][kStageLd]: a 32-column chunk of fp32 accumulators for the conv epilogue.
-    // The same bytes (group g at g * kGroupStage) stage 64-column bf16 tiles for the bulk stores.
+    // Per drain group: [128 rows][kStageLd] fp32, a 32-column chunk of accumulators for the conv
+    // walks; the same bytes hold [128 rows][128 bytes] in the 128-byte swizzle (piece c of row r at
+    // c ^ (r % 8)), a 64-column bf16 (or 32-column fp32) unit for the bulk stores.
     constexpr int kGroupStage = CONV ? kBM * kStageLd * 4 : kBM * 128;  // both multiples of 1024
     float* stage = reinterpret_cast<float*>(smem + STAGES * STAGE_BYTES);
     // answers of the launch-control requests (one per tile position, kTileRing in flight at most)
@@ -160,6 +179,7 @@ __global__ void __launch_bounds__(320, 1)
         fence_mbar_init();
         prefetch_tmap(&mapA);
         prefetch_tmap(&mapB);
+        if (p.pair_tiles) prefetch_tmap(&mapB2);
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, TMEM_COLS);
@@ -211,7 +231,12 @@ __global__ void __launch_bounds__(320, 1)
                     uint8_t* sa = smem + s * STAGE_BYTES;
                     mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
                     tma_load_2d(sa, &mapA, &full[s], kt * kBK, arow);
-                    tma_load_2d(sa + A_BYTES, &mapB, &full[s], kt * kBK, t.b_row);
+                    if (t.seg2 >= 0) {  // two half-height boxes: the store rows, then the conv rows
+                        tma_load_2d(sa + A_BYTES, &mapB2, &full[s], kt * kBK, t.b_row);
+                        tma_load_2d(sa + A_BYTES + B_BYTES / 2, &mapB2, &full[s], kt * kBK, t.b_row2);
+                    } else {
+                        tma_load_2d(sa + A_BYTES, &mapB, &full[s], kt * kBK, t.b_row);
+                    }
                 }
                 if (!mbar_wait(&cfull[cs], (j / kTileRing) & 1, abort)) {
                     raise_timeout(abort, p.status);
@@ -238,7 +263,7 @@ __global__ void __launch_bounds__(320, 1)
                 }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem + buf * BN;
-                const int nmma = (t.nvalid + 15) & ~15;
+                const int nmma = t.seg2 >= 0 ? BN : (t.nvalid + 15) & ~15;
                 const uint32_t idesc = idesc_bf16(kBM, nmma, 0, 0);
                 for (int kt = 0; kt < p.ktiles; ++kt, ++it) {
                     const int s = it % STAGES;
@@ -272,6 +297,9 @@ __global__ void __launch_bounds__(320, 1)
             const TileInfo<BN> t = tile_info<BN>(p, tile);
             const int buf = tc & 1;
             const TcSeg& sg = p.seg[t.seg];
+            const bool paired = t.seg2 >= 0;
+            const TcSeg& cs = p.seg[paired ? t.seg2 : t.seg];  // the segment of the chunk loop's columns
+            const int cbase = paired ? BN / 2 : 0;            // and their first accumulator column
             const int64_t m = (int64_t)t.mt * p.rows - p.shift + r;  // token of this row
             const bool row_ok = r >= p.shift && m < p.M;
             // the row scale does not depend on the accumulator: its loads go out before the wait
@@ -291,47 +319,50 @@ __global__ void __launch_bounds__(320, 1)
                 }
                 scale = rsqrtf(ss * ex.rs_inv_n + ex.rs_eps);
             }
-            // Conv tiles: this thread's walk (rows [16 rb, 16 rb + 16) of the tile, rb = 2 q + lane / 16,
-            // outputs from w_fr on, past the tile's halo), the token of its first output, that token's
-            // position in its sequence, its valid outputs, and its path: 1 = every output's three
-            // history rows are earlier rows of the walk's window in the same sequence (and no output is
-            // one of the last K-1 of its sequence when the conv state is written), 2 = the walk meets a
-            // sequence start or the end of the tokens, 0 = anything else.  The filters and biases of
-            // the thread's column pair in each of its group's chunks are loaded before the accumulator
-            // wait, so that their latency hides behind it.
-            constexpr int kChunks = BN / 64;
+            // Conv tiles: this thread's walk stores outputs at rows [wr0, wr0 + 16) of the tile
+            // (wr0 = 16 rb, rb = 2 q + lane / 16) from a window of rows [wr0 - 3, wr0 + 16).  Outputs
+            // [w_ilo, w_ihi) are stored: the top walk's first rows are the tile's halo, and rows past
+            // the last token are no tokens.  w_m0, w_tp0: the token of row wr0 and its position in its
+            // sequence.  Path 1: every stored output's three history rows are earlier rows of its own
+            // sequence in the window (and none is one of the last K-1 of its sequence when the conv
+            // state is written); path 2: the walk meets a sequence start or the end of the tokens;
+            // path 0: anything else.
             const int wrb = 2 * q + (lane >> 4), wr0 = 16 * wrb;
-            const int w_fr = max(wr0, p.shift), w_n = wr0 + 16 - w_fr;
             const int lc = 2 * (lane & 15);  // the walk's column pair within a chunk
             int64_t w_m0 = 0;
-            int w_tp0 = 0, w_nout = 0, w_path = 0;
-            uint2 fwa[kChunks], fwb[kChunks];
-            uint32_t fbias[kChunks];
-            if (CONV && sg.kind == kEpiConv) {
-                w_m0 = (int64_t)t.mt * p.rows - p.shift + w_fr;
+            int w_tp0 = 0, w_ilo = 0, w_ihi = 0, w_path = 0;
+            if (CONV && cs.kind == kEpiConv) {
+                w_m0 = (int64_t)t.mt * p.rows - p.shift + wr0;
                 w_tp0 = (int)(((w_m0 % ex.L) + ex.L) % ex.L);
-                const int64_t left = (int64_t)p.M - w_m0;  // tokens from the walk's first output on
-                w_nout = left <= 0 ? 0 : (left < w_n ? (int)left : w_n);
-                const bool vec = sg.vec_ok && p.shift == 3 && w_m0 >= 0;
+                w_ilo = wr0 < p.shift ? p.shift - wr0 : 0;
+                const int64_t left = (int64_t)p.M - w_m0;  // tokens from row wr0 on
+                w_ihi = left <= 0 ? 0 : (left < 16 ? (int)left : 16);
+                const int tpf = (w_tp0 + w_ilo) % ex.L;  // position of the first stored output
+                const bool vec = cs.vec_ok && p.shift == 3;
                 const int tail = ex.conv_state_out ? 3 : 0;
-                if (vec && w_nout == w_n && w_tp0 >= 3 && w_tp0 + w_n - 1 + tail < ex.L) w_path = 1;
-                else if (vec && ex.L >= 19 && w_nout > 0) w_path = 2;
-                const __nv_bfloat16* cw = static_cast<const __nv_bfloat16*>(ex.conv_w);
-                const __nv_bfloat16* cb = static_cast<const __nv_bfloat16*>(ex.conv_b);
-#pragma unroll
-                for (int j = 0; j < kChunks; ++j) {
-                    const int cc = 32 * eg + 64 * j + lc;  // tile column of the pair in chunk j
-                    fwa[j] = fwb[j] = make_uint2(0, 0);
-                    fbias[j] = 0;
-                    if (w_path && cc + 1 < t.nvalid) {
-                        const int crow = sg.conv_row0 + t.n0 + cc;
-                        fwa[j] = *reinterpret_cast<const uint2*>(cw + (int64_t)crow * 4);
-                        fwb[j] = *reinterpret_cast<const uint2*>(cw + (int64_t)(crow + 1) * 4);
-                        fbias[j] = (uint32_t)__bfloat16_as_ushort(cb[crow]) |
-                                   ((uint32_t)__bfloat16_as_ushort(cb[crow + 1]) << 16);
-                    }
-                }
+                if (vec && w_ihi == 16 && tpf >= 3 && tpf + (15 - w_ilo) + tail < ex.L) w_path = 1;
+                else if (vec && ex.L >= 19 && w_ihi > w_ilo) w_path = 2;
             }
+            // filters and biases of the pair in the group's chunk j (zeros when the walk does not use them)
+            auto load_filters = [&](int j, uint2& fa, uint2& fb, uint32_t& fbi) {
+                const int cc = 32 * eg + 64 * j + lc;  // column of the pair in the chunk loop's columns
+                fa = fb = make_uint2(0, 0);
+                fbi = 0;
+                if (CONV && cs.kind == kEpiConv && w_path && cc + 1 < t.nvalid) {
+                    const __nv_bfloat16* cw = static_cast<const __nv_bfloat16*>(ex.conv_w);
+                    const __nv_bfloat16* cb = static_cast<const __nv_bfloat16*>(ex.conv_b);
+                    const int crow = cs.conv_row0 + t.n0 + cc;
+                    fa = *reinterpret_cast<const uint2*>(cw + (int64_t)crow * 4);
+                    fb = *reinterpret_cast<const uint2*>(cw + (int64_t)(crow + 1) * 4);
+                    fbi = (uint32_t)__bfloat16_as_ushort(cb[crow]) | ((uint32_t)__bfloat16_as_ushort(cb[crow + 1]) << 16);
+                }
+            };
+            // the first two chunks' filters go out before the accumulator wait; each chunk then
+            // fetches the filters of the chunk after next
+            uint2 fwa[2], fwb[2];
+            uint32_t fbias[2];
+            load_filters(0, fwa[0], fwb[0], fbias[0]);
+            load_filters(1, fwa[1], fwb[1], fbias[1]);
             // dt biases of the group's first 16-column chunk of a softplus tile, loaded before the wait
             float dtb[16];
 #pragma unroll
@@ -410,7 +441,8 @@ __global__ void __launch_bounds__(320, 1)
             if (sg.tma == 1 && tile_row0 >= 0) {
                 // 64-column units (group eg takes units eg, eg + 2, ...): rows staged as bf16 in the
                 // 128-byte-swizzled layout, then one bulk store per unit.  Halo rows above the tile's
-                // outputs rewrite the identical values the previous row block wrote.
+                // outputs rewrite the identical values the previous row block wrote.  A paired tile
+                // stores its first half this way and goes on to its conv half.
                 uint8_t* stg = reinterpret_cast<uint8_t*>(stage) + eg * kGroupStage;
                 for (int u = eg; 64 * u < t.nvalid; u += 2) {
                     // the previous unit's store has read the staging rows (its issuer waited)
@@ -447,16 +479,31 @@ __global__ void __launch_bounds__(320, 1)
                 }
                 // the last store has read the staging rows before the group writes them again
                 asm volatile("bar.sync %0, 128;" ::"r"(2 + eg) : "memory");
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&tempty[buf]);
-                continue;
+                if (!paired) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&tempty[buf]);
+                    continue;
+                }
+            } else if (paired) {  // first half of a paired tile at the top row block: plain stores
+                for (int c0 = 32 * eg; c0 < t.nvalid; c0 += 64) {
+                    if (!ok) continue;
+                    uint32_t raw[32];
+                    tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + buf * BN + c0, raw);
+                    tmem_ld_wait();
+                    float v[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(raw[i]);
+                    if (row_ok)
+                        store_bf16_chunk(static_cast<__nv_bfloat16*>(sg.out) + m * sg.ldo + t.n0 + c0,
+                                         min(32, t.nvalid - c0), sg.vec_ok, v);
+                }
             }
             for (int c0 = 32 * eg; c0 < t.nvalid; c0 += 64) {
                 float v[32];
                 if (ok) {
                     uint32_t raw[32];
-                    tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + buf * BN + c0, raw);
+                    tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + buf * BN + cbase + c0, raw);
                     tmem_ld_wait();
 #pragma unroll
                     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(raw[i]);
@@ -470,21 +517,23 @@ __global__ void __launch_bounds__(320, 1)
                 }
                 const int ncols = min(32, t.nvalid - c0);
                 const int col = t.n0 + c0;
-                if (CONV && sg.kind == kEpiConv) {
+                if (CONV && cs.kind == kEpiConv) {
                     // The chunk goes through shared memory so that each thread can walk down the token
                     // axis over its column pair, keeping a window of pre-conv values in registers.
                     // Taps never cross a sequence start: there the window restarts from the given
                     // history (or zeros).
                     float* st = stage + eg * (kBM * kStageLd);
+                    // the pre-conv values of columns lc, lc + 1 (lc even) in row `row` of the chunk
+                    auto xat = [st](int row, int lc2) -> float2 {
+                        return *reinterpret_cast<const float2*>(st + row * kStageLd + lc2);
+                    };
                     // this chunk's filters and biases; the next chunk's move to the front
                     const uint2 wa = fwa[0], wb = fwb[0];
                     const uint32_t bab = fbias[0];
-#pragma unroll
-                    for (int j = 0; j + 1 < kChunks; ++j) {
-                        fwa[j] = fwa[j + 1];
-                        fwb[j] = fwb[j + 1];
-                        fbias[j] = fbias[j + 1];
-                    }
+                    fwa[0] = fwa[1];
+                    fwb[0] = fwb[1];
+                    fbias[0] = fbias[1];
+                    load_filters((c0 - 32 * eg) / 64 + 2, fwa[1], fwb[1], fbias[1]);
                     if (ok) {
 #pragma unroll
                         for (int c = 0; c < 8; ++c)
@@ -496,32 +545,35 @@ __global__ void __launch_bounds__(320, 1)
                         const float a0 = bf_lo_u(wa.x), a1 = bf_hi_u(wa.x), a2 = bf_lo_u(wa.y), a3 = bf_hi_u(wa.y);
                         const float b0 = bf_lo_u(wb.x), b1 = bf_hi_u(wb.x), b2 = bf_lo_u(wb.y), b3 = bf_hi_u(wb.y);
                         const float biasa = bf_lo_u(bab), biasb = bf_hi_u(bab);
-                        // rows w_fr - 3 .. w_fr + 15 of the staged chunk (all inside the tile; the top
-                        // walk reads three rows past its 13 outputs and ignores them)
-                        const float* sr = st + (w_fr - 3) * kStageLd + lc;
+                        // the window, rows wr0 - 3 .. wr0 + 15 of the staged chunk.  The top walk's rows
+                        // -3..-1 lie before the group's staging rows (still inside the CTA's shared
+                        // memory) and feed only its halo outputs, which are not stored.
+                        const float* wbase = st + (wr0 - 3) * kStageLd + lc;
                         float2 xw[19];
 #pragma unroll
-                        for (int i = 0; i < 19; ++i) xw[i] = *reinterpret_cast<const float2*>(sr + i * kStageLd);
-                        uint32_t* o = reinterpret_cast<uint32_t*>(static_cast<__nv_bfloat16*>(sg.out) + w_m0 * sg.ldo +
-                                                                  col + lc);
-                        const int64_t step = sg.ldo / 2;  // output row pitch in bf16 pairs
+                        for (int i = 0; i < 19; ++i) xw[i] = *reinterpret_cast<const float2*>(wbase + i * kStageLd);
+                        // output i goes to row (i - w_ilo) from the first stored one
+                        uint32_t* o = reinterpret_cast<uint32_t*>(static_cast<__nv_bfloat16*>(cs.out) +
+                                                                  (w_m0 + w_ilo) * cs.ldo + col + lc);
+                        const int64_t step = cs.ldo / 2;  // output row pitch in bf16 pairs
                         if (w_path == 1) {
                             // every output's taps are rows of the window
 #pragma unroll
                             for (int i = 0; i < 16; ++i) {
                                 float oa = fmaf(a3, xw[i + 3].x, fmaf(a2, xw[i + 2].x, fmaf(a1, xw[i + 1].x, fmaf(a0, xw[i].x, biasa))));
                                 float ob = fmaf(b3, xw[i + 3].y, fmaf(b2, xw[i + 2].y, fmaf(b1, xw[i + 1].y, fmaf(b0, xw[i].y, biasb))));
-                                if (i < w_n) o[i * step] = pack_bf16(silu_fast(oa), silu_fast(ob));
+                                if (i >= w_ilo) o[(i - w_ilo) * step] = pack_bf16(silu_fast(oa), silu_fast(ob));
                             }
                         } else {
                             // A sequence whose first outputs reach into the history starts at output kst:
-                            // 0..2 tokens before the walk (kst = -position of the first output) or inside
-                            // it (one start at most: sequences are at least 19 tokens long).  Its history
-                            // (the K-1 pre-conv values before its first token, oldest first) comes from
-                            // the given conv state or is zero.
+                            // up to 2 rows before the first stored output, or after it (one start at most:
+                            // sequences are at least 19 tokens long).  Its history (the K-1 pre-conv values
+                            // before its first token, oldest first) comes from the given conv state or is
+                            // zero.
                             const int L = ex.L;
-                            const int kst = w_tp0 < 3 ? -w_tp0 : (L - w_tp0 < w_nout ? L - w_tp0 : 16);
-                            const int crow = sg.conv_row0 + col + lc;
+                            const int tpf = (w_tp0 + w_ilo) % L;
+                            const int kst = tpf < 3 ? w_ilo - tpf : (L - tpf < w_ihi - w_ilo ? w_ilo + L - tpf : 16);
+                            const int crow = cs.conv_row0 + col + lc;
                             float2 h0 = make_float2(0.f, 0.f), h1 = h0, h2 = h0;
                             const __nv_bfloat16* cin = static_cast<const __nv_bfloat16*>(ex.conv_state_in);
                             if (kst < 16 && cin) {
@@ -548,7 +600,7 @@ __global__ void __launch_bounds__(320, 1)
                                 const float2 cur = xw[i + 3];
                                 float oa = fmaf(a3, cur.x, fmaf(a2, p1.x, fmaf(a1, p2.x, fmaf(a0, p3.x, biasa))));
                                 float ob = fmaf(b3, cur.y, fmaf(b2, p1.y, fmaf(b1, p2.y, fmaf(b0, p3.y, biasb))));
-                                if (i < w_nout) o[i * step] = pack_bf16(silu_fast(oa), silu_fast(ob));
+                                if (i >= w_ilo && i < w_ihi) o[(i - w_ilo) * step] = pack_bf16(silu_fast(oa), silu_fast(ob));
                                 p3 = p2;
                                 p2 = p1;
                                 p1 = cur;
@@ -558,17 +610,17 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
                                 for (int sl = 0; sl < 3; ++sl) {
                                     const int i = ((L - 3 + sl - w_tp0) % L + L) % L;  // output at position L-3+sl
-                                    if (i < w_nout) {
+                                    if (i >= w_ilo && i < w_ihi) {
                                         const int64_t bq = (w_m0 + i) / L;
-                                        const float2 xv = *reinterpret_cast<const float2*>(st + (w_fr + i) * kStageLd + lc);
+                                        const float2 xv = xat(wr0 + i, lc);
                                         cout[(bq * ex.conv_rows + crow) * 3 + sl] = __float2bfloat16_rn(xv.x);
                                         cout[(bq * ex.conv_rows + crow + 1) * 3 + sl] = __float2bfloat16_rn(xv.y);
                                     }
                                 }
                             }
                         }
-                    } else if (ok && lc < ncols && w_nout > 0) {
-                        const int crow = sg.conv_row0 + col + lc;
+                    } else if (ok && lc < ncols && w_ihi > w_ilo) {
+                        const int crow = cs.conv_row0 + col + lc;
                         const bool two = lc + 1 < ncols;
                         const __nv_bfloat16* cw = static_cast<const __nv_bfloat16*>(ex.conv_w);
                         const __nv_bfloat16* cbias = static_cast<const __nv_bfloat16*>(ex.conv_b);
@@ -584,9 +636,9 @@ __global__ void __launch_bounds__(320, 1)
                         const int r0 = wr0;
                         float xa3 = 0.f, xa2 = 0.f, xa1 = 0.f, xb3 = 0.f, xb2 = 0.f, xb1 = 0.f;
                         if (r0 >= 3) {
-                            const float2 p3 = *reinterpret_cast<const float2*>(st + (r0 - 3) * kStageLd + lc);
-                            const float2 p2 = *reinterpret_cast<const float2*>(st + (r0 - 2) * kStageLd + lc);
-                            const float2 p1 = *reinterpret_cast<const float2*>(st + (r0 - 1) * kStageLd + lc);
+                            const float2 p3 = xat(r0 - 3, lc);
+                            const float2 p2 = xat(r0 - 2, lc);
+                            const float2 p1 = xat(r0 - 1, lc);
                             xa3 = p3.x; xb3 = p3.y; xa2 = p2.x; xb2 = p2.y; xa1 = p1.x; xb1 = p1.y;
                         }
                         int64_t m_r = (int64_t)t.mt * p.rows - p.shift + r0;  // token of row r0
@@ -594,7 +646,7 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll 4
                         for (int i = 0; i < 16; ++i, ++m_r) {
                             const int rr = r0 + i;
-                            const float2 xv = *reinterpret_cast<const float2*>(st + rr * kStageLd + lc);
+                            const float2 xv = xat(rr, lc);
                             if (tp == 0) {  // sequence start: history from the given state, or zeros
                                 const int64_t bq = m_r / ex.L;
                                 if (cin && m_r >= 0 && m_r < p.M) {
@@ -614,7 +666,7 @@ __global__ void __launch_bounds__(320, 1)
                                 float ob = fmaf(b3, xv.y, fmaf(b2, xb1, fmaf(b1, xb2, fmaf(b0, xb3, biasb))));
                                 oa = silu_fast(oa);
                                 ob = silu_fast(ob);
-                                __nv_bfloat16* o = static_cast<__nv_bfloat16*>(sg.out) + m_r * sg.ldo + col + lc;
+                                __nv_bfloat16* o = static_cast<__nv_bfloat16*>(cs.out) + m_r * cs.ldo + col + lc;
                                 if (two) *reinterpret_cast<uint32_t*>(o) = pack_bf16(oa, ob);
                                 else *o = __float2bfloat16_rn(oa);
                                 if (cout && tp >= ex.L - 3) {  // last K-1 pre-conv inputs of the sequence
@@ -757,18 +809,36 @@ template <int BN, int STAGES, bool CONV>
 static cudaError_t launch_bn(const GemmDesc& g, const TcParams& p0, cudaStream_t s, int* status)
 {
     TcParams p = p0;
-    p.ntiles = 0;
+    // Pair the conv columns of in_proj with the plain store columns of the same width: every
+    // tile then drains half cheap stores and half conv walks, instead of alternating tiles whose
+    // drains differ threefold (with two accumulators, the slow drains would hold up the MMAs).
+    p.pair_tiles = 0;
+    p.pair_a = p.pair_b = 0;
+    if (CONV && BN == 256) {
+        for (int a = 0; a < p.nseg && !p.pair_tiles; ++a)
+            for (int b = 0; b < p.nseg; ++b)
+                if (p.seg[a].kind == kEpiStore && !p.seg[a].out_f32 && !p.seg[a].accumulate &&
+                    p.seg[b].kind == kEpiConv && p.seg[a].n == p.seg[b].n) {
+                    p.pair_a = a;
+                    p.pair_b = b;
+                    p.pair_tiles = (p.seg[a].n + BN / 2 - 1) / (BN / 2);
+                    break;
+                }
+    }
+    p.ntiles = p.pair_tiles;
     for (int i = 0; i < p.nseg; ++i) {
-        p.seg[i].ntiles = (p.seg[i].n + BN - 1) / BN;
+        const bool in_pair = p.pair_tiles && (i == p.pair_a || i == p.pair_b);
+        p.seg[i].ntiles = in_pair ? 0 : (p.seg[i].n + BN - 1) / BN;
         p.ntiles += p.seg[i].ntiles;
     }
     p.status = status;
     const char* base = static_cast<const char*>(g.seg[0].B);
     int64_t rows = 0;
     for (int i = 0; i < p.nseg; ++i) rows = max(rows, (int64_t)p.seg[i].b_row0 + p.seg[i].n);
-    CUtensorMap mapA, mapB;
+    CUtensorMap mapA, mapB, mapB2;
     if (!make_tmap_bf16(&mapA, g.A, g.K, g.M, g.lda * 2, kBK, kBM)) return cudaErrorInvalidValue;
     if (!make_tmap_bf16(&mapB, base, g.ldb, rows, g.ldb * 2, kBK, BN)) return cudaErrorInvalidValue;
+    if (!make_tmap_bf16(&mapB2, base, g.ldb, rows, g.ldb * 2, kBK, BN / 2)) return cudaErrorInvalidValue;
     OutMaps om;
     std::memset(&om, 0, sizeof(om));
     for (int i = 0; i < p.nseg; ++i) {  // plain outputs leave through bulk stores (fp32: or bulk adds)
@@ -794,7 +864,7 @@ static cudaError_t launch_bn(const GemmDesc& g, const TcParams& p0, cudaStream_t
         attr_set |= 1ull << dev;
     }
     // one CTA per tile: the CTAs that start first take over the others' tiles as they go
-    gemm_tc_kernel<BN, STAGES, CONV><<<p.mtiles * p.ntiles, 320, smem, s>>>(mapA, mapB, om, p);
+    gemm_tc_kernel<BN, STAGES, CONV><<<p.mtiles * p.ntiles, 320, smem, s>>>(mapA, mapB, mapB2, om, p);
     return cudaGetLastError();
 }
 
