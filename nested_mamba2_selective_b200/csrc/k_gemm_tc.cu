@@ -131,14 +131,18 @@ __device__ __forceinline__ void store_bf16_chunk(__nv_bfloat16* o, int ncols, bo
     }
 }
 
-template <int BN, int STAGES, bool CONV>
+// PAIR: the kernel runs as clusters of two CTAs sharing each MMA (M = 256 over the pair).  CTA r
+// of a cluster takes row block 2 m + r of tile pair (m, j), loads its own A rows and half of the
+// tile's B rows (the first half in the even CTA, the second in the odd one), and drains its own
+// accumulator rows; the even CTA issues the MMAs.  The walk over tile pairs is static.
+template <int BN, int STAGES, bool CONV, bool PAIR>
 __global__ void __launch_bounds__(320, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
                    const __grid_constant__ CUtensorMap mapB2, const __grid_constant__ OutMaps omaps, const TcParams p)
 {
     constexpr int A_BYTES = kBM * kBK * 2;
     constexpr int B_BYTES = BN * kBK * 2;
-    constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    constexpr int STAGE_BYTES = A_BYTES + (PAIR ? B_BYTES / 2 : B_BYTES);  // this CTA's bytes of a stage
     constexpr uint32_t TMEM_COLS = 2 * BN;
 
     extern __shared__ uint8_t smem_raw[];
@@ -161,14 +165,15 @@ __global__ void __launch_bounds__(320, 1)
     volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = PAIR ? cluster_ctarank() : 0;  // 0 issues the pair's MMAs
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&full[s], 1);
+            mbar_init(&full[s], PAIR ? 2 : 1);  // the pair: both producers arrive on the even CTA's
             mbar_init(&empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&tfull[b], 1);
-            mbar_init(&tempty[b], 8);
+            mbar_init(&tempty[b], PAIR ? 16 : 8);  // the pair: both CTAs' drain warps
         }
         for (int j = 0; j < kTileRing; ++j) {
             mbar_init(&cfull[j], 1);
@@ -182,14 +187,31 @@ __global__ void __launch_bounds__(320, 1)
         if (p.pair_tiles) prefetch_tmap(&mapB2);
     }
     if (warp == 1) {
-        tmem_alloc(tmem_slot, TMEM_COLS);
-        tmem_relinquish();
+        if (PAIR) {
+            tmem_alloc_pair(tmem_slot, TMEM_COLS);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(tmem_slot, TMEM_COLS);
+            tmem_relinquish();
+        }
     }
     tc_fence_before();
     __syncthreads();
+    if (PAIR) cluster_sync();  // both CTAs' barriers are initialised before any arrives on them
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const int total = p.mtiles * p.ntiles;
+    // the pair's static walk: tile pair tp = (row-block pair tp / ntiles, N tile tp % ntiles)
+    const int total_pairs = ((p.mtiles + 1) / 2) * p.ntiles;
+    const int ncl = (int)gridDim.x / 2, cl = (int)blockIdx.x / 2;
+    auto pair_tile = [&](int tp) -> int { return ((tp / p.ntiles) * 2 + (int)rank) * p.ntiles + tp % p.ntiles; };
+    // the even CTA's accumulator barriers and stage barriers, in cluster space
+    const uint32_t tempty_l = PAIR ? map_to_rank(tempty, 0) : 0;
+    const uint32_t full_l = PAIR ? map_to_rank(full, 0) : 0;
+    auto release_acc = [&](int b) {  // this drain warp is done with accumulator b
+        if (PAIR && rank != 0) mbar_arrive_cluster(tempty_l + 8u * b);
+        else mbar_arrive(&tempty[b]);
+    };
     // The tile of position j + 1 (`total` once the walk is over) from the scheduler's answer j;
     // each reader then releases the answer's slot (the MMA lane alone, or a drain warp once all
     // its lanes have read).  The wait ignores the abort flag, so every reader of an answer that
@@ -205,7 +227,31 @@ __global__ void __launch_bounds__(320, 1)
     };
 
     if (warp == 0) {
-        if (lane == 0) {  // ---------------- tile scheduler and TMA producer
+        if (PAIR && lane == 0) {  // ---------------- TMA producer of a pair CTA
+            int it = 0;
+            for (int j = 0; cl + j * ncl < total_pairs && !*abort; ++j) {
+                const TileInfo<BN> t = tile_info<BN>(p, pair_tile(cl + j * ncl));
+                const int arow = t.mt * p.rows - p.shift;  // rows outside [0, M) load as zeros
+                const int brow = t.seg2 >= 0 ? (rank ? t.b_row2 : t.b_row) : t.b_row + (int)rank * (BN / 2);
+                for (int kt = 0; kt < p.ktiles; ++kt, ++it) {
+                    const int s = it % STAGES;
+                    if (!mbar_wait(&empty[s], ((it / STAGES) & 1) ^ 1, abort)) {
+                        raise_timeout(abort, p.status);
+                        break;
+                    }
+                    uint8_t* sa = smem + s * STAGE_BYTES;
+                    const uint32_t fb = full_l + 8u * s;
+                    if (rank == 0) mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
+                    else mbar_arrive_expect_tx_cluster(fb, STAGE_BYTES);
+                    tma_load_2d_pair(sa, &mapA, fb, kt * kBK, arow);
+                    tma_load_2d_pair(sa + A_BYTES, &mapB2, fb, kt * kBK, brow);
+                }
+            }
+            // the even CTA sees every load of both CTAs land (bounded); the odd CTA's loads have
+            // landed before the even CTA reaches the closing cluster barrier
+            if (rank == 0)
+                for (int i = max(0, it - STAGES); i < it; ++i) mbar_wait(&full[i % STAGES], (i / STAGES) & 1, nullptr);
+        } else if (!PAIR && lane == 0) {  // ---------------- tile scheduler and TMA producer
             // Tile position 0 is this CTA's own index; the tile of position j + 1 is the index of a
             // CTA that had not started yet, cancelled by a launch-control request made while tile j
             // loads.  An answer that cancelled nothing ends the walk (the grid has one CTA per tile).
@@ -252,7 +298,37 @@ __global__ void __launch_bounds__(320, 1)
             for (int i = max(0, it - STAGES); i < it; ++i) mbar_wait(&full[i % STAGES], (i / STAGES) & 1, nullptr);
         }
     } else if (warp == 1) {
-        if (lane == 0) {  // ---------------- MMA issuer
+        if (PAIR && lane == 0 && rank == 0) {  // ---------------- MMA issuer of the pair
+            int it = 0;
+            const uint32_t idesc = idesc_bf16(2 * kBM, BN, 0, 0);
+            for (int j = 0; cl + j * ncl < total_pairs && !*abort; ++j) {
+                const int buf = j & 1;
+                if (!mbar_wait(&tempty[buf], ((j >> 1) & 1) ^ 1, abort)) {
+                    raise_timeout(abort, p.status);
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem + buf * BN;
+                for (int kt = 0; kt < p.ktiles; ++kt, ++it) {
+                    const int s = it % STAGES;
+                    if (!mbar_wait(&full[s], (it / STAGES) & 1, abort)) {
+                        raise_timeout(abort, p.status);
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a0 = smem_u32(smem + s * STAGE_BYTES);
+                    const uint32_t b0 = a0 + A_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < kBK / 16; ++kk)
+                        mma_ss_pair(d_tmem, desc_sw128(a0 + kk * 32, 16, 1024), desc_sw128(b0 + kk * 32, 16, 1024),
+                                    idesc, (kt | kk) != 0);
+                    mma_commit_pair(&empty[s]);
+                }
+                mma_commit_pair(&tfull[buf]);
+            }
+            mma_commit_pair(done);
+            mbar_wait(done, 0, nullptr);
+        } else if (!PAIR && lane == 0) {  // ---------------- MMA issuer
             int it = 0, tc = 0;
             for (int tile = blockIdx.x; tile < total && !*abort; ++tc) {
                 const TileInfo<BN> t = tile_info<BN>(p, tile);
@@ -293,7 +369,10 @@ __global__ void __launch_bounds__(320, 1)
         const int r = q * 32 + lane;  // tile row = TMEM lane
         const GemmExtra& ex = p.ex;
         int tc = 0;
-        for (int tile = blockIdx.x; tile < total; tile = next_tile(tc++, false)) {
+        // the walk: the pair's static one over tile pairs, else the scheduler's answers
+        auto in_walk = [&](int j, int tl) -> bool { return PAIR ? cl + j * ncl < total_pairs : tl < total; };
+        auto advance = [&](int j) -> int { return PAIR ? pair_tile(cl + (j + 1) * ncl) : next_tile(j, false); };
+        for (int tile = PAIR ? pair_tile(cl) : (int)blockIdx.x; in_walk(tc, tile); tile = advance(tc++)) {
             const TileInfo<BN> t = tile_info<BN>(p, tile);
             const int buf = tc & 1;
             const TcSeg& sg = p.seg[t.seg];
@@ -396,11 +475,11 @@ __global__ void __launch_bounds__(320, 1)
                 }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&tempty[buf]);
+                if (lane == 0) release_acc(buf);
                 continue;
             }
             const int64_t tile_row0 = (int64_t)t.mt * p.rows - p.shift;  // token of tile row 0
-            if (sg.tma >= 2 && tile_row0 >= 0) {
+            if (sg.tma >= 2 && tile_row0 >= 0 && tile_row0 < p.M) {
                 // fp32 outputs: 32-column units (group eg takes units eg, eg + 2, ...), rows staged in
                 // the 128-byte-swizzled layout, then one bulk store or bulk add per unit.  Each output
                 // element gets exactly one add per launch, the same fp32 add as a read-modify-write.
@@ -435,10 +514,10 @@ __global__ void __launch_bounds__(320, 1)
                 asm volatile("bar.sync %0, 128;" ::"r"(2 + eg) : "memory");  // last unit's rows read
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&tempty[buf]);
+                if (lane == 0) release_acc(buf);
                 continue;
             }
-            if (sg.tma == 1 && tile_row0 >= 0) {
+            if (sg.tma == 1 && tile_row0 >= 0 && tile_row0 < p.M) {
                 // 64-column units (group eg takes units eg, eg + 2, ...): rows staged as bf16 in the
                 // 128-byte-swizzled layout, then one bulk store per unit.  Halo rows above the tile's
                 // outputs rewrite the identical values the previous row block wrote.  A paired tile
@@ -482,7 +561,7 @@ __global__ void __launch_bounds__(320, 1)
                 if (!paired) {
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&tempty[buf]);
+                    if (lane == 0) release_acc(buf);
                     continue;
                 }
             } else if (paired) {  // first half of a paired tile at the top row block: plain stores
@@ -703,14 +782,18 @@ __global__ void __launch_bounds__(320, 1)
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&tempty[buf]);
+            if (lane == 0) release_acc(buf);
         }
     }
     if (warp >= 2 && (warp & 3) == 2 && lane == 0) bulk_wait0();  // this group's bulk stores are complete
     tc_fence_before();
     __syncthreads();
+    if (PAIR) cluster_sync();  // the pair's MMAs, loads and arrives are all done
     tc_fence_after();
-    if (warp == 1) tmem_dealloc(tmem, TMEM_COLS);
+    if (warp == 1) {
+        if (PAIR) tmem_dealloc_pair(tmem, TMEM_COLS);
+        else tmem_dealloc(tmem, TMEM_COLS);
+    }
 }
 
 // --------------------------------------------------------------------------- host side
@@ -805,7 +888,7 @@ static bool tc_shape_ok(const GemmDesc& g)
 
 bool gemm_tc_supported(const GemmDesc& g) { return tc_shape_ok(g) && encode_fn() != nullptr; }
 
-template <int BN, int STAGES, bool CONV>
+template <int BN, int STAGES, bool CONV, bool PAIR>
 static cudaError_t launch_bn(const GemmDesc& g, const TcParams& p0, cudaStream_t s, int* status)
 {
     TcParams p = p0;
@@ -852,20 +935,48 @@ static cudaError_t launch_bn(const GemmDesc& g, const TcParams& p0, cudaStream_t
             t.tma = make_tmap_f32(&om.m[i], t.out, (uint64_t)t.n, (uint64_t)g.M, (uint64_t)t.ldo * 4, 32, kBM)
                         ? (t.accumulate ? 3 : 2) : 0;
     }
-    constexpr int smem = STAGES * (kBM + BN) * kBK * 2 + (CONV ? 2 * kBM * kStageLd * 4 : 2 * kBM * 128) + 1024 + 512;
+    constexpr int smem = STAGES * (kBM + (PAIR ? BN / 2 : BN)) * kBK * 2 +
+                         (CONV ? 2 * kBM * kStageLd * 4 : 2 * kBM * 128) + 1024 + 512;
     static_assert(smem <= 232448, "GEMM configuration exceeds 227 KB of shared memory");
+    auto kernel = gemm_tc_kernel<BN, STAGES, CONV, PAIR>;
     int dev = 0;
     cudaGetDevice(&dev);
     static unsigned long long attr_set = 0;  // one bit per device
-    if (dev < 64 && !(attr_set >> dev & 1ull)) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, STAGES, CONV>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    static int max_clusters[64] = {};        // co-resident clusters of two (pair kernels)
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!(attr_set >> dev & 1ull)) {
+        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
         attr_set |= 1ull << dev;
     }
-    // one CTA per tile: the CTAs that start first take over the others' tiles as they go
-    gemm_tc_kernel<BN, STAGES, CONV><<<p.mtiles * p.ntiles, 320, smem, s>>>(mapA, mapB, mapB2, om, p);
-    return cudaGetLastError();
+    if (!PAIR) {
+        // one CTA per tile: the CTAs that start first take over the others' tiles as they go
+        kernel<<<p.mtiles * p.ntiles, 320, smem, s>>>(mapA, mapB, mapB2, om, p);
+        return cudaGetLastError();
+    }
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(320, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (max_clusters[dev] <= 0) {  // as many clusters as can be resident at once (a static walk)
+        int sms = 148, n = 0;
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        cfg.gridDim = dim3(2 * (sms / 2), 1, 1);
+        cudaError_t e = cudaOccupancyMaxActiveClusters(&n, kernel, &cfg);
+        if (e != cudaSuccess) return e;
+        if (n <= 0) return cudaErrorInvalidConfiguration;
+        max_clusters[dev] = n;
+    }
+    const int total_pairs = ((p.mtiles + 1) / 2) * p.ntiles;
+    cfg.gridDim = dim3(2 * min(total_pairs, max_clusters[dev]), 1, 1);
+    return cudaLaunchKernelEx(&cfg, kernel, mapA, mapB, mapB2, om, p);
 }
 
 cudaError_t launch_gemm_tc(const GemmDesc& g, cudaStream_t s)
@@ -901,9 +1012,16 @@ cudaError_t launch_gemm_tc(const GemmDesc& g, cudaStream_t s)
     // Wide tiles when they still give every SM work; narrow ones for skinny problems.
     const int tiles256 = p.mtiles * ((n_total + 255) / 256);
     const bool conv = p.shift > 0;
+    // Wide tiles could go to CTA pairs (each CTA loads half of B; two row blocks needed).  The pair
+    // mode gives the right results on B200 but was measured slower than one CTA per tile on the
+    // b8 x L2048 block at width 768 (in_proj 151 vs 107.5 us, out_proj 70 vs 40 us, with all 74
+    // clusters resident), so it stays off until the cause is found.
+    constexpr bool kPairMma = false;
+    if (kPairMma && tiles256 >= 148 && p.mtiles >= 2)
+        return conv ? launch_bn<256, 5, true, true>(g, p, s, status) : launch_bn<256, 6, false, true>(g, p, s, status);
     if (tiles256 >= 148)
-        return conv ? launch_bn<256, 3, true>(g, p, s, status) : launch_bn<256, 4, false>(g, p, s, status);
-    return conv ? launch_bn<128, 5, true>(g, p, s, status) : launch_bn<128, 6, false>(g, p, s, status);
+        return conv ? launch_bn<256, 3, true, false>(g, p, s, status) : launch_bn<256, 4, false, false>(g, p, s, status);
+    return conv ? launch_bn<128, 5, true, false>(g, p, s, status) : launch_bn<128, 6, false, false>(g, p, s, status);
 }
 
 }  // namespace mm
