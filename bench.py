@@ -44,7 +44,12 @@ def parse():
     ap.add_argument("--ncu-summary", metavar="CSV", default=None,
                     help="print a per-kernel table (launches, device time, share, DRAM bytes per launch) of an "
                          "ncu --csv log and exit")
+    ap.add_argument("--stub", action="store_true",
+                    help="launcher check on CPU: every rank times a small host matmul over gloo and rank 0 prints "
+                         "the rank count and the whole-job rate (no GPU, no library)")
     a = ap.parse_args()
+    if a.gpus < 1:
+        ap.error("--gpus must be at least 1")
     if a.only is None:
         a.warmup = max(a.warmup, 3)
     return a
@@ -591,9 +596,69 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def launch_ranks(args):
+    """Start one rank per GPU when --gpus N > 1 and this process is not already a rank.
+
+    Returns None when this process should run the benchmark itself (N = 1, or a rank started by
+    torch.distributed.run whose WORLD_SIZE agrees with N), else an exit status: that of the
+    launched job, or 2 when WORLD_SIZE and --gpus disagree."""
+    env_world = os.environ.get("WORLD_SIZE")
+    if env_world is not None:
+        if int(env_world) != args.gpus:
+            sys.stderr.write("bench.py: --gpus %d but WORLD_SIZE=%s; launch one rank per GPU with matching counts\n"
+                             % (args.gpus, env_world))
+            return 2
+        return None
+    if args.gpus == 1:
+        return None
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", str(args.gpus),
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__), *sys.argv[1:]]
+    try:
+        return subprocess.run(cmd, timeout=3600).returncode
+    except subprocess.TimeoutExpired:
+        sys.stderr.write("bench.py: the %d-rank job did not finish within an hour\n" % args.gpus)
+        return 3
+
+
+def run_stub(args):
+    """Launcher check without a GPU: ranks over gloo, a host matmul as the step."""
+    import numpy as np
+    import torch.distributed as dist
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("gloo", timeout=timedelta(seconds=60))
+    a = np.random.default_rng(rank).standard_normal((128, 128))
+    for _ in range(args.warmup):
+        a = np.tanh(a @ a)
+    if world > 1:
+        dist.barrier()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        a = np.tanh(a @ a)
+    slowest = max_over_ranks(time.perf_counter() - t0, world, dist, "cpu")
+    if rank == 0:
+        print(json.dumps({"impl": "stub", "metric": "host matmul steps/s (launcher check)", "n_gpus": world,
+                          "value": whole_job_rate(1, args.steps, world, slowest), "unit": "steps/s",
+                          "steps": args.steps, "warmup": args.warmup, "data": "stub"}), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 if __name__ == "__main__":
     a = parse()
-    if a.ncu_summary:
+    rc = None if a.ncu_summary else launch_ranks(a)
+    if rc is not None:
+        sys.exit(rc)
+    if a.stub:
+        run_stub(a)
+    elif a.ncu_summary:
         ncu_summary(a.ncu_summary)
     elif a.impl == "reference":
         run_reference(a)

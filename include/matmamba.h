@@ -209,16 +209,19 @@ int ssd_scan(int dtype, const void* x, int64_t x_stride, const float* dt, int64_
  * a latency-critical loop that must avoid the device-wide synchronisation
  * cudaMalloc / cudaFree may cause.  The paper has no counterpart; it is a
  * deployment convenience of this library.
- * Same arguments and results as ssd_scan.  Scratch comes from a fixed 16 MiB
- * device array inside the library (held by every GPU that loads it, until
- * exit); a call needing more than that (see ssd_scan_workspace) returns
- * MM_ERR_WORKSPACE and launches nothing.  Allocates nothing itself.
+ * Same arguments and results as ssd_scan.  Scratch comes from a fixed device
+ * array of MM_SCAN_STATIC_SCRATCH_BYTES inside the library (held by every GPU
+ * that loads it, until exit); a call whose scan needs more than that (its
+ * ssd_scan_workspace figure for the same arguments) returns MM_ERR_WORKSPACE
+ * and launches nothing.  Allocates nothing itself.
  * All calls on a device share the array and it keeps the last call's
  * contents (the scan writes every scratch byte before reading it): calls that
  * overlap on the GPU race and must be serialised by the caller.  The first
  * call on a device looks up the array's device address and caches it; make
  * that first call before any stream capture.
  */
+#define MM_SCAN_STATIC_SCRATCH_BYTES ((size_t)16 << 20) /* 16 MiB per device */
+
 int ssd_scan_static(int dtype, const void* x, int64_t x_stride, const float* dt, int64_t dt_stride, const float* A,
                     const void* B, int64_t B_stride, const void* C, int64_t C_stride, const float* D, int batch,
                     int L, int h, int P, int N, int G, int heads_per_group, int chunk, const float* init_state,

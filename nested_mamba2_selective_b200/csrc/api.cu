@@ -34,6 +34,14 @@ bool dtype_ok(int dtype) { return dtype == MM_F32 || dtype == MM_BF16; }
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 size_t round_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
+// True when the byte ranges [a, a + na) and [b, b + nb) share a byte (null or empty ranges never do).
+bool ranges_overlap(const void* a, size_t na, const void* b, size_t nb)
+{
+    if (!a || !b || !na || !nb) return false;
+    const uintptr_t pa = reinterpret_cast<uintptr_t>(a), pb = reinterpret_cast<uintptr_t>(b);
+    return pa < pb + nb && pb < pa + na;
+}
+
 // Sequential carving of the caller's workspace into 256-byte aligned pieces.
 struct Carver {
     char* base;
@@ -421,8 +429,12 @@ int matmamba_block_fwd(const mm_block_params* p, const void* u, int batch, int L
     if (batch <= 0 || L <= 0) return MM_ERR_SHAPE;
     if ((rc = check_chunk(chunk))) return rc;
     if (p->dtype == MM_BF16 && (!aligned16(u) || !aligned16(out))) return MM_ERR_ALIGN;
-    if ((ssm_state_out && (const void*)ssm_state_out == (const void*)ssm_state_in) ||
-        (conv_state_out && conv_state_out == conv_state_in))
+    // a state output may not share a byte with its input: CTAs write one sequence's output while
+    // others still read their input
+    const size_t ssm_bytes = (size_t)batch * v.H * v.P * v.N * 4;
+    const size_t conv_bytes = (size_t)batch * (v.E + 2 * v.GN) * (v.K - 1) * esize(p->dtype);
+    if (ranges_overlap(ssm_state_out, ssm_bytes, ssm_state_in, ssm_bytes) ||
+        ranges_overlap(conv_state_out, conv_bytes, conv_state_in, conv_bytes))
         return MM_ERR_SHAPE;
     size_t need;
     matmamba_block_workspace(p, batch, L, m_i, chunk, &need);
@@ -513,7 +525,10 @@ int ssd_scan(int dtype, const void* x, int64_t x_stride, const float* dt, int64_
     int rc = scan_args_check(dtype, x, x_stride, dt, dt_stride, A, B, B_stride, C, C_stride, batch, L, h, P, N, G,
                              heads_per_group, chunk, state_stride, y, y_stride, init_state || final_state);
     if (rc) return rc;
-    if (init_state && final_state && (const void*)init_state == (const void*)final_state) return MM_ERR_SHAPE;
+    {  // final_state may not share a byte with init_state (one CTA's output is another's input)
+        const size_t st_bytes = ((size_t)(batch - 1) * state_stride + (size_t)h * P * N) * 4;
+        if (ranges_overlap(final_state, st_bytes, init_state, st_bytes)) return MM_ERR_SHAPE;
+    }
     ScanArgs a = make_scan_args(x, x_stride, dt, dt_stride, A, B, B_stride, C, C_stride, D, batch, L, h, P, N, G,
                                 heads_per_group, chunk, init_state, state_stride, y, y_stride, final_state);
     const size_t need = scan_ws_bytes(dtype, a);

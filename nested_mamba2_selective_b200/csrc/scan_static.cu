@@ -10,9 +10,10 @@
 // loads the library holds until the process exits.
 //
 // Rules of use:
-//  - The array holds kScanScratchBytes; a call whose scan would need more is
-//    rejected with MM_ERR_WORKSPACE before anything is launched (the
-//    ssd_scan_workspace query gives the need).
+//  - The array holds kScanScratchBytes (MM_SCAN_STATIC_SCRATCH_BYTES); a call
+//    whose scan needs more is rejected with MM_ERR_WORKSPACE before anything
+//    is launched: ssd_scan compares the need of these very arguments with the
+//    array's size.
 //  - All calls on a device share the one array and it keeps whatever the last
 //    call left in it.  The scan writes every scratch byte before reading it,
 //    so nothing has to start at zero, but calls that overlap on the GPU (two
@@ -25,7 +26,7 @@
 
 namespace {
 
-constexpr size_t kScanScratchBytes = size_t(16) << 20;  // 16 MiB per device
+constexpr size_t kScanScratchBytes = MM_SCAN_STATIC_SCRATCH_BYTES;
 
 // In host code this name is only a stand-in for the device array; kernels are
 // given the address that cudaGetSymbolAddress returns for the current device.
@@ -54,10 +55,8 @@ extern "C" int ssd_scan_static(int dtype, const void* x, int64_t x_stride, const
                                int chunk, const float* init_state, int64_t state_stride, void* y, int64_t y_stride,
                                float* final_state, void* stream)
 {
-    size_t need = 0;
-    int rc = ssd_scan_workspace(dtype, batch, L, h, P, N, G, chunk, &need);
-    if (rc) return rc;
-    if (need > kScanScratchBytes) return MM_ERR_WORKSPACE;
+    // ssd_scan validates the arguments and rejects, before any launch, a scan whose scratch need
+    // (worked out from these very arguments) exceeds the array
     void* scratch = scratch_address();
     if (!scratch) return MM_ERR_CUDA;
     return ssd_scan(dtype, x, x_stride, dt, dt_stride, A, B, B_stride, C, C_stride, D, batch, L, h, P, N, G,

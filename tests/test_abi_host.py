@@ -90,6 +90,24 @@ def test_rejected_calls_launch_nothing(lib):
                         128, 1, 1, 256, None, 0, fake, 64, None, None, 0, None) == 4
 
 
+def test_overlapping_state_buffers_are_rejected(lib):
+    """A final state that shares bytes with the initial state is refused before any launch; disjoint
+    buffers pass validation (and would launch, so they are not called here)."""
+    base = 1 << 24
+    x, dt, a_, bc, y = (ctypes.c_void_p(base + i * (1 << 22)) for i in range(5))
+    init = ctypes.c_void_p(base + 8 * (1 << 22))
+    for shift in (0, 64, (1 << 15) - 4):    # same start, inside, last float of the first head
+        final = ctypes.c_void_p(init.value + shift)
+        assert lib.ssd_scan(1, x, 64, dt, 1, a_, bc, 128, bc, 128, None, 1, 64, 1, 64, 128, 1, 1, 256, init,
+                            64 * 128, y, 64, final, None, 0, None) == 2
+    p = params()
+    fake = ctypes.c_void_p(1 << 20)
+    s_in = ctypes.c_void_p(1 << 26)
+    s_out = ctypes.c_void_p((1 << 26) + 4096)
+    assert lib.matmamba_block_fwd(ctypes.byref(p), fake, 2, 16, 768, 256, fake, s_in, None, s_out, None, fake,
+                                  1 << 30, None) == 2
+
+
 def test_status_strings(lib):
     for s in range(10):
         assert lib.mm_status_string(s)

@@ -50,10 +50,11 @@ def test_block_tiny_f32_every_width(orc, m):
     assert max_abs_rel(to_np(c_out), c_ref) <= TOL["f32"]
 
 
-@pytest.mark.parametrize("m", [768, 384, 192, 96])
+@pytest.mark.parametrize("m", [768, 736, 384, 192, 96])
 def test_block_130m_reduced_batch(orc, m):
     """130M-class block (d_model 768, 24 heads of 64, d_state 128) on b2 L640: several chunks
-    and a ragged tail (640 = 2*256 + 128)."""
+    and a ragged tail (640 = 2*256 + 128).  m = 736 is a width outside the trained set that still
+    gives whole heads (23, an odd count), as Mix'n'Match allows."""
     w = synth.WORKLOADS["block_130m_b8_L2048"]
     wt, p64 = make_block(w)
     u = synth.activations((2, 640, w.d_model), "bf16", seed=w.seed + 20)
@@ -64,16 +65,19 @@ def test_block_130m_reduced_batch(orc, m):
 
 
 @pytest.mark.parametrize("m", [768, 96])
-def test_block_130m_full_size_sampled(orc, m):
-    """Full workload (b8 L2048) in one launch; the oracle checks batch row 7 over a causal
-    prefix of 300 tokens (exact for those outputs by causality and batch independence)."""
+def test_block_130m_full_size_whole_rows(orc, m):
+    """Full workload (b8 L2048) in the launch configuration the benchmark times; the oracle checks
+    batch rows 0 and 7 over all 2048 tokens (rows are independent), so every 128-token scan block,
+    segment and GEMM tile row of those sequences is compared."""
     w = synth.WORKLOADS["block_130m_b8_L2048"]
     wt, p64 = make_block(w)
     u = synth.activations((w.batch, w.seqlen, w.d_model), "bf16", seed=w.seed + 30)
     out = run_block(orc, w, wt, p64, u, m, w.chunk)
-    ref = orc.block_fwd(dims_of(w), p64, u[7:8, :300], m)
-    assert max_abs_rel(to_np(out[7:8, :300]), ref) <= TOL["bf16"]
     assert torch.isfinite(out.float()).all()
+    on = to_np(out)
+    for row in (0, 7):
+        ref = orc.block_fwd(dims_of(w), p64, u[row:row + 1], m)
+        assert max_abs_rel(on[row:row + 1], ref) <= TOL["bf16"], row
 
 
 def sliced_weights(wt: BlockWeights, d, h):
@@ -194,3 +198,42 @@ def test_repeated_calls_are_bit_identical():
     b = matmamba_block_fwd(wt, u, 768, 256)
     torch.cuda.synchronize()
     assert torch.equal(a, b)
+
+
+def guarded(shape, dtype, fill, pad=4096):
+    """A tensor of `shape` inside a larger buffer whose other elements hold `fill`."""
+    n = int(np.prod(shape))
+    flat = torch.full((pad + n + pad,), fill, dtype=dtype, device="cuda")
+    return flat, flat[pad:pad + n].view(*shape), (pad, pad + n)
+
+
+def assert_outside_untouched(flat, span, fill):
+    lo, hi = span
+    assert torch.all(flat[:lo] == fill) and torch.all(flat[hi:] == fill), "write outside the output region"
+
+
+@pytest.mark.parametrize("m,L", [(736, 300), (96, 131)])
+def test_block_writes_nothing_outside_its_outputs(orc, m, L):
+    """out, ssm_state_out and conv_state_out each sit inside a larger buffer filled with a sentinel;
+    with a ragged length and an odd head count (23 or 3 heads) no byte outside the outputs (nor an
+    inactive head or conv row) changes, and the outputs match the oracle."""
+    w = synth.WORKLOADS["block_130m_b8_L2048"]
+    wt, p64 = make_block(w)
+    dims = dims_of(w)
+    H, P, N, E = dims.nheads, w.d_head, w.d_state, w.d_inner
+    rows = E + 2 * N
+    u = synth.activations((3, L, w.d_model), "bf16", seed=80 + m)
+    fo, out, so = guarded((3, L, w.d_model), torch.bfloat16, -7.0)
+    fs, s_out, ss = guarded((3, H, P, N), torch.float32, 11.5)
+    fc, c_out, sc = guarded((3, rows, 3), torch.bfloat16, -5.0)
+    run_block(orc, w, wt, p64, u, m, 256, out=out, ssm_state_out=s_out, conv_state_out=c_out)
+    d, h = orc.width(dims, m)
+    s_ref, c_ref = np.zeros((3, H, P, N)), np.zeros((3, rows, 3))
+    ref = orc.block_fwd(dims, p64, u, m, ssm_state_out=s_ref, conv_state_out=c_ref)
+    assert max_abs_rel(to_np(out), ref) <= TOL["bf16"]
+    assert max_abs_rel(to_np(s_out[:, :h]), s_ref[:, :h]) <= TOL["bf16"]
+    active = list(range(d)) + list(range(E, rows))
+    assert max_abs_rel(to_np(c_out[:, active]), c_ref[:, active]) <= TOL["bf16"]
+    assert torch.all(s_out[:, h:] == 11.5) and torch.all(c_out[:, d:E] == -5.0)
+    for flat, span, fill in ((fo, so, -7.0), (fs, ss, 11.5), (fc, sc, -5.0)):
+        assert_outside_untouched(flat, span, fill)

@@ -54,6 +54,30 @@ def test_steps_match_oracle_and_leave_inactive_state(orc, block, m):
     np.testing.assert_array_equal(to_np(c_gpu[:, d:E]), c_np[:, d:E].astype(np.float64))
 
 
+@pytest.mark.parametrize("m", [2048, 512])
+def test_64_consecutive_steps_match_oracle(orc, block, m):
+    """64 recurrent tokens in a row on 4 sequences from a prefilled random state: the state carried
+    through the GPU's own updates stays on the oracle's trajectory (every step's output and the
+    final states are compared)."""
+    wt, p64 = block
+    dims = dims_of(W)
+    s_np, c_np = states(4, seed=340 + m)
+    s_gpu, c_gpu = torch.from_numpy(s_np).cuda(), to_device(c_np, "bf16")
+    s_ref, c_ref = s_np.astype(np.float64), c_np.astype(np.float64)
+    d, h = orc.width(dims, m)
+    us = synth.activations((64, 4, W.d_model), "bf16", seed=350 + m)
+    worst = 0.0
+    for step in range(64):
+        out = ssd_step(wt, s_gpu, c_gpu, to_device(us[step], "bf16"), m)
+        ref = orc.block_step(dims, p64, us[step], m, s_ref, c_ref)
+        worst = max(worst, max_abs_rel(to_np(out), ref))
+    assert worst <= TOL["bf16"], worst
+    assert max_abs_rel(to_np(s_gpu[:, :h]), s_ref[:, :h]) <= TOL["bf16"]
+    E = W.d_inner
+    active = list(range(d)) + list(range(E, E + 2 * W.d_state))
+    assert max_abs_rel(to_np(c_gpu[:, active]), c_ref[:, active]) <= TOL["bf16"]
+
+
 def test_full_batch_step_sampled(orc, block):
     """256 sequences in one launch; the oracle checks three of them (sequences are independent)."""
     wt, p64 = block

@@ -159,3 +159,27 @@ def test_scan_steep_decay_blocks(orc):
     for i in range(6):  # per head: the steep token's large output must not hide errors elsewhere
         assert max_abs_rel(yn[:, :, i], ref[:, :, i]) <= TOL["bf16"], i
         assert max_abs_rel(fsn[:, i], fs_ref[:, i]) <= TOL["bf16"], i
+
+
+@pytest.mark.parametrize("h,L", [(5, 1000), (3, 131), (23, 384)])
+def test_scan_writes_nothing_outside_its_outputs(orc, h, L):
+    """y has a row pitch of h+1 heads (y_stride > h*P) and sits with the final state inside larger
+    buffers filled with a sentinel; odd head counts and ragged lengths leave every byte outside the
+    outputs, and the padding head of every row, unchanged."""
+    b = 2
+    inp = synth.long_memory(synth.ssd_inputs(b, L, h, 64, 128, 1, "bf16", seed=210 + h))
+    g = upload(inp, "bf16")
+    pad = 8192
+    ny, ns = b * L * (h + 1) * 64, b * h * 64 * 128
+    fy = torch.full((pad + ny + pad,), -9.0, dtype=torch.bfloat16, device="cuda")
+    fsf = torch.full((pad + ns + pad,), 13.0, device="cuda")
+    y = fy[pad:pad + ny].view(b, L, h + 1, 64)
+    fs = fsf[pad:pad + ns].view(b, h, 64, 128)
+    ssd_scan(g["x"], g["dt"], g["A"], g["B"], g["C"], g["D"], h=h, chunk=256, y=y, final_state=fs)
+    torch.cuda.synchronize()
+    ref, fs_ref = oracle_scan(orc, inp, h)
+    assert max_abs_rel(to_np(y[:, :, :h]), ref) <= TOL["bf16"]
+    assert max_abs_rel(to_np(fs), fs_ref) <= TOL["bf16"]
+    assert torch.all(y[:, :, h:] == -9.0), "write into the padding columns of a y row"
+    for flat, fill in ((fy, -9.0), (fsf, 13.0)):
+        assert torch.all(flat[:pad] == fill) and torch.all(flat[-pad:] == fill), "write outside an output"

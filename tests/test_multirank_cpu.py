@@ -40,3 +40,37 @@ def test_single_rank_needs_no_process_group():
     import bench
     assert bench.max_over_ranks(0.5, 1) == 0.5
     assert bench.whole_job_rate(100, 4, 1, 2.0) == 200.0
+
+
+def _bench(args, env_extra=None):
+    import json
+    import subprocess
+    env = dict(os.environ)
+    for k in ("RANK", "WORLD_SIZE", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT"):
+        env.pop(k, None)
+    env.update(env_extra or {})
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), *args], capture_output=True, text=True,
+                       env=env, timeout=300)
+    lines = [json.loads(l) for l in r.stdout.splitlines() if l.startswith("{")]
+    return r.returncode, lines, r.stderr
+
+
+def test_gpus_flag_launches_one_rank_per_device_count():
+    """bench.py --gpus 2 started as a plain process launches two ranks itself (torch.distributed.run),
+    and rank 0 alone prints one line that counts both."""
+    rc, lines, err = _bench(["--gpus", "2", "--stub", "--steps", "3", "--warmup", "1"])
+    assert rc == 0, err[-2000:]
+    assert len(lines) == 1
+    assert lines[0]["n_gpus"] == 2 and lines[0]["value"] > 0
+
+
+def test_gpus_flag_and_world_size_must_agree():
+    rc, lines, err = _bench(["--gpus", "2", "--stub"], {"WORLD_SIZE": "3", "RANK": "0"})
+    assert rc == 2 and not lines
+    assert "WORLD_SIZE" in err
+
+
+def test_single_gpu_runs_in_process():
+    rc, lines, err = _bench(["--stub", "--steps", "2", "--warmup", "1"])
+    assert rc == 0, err[-2000:]
+    assert lines[0]["n_gpus"] == 1

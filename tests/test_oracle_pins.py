@@ -262,6 +262,21 @@ def test_rmsnorm_unit_rms_and_scale_invariance(orc):
     np.testing.assert_allclose(orc.rmsnorm_rows(v, w2, 0.0), n * w2, rtol=1e-13)
 
 
+def test_rmsnorm_with_eps_closed_form(orc):
+    """With eps > 0 the output keeps each row's direction and has RMS 1/sqrt(1 + eps/mean(v^2)): the
+    textbook definition v / sqrt(mean(v^2) + eps), checked through that closed form."""
+    rng = np.random.default_rng(31)
+    v = rng.standard_normal((6, 40)) * np.array([1e-3, 0.1, 1.0, 3.0, 10.0, 0.02])[:, None]
+    w = np.ones(40)
+    for eps in (1e-5, 1e-2, 0.5):
+        n = orc.rmsnorm_rows(v, w, eps)
+        ms = np.mean(v * v, -1)
+        np.testing.assert_allclose(np.sqrt(np.mean(n * n, -1)), 1.0 / np.sqrt(1.0 + eps / ms), rtol=1e-12)
+        ratio = n / v
+        np.testing.assert_allclose(ratio, np.broadcast_to(ratio[:, :1], ratio.shape), rtol=1e-12)
+        assert np.all(ratio > 0)
+
+
 def sliced_params(dims, p, d, h):
     E, GN = dims.d_inner, dims.ngroups * dims.d_state
     W = p["W_in"]
@@ -357,6 +372,26 @@ def test_stack_composition_and_mix_n_match(orc):
         n = x / np.sqrt(np.mean(x * x, -1, keepdims=True) + 1e-5) * wts[l]
         x = x + orc.block_fwd(dims, params[l], n, ms[l])
     assert rel_err(out, x) < 1e-13
+
+
+def test_stack_with_zero_output_projections_is_the_identity(orc):
+    """All W_out = 0: every block adds exactly zero to the residual stream, so the stack returns its
+    input bit for bit, whatever the other weights and widths (a dropped or doubled residual, or a
+    residual added to the normed stream, fails)."""
+    dims = tiny_dims(orc)
+    params = []
+    for l in range(4):
+        p = tiny_params(dims, seed=120 + l)
+        p["W_out"] = np.zeros_like(p["W_out"])
+        params.append(p)
+    wts = [1.0 + 0.3 * np.random.default_rng(130 + l).standard_normal(16) for l in range(4)]
+    u = np.random.default_rng(140).standard_normal((2, 9, 16)) * 3.0
+    out = orc.stack_fwd(dims, 4, lambda l: params[l], lambda l: wts[l], u, [16, 4, 12, 8])
+    np.testing.assert_array_equal(out, u)
+    # and a single non-zero W_out changes it: the pin is not vacuous
+    params[2] = tiny_params(dims, seed=122)
+    out2 = orc.stack_fwd(dims, 4, lambda l: params[l], lambda l: wts[l], u, [16, 4, 12, 8])
+    assert np.max(np.abs(out2 - u)) > 1e-6
 
 
 @pytest.mark.parametrize("name,expect", [("block_tiny_f32", 0.966), ("block_130m_b8_L2048", 0.997),
