@@ -8,7 +8,7 @@ prefix).  Inputs are seeded synthetic tensors already resident in HBM; L2 is
 flushed (256 MiB write) before every timed step and each step is timed with
 CUDA events on the launching stream.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--extended]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
 With N > 1 (launched by torch.distributed.run) every rank runs an independent
 replica on its own GPU (sequences shard with no exchange), and value is the
@@ -36,9 +36,10 @@ def parse():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--extended", action="store_true", help="also time the 48-layer stack and the decode step")
+    ap.add_argument("--skip-stack-decode", action="store_true",
+                    help="leave out the 48-layer stack and the decode step (profiling aid)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["block", "scan"], default=None,
+    ap.add_argument("--only", choices=["block", "scan", "decode"], default=None,
                     help="profiling aid: run just the headline block or just the standalone scan, print per-stage "
                          "times and no benchmark line")
     ap.add_argument("--ncu-summary", metavar="CSV", default=None,
@@ -142,6 +143,53 @@ def block_work(m, T, Dm=768, E=1536, P=64, N=128):
         "gate_rmsnorm": ("hbm", T * d * 2 * 3),
         "out_proj": ("tensor", 2.0 * T * d * Dm),
     }
+
+
+STACK = dict(workload="stack48_1p4b_b4_L4096", batch=4, seq_len=4096, d_model=2048, d_inner=4096, d_head=64,
+             d_state=128, nlayers=48, chunk=256, widths=[2048, 1024, 512, 256])
+DECODE = dict(workload="decode_b256_1p4b", batch=256, d_model=2048, d_inner=4096, d_head=64, d_state=128,
+              steps=1000, graph_steps=100, widths=[2048, 1024, 512])
+
+
+def stack_work(m, T, Dm=2048, E=4096, P=64, N=128):
+    """Algorithmic work of each launch stage of one stack layer on T tokens at width m: the block's stages
+    (out_proj adds into the fp32 residual) and the pre-norm (fp32 residual read, bf16 row written)."""
+    w = block_work(m, T, Dm, E, P, N)
+    w["prenorm"] = ("hbm", T * Dm * (4 + 2))
+    return w
+
+
+def decode_work(m, Bt, Dm=2048, E=4096, P=64, N=128, K=4):
+    """HBM bytes of each launch stage of one recurrent step for Bt sequences at width m."""
+    d = E * m // Dm
+    h = d // P
+    nconv = d + 2 * N
+    return {
+        "step_in_proj": ("hbm", (2 * d + 2 * N + h) * Dm * 2 + Bt * Dm * 2 + Bt * ((d + nconv) * 2 + h * 4)),
+        "step_conv_dt": ("hbm", Bt * (nconv * (K - 1) * 2 * 2 + nconv * 2 * 2 + h * 4 * 2)),
+        "step_scan": ("hbm", Bt * (h * P * N * 4 * 2 + nconv * 2 + h * 4 + d * 2)),
+        "step_gate_rmsnorm": ("hbm", Bt * d * 2 * 3),
+        "step_out_proj": ("hbm", Dm * d * 2 + Bt * d * 2 + Bt * Dm * 2),
+    }
+
+
+def stage_table(stages, work, pk, per_launch_divisor=1):
+    """Per traced stage: mean launch time, share of the traced time, and achieved work against the peak
+    (bf16 tensor FLOP/s or HBM GB/s).  per_launch_divisor splits a stage's launches into the unit the work
+    is quoted for (e.g. 48 layers)."""
+    tot_ms = sum(v[2] for v in stages.values()) or 1.0
+    out = {}
+    for k, (n, kern, ms) in stages.items():
+        kd, amt = work.get(k, (None, 0.0))
+        per = ms / n
+        row = {"ms_per_launch": per, "launches": n, "share": ms / tot_ms}
+        if kd is not None:
+            ach = amt / (per / 1e3) / (1e12 if kd == "tensor" else 1e9)
+            peak = pk["bf16_tflops"] if kd == "tensor" else pk["hbm_gbs"]
+            row.update({"bound": kd, "achieved": ach, "unit": "TFLOP/s" if kd == "tensor" else "GB/s",
+                        "frac": ach / peak})
+        out[k] = row
+    return out
 
 
 def scan_bytes(T, h, P=64, N=128):
@@ -351,7 +399,8 @@ def run_ours(args):
         ms, tr = timed(fn, args.steps, args.warmup, trace=True)
         total = slowest(sum(ms))
         per_width[str(m)] = {"tokens_per_s": whole_job_rate(T, args.steps, world, total / 1e3),
-                             "ms_per_step": total / args.steps}
+                             "ms_per_step": total / args.steps,
+                             "stages": stage_table(tr[0], block_work(m, T), pk)}
         if m == B["widths"][0]:
             head = (ms, total, tr)
     ms, total, (stages, kernels) = head
@@ -360,25 +409,14 @@ def run_ours(args):
 
     # dominant stage of the headline step -> roofline object
     work = block_work(m0, T)
+    stage_rows = stage_table(stages, work, pk)
     dom = max(stages, key=lambda k: stages[k][2])
-    kind, amount = work.get(dom, ("hbm", 0.0))
     avg_ms = stages[dom][2] / stages[dom][0]
-    if kind == "tensor":
-        achieved = amount / (avg_ms / 1e3) / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"], "unit": "TFLOP/s"}
-    else:
-        achieved = amount / (avg_ms / 1e3) / 1e9
-        roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s"}
-    roof.update({"frac": roof["achieved"] / roof["peak"], "traffic": traffic_for(dom), "kernel": dom,
-                 "peak_source": pk_src, "avg_launch_ms": avg_ms})
-    stage_table = {}
-    for k, (n, kern, tot) in stages.items():
-        kd, amt = work.get(k, ("hbm", 0.0))
-        per = tot / n
-        ach = amt / (per / 1e3) / (1e12 if kd == "tensor" else 1e9)
-        stage_table[k] = {"ms_per_launch": per, "share": tot / sum(v[2] for v in stages.values()), "bound": kd,
-                          "achieved": ach, "unit": "TFLOP/s" if kd == "tensor" else "GB/s",
-                          "frac": ach / (pk["bf16_tflops"] if kd == "tensor" else pk["hbm_gbs"])}
+    sr = stage_rows[dom]
+    roof = {"bound": sr["bound"], "achieved": sr["achieved"],
+            "peak": pk["bf16_tflops"] if sr["bound"] == "tensor" else pk["hbm_gbs"], "unit": sr["unit"],
+            "frac": sr["frac"], "traffic": traffic_for(dom), "kernel": dom, "peak_source": pk_src,
+            "avg_launch_ms": avg_ms}
 
     # ---------------- standalone SSD scan (the graded scan roofline)
     S = SCAN
@@ -394,14 +432,16 @@ def run_ours(args):
                                                     S["chunk"]), 1), dtype=torch.uint8, device=dev)
         fn = lambda h=h, y=y, sws=sws: mm.ssd_scan(g["x"], g["dt"], g["A"], g["B"], g["C"], g["D"], h=h,  # noqa
                                                    chunk=S["chunk"], y=y, workspace=sws)
-        sms, _ = timed(fn, args.steps, args.warmup)
+        sms, str_ = timed(fn, args.steps, args.warmup, trace=True)
         avg = slowest(sum(sms)) / args.steps
         nbytes = scan_bytes(Ts, h)
         scan[str(h)] = {"tokens_per_s": world * Ts / (avg / 1e3), "us_per_call": avg * 1e3,
+                        "kernels_per_call": str_[1] // args.steps,
                         "roofline": {"bound": "hbm", "achieved": nbytes / (avg / 1e3) / 1e9, "peak": pk["hbm_gbs"],
                                      "unit": "GB/s", "frac": nbytes / (avg / 1e3) / 1e9 / pk["hbm_gbs"],
                                      "algorithmic_bytes": nbytes, "traffic": traffic_for("ssd_scan_h%d" % h),
                                      "peak_source": pk_src}}
+    del g, inp
 
     # ---------------- end to end through the host-buffer entry point
     u_host = torch.from_numpy(u_np).bfloat16().pin_memory()
@@ -416,10 +456,12 @@ def run_ours(args):
         e2e_fn()
     e2e_s = slowest(time.perf_counter() - t0)
     io_bytes = T * B["d_model"] * 2
+    del ws, u_dev, out_dev
 
-    extended = {}
-    if args.extended:
-        extended = run_extended(args, mm, synth, torch, dev, timed, slowest, world)
+    stack = decode = None
+    if not args.skip_stack_decode:
+        stack = run_stack(args, mm, torch, dev, timed, slowest, world, pk)
+        decode = run_decode(args, mm, torch, dev, timed, slowest, world, pk)
     clk.__exit__(None, None, None)
     clocks = clk.summary()
 
@@ -430,30 +472,149 @@ def run_ours(args):
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": B["workload"], "batch": B["batch"], "seq_len": B["seq_len"],
                        "d_model": B["d_model"], "d_inner": B["d_inner"], "d_head": B["d_head"],
-                       "d_state": B["d_state"], "ngroups": 1, "d_conv": 4, "chunk": B["chunk"], "width": m0,
-                       "parallelism": "replicas%d" % world,
+                       "d_state": B["d_state"], "ngroups": 1, "d_conv": 4, "chunk": B["chunk"],
+                       "scan_block_tokens": 128,
+                       "chunk_note": "the chunked scan's result does not depend on chunk; the bf16 kernels "
+                                     "evaluate every chunk of 256 as two 128-token blocks",
+                       "width": m0, "parallelism": "replicas%d" % world,
                        "l2": "flushed (256 MiB write) before every timed step"},
             "per_width": per_width,
             "roofline": roof,
-            "stages": stage_table,
+            "stages": stage_rows,
             "ssd_scan": {"workload": S["workload"], "by_heads": scan},
-            "e2e": {"value": whole_job_rate(T, args.steps, world, e2e_s), "unit": "tokens/s", "h2d_bytes_per_step": io_bytes,
-                    "d2h_bytes_per_step": io_bytes},
+            "e2e": {"value": whole_job_rate(T, args.steps, world, e2e_s), "unit": "tokens/s",
+                    "h2d_bytes_per_step": io_bytes, "d2h_bytes_per_step": io_bytes},
             "gpu_launches": kernels,
             "clocks": clocks,
         }
-        if extended:
-            line["extended"] = extended
+        if stack:
+            line["stack48"] = stack
+        if decode:
+            line["decode"] = decode
         if not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(arrays, u_np, m0)
+            line["cpu_baseline_scan"] = cpu_baseline_scan()
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
 
 
+def device_block_weights(mm, torch, gen, Dm, E, P, N, dev, K=4):
+    """Full-width block weights drawn on the device from a seeded generator with the synthetic recipe
+    (weights ~ N(0, 0.02) in bf16, norm_w = 1 + N(0, 0.02), A = -exp(U(log 1, log 16)), dt_bias =
+    softplus^-1 of a log-uniform dt in [1e-3, 1e-1], D ~ N(0, 1))."""
+    H = E // P
+
+    def nrm(*shape, std=0.02, mean=0.0):
+        return (torch.randn(*shape, generator=gen, device=dev) * std + mean).bfloat16().contiguous()
+
+    def uni(n, lo, hi):
+        return torch.rand(n, generator=gen, device=dev) * (hi - lo) + lo
+
+    import math
+    dt0 = torch.exp(uni(H, math.log(1e-3), math.log(1e-1))).double()
+    return mm.BlockWeights(Dm, E, P, N, 1, K, 1e-5, nrm(2 * E + 2 * N + H, Dm), nrm(E + 2 * N, K), nrm(E + 2 * N),
+                           (dt0 + torch.log(-torch.expm1(-dt0))).float().contiguous(),
+                           (-torch.exp(uni(H, 0.0, math.log(16.0)))).contiguous(),
+                           torch.randn(H, generator=gen, device=dev).contiguous(), nrm(E, mean=1.0), nrm(Dm, E))
+
+
+def graph_of(torch, fn, reps=1):
+    """Capture `reps` consecutive calls in one CUDA graph (after an eager call that does the per-device
+    set-up)."""
+    fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for _ in range(reps):
+            fn()
+    torch.cuda.synchronize()
+    return g
+
+
+def run_stack(args, mm, torch, dev, timed, slowest, world, pk):
+    """48-layer pre-norm stack (b4 L4096, d_model 2048, 64 heads) per width: the forward timed as CUDA-graph
+    replays (L2 flushed before each), and each stage's roofline fraction from one traced eager forward."""
+    S = STACK
+    Dm, E, nl = S["d_model"], S["d_inner"], S["nlayers"]
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(1003)
+    layers = [device_block_weights(mm, torch, gen, Dm, E, S["d_head"], S["d_state"], dev) for _ in range(nl)]
+    pws = [(1.0 + 0.02 * torch.randn(Dm, generator=gen, device=dev)).bfloat16() for _ in range(nl)]
+    u = torch.randn(S["batch"], S["seq_len"], Dm, generator=gen, device=dev).bfloat16()
+    out = torch.empty_like(u)
+    T = S["batch"] * S["seq_len"]
+    ws = torch.empty(max(mm.matmamba_stack_workspace(layers, [m] * nl, S["batch"], S["seq_len"])
+                         for m in S["widths"]), dtype=torch.uint8, device=dev)
+    res = {"workload": S["workload"], "timing": "CUDA-graph replay of the 48-layer forward, L2 flushed before each",
+           "by_width": {}}
+    for m in S["widths"]:
+        ms_list = [m] * nl
+        fn = lambda ms_list=ms_list: mm.matmamba_stack_fwd(layers, pws, u, ms_list, out=out, workspace=ws)  # noqa
+        steps = max(2, min(args.steps, 5))
+        g = graph_of(torch, fn)
+        ms, _ = timed(g.replay, steps, 1)
+        avg = slowest(sum(ms)) / steps
+        del g
+        mm.mm_trace_enable(nl * 8 + 16)
+        fn()
+        torch.cuda.synchronize()
+        stg, kern = mm.mm_trace_collect()
+        mm.mm_trace_enable(0)
+        res["by_width"][str(m)] = {"ms_per_forward": avg, "tokens_per_s": world * T / (avg / 1e3),
+                                   "kernels_per_forward": kern,
+                                   "stages_per_layer": stage_table(stg, stack_work(m, T, Dm, E), pk)}
+    del layers, ws
+    return res
+
+
+def run_decode(args, mm, torch, dev, timed, slowest, world, pk):
+    """1000 consecutive recurrent steps of the 1.4B-class block for 256 sequences per width, from a
+    prefilled N(0, 1) state: ten replays of a CUDA graph of 100 steps form the timed region (the state,
+    537 MB, exceeds L2); each stage's roofline fraction from traced eager steps."""
+    D = DECODE
+    Dm, E, Bt = D["d_model"], D["d_inner"], D["batch"]
+    H = E // D["d_head"]
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(1004)
+    w = device_block_weights(mm, torch, gen, Dm, E, D["d_head"], D["d_state"], dev)
+    res = {"workload": D["workload"], "steps": D["steps"],
+           "timing": "%d CUDA-graph replays of %d consecutive steps (state larger than L2, no flush)"
+                     % (D["steps"] // D["graph_steps"], D["graph_steps"]), "by_width": {}}
+    for m in D["widths"]:
+        s = torch.randn(Bt, H, D["d_head"], D["d_state"], generator=gen, device=dev)
+        c = torch.randn(Bt, E + 2 * D["d_state"], 3, generator=gen, device=dev).bfloat16()
+        ut = torch.randn(Bt, Dm, generator=gen, device=dev).bfloat16()
+        ot = torch.empty_like(ut)
+        ws = torch.empty(mm.ssd_step_workspace(w, Bt, m), dtype=torch.uint8, device=dev)
+        fn = lambda m=m, s=s, c=c, ut=ut, ot=ot, ws=ws: mm.ssd_step(w, s, c, ut, m, out_t=ot, workspace=ws)  # noqa
+        g = graph_of(torch, fn, D["graph_steps"])
+        reps = D["steps"] // D["graph_steps"]
+
+        def run_all():
+            for _ in range(reps):
+                g.replay()
+        ms, _ = timed(run_all, 1, 1)
+        total_ms = slowest(ms[0])
+        del g
+        _, (stg, _) = timed(fn, 5, 2, trace=True)
+        per = total_ms / D["steps"]
+        res["by_width"][str(m)] = {"us_per_step": per * 1e3, "tokens_per_s": world * Bt / (per / 1e3),
+                                   "stages": stage_table(stg, decode_work(m, Bt, Dm, E), pk)}
+    return res
+
+
 def run_only(args, mm, synth, torch, dev, timed):
     """One workload piece with few launches, for ncu captures; prints per-stage device times."""
+    if args.only == "decode":
+        pk, _ = peaks()
+        res = run_decode(args, mm, torch, dev, timed, lambda v: v, 1, pk)
+        print(json.dumps({"only": "decode", "by_width": {m: {"us_per_step": v["us_per_step"],
+                                                            "stages_us": {k: s["ms_per_launch"] * 1e3
+                                                                          for k, s in v["stages"].items()}}
+                                                        for m, v in res["by_width"].items()}}))
+        return
     if args.only == "block":
         B = BLOCK
         arrays = synth.block_params(B["d_model"], B["d_inner"], B["d_head"], B["d_state"], dtype="bf16", seed=1002)
@@ -473,69 +634,38 @@ def run_only(args, mm, synth, torch, dev, timed):
     print(json.dumps({"only": args.only, "ms_per_step": sum(ms) / len(ms), "stages": stages, "kernels": kernels}))
 
 
-def run_extended(args, mm, synth, torch, dev, timed, slowest, world):
-    """48-layer stack (b4 L4096, d_model 2048) per width and the 256-sequence decode step per width."""
+def cpu_baseline_scan(budget_s=6.0):
+    """The fp64 oracle's sequential scan on rows of the standalone-scan workload (24 heads): whole 8192-token
+    batch rows with every OpenMP thread for about budget_s, and one 2048-token prefix of a row on a single
+    thread (a separate process started with OMP_NUM_THREADS=1)."""
     import numpy as np
-    res = {}
-    Dm, E = 2048, 4096
 
-    def graph_of(fn):
-        """Capture one call in a CUDA graph (after an eager call that does the per-device set-up)."""
-        fn()
-        torch.cuda.synchronize()
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            fn()
-        torch.cuda.synchronize()
-        return g
-
-    layers, pws = [], []
-    for l in range(48):
-        a = synth.block_params(Dm, E, 64, 128, dtype="bf16", seed=1003 * 1000 + l)
-        layers.append(mm.BlockWeights.from_arrays(a, Dm, E, 64, 128, dtype=torch.bfloat16, device=dev))
-        pws.append(torch.from_numpy(synth.round_to(1.0 + 0.02 * np.random.default_rng(1003 * 1000 + 500 + l)
-                                                   .standard_normal(Dm), "bf16")).to(dev).bfloat16())
-    u = torch.from_numpy(synth.activations((4, 4096, Dm), "bf16", seed=402)).to(dev).bfloat16()
-    out = torch.empty_like(u)
-    stack = {}
-    for m in (2048, 1024, 512, 256):
-        ms_list = [m] * 48
-        ws = torch.empty(mm.matmamba_stack_workspace(layers, ms_list, 4, 4096), dtype=torch.uint8, device=dev)
-        fn = lambda: mm.matmamba_stack_fwd(layers, pws, u, ms_list, out=out, workspace=ws)  # noqa: E731
-        steps = max(2, min(args.steps, 5))
-        g = graph_of(fn)
-        ms, _ = timed(g.replay, steps, 1)
-        avg = slowest(sum(ms)) / steps
-        del g
-        # one eager forward, traced: the summed device time of each stage over the 48 layers
-        mm.mm_trace_enable(48 * 8 + 16)
-        fn()
-        torch.cuda.synchronize()
-        stg, _ = mm.mm_trace_collect()
-        mm.mm_trace_enable(0)
-        stack[str(m)] = {"ms_per_forward": avg, "tokens_per_s": world * 4 * 4096 / (avg / 1e3),
-                         "timing": "CUDA graph replay of the 48-layer forward",
-                         "stages_eager_ms": {k: round(v[2], 3) for k, v in stg.items()}}
-    res["stack48_1p4b_b4_L4096"] = stack
-    dec = {}
-    w = layers[0]
-    for m in (2048, 1024, 512):
-        s_np, c_np = synth.states(256, 64, 64, 128, E + 256, 4, "bf16", seed=320)
-        s = torch.from_numpy(s_np).to(dev)
-        c = torch.from_numpy(c_np).to(dev).bfloat16()
-        ut = torch.from_numpy(synth.activations((256, Dm), "bf16", seed=321)).to(dev).bfloat16()
-        ot = torch.empty_like(ut)
-        ws = torch.empty(mm.ssd_step_workspace(w, 256, m), dtype=torch.uint8, device=dev)
-        fn = lambda: mm.ssd_step(w, s, c, ut, m, out_t=ot, workspace=ws)  # noqa: E731
-        g = graph_of(fn)
-        ms, _ = timed(g.replay, args.steps, args.warmup)
-        avg = slowest(sum(ms)) / args.steps
-        del g
-        _, (stg, _) = timed(fn, 3, 1, trace=True)  # eager, traced: where a step's time goes
-        dec[str(m)] = {"us_per_step": avg * 1e3, "tokens_per_s": world * 256 / (avg / 1e3),
-                       "timing": "CUDA graph replay of one step, L2 flushed before each",
-                       "stages_eager_us": {k: round(v[2] / v[0] * 1e3, 1) for k, v in stg.items()}}
-    res["decode_b256_1p4b"] = dec
+    import oracle
+    from nested_mamba2_selective_b200 import synth
+    S = SCAN
+    inp = synth.ssd_inputs(S["batch"], S["seq_len"], S["heads"], S["d_head"], S["d_state"], 1, "bf16", seed=1001)
+    rows, t0 = 0, time.perf_counter()
+    while rows < S["batch"] and time.perf_counter() - t0 < budget_s:
+        sl = slice(rows, rows + 1)
+        oracle.ssd_scan(inp["x"][sl], inp["dt"][sl], inp["A"], inp["B"][sl], inp["C"][sl], inp["D"])
+        rows += 1
+    el = time.perf_counter() - t0
+    res = {"value": rows * S["seq_len"] / el, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+           "sample": "%d of %d batch rows x %d tokens, 24 heads (fp64 sequential scan, OpenMP)"
+                     % (rows, S["batch"], S["seq_len"])}
+    code = ("import sys, time; sys.path.insert(0, %r)\n"
+            "import oracle\nfrom nested_mamba2_selective_b200 import synth\n"
+            "i = synth.ssd_inputs(1, 2048, 24, 64, 128, 1, 'bf16', seed=1001)\n"
+            "t = time.perf_counter(); oracle.ssd_scan(i['x'], i['dt'], i['A'], i['B'], i['C'], i['D'])\n"
+            "print(2048 / (time.perf_counter() - t), oracle.num_threads())\n" % ROOT)
+    try:
+        r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=120,
+                           env=dict(os.environ, OMP_NUM_THREADS="1"))
+        v, c = r.stdout.split()
+        res["one_core"] = {"value": float(v), "unit": "tokens/s", "cores": int(c),
+                           "sample": "one batch row x 2048 tokens, 24 heads"}
+    except Exception as e:  # noqa: BLE001 - the 1-core figure is informative only
+        res["one_core"] = {"error": str(e)[:200]}
     return res
 
 

@@ -158,9 +158,16 @@ int matmamba_block_fwd(const mm_block_params* p, const void* u, int batch, int L
 
 /*
  * Same computation with u and out in HOST memory: copies u to u_dev, runs
- * matmamba_block_fwd, copies out_dev back to out_host and waits for the
- * stream.  u_dev and out_dev are caller-owned device buffers of the same
- * shapes.  Pinned host buffers give asynchronous copies.
+ * matmamba_block_fwd, copies out_dev back to out_host and waits.  u_dev and
+ * out_dev are caller-owned device buffers of the same shapes.  The batch is
+ * cut into up to four sub-batches of whole sequences (sequences are
+ * independent; a sub-batch may take another scan schedule, so results match
+ * a single call up to rounding): sub-batch i computes on
+ * `stream` while sub-batch i+1 is uploaded and sub-batch i-1 downloaded on two
+ * copy streams the library creates once per device, so with pinned host
+ * buffers the transfers in both directions overlap the compute.  The call
+ * orders itself after earlier work on `stream` and returns once out_host
+ * holds the result.
  */
 int matmamba_block_fwd_host(const mm_block_params* p, const void* u_host, int batch, int L, int m_i, int chunk,
                             void* out_host, void* u_dev, void* out_dev, void* workspace, size_t ws_bytes,

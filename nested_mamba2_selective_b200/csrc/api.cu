@@ -445,6 +445,42 @@ int matmamba_block_fwd(const mm_block_params* p, const void* u, int batch, int L
                       static_cast<cudaStream_t>(stream));
 }
 
+// Streams and events of the host-buffer entry point, created once per device (no device memory):
+// copies in and out run on their own streams so that sub-batch i's compute overlaps the upload of
+// sub-batch i+1 and the download of sub-batch i-1.
+namespace {
+constexpr int kMaxSub = 8;
+struct HostPipe {
+    cudaStream_t in = nullptr, out = nullptr;
+    cudaEvent_t start = nullptr, done = nullptr, up[kMaxSub] = {}, comp[kMaxSub] = {};
+    bool ready = false;
+};
+HostPipe g_pipes[64];
+
+cudaError_t host_pipe(HostPipe** out)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    HostPipe& hp = g_pipes[dev];
+    if (!hp.ready) {
+        const unsigned ef = cudaEventDisableTiming;
+        if ((e = cudaStreamCreateWithFlags(&hp.in, cudaStreamNonBlocking)) != cudaSuccess) return e;
+        if ((e = cudaStreamCreateWithFlags(&hp.out, cudaStreamNonBlocking)) != cudaSuccess) return e;
+        if ((e = cudaEventCreateWithFlags(&hp.start, ef)) != cudaSuccess) return e;
+        if ((e = cudaEventCreateWithFlags(&hp.done, ef)) != cudaSuccess) return e;
+        for (int i = 0; i < kMaxSub; ++i) {
+            if ((e = cudaEventCreateWithFlags(&hp.up[i], ef)) != cudaSuccess) return e;
+            if ((e = cudaEventCreateWithFlags(&hp.comp[i], ef)) != cudaSuccess) return e;
+        }
+        hp.ready = true;
+    }
+    *out = &hp;
+    return cudaSuccess;
+}
+}  // namespace
+
 int matmamba_block_fwd_host(const mm_block_params* p, const void* u_host, int batch, int L, int m_i, int chunk,
                             void* out_host, void* u_dev, void* out_dev, void* workspace, size_t ws_bytes, void* stream)
 {
@@ -454,15 +490,45 @@ int matmamba_block_fwd_host(const mm_block_params* p, const void* u_host, int ba
     if (rc) return rc;
     if (batch <= 0 || L <= 0) return MM_ERR_SHAPE;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const size_t bytes = (size_t)batch * L * v.Dm * esize(p->dtype);
+    const size_t row_bytes = (size_t)L * v.Dm * esize(p->dtype);  // one sequence of u or out
     size_t need;
     if ((rc = matmamba_block_workspace(p, batch, L, m_i, chunk, &need))) return rc;
     if (!workspace || ws_bytes < need) return MM_ERR_WORKSPACE;
-    MM_TRY(cudaMemcpyAsync(u_dev, u_host, bytes, cudaMemcpyHostToDevice, s));
-    rc = matmamba_block_fwd(p, u_dev, batch, L, m_i, chunk, out_dev, nullptr, nullptr, nullptr, nullptr, workspace,
-                            ws_bytes, stream);
-    if (rc) return rc;
-    MM_TRY(cudaMemcpyAsync(out_host, out_dev, bytes, cudaMemcpyDeviceToHost, s));
+    // sub-batches of whole sequences (sequences are independent); each must fit the workspace
+    int nsub = batch < 4 ? batch : 4;
+    for (; nsub > 1; --nsub) {
+        const int per = (batch + nsub - 1) / nsub;
+        size_t sub_need;
+        if (!matmamba_block_workspace(p, per, L, m_i, chunk, &sub_need) && sub_need <= ws_bytes) break;
+    }
+    HostPipe* hp;
+    MM_TRY(host_pipe(&hp));
+    MM_TRY(cudaEventRecord(hp->start, s));  // earlier work on s (users of u_dev / out_dev) comes first
+    MM_TRY(cudaStreamWaitEvent(hp->in, hp->start, 0));
+    MM_TRY(cudaStreamWaitEvent(hp->out, hp->start, 0));
+    const int per = (batch + nsub - 1) / nsub;
+    for (int i = 0, b0 = 0; b0 < batch; ++i, b0 += per) {
+        const int nb = batch - b0 < per ? batch - b0 : per;
+        const size_t off = (size_t)b0 * row_bytes, bytes = (size_t)nb * row_bytes;
+        char* ud = static_cast<char*>(u_dev) + off;
+        char* od = static_cast<char*>(out_dev) + off;
+        MM_TRY(cudaMemcpyAsync(ud, static_cast<const char*>(u_host) + off, bytes, cudaMemcpyHostToDevice, hp->in));
+        MM_TRY(cudaEventRecord(hp->up[i], hp->in));
+        MM_TRY(cudaStreamWaitEvent(s, hp->up[i], 0));
+        rc = matmamba_block_fwd(p, ud, nb, L, m_i, chunk, od, nullptr, nullptr, nullptr, nullptr, workspace, ws_bytes,
+                                stream);
+        if (rc) {
+            cudaStreamSynchronize(hp->in);
+            cudaStreamSynchronize(s);
+            cudaStreamSynchronize(hp->out);
+            return rc;
+        }
+        MM_TRY(cudaEventRecord(hp->comp[i], s));
+        MM_TRY(cudaStreamWaitEvent(hp->out, hp->comp[i], 0));
+        MM_TRY(cudaMemcpyAsync(static_cast<char*>(out_host) + off, od, bytes, cudaMemcpyDeviceToHost, hp->out));
+    }
+    MM_TRY(cudaEventRecord(hp->done, hp->out));
+    MM_TRY(cudaStreamWaitEvent(s, hp->done, 0));
     MM_TRY(cudaStreamSynchronize(s));
     return MM_OK;
 }
@@ -556,17 +622,39 @@ int mm_linear(int dtype, const void* A, int64_t lda, int M, int K, const void* W
     return cuda_status(stage("linear", 1, s, [&] { return run_gemm(dtype, g, s); }));
 }
 
+// Buffers of one recurrent step in the caller's workspace.
+struct StepBufs {
+    void *zxbc, *xbc, *y, *nrm;
+    float *dt_raw, *dt, *row_parts;
+};
+
+static StepBufs carve_step(Carver& c, const View& v, const mm_block_params* p, int batch)
+{
+    const size_t es = esize(p->dtype);
+    StepBufs b{};
+    b.zxbc = c.take((size_t)batch * (v.d + v.nconv) * es);
+    b.dt_raw = static_cast<float*>(c.take((size_t)batch * v.h * 4));
+    b.xbc = c.take((size_t)batch * v.nconv * es);
+    b.dt = static_cast<float*>(c.take((size_t)batch * v.h * 4));
+    b.y = c.take((size_t)batch * v.d * es);
+    b.nrm = c.take((size_t)batch * v.d * es);
+    b.row_parts = static_cast<float*>(c.take((size_t)batch * 2 * v.h * 4));
+    return b;
+}
+
 static size_t step_ws(const View& v, const mm_block_params* p, int batch)
 {
     Carver c(nullptr);
-    const size_t es = esize(p->dtype);
-    c.take((size_t)batch * (v.d + v.nconv) * es);
-    c.take((size_t)batch * v.h * 4);
-    c.take((size_t)batch * v.nconv * es);
-    c.take((size_t)batch * v.h * 4);
-    c.take((size_t)batch * v.d * es);
-    c.take((size_t)batch * v.d * es);
+    carve_step(c, v, p, batch);
     return c.used;
+}
+
+// The gate and norm fold into the step's scan and out_proj (bf16, d_head 64, d_state 128, aligned state
+// rows, tensor-core out_proj).
+static bool step_gated_ok(const View& v, const mm_block_params* p, const float* ssm_state, const GemmDesc& go)
+{
+    return p->dtype == MM_BF16 && v.P == 64 && v.N == 128 && (reinterpret_cast<uintptr_t>(ssm_state) & 15u) == 0 &&
+           gemm_tc_supported(go);
 }
 
 int ssd_step_workspace(const mm_block_params* p, int batch, int m_i, size_t* bytes)
@@ -592,28 +680,37 @@ int ssd_step(const mm_block_params* p, float* ssm_state, void* conv_state, const
     if (!workspace || ws_bytes < step_ws(v, p, batch)) return MM_ERR_WORKSPACE;
     if (reinterpret_cast<uintptr_t>(workspace) % kAlign) return MM_ERR_ALIGN;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const size_t es = esize(p->dtype);
     Carver c(workspace);
-    void* zxbc = c.take((size_t)batch * (v.d + v.nconv) * es);
-    float* dt_raw = static_cast<float*>(c.take((size_t)batch * v.h * 4));
-    void* xbc = c.take((size_t)batch * v.nconv * es);
-    float* dt = static_cast<float*>(c.take((size_t)batch * v.h * 4));
-    void* y = c.take((size_t)batch * v.d * es);
-    void* nrm = c.take((size_t)batch * v.d * es);
-    MM_TRY(stage("step_in_proj", 1, s, [&] { return run_gemm(p->dtype, in_proj_desc(v, p, u_t, batch, zxbc, dt_raw), s); }));
+    const StepBufs b = carve_step(c, v, p, batch);
+    MM_TRY(stage("step_in_proj", 1, s,
+                 [&] { return run_gemm(p->dtype, in_proj_desc(v, p, u_t, batch, b.zxbc, b.dt_raw), s); }));
     MM_TRY(stage("step_conv_dt", 1, s, [&] {
-        return launch_step_conv_dt(p->dtype, zxbc, v.d + v.nconv, v.d, dt_raw, p->conv_w, p->conv_b, p->dt_bias, v.E,
-                                   v.d, v.nconv, v.h, v.K, batch, conv_state, v.E + 2 * v.GN, xbc, dt, s);
+        return launch_step_conv_dt(p->dtype, b.zxbc, v.d + v.nconv, v.d, b.dt_raw, p->conv_w, p->conv_b, p->dt_bias,
+                                   v.E, v.d, v.nconv, v.h, v.K, batch, conv_state, v.E + 2 * v.GN, b.xbc, b.dt, s);
     }));
+    GemmDesc go = out_proj_desc(v, p, b.nrm, batch, out_t, 0);
+    if (step_gated_ok(v, p, ssm_state, go)) {
+        // scan with the gate in its output, out_proj scaling rows by 1/RMS from the partial sums
+        MM_TRY(stage("step_scan_gate", 1, s, [&] {
+            return launch_step_scan_gated(b.xbc, v.nconv, v.d, b.dt, p->A, p->D, ssm_state, v.H, v.h, v.GN, v.hpg,
+                                          batch, b.zxbc, v.d + v.nconv, p->norm_w, b.nrm, b.row_parts, s);
+        }));
+        go.ex.row_parts = b.row_parts;
+        go.ex.nparts = 2 * v.h;
+        go.ex.rs_inv_n = 1.0f / (float)v.d;
+        go.ex.rs_eps = p->norm_eps;
+        MM_TRY(stage("step_out_proj_norm", 1, s, [&] { return launch_gemm_tc(go, s); }));
+        return MM_OK;
+    }
     MM_TRY(stage("step_scan", 1, s, [&] {
-        return launch_step_scan(p->dtype, xbc, v.nconv, v.d, dt, p->A, p->D, ssm_state, v.H, v.h, v.P, v.N, v.GN,
-                                v.hpg, batch, y, s);
+        return launch_step_scan(p->dtype, b.xbc, v.nconv, v.d, b.dt, p->A, p->D, ssm_state, v.H, v.h, v.P, v.N, v.GN,
+                                v.hpg, batch, b.y, s);
     }));
     MM_TRY(stage("step_gate_rmsnorm", 1, s, [&] {
-        return launch_gate_rmsnorm(p->dtype, y, v.d, zxbc, v.d + v.nconv, p->norm_w, p->norm_eps, v.d, batch, nrm, v.d,
-                                   s);
+        return launch_gate_rmsnorm(p->dtype, b.y, v.d, b.zxbc, v.d + v.nconv, p->norm_w, p->norm_eps, v.d, batch,
+                                   b.nrm, v.d, s);
     }));
-    MM_TRY(stage("step_out_proj", 1, s, [&] { return run_gemm(p->dtype, out_proj_desc(v, p, nrm, batch, out_t, 0), s); }));
+    MM_TRY(stage("step_out_proj", 1, s, [&] { return run_gemm(p->dtype, go, s); }));
     return MM_OK;
 }
 

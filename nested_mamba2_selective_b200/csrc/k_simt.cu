@@ -548,6 +548,110 @@ __global__ void __launch_bounds__(256) step_scan_kernel(const T* __restrict__ xb
     }
 }
 
+// The same update with the gate folded into its output (bf16, N == 128, P == 64, 16-byte aligned
+// state rows): instead of y it stores n = (y * SiLU(z)) * norm_w and, per (sequence, head, 32-channel
+// half), the sum of squares of y * SiLU(z) into row_parts[b * 2h + 2 i + half]; the output projection
+// then scales each row by 1/RMS.  The per-warp partial sums are added in warp order (deterministic).
+__global__ void __launch_bounds__(256) step_scan_gated_kernel(const __nv_bfloat16* __restrict__ xbc, int nconv, int d,
+                                                              const float* __restrict__ dt, const float* __restrict__ A,
+                                                              const float* __restrict__ D, float* __restrict__ ssm_state,
+                                                              int H, int h, int GN, int hpg,
+                                                              const __nv_bfloat16* __restrict__ z, int64_t ldz,
+                                                              const __nv_bfloat16* __restrict__ norm_w,
+                                                              __nv_bfloat16* __restrict__ nrm, float* __restrict__ row_parts)
+{
+    constexpr int P = 64, N = 128;
+    __shared__ float part[8][2];
+    const int b = blockIdx.x / h, i = blockIdx.x % h;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = i / hpg;
+    const __nv_bfloat16* xr = xbc + (int64_t)b * nconv;
+    const __nv_bfloat16* zr = z + (int64_t)b * ldz;
+    const float dtv = dt[(int64_t)b * h + i];
+    const float av = expf(dtv * A[i]);
+    const float Di = D[i];
+    const __nv_bfloat16* Bv = xr + d + g * N;
+    const __nv_bfloat16* Cv = xr + d + GN + g * N;
+    float* st = ssm_state + ((int64_t)b * H + i) * P * N;
+    float bq[4], cq[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        bq[e] = to_f32(Bv[4 * lane + e]);
+        cq[e] = to_f32(Cv[4 * lane + e]);
+    }
+    // this warp's rows are p = warp + 8 j (j < 8); lane j < 8 fetches z and norm_w of row j up front and
+    // later gates that row, so no dependent global load sits in the state loop
+    float zr_l = 0.0f, nw_l = 0.0f;
+    if (lane < 8) {
+        const int c = i * P + warp + 8 * lane;
+        zr_l = silu_f(to_f32(zr[c]));
+        nw_l = to_f32(norm_w[c]);
+    }
+    float ssq = 0.0f;  // lane j's row (lanes < 8)
+#pragma unroll 1
+    for (int p0 = warp; p0 < P; p0 += 16) {  // rows p0 and p0 + 8: both in the same half
+        const int p1 = p0 + 8;
+        float4* r0 = reinterpret_cast<float4*>(st + (int64_t)p0 * N) + lane;
+        float4* r1 = reinterpret_cast<float4*>(st + (int64_t)p1 * N) + lane;
+        float4 s0 = *r0, s1 = *r1;
+        const float x0 = to_f32(xr[i * P + p0]), x1 = to_f32(xr[i * P + p1]);
+        const float d0 = dtv * x0, d1 = dtv * x1;
+        s0.x = fmaf(av, s0.x, d0 * bq[0]); s0.y = fmaf(av, s0.y, d0 * bq[1]);
+        s0.z = fmaf(av, s0.z, d0 * bq[2]); s0.w = fmaf(av, s0.w, d0 * bq[3]);
+        s1.x = fmaf(av, s1.x, d1 * bq[0]); s1.y = fmaf(av, s1.y, d1 * bq[1]);
+        s1.z = fmaf(av, s1.z, d1 * bq[2]); s1.w = fmaf(av, s1.w, d1 * bq[3]);
+        *r0 = s0;
+        *r1 = s1;
+        float a0 = fmaf(cq[3], s0.w, fmaf(cq[2], s0.z, fmaf(cq[1], s0.y, cq[0] * s0.x)));
+        float a1 = fmaf(cq[3], s1.w, fmaf(cq[2], s1.z, fmaf(cq[1], s1.y, cq[0] * s1.x)));
+#pragma unroll
+        for (int o = 16; o; o >>= 1) {
+            a0 += __shfl_xor_sync(0xffffffffu, a0, o);
+            a1 += __shfl_xor_sync(0xffffffffu, a1, o);
+        }
+        // row p0 is lane j0 = (p0 - warp) / 8's, row p1 lane j0 + 1's
+        const int j0 = (p0 - warp) >> 3;
+        if (lane == j0 || lane == j0 + 1) {
+            const bool second = lane == j0 + 1;
+            const float q = fmaf(Di, second ? x1 : x0, second ? a1 : a0) * zr_l;
+            ssq = q * q;
+            nrm[(int64_t)b * d + i * P + (second ? p1 : p0)] = from_f32<__nv_bfloat16>(q * nw_l);
+        }
+    }
+    // half 0 holds rows p < 32 (lanes 0-3), half 1 rows p >= 32 (lanes 4-7); summed in lane order
+    float h0 = 0.0f, h1 = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const float v = __shfl_sync(0xffffffffu, ssq, j);
+        if (j < 4) h0 += v;
+        else h1 += v;
+    }
+    const float ssq2[2] = {h0, h1};
+    if (lane == 0) {
+        part[warp][0] = ssq2[0];
+        part[warp][1] = ssq2[1];
+    }
+    __syncthreads();
+    if (threadIdx.x < 2) {
+        float tot = 0.0f;
+        for (int w = 0; w < 8; ++w) tot += part[w][threadIdx.x];
+        row_parts[(int64_t)b * 2 * h + 2 * i + threadIdx.x] = tot;
+    }
+}
+
+cudaError_t launch_step_scan_gated(const void* xbc, int nconv, int d, const float* dt, const float* A, const float* D,
+                                   float* ssm_state, int H, int h, int GN, int hpg, int batch, const void* z,
+                                   int64_t ldz, const void* norm_w, void* nrm, float* row_parts, cudaStream_t s)
+{
+    const int64_t heads = (int64_t)batch * h;
+    if (heads == 0) return cudaSuccess;
+    if (heads > 0x7fffffff) return cudaErrorInvalidValue;
+    step_scan_gated_kernel<<<(unsigned)heads, 256, 0, s>>>(
+        (const __nv_bfloat16*)xbc, nconv, d, dt, A, D, ssm_state, H, h, GN, hpg, (const __nv_bfloat16*)z, ldz,
+        (const __nv_bfloat16*)norm_w, (__nv_bfloat16*)nrm, row_parts);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_step_scan(int dtype, const void* xbc, int nconv, int d, const float* dt, const float* A,
                              const float* D, float* ssm_state, int H, int h, int P, int N, int GN, int hpg, int batch,
                              void* y, cudaStream_t s)

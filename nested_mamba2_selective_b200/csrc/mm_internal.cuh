@@ -117,6 +117,10 @@ cudaError_t launch_step_scan(int dtype, const void* xbc, int nconv, int d, const
                              const float* D, float* ssm_state, int H, int h, int P, int N, int GN, int hpg, int batch,
                              void* y, cudaStream_t s);
 
+cudaError_t launch_step_scan_gated(const void* xbc, int nconv, int d, const float* dt, const float* A, const float* D,
+                                   float* ssm_state, int H, int h, int GN, int hpg, int batch, const void* z,
+                                   int64_t ldz, const void* norm_w, void* nrm, float* row_parts, cudaStream_t s);
+
 // Device status word of the current device (MM_OK or a code a kernel recorded).
 int* device_status_ptr();
 bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint64_t pitch,
