@@ -625,7 +625,7 @@ int mm_linear(int dtype, const void* A, int64_t lda, int M, int K, const void* W
 // Buffers of one recurrent step in the caller's workspace.
 struct StepBufs {
     void *zxbc, *xbc, *y, *nrm;
-    float *dt_raw, *dt, *row_parts;
+    float *dt_raw, *dt, *row_parts, *out32;
 };
 
 static StepBufs carve_step(Carver& c, const View& v, const mm_block_params* p, int batch)
@@ -639,6 +639,7 @@ static StepBufs carve_step(Carver& c, const View& v, const mm_block_params* p, i
     b.y = c.take((size_t)batch * v.d * es);
     b.nrm = c.take((size_t)batch * v.d * es);
     b.row_parts = static_cast<float*>(c.take((size_t)batch * 2 * v.h * 4));
+    b.out32 = static_cast<float*>(c.take((size_t)batch * v.Dm * 4));
     return b;
 }
 
@@ -649,8 +650,9 @@ static size_t step_ws(const View& v, const mm_block_params* p, int batch)
     return c.used;
 }
 
-// The gate and norm fold into the step's scan and out_proj (bf16, d_head 64, d_state 128, aligned state
-// rows, tensor-core out_proj).
+// The gate and norm fold into the step's scan and out_proj (bf16, d_head 64, d_state 128, 16-byte
+// aligned state rows, tensor-core out_proj).  out_proj then adds its K slices (few rows, a long K)
+// into an fp32 buffer with the 1/RMS row scale, which is rounded to the output afterwards.
 static bool step_gated_ok(const View& v, const mm_block_params* p, const float* ssm_state, const GemmDesc& go)
 {
     return p->dtype == MM_BF16 && v.P == 64 && v.N == 128 && (reinterpret_cast<uintptr_t>(ssm_state) & 15u) == 0 &&
@@ -688,18 +690,22 @@ int ssd_step(const mm_block_params* p, float* ssm_state, void* conv_state, const
         return launch_step_conv_dt(p->dtype, b.zxbc, v.d + v.nconv, v.d, b.dt_raw, p->conv_w, p->conv_b, p->dt_bias,
                                    v.E, v.d, v.nconv, v.h, v.K, batch, conv_state, v.E + 2 * v.GN, b.xbc, b.dt, s);
     }));
-    GemmDesc go = out_proj_desc(v, p, b.nrm, batch, out_t, 0);
+    GemmDesc go = out_proj_desc(v, p, b.nrm, batch, b.out32, 1);
+    go.ex.row_parts = b.row_parts;
+    go.ex.nparts = 2 * v.h;
+    go.ex.rs_inv_n = 1.0f / (float)v.d;
+    go.ex.rs_eps = p->norm_eps;
     if (step_gated_ok(v, p, ssm_state, go)) {
-        // scan with the gate in its output, out_proj scaling rows by 1/RMS from the partial sums
         MM_TRY(stage("step_scan_gate", 1, s, [&] {
             return launch_step_scan_gated(b.xbc, v.nconv, v.d, b.dt, p->A, p->D, ssm_state, v.H, v.h, v.GN, v.hpg,
                                           batch, b.zxbc, v.d + v.nconv, p->norm_w, b.nrm, b.row_parts, s);
         }));
-        go.ex.row_parts = b.row_parts;
-        go.ex.nparts = 2 * v.h;
-        go.ex.rs_inv_n = 1.0f / (float)v.d;
-        go.ex.rs_eps = p->norm_eps;
-        MM_TRY(stage("step_out_proj_norm", 1, s, [&] { return launch_gemm_tc(go, s); }));
+        MM_TRY(stage("step_out_proj_norm", 2, s, [&] {
+            cudaError_t e = cudaMemsetAsync(b.out32, 0, (size_t)batch * v.Dm * 4, s);
+            if (e == cudaSuccess) e = launch_gemm_tc(go, s);
+            if (e == cudaSuccess) e = launch_from_f32(p->dtype, b.out32, out_t, (int64_t)batch * v.Dm, s);
+            return e;
+        }));
         return MM_OK;
     }
     MM_TRY(stage("step_scan", 1, s, [&] {
@@ -710,7 +716,8 @@ int ssd_step(const mm_block_params* p, float* ssm_state, void* conv_state, const
         return launch_gate_rmsnorm(p->dtype, b.y, v.d, b.zxbc, v.d + v.nconv, p->norm_w, p->norm_eps, v.d, batch,
                                    b.nrm, v.d, s);
     }));
-    MM_TRY(stage("step_out_proj", 1, s, [&] { return run_gemm(p->dtype, go, s); }));
+    MM_TRY(stage("step_out_proj", 1, s,
+                 [&] { return run_gemm(p->dtype, out_proj_desc(v, p, b.nrm, batch, out_t, 0), s); }));
     return MM_OK;
 }
 

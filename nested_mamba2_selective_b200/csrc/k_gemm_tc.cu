@@ -60,6 +60,9 @@ struct OutMaps {
 
 struct TcParams {
     int M, K, ktiles, mtiles, ntiles, nseg;
+    // split K: tiles come in ksplit K slices of kper k-tiles each; every slice adds its partial
+    // product into the (fp32, bulk-add) output, so only single-segment accumulating outputs split
+    int ksplit, kper;
     int shift;  // halo rows at the top of each tile (K-1 with a conv segment, else 0)
     int rows;   // output rows per tile = 128 - shift
     // Paired tiles (the first pair_tiles tiles of a row block): columns [n0, n0 + BN/2) of segment
@@ -76,12 +79,18 @@ template <int BN>
 struct TileInfo {
     int mt, seg, n0, nvalid, b_row;
     int seg2, b_row2;  // paired tile: the conv segment and its B row (else seg2 = -1)
+    int k0, k1;        // k-tiles [k0, k1) of this tile's K slice
 };
 
 template <int BN>
 __device__ __forceinline__ TileInfo<BN> tile_info(const TcParams& p, int tile)
 {
     TileInfo<BN> t;
+    const int per_slice = p.mtiles * p.ntiles;
+    const int ks = tile / per_slice;
+    tile -= ks * per_slice;
+    t.k0 = ks * p.kper;
+    t.k1 = min(p.ktiles, t.k0 + p.kper);
     // row-block major: the N tiles of a row block are consecutive, so CTAs working at the same
     // time share its A rows in L2
     t.mt = tile / p.ntiles;
@@ -131,18 +140,14 @@ __device__ __forceinline__ void store_bf16_chunk(__nv_bfloat16* o, int ncols, bo
     }
 }
 
-// PAIR: the kernel runs as clusters of two CTAs sharing each MMA (M = 256 over the pair).  CTA r
-// of a cluster takes row block 2 m + r of tile pair (m, j), loads its own A rows and half of the
-// tile's B rows (the first half in the even CTA, the second in the odd one), and drains its own
-// accumulator rows; the even CTA issues the MMAs.  The walk over tile pairs is static.
-template <int BN, int STAGES, bool CONV, bool PAIR>
+template <int BN, int STAGES, bool CONV>
 __global__ void __launch_bounds__(320, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
                    const __grid_constant__ CUtensorMap mapB2, const __grid_constant__ OutMaps omaps, const TcParams p)
 {
     constexpr int A_BYTES = kBM * kBK * 2;
     constexpr int B_BYTES = BN * kBK * 2;
-    constexpr int STAGE_BYTES = A_BYTES + (PAIR ? B_BYTES / 2 : B_BYTES);  // this CTA's bytes of a stage
+    constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
     constexpr uint32_t TMEM_COLS = 2 * BN;
 
     extern __shared__ uint8_t smem_raw[];
@@ -165,15 +170,14 @@ __global__ void __launch_bounds__(320, 1)
     volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const uint32_t rank = PAIR ? cluster_ctarank() : 0;  // 0 issues the pair's MMAs
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&full[s], PAIR ? 2 : 1);  // the pair: both producers arrive on the even CTA's
+            mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&tfull[b], 1);
-            mbar_init(&tempty[b], PAIR ? 16 : 8);  // the pair: both CTAs' drain warps
+            mbar_init(&tempty[b], 8);
         }
         for (int j = 0; j < kTileRing; ++j) {
             mbar_init(&cfull[j], 1);
@@ -187,31 +191,16 @@ __global__ void __launch_bounds__(320, 1)
         if (p.pair_tiles) prefetch_tmap(&mapB2);
     }
     if (warp == 1) {
-        if (PAIR) {
-            tmem_alloc_pair(tmem_slot, TMEM_COLS);
-            tmem_relinquish_pair();
-        } else {
-            tmem_alloc(tmem_slot, TMEM_COLS);
-            tmem_relinquish();
-        }
+        tmem_alloc(tmem_slot, TMEM_COLS);
+        tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
-    if (PAIR) cluster_sync();  // both CTAs' barriers are initialised before any arrives on them
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const int total = p.mtiles * p.ntiles;
-    // the pair's static walk: tile pair tp = (row-block pair tp / ntiles, N tile tp % ntiles)
-    const int total_pairs = ((p.mtiles + 1) / 2) * p.ntiles;
-    const int ncl = (int)gridDim.x / 2, cl = (int)blockIdx.x / 2;
-    auto pair_tile = [&](int tp) -> int { return ((tp / p.ntiles) * 2 + (int)rank) * p.ntiles + tp % p.ntiles; };
-    // the even CTA's accumulator barriers and stage barriers, in cluster space
-    const uint32_t tempty_l = PAIR ? map_to_rank(tempty, 0) : 0;
-    const uint32_t full_l = PAIR ? map_to_rank(full, 0) : 0;
-    auto release_acc = [&](int b) {  // this drain warp is done with accumulator b
-        if (PAIR && rank != 0) mbar_arrive_cluster(tempty_l + 8u * b);
-        else mbar_arrive(&tempty[b]);
-    };
+    // tiles: (K slice, row block, N tile), K slices slowest
+    const int total = p.mtiles * p.ntiles * p.ksplit;
+    auto release_acc = [&](int b) { mbar_arrive(&tempty[b]); };  // this drain warp is done with accumulator b
     // The tile of position j + 1 (`total` once the walk is over) from the scheduler's answer j;
     // each reader then releases the answer's slot (the MMA lane alone, or a drain warp once all
     // its lanes have read).  The wait ignores the abort flag, so every reader of an answer that
@@ -227,31 +216,7 @@ __global__ void __launch_bounds__(320, 1)
     };
 
     if (warp == 0) {
-        if (PAIR && lane == 0) {  // ---------------- TMA producer of a pair CTA
-            int it = 0;
-            for (int j = 0; cl + j * ncl < total_pairs && !*abort; ++j) {
-                const TileInfo<BN> t = tile_info<BN>(p, pair_tile(cl + j * ncl));
-                const int arow = t.mt * p.rows - p.shift;  // rows outside [0, M) load as zeros
-                const int brow = t.seg2 >= 0 ? (rank ? t.b_row2 : t.b_row) : t.b_row + (int)rank * (BN / 2);
-                for (int kt = 0; kt < p.ktiles; ++kt, ++it) {
-                    const int s = it % STAGES;
-                    if (!mbar_wait(&empty[s], ((it / STAGES) & 1) ^ 1, abort)) {
-                        raise_timeout(abort, p.status);
-                        break;
-                    }
-                    uint8_t* sa = smem + s * STAGE_BYTES;
-                    const uint32_t fb = full_l + 8u * s;
-                    if (rank == 0) mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
-                    else mbar_arrive_expect_tx_cluster(fb, STAGE_BYTES);
-                    tma_load_2d_pair(sa, &mapA, fb, kt * kBK, arow);
-                    tma_load_2d_pair(sa + A_BYTES, &mapB2, fb, kt * kBK, brow);
-                }
-            }
-            // the even CTA sees every load of both CTAs land (bounded); the odd CTA's loads have
-            // landed before the even CTA reaches the closing cluster barrier
-            if (rank == 0)
-                for (int i = max(0, it - STAGES); i < it; ++i) mbar_wait(&full[i % STAGES], (i / STAGES) & 1, nullptr);
-        } else if (!PAIR && lane == 0) {  // ---------------- tile scheduler and TMA producer
+        if (lane == 0) {  // ---------------- tile scheduler and TMA producer
             // Tile position 0 is this CTA's own index; the tile of position j + 1 is the index of a
             // CTA that had not started yet, cancelled by a launch-control request made while tile j
             // loads.  An answer that cancelled nothing ends the walk (the grid has one CTA per tile).
@@ -268,7 +233,7 @@ __global__ void __launch_bounds__(320, 1)
                 asked = true;
                 const TileInfo<BN> t = tile_info<BN>(p, tile);
                 const int arow = t.mt * p.rows - p.shift;  // may be negative: rows above 0 load as zeros
-                for (int kt = 0; kt < p.ktiles; ++kt, ++it) {
+                for (int kt = t.k0; kt < t.k1; ++kt, ++it) {
                     const int s = it % STAGES;
                     if (!mbar_wait(&empty[s], ((it / STAGES) & 1) ^ 1, abort)) {
                         raise_timeout(abort, p.status);
@@ -298,37 +263,7 @@ __global__ void __launch_bounds__(320, 1)
             for (int i = max(0, it - STAGES); i < it; ++i) mbar_wait(&full[i % STAGES], (i / STAGES) & 1, nullptr);
         }
     } else if (warp == 1) {
-        if (PAIR && lane == 0 && rank == 0) {  // ---------------- MMA issuer of the pair
-            int it = 0;
-            const uint32_t idesc = idesc_bf16(2 * kBM, BN, 0, 0);
-            for (int j = 0; cl + j * ncl < total_pairs && !*abort; ++j) {
-                const int buf = j & 1;
-                if (!mbar_wait(&tempty[buf], ((j >> 1) & 1) ^ 1, abort)) {
-                    raise_timeout(abort, p.status);
-                    break;
-                }
-                tc_fence_after();
-                const uint32_t d_tmem = tmem + buf * BN;
-                for (int kt = 0; kt < p.ktiles; ++kt, ++it) {
-                    const int s = it % STAGES;
-                    if (!mbar_wait(&full[s], (it / STAGES) & 1, abort)) {
-                        raise_timeout(abort, p.status);
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint32_t a0 = smem_u32(smem + s * STAGE_BYTES);
-                    const uint32_t b0 = a0 + A_BYTES;
-#pragma unroll
-                    for (int kk = 0; kk < kBK / 16; ++kk)
-                        mma_ss_pair(d_tmem, desc_sw128(a0 + kk * 32, 16, 1024), desc_sw128(b0 + kk * 32, 16, 1024),
-                                    idesc, (kt | kk) != 0);
-                    mma_commit_pair(&empty[s]);
-                }
-                mma_commit_pair(&tfull[buf]);
-            }
-            mma_commit_pair(done);
-            mbar_wait(done, 0, nullptr);
-        } else if (!PAIR && lane == 0) {  // ---------------- MMA issuer
+        if (lane == 0) {  // ---------------- MMA issuer
             int it = 0, tc = 0;
             for (int tile = blockIdx.x; tile < total && !*abort; ++tc) {
                 const TileInfo<BN> t = tile_info<BN>(p, tile);
@@ -341,7 +276,7 @@ __global__ void __launch_bounds__(320, 1)
                 const uint32_t d_tmem = tmem + buf * BN;
                 const int nmma = t.seg2 >= 0 ? BN : (t.nvalid + 15) & ~15;
                 const uint32_t idesc = idesc_bf16(kBM, nmma, 0, 0);
-                for (int kt = 0; kt < p.ktiles; ++kt, ++it) {
+                for (int kt = t.k0; kt < t.k1; ++kt, ++it) {
                     const int s = it % STAGES;
                     if (!mbar_wait(&full[s], (it / STAGES) & 1, abort)) {
                         raise_timeout(abort, p.status);
@@ -353,7 +288,7 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
                     for (int kk = 0; kk < kBK / 16; ++kk)
                         mma_ss(d_tmem, desc_sw128(a0 + kk * 32, 16, 1024), desc_sw128(b0 + kk * 32, 16, 1024), idesc,
-                               (kt | kk) != 0);
+                               (kt != t.k0 || kk != 0) ? 1u : 0u);
                     mma_commit(&empty[s]);
                 }
                 mma_commit(&tfull[buf]);
@@ -369,10 +304,8 @@ __global__ void __launch_bounds__(320, 1)
         const int r = q * 32 + lane;  // tile row = TMEM lane
         const GemmExtra& ex = p.ex;
         int tc = 0;
-        // the walk: the pair's static one over tile pairs, else the scheduler's answers
-        auto in_walk = [&](int j, int tl) -> bool { return PAIR ? cl + j * ncl < total_pairs : tl < total; };
-        auto advance = [&](int j) -> int { return PAIR ? pair_tile(cl + (j + 1) * ncl) : next_tile(j, false); };
-        for (int tile = PAIR ? pair_tile(cl) : (int)blockIdx.x; in_walk(tc, tile); tile = advance(tc++)) {
+        // the walk: this CTA's own tile, then the scheduler's answers
+        for (int tile = (int)blockIdx.x; tile < total; tile = next_tile(tc++, false)) {
             const TileInfo<BN> t = tile_info<BN>(p, tile);
             const int buf = tc & 1;
             const TcSeg& sg = p.seg[t.seg];
@@ -748,19 +681,22 @@ __global__ void __launch_bounds__(320, 1)
                                 __nv_bfloat16* o = static_cast<__nv_bfloat16*>(cs.out) + m_r * cs.ldo + col + lc;
                                 if (two) *reinterpret_cast<uint32_t*>(o) = pack_bf16(oa, ob);
                                 else *o = __float2bfloat16_rn(oa);
-                                if (cout && tp >= ex.L - 3) {  // last K-1 pre-conv inputs of the sequence
-                                    const int64_t bq = m_r / ex.L;
-                                    const int slot = tp - (ex.L - 3);
-                                    cout[(bq * ex.conv_rows + crow) * 3 + slot] = __float2bfloat16_rn(xv.x);
-                                    if (two) cout[(bq * ex.conv_rows + crow + 1) * 3 + slot] = __float2bfloat16_rn(xv.y);
-                                }
-                                if (cout && tp == 0 && ex.L < 3) {  // older entries shift in from the history
+                                // the new conv state: older entries shift in from the history first, then
+                                // the sequence's own last inputs (this order also holds with the state
+                                // updated in place)
+                                if (cout && tp == 0 && ex.L < 3) {
                                     const int64_t bq = m_r / ex.L;
                                     for (int e = 0; e < 3 - ex.L; ++e) {
                                         const int64_t ba = (bq * ex.conv_rows + crow) * 3;
                                         cout[ba + e] = cin ? cin[ba + e + ex.L] : __float2bfloat16_rn(0.0f);
                                         if (two) cout[ba + 3 + e] = cin ? cin[ba + 3 + e + ex.L] : __float2bfloat16_rn(0.0f);
                                     }
+                                }
+                                if (cout && tp >= ex.L - 3) {  // last K-1 pre-conv inputs of the sequence
+                                    const int64_t bq = m_r / ex.L;
+                                    const int slot = tp - (ex.L - 3);
+                                    cout[(bq * ex.conv_rows + crow) * 3 + slot] = __float2bfloat16_rn(xv.x);
+                                    if (two) cout[(bq * ex.conv_rows + crow + 1) * 3 + slot] = __float2bfloat16_rn(xv.y);
                                 }
                             }
                             xa3 = xa2; xa2 = xa1; xa1 = xv.x;
@@ -788,12 +724,8 @@ __global__ void __launch_bounds__(320, 1)
     if (warp >= 2 && (warp & 3) == 2 && lane == 0) bulk_wait0();  // this group's bulk stores are complete
     tc_fence_before();
     __syncthreads();
-    if (PAIR) cluster_sync();  // the pair's MMAs, loads and arrives are all done
     tc_fence_after();
-    if (warp == 1) {
-        if (PAIR) tmem_dealloc_pair(tmem, TMEM_COLS);
-        else tmem_dealloc(tmem, TMEM_COLS);
-    }
+    if (warp == 1) tmem_dealloc(tmem, TMEM_COLS);
 }
 
 // --------------------------------------------------------------------------- host side
@@ -888,7 +820,7 @@ static bool tc_shape_ok(const GemmDesc& g)
 
 bool gemm_tc_supported(const GemmDesc& g) { return tc_shape_ok(g) && encode_fn() != nullptr; }
 
-template <int BN, int STAGES, bool CONV, bool PAIR>
+template <int BN, int STAGES, bool CONV>
 static cudaError_t launch_bn(const GemmDesc& g, const TcParams& p0, cudaStream_t s, int* status)
 {
     TcParams p = p0;
@@ -935,48 +867,26 @@ static cudaError_t launch_bn(const GemmDesc& g, const TcParams& p0, cudaStream_t
             t.tma = make_tmap_f32(&om.m[i], t.out, (uint64_t)t.n, (uint64_t)g.M, (uint64_t)t.ldo * 4, 32, kBM)
                         ? (t.accumulate ? 3 : 2) : 0;
     }
-    constexpr int smem = STAGES * (kBM + (PAIR ? BN / 2 : BN)) * kBK * 2 +
+    if (p.ksplit > 1 && p.seg[0].tma != 3) {  // K slices add their partials only through bulk adds
+        p.ksplit = 1;
+        p.kper = p.ktiles;
+    }
+    constexpr int smem = STAGES * (kBM + BN) * kBK * 2 +
                          (CONV ? 2 * kBM * kStageLd * 4 : 2 * kBM * 128) + 1024 + 512;
     static_assert(smem <= 232448, "GEMM configuration exceeds 227 KB of shared memory");
-    auto kernel = gemm_tc_kernel<BN, STAGES, CONV, PAIR>;
+    auto kernel = gemm_tc_kernel<BN, STAGES, CONV>;
     int dev = 0;
     cudaGetDevice(&dev);
     static unsigned long long attr_set = 0;  // one bit per device
-    static int max_clusters[64] = {};        // co-resident clusters of two (pair kernels)
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     if (!(attr_set >> dev & 1ull)) {
         cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
         attr_set |= 1ull << dev;
     }
-    if (!PAIR) {
-        // one CTA per tile: the CTAs that start first take over the others' tiles as they go
-        kernel<<<p.mtiles * p.ntiles, 320, smem, s>>>(mapA, mapB, mapB2, om, p);
-        return cudaGetLastError();
-    }
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cudaLaunchConfig_t cfg = {};
-    cfg.blockDim = dim3(320, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = s;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (max_clusters[dev] <= 0) {  // as many clusters as can be resident at once (a static walk)
-        int sms = 148, n = 0;
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        cfg.gridDim = dim3(2 * (sms / 2), 1, 1);
-        cudaError_t e = cudaOccupancyMaxActiveClusters(&n, kernel, &cfg);
-        if (e != cudaSuccess) return e;
-        if (n <= 0) return cudaErrorInvalidConfiguration;
-        max_clusters[dev] = n;
-    }
-    const int total_pairs = ((p.mtiles + 1) / 2) * p.ntiles;
-    cfg.gridDim = dim3(2 * min(total_pairs, max_clusters[dev]), 1, 1);
-    return cudaLaunchKernelEx(&cfg, kernel, mapA, mapB, mapB2, om, p);
+    // one CTA per tile: the CTAs that start first take over the others' tiles as they go
+    kernel<<<p.mtiles * p.ntiles * p.ksplit, 320, smem, s>>>(mapA, mapB, mapB2, om, p);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_gemm_tc(const GemmDesc& g, cudaStream_t s)
@@ -1009,19 +919,32 @@ cudaError_t launch_gemm_tc(const GemmDesc& g, cudaStream_t s)
         n_total += sg.n;
     }
     int* status = device_status_ptr();
-    // Wide tiles when they still give every SM work; narrow ones for skinny problems.
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    // One tcgen05.mma of N = 128 columns costs about as much as one of N = 256 (measured on B200:
+    // about 170-190 cycles each from one CTA), so a tile's MMA time depends on K alone and wide tiles
+    // do twice the work per instruction.  Narrow tiles only when they take no more waves over the
+    // SMs than wide ones (each SM then drains half as many columns).
     const int tiles256 = p.mtiles * ((n_total + 255) / 256);
+    const int tiles128 = p.mtiles * ((n_total + 127) / 128);
+    auto waves = [&](int t) { return (t + sms - 1) / sms; };
     const bool conv = p.shift > 0;
-    // Wide tiles could go to CTA pairs (each CTA loads half of B; two row blocks needed).  The pair
-    // mode gives the right results on B200 but was measured slower than one CTA per tile on the
-    // b8 x L2048 block at width 768 (in_proj 151 vs 107.5 us, out_proj 70 vs 40 us, with all 74
-    // clusters resident), so it stays off until the cause is found.
-    constexpr bool kPairMma = false;
-    if (kPairMma && tiles256 >= 148 && p.mtiles >= 2)
-        return conv ? launch_bn<256, 5, true, true>(g, p, s, status) : launch_bn<256, 6, false, true>(g, p, s, status);
-    if (tiles256 >= 148)
-        return conv ? launch_bn<256, 3, true, false>(g, p, s, status) : launch_bn<256, 4, false, false>(g, p, s, status);
-    return conv ? launch_bn<128, 5, true, false>(g, p, s, status) : launch_bn<128, 6, false, false>(g, p, s, status);
+    bool wide = waves(tiles256) < waves(tiles128);
+    // Too few tiles for the SMs and a long K: a single accumulating fp32 output splits K into
+    // slices whose partial products add into it (bulk tensor adds, performed in L2).
+    p.ksplit = 1;
+    p.kper = p.ktiles;
+    if (g.nseg == 1 && g.seg[0].out_f32 && g.seg[0].accumulate && g.seg[0].kind == kEpiStore && !conv &&
+        tiles256 * 2 <= sms && p.ktiles >= 4) {
+        wide = true;
+        const int ks = min(sms / tiles256, p.ktiles / 2);  // at least two k-tiles per slice
+        p.kper = (p.ktiles + ks - 1) / ks;
+        p.ksplit = (p.ktiles + p.kper - 1) / p.kper;
+    }
+    if (wide)
+        return conv ? launch_bn<256, 3, true>(g, p, s, status) : launch_bn<256, 4, false>(g, p, s, status);
+    return conv ? launch_bn<128, 5, true>(g, p, s, status) : launch_bn<128, 6, false>(g, p, s, status);
 }
 
 }  // namespace mm
