@@ -4,12 +4,16 @@
 // The scan H_t = exp(dt_t A) H_{t-1} + dt_t B_t x_t^T, y_t = C_t^T H_t + D x_t
 // ("MatMamba: A Matryoshka State Space Model", block-definition paragraph:
 // "chunk + selective scan", A and D learnable) is evaluated on blocks of
-// Q = 128 tokens.  With cs_t the running sum of dt*A inside a block:
-//   Y_diag = (Lmask o C B^T) (dt o X),  Lmask[t,s] = exp(cs_t - cs_s), s <= t
-//   Y_off  = exp(cs_t) C_t^T H_prev
-//   H_next = exp(cs_end) H_prev + B^T (w o X),  w_s = exp(cs_end - cs_s) dt_s
-// which unrolls the recurrence exactly.  The sequence is cut into segments of
-// whole blocks so that (batch, head, segment) CTAs fill the GPU:
+// Q = 128 tokens.  With cs_t the running sum of dt*A inside a block and a the
+// value of cs at the block's middle row, the chunk scan's fast blocks use
+//   y_t    = 2^(cs_t - a) [ (Gc X~)_t + C_t (2^a H_prev) ] + D x_t
+//   H_next = 2^(tot - a) [ 2^a H_prev + B^T X~ ],   X~_s = 2^(a - cs_s) dt_s x_s
+// with Gc the causally masked C B^T (log2 units): the decay becomes per-token
+// scales of x and per-row scales of y, and one contraction serves both heads of
+// a CTA.  Blocks whose decay across half a block exceeds 2^64 use exact
+// per-element decay matrices instead (see ssd_chunk_kernel).  Both unroll the
+// recurrence exactly.  The sequence is cut into segments of whole blocks so
+// that (batch, head pair, segment) CTAs fill the GPU:
 //   1. seg_state  : each segment's end state from a zero start (tcgen05)
 //   2. chunk_scan : every segment from its true start state (the initial state
 //                   carried over the earlier segments' end states at the CTA's
@@ -44,11 +48,10 @@ constexpr int kTileQP = kQ * kP * 2;              // x, X' or H block of one hea
 constexpr int kOffC = 0, kOffB = kTileQN, kOffX = 2 * kTileQN;
 constexpr int kStage = 2 * kTileQN + 2 * kTileQP; // C | B | x of two heads
 constexpr int kNStage = 2;
-constexpr int kOffHX = kNStage * kStage;          // H (then X') of two heads
 
-// TMEM columns: G = C B^T, overwritten in place by the masked M_0 | M_1 (A operands);
-// Y_0 | Y_1; Y_off of both heads; S of both heads.
-constexpr uint32_t kTG = 0, kTY = 128, kTYO = 256, kTS = 384, kTCols = 512;
+// TMEM columns: G = C B^T, overwritten in place by Gc or M_0 | M_1 (A operands); two output
+// accumulators of both heads (Y buffer i at kTY0 + 128 i); the state S of both heads.
+constexpr uint32_t kTG = 0, kTY0 = 128, kTS = 384, kTCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct ScanTcParams {
@@ -101,25 +104,41 @@ __device__ __forceinline__ float silu_approx(float x)
 __device__ __forceinline__ float bf_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
 
-// Chunk scan.  A CTA takes two heads of one (batch, segment); 512 threads in roles:
-//   warps 0-7   M builders, except warp 4: thread (quarter q = warp % 4, lane) owns TMEM lane and
-//               token row r = 32 q + lane and builds, for both heads, the masked decay matrix M
-//               over some of its row's 32-token column blocks, in place over G = C B^T.  The two
-//               warps of a quarter split the causal blocks (at most two blocks of both heads per
-//               warp) and one of them writes the zero blocks above the diagonal.
-//   warp 4      control: one lane issues the TMA loads and the tcgen05.mma; the warp owns TMEM
-//   warps 8-15  state warps: thread (q, lane, head hf) owns row r of head hf: decay scan, state
-//               read-back (bf16 copy for Y_off, decayed fp32 state for the S MMA), X', epilogue
-// The M builders work on block k while the state warps finish block k-1's epilogue.  Per block
-// k the tensor core runs G = C B^T (once Y of block k-1 has consumed M), Y_off = C [H_0 | H_1]
-// (after the read-back), then Y_j = M_j X_j and S += B^T [X'_0 | X'_1] (after M and X').
-// M factors the decay through the anchor of each 32-token column block cb (a_cb = cs at row
-// 32 cb): 2^(cs_t - cs_s) dt_s = 2^(cs_t - a_cb) * (2^(a_cb - cs_s) dt_s) for s in block cb,
-// s <= t.  The first factor is <= 1; the second, g_s, is a per-token table bounded by the decay
-// across one 32-token block.  A block whose decay exceeds 2^-kDropMax would overflow g and
-// takes direct exponentials instead (g_s = dt_s, M = G 2^min(cs_t - cs_s, 0) g_s).
+// Chunk scan.  A CTA takes two heads of one (batch, segment) and walks the segment's 128-token
+// blocks in order, carrying the fp32 state of both heads in TMEM.
+//
+// Fast blocks.  With cs_t the running sum of dt A (log2 units) from the block's start and a the
+// anchor cs at the block's middle row (63),
+//   y_t    = 2^(cs_t - a) [ sum_{s<=t} G[t,s] X~_s + C_t (2^a H) ] + D x_t,
+//   X~_s   = 2^(a - cs_s) dt_s x_s,    G = C B^T,
+//   H_next = 2^(tot - a) [ 2^a H + B^T X~ ],
+// which unrolls the recurrence exactly.  The causally masked G (Gc) does not depend on the head,
+// so one tensor-core contraction [Gc | C] . [X~ ; 2^a H] of K = 256 and N = 128 gives both heads'
+// outputs, and the per-head decay reduces to per-token scales of x (X~) and per-row scales of the
+// output.  Every exponent stays within the decay across half a block, which fast blocks bound by
+// 2^kFastMax (64 in log2 units) for both heads.
+// Steep blocks (either half of a head decays faster than that) take the direct form instead:
+// per-head masked decay matrices M_j[t,s] = G[t,s] 2^(cs_t - cs_s) dt_s with exact exponentials,
+//   y_t = M_j x + 2^(cs_t) C_t H + D x_t,   H_next = 2^tot H + B^T X',  X'_s = 2^(tot - cs_s) dt_s x_s,
+// with the state term in a second output accumulator.
+//
+// 512 threads in roles:
+//   warp 0      TMA producer (one lane)
+//   warp 1      tcgen05.mma issuer (one lane); the warp owns the TMEM allocation
+//   warps 2-7   builders: thread (quarter q = warp % 4, lane) owns TMEM lane and token row
+//               r = 32 q + lane, and turns G into Gc (fast) or M_0 | M_1 (steep) in place over
+//               some of its row's 32-token column blocks; warps 2 and 3 take the upper column
+//               blocks of quarters 2 and 3, and the lower quarters also write the zero blocks
+//   warps 8-15  state warps: thread (q, lane, head hf) owns row r of head hf: decay scan and the
+//               block's mode, state read-back (bf16 copy of the state for the C.H term, scaled
+//               fp32 state back for the state MMA), X~ (in place over x) or X', epilogue
+// Per block k the tensor core runs G = C B^T (once block k-1's G columns are consumed), then for
+// fast blocks S += B^T X~, Y = C . [2^a H_0 | 2^a H_1] and Y += Gc . [X~_0 | X~_1]; for steep
+// blocks Yoff = C . [H_0 | H_1], S += B^T X', Y_j = M_j x_j.  The two output accumulators
+// alternate between blocks, so block k-1's epilogue runs under block k's tensor work.
 // Element-wise products use the paired fp32 instructions (mul/fma .f32x2, rounded per lane
 // exactly like their scalar forms).
+
 // Blocks [c_begin, c_end) of segment `seg`.
 __device__ __forceinline__ void seg_range(const ScanTcParams& p, int seg, int* c_begin, int* c_end)
 {
@@ -133,37 +152,68 @@ __device__ __forceinline__ void grid_launch_dependents() { asm volatile("griddep
 __device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 constexpr int kChunkThreads = 512;
-constexpr int kCtlWarp = 4;
-constexpr float kDropMax = 100.0f;  // log2 units
-// small tables after the H/X' buffers (floats): state-warp scan totals [2 parity][2 heads][4],
-// M-builder scan totals [2][2][4], g [2 heads][128], cs [2][128], anchors [2][4], fallback flags [2][4]
-constexpr int kTabWtotS = 0, kTabWtotM = 16, kTabG = 32, kTabC = 288, kTabAnch = 544, kTabFlag = 552, kTabFloats = 560;
-constexpr int kOffTab = kOffHX + 2 * kTileQP;
+constexpr float kFastMax = 64.0f;  // log2 units
+// small tables after the H buffer (floats): state-warp scan totals [2 parity][2 heads][4], block
+// mode [2 parity], builder tables for steep blocks: cs [2 heads][128], dt [2 heads][128], builder
+// scan totals [2 heads][4]
+constexpr int kTabPart = 0, kTabMode = 16, kTabCs = 20, kTabDt = 276, kTabBPart = 532, kTabFloats = 540;
+constexpr int kOffH = kNStage * kStage;  // bf16 state copy of two heads (steep blocks: then X')
+constexpr int kOffTab = kOffH + 2 * kTileQP;
 constexpr int kOffBar = kOffTab + kTabFloats * 4;
-constexpr int kChunkSmem = kOffBar + 11 * 8 + 16;
+constexpr int kNumBars = 18;
+constexpr int kChunkSmem = kOffBar + kNumBars * 8 + 16;
 static_assert(kChunkSmem <= 232448, "chunk scan exceeds the 227 KB of shared memory a CTA can have");
+static_assert(kOffBar % 8 == 0, "mbarriers need 8-byte alignment");
 
 __device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
 __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
 __device__ __forceinline__ float2 bf2(uint32_t v) { return make_float2(bf_lo(v), bf_hi(v)); }
 __device__ __forceinline__ uint32_t pack2(float2 v) { return pack_bf16(v.x, v.y); }
 
+// Inclusive prefix sum over the 32 lanes of a warp.
+__device__ __forceinline__ float warp_incl_scan(float v, int lane)
+{
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const float u = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += u;
+    }
+    return v;
+}
+
+// Fast-block test of one head from its four 32-row partial sums (log2 units, each <= 0): the
+// anchor a (cs at row 63) and the total; exponents of the fast form stay within [-64, 64].
+__device__ __forceinline__ bool fast_head(const float* part, float* a_out, float* tot_out)
+{
+    const float a = part[0] + part[1];
+    const float tot = a + part[2] + part[3];
+    *a_out = a;
+    *tot_out = tot;
+    return a - tot <= kFastMax && -a <= kFastMax;
+}
+
+template <bool GATED>
 __global__ void __launch_bounds__(kChunkThreads, 1)
     ssd_chunk_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CUtensorMap mapB,
                      const __grid_constant__ CUtensorMap mapC, const __grid_constant__ CUtensorMap mapY,
-                     const ScanTcParams p)
+                     const __grid_constant__ CUtensorMap mapZ, const ScanTcParams p)
 {
     extern __shared__ __align__(1024) uint8_t sm[];
     float* tab = reinterpret_cast<float*>(sm + kOffTab);
-    uint64_t* full = reinterpret_cast<uint64_t*>(sm + kOffBar);
-    uint64_t* empty = full + kNStage;
-    uint64_t* g_done = empty + kNStage;
-    uint64_t* h_ready = g_done + 1;
-    uint64_t* yo_done = h_ready + 1;
-    uint64_t* mx_ready = yo_done + 1;
-    uint64_t* ys_full = mx_ready + 1;  // all MMAs of the block done (Y, then S)
-    uint64_t* y_done = ys_full + 1;    // Y of the block done (S may still run)
-    uint64_t* done = y_done + 1;
+    uint64_t* full = reinterpret_cast<uint64_t*>(sm + kOffBar);  // [2] stage loaded (TMA transaction)
+    uint64_t* empty = full + 2;                                   // [2] stage free: its y tile stored (8 warps)
+    uint64_t* g_done = empty + 2;                                 // G of the block done (commit)
+    uint64_t* m_ready = g_done + 1;                               // Gc or M built (6 builder warps)
+    uint64_t* mode_rdy = m_ready + 1;                             // block mode written (1 state thread)
+    uint64_t* h_ready = mode_rdy + 1;                             // read-back done (8 state warps)
+    uint64_t* h_free = h_ready + 1;                               // state MMA and H copy consumed (commit)
+    uint64_t* yo_done = h_free + 1;                               // steep blocks: C.H done (commit)
+    uint64_t* x_ready = yo_done + 1;                              // X~ or X' written (8 state warps)
+    uint64_t* y_done = x_ready + 1;                               // [2] every MMA of a block using output
+                                                                  // accumulator i done (commit)
+    uint64_t* yfree = y_done + 2;                                 // [2] output accumulator read (8 warps)
+    uint64_t* zfull = yfree + 2;                                  // [2] gated: z tile in the C region (TMA)
+    uint64_t* done = zfull + 2;                                   // drain (commit)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
     volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -182,13 +232,17 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
         for (int s = 0; s < kNStage; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 8);
+            mbar_init(&yfree[s], 8);
+            mbar_init(&y_done[s], 1);
+            mbar_init(&zfull[s], 1);
         }
         mbar_init(g_done, 1);
+        mbar_init(m_ready, 6);
+        mbar_init(mode_rdy, 1);
         mbar_init(h_ready, 8);
+        mbar_init(h_free, 1);
         mbar_init(yo_done, 1);
-        mbar_init(mx_ready, 15);  // 7 M-builder warps and 8 state warps
-        mbar_init(ys_full, 1);
-        mbar_init(y_done, 1);
+        mbar_init(x_ready, 8);
         mbar_init(done, 1);
         *abort = (smem_u32(sm) & 1023u) ? 1 : 0;  // tiles need 1024-byte alignment; never fault on it
         if (*abort) raise_timeout(abort, p.status);
@@ -197,8 +251,9 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
         prefetch_tmap(&mapB);
         prefetch_tmap(&mapC);
         if (p.y_tma) prefetch_tmap(&mapY);
+        if (GATED) prefetch_tmap(&mapZ);
     }
-    if (warp == kCtlWarp) {
+    if (warp == 1) {
         tmem_alloc(tmem_slot, kTCols);
         tmem_relinquish();
     }
@@ -206,18 +261,32 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    uint8_t* sHX = sm + kOffHX;  // [2 heads] x 16 KB: bf16 state copy H, then X' of the current block
+    uint8_t* sH = sm + kOffH;
 
-    if (warp == kCtlWarp) {
-        if (lane == 0 && !*abort) {  // ------------------------------------ TMA loads and tcgen05.mma
-            const uint32_t id_g = idesc_bf16(128, 128, 0, 0);   // C (K-major) x B (K-major)
-            const uint32_t id_o = idesc_bf16(128, 128, 0, 1);   // C (K-major) x [H_0 | H_1] (MN-major)
-            const uint32_t id_y = idesc_bf16(128, 64, 0, 1);    // M_j (TMEM) x X_j (MN-major)
-            const uint32_t id_s = idesc_bf16(128, 128, 1, 1);   // B^T (MN-major) x [X'_0 | X'_1] (MN-major)
-            const uint32_t aHX = smem_u32(sHX);
-            auto load = [&](int c) {  // block c of the segment into stage c % 2
-                const int s = c % kNStage;
-                const int row = (int)(tok0 + (int64_t)(c_begin + c) * kQ);
+    if (warp == 0) {
+        if (lane == 0 && !*abort) {  // ------------------------------------------------ TMA producer
+            // gated: block j's z tile goes into its stage's C region once the C.H MMA has read C
+            int zk = 0;  // z tiles issued
+            auto load_z = [&](int j) -> bool {
+                if (!mbar_wait(h_free, j & 1, abort)) return false;
+                const int sj = j % kNStage;
+                const int zrow = (int)(tok0 + (int64_t)(c_begin + j) * kQ);
+                uint8_t* zb = sm + sj * kStage + kOffC;
+                mbar_arrive_expect_tx(&zfull[sj], 2 * kTileQP);
+                tma_load_2d(zb, &mapZ, &zfull[sj], head0 * kP, zrow);
+                tma_load_2d(zb + kTileQP, &mapZ, &zfull[sj], min(head0 + 1, p.h - 1) * kP, zrow);
+                ++zk;
+                return true;
+            };
+            int k = 0;
+            for (; k < nch; ++k) {
+                const int s = k % kNStage;
+                // block k goes into the stage block k-2 used, once its epilogue released it
+                if (k >= kNStage && !mbar_wait(&empty[s], ((k / kNStage) - 1) & 1, abort)) {
+                    raise_timeout(abort, p.status);
+                    break;
+                }
+                const int row = (int)(tok0 + (int64_t)(c_begin + k) * kQ);
                 uint8_t* base = sm + s * kStage;
                 mbar_arrive_expect_tx(&full[s], kStage);
                 tma_load_2d(base + kOffC, &mapC, &full[s], grp * kN, row);
@@ -227,135 +296,170 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
                 tma_load_2d(base + kOffX, &mapX, &full[s], head0 * kP, row);
                 // a pair's second head past the last head reloads the last head (its dt is zero)
                 tma_load_2d(base + kOffX + kTileQP, &mapX, &full[s], min(head0 + 1, p.h - 1) * kP, row);
-            };
-            int loaded = 0;  // blocks whose loads were issued
-            for (; loaded < nch && loaded < kNStage; ++loaded) load(loaded);
-            for (int k = 0; k < nch; ++k) {
-                const int s = k % kNStage;
-                // stage k is loaded, and block k-1's Y MMAs (which read M from the G columns) are done;
-                // its S MMAs may still run, ahead of G in the tensor pipe
-                if (!mbar_wait(&full[s], (k / kNStage) & 1, abort) ||
-                    (k > 0 && !mbar_wait(y_done, (k - 1) & 1, abort))) {
+                if (GATED && k > 0 && !load_z(k - 1)) {  // block k-1's z, once its C.H MMA is done
                     raise_timeout(abort, p.status);
+                    break;
+                }
+            }
+            if (GATED && k == nch && nch > 0 && !load_z(nch - 1)) raise_timeout(abort, p.status);
+            // every issued load lands before the CTA can exit (bounded; only the last two can be pending)
+            for (int j = max(0, k - kNStage); j < k; ++j) mbar_wait(&full[j % kNStage], (j / kNStage) & 1, nullptr);
+            for (int j = max(0, zk - kNStage); j < zk; ++j) mbar_wait(&zfull[j % kNStage], (j / kNStage) & 1, nullptr);
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && !*abort) {  // -------------------------------------------------- tcgen05.mma
+            const uint32_t id_g = idesc_bf16(128, 128, 0, 0);   // C (K-major) x B (K-major)
+            const uint32_t id_o = idesc_bf16(128, 128, 0, 1);   // C (K-major) x [H_0 | H_1] (MN-major)
+            const uint32_t id_s = idesc_bf16(128, 128, 1, 1);   // B^T (MN-major) x [X_0 | X_1] (MN-major)
+            const uint32_t id_y = idesc_bf16(128, 64, 0, 1);    // M_j (TMEM) x x_j (MN-major)
+            const uint32_t aH = smem_u32(sH);
+            uint32_t nuse[2] = {0u, 0u};  // uses of each output accumulator so far
+            auto acc_free = [&](int i) -> bool {  // earlier use of accumulator i read by its epilogue
+                if (nuse[i] > 0 && !mbar_wait(&yfree[i], (nuse[i] - 1) & 1, abort)) return false;
+                ++nuse[i];
+                return true;
+            };
+            bool ok = true;
+            for (int k = 0; ok && k < nch; ++k) {
+                const int s = k % kNStage, yi = k & 1;
+                // stage k is loaded, and block k-1's output MMAs (the last readers of the G columns) are done
+                if (!mbar_wait(&full[s], (k / kNStage) & 1, abort) ||
+                    (k > 0 && !mbar_wait(&y_done[(k - 1) & 1], ((k - 1) >> 1) & 1, abort))) {
+                    ok = false;
                     break;
                 }
                 tc_fence_after();
                 const uint32_t aS = smem_u32(sm + s * kStage);
                 const uint32_t aC = aS + kOffC, aB = aS + kOffB, aX = aS + kOffX;
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {  // G = C . B^T
+                for (int kk = 0; kk < 8; ++kk) {  // G = C . B^T over the state dim
                     const uint32_t off = (kk & 3) * 32 + (kk >> 2) * (kTileQN / 2);
                     mma_ss(tmem + kTG, desc_sw128(aC + off, 16, 1024), desc_sw128(aB + off, 16, 1024), id_g, kk > 0);
                 }
                 mma_commit(g_done);
-                if (!mbar_wait(h_ready, k & 1, abort)) {
-                    raise_timeout(abort, p.status);
+                if (!mbar_wait(h_ready, k & 1, abort)) {  // read-back done; the block's mode is written
+                    ok = false;
                     break;
                 }
                 tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {  // Y_off = C . [H_0 | H_1] over the state dim
-                    const uint32_t off = (kk & 3) * 32 + (kk >> 2) * (kTileQN / 2);
-                    mma_ss(tmem + kTYO, desc_sw128(aC + off, 16, 1024), desc_sw128(aHX + kk * 2048, kTileQP, 1024),
-                           id_o, kk > 0);
-                }
-                mma_commit(yo_done);
-                // block k+1 goes into the stage block k-1 used, free once its epilogue has read x and
-                // its y tile has left (released after the read-back that h_ready waited for)
-                if (loaded == k + 1 && loaded < nch) {
-                    if (!mbar_wait(&empty[loaded % kNStage], ((loaded / kNStage) & 1) ^ 1, abort)) {
-                        raise_timeout(abort, p.status);
+                const bool fast = tab[kTabMode + (k & 1)] != 0.0f;
+                const uint32_t yacc = tmem + kTY0 + 128 * yi;
+                if (fast) {
+                    if (!mbar_wait(x_ready, k & 1, abort)) {
+                        ok = false;
                         break;
                     }
-                    load(loaded++);
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)  // S += B^T . [X~_0 | X~_1] over the block's tokens
+                        mma_ss(tmem + kTS, desc_sw128(aB + kk * 2048, kTileQN / 2, 1024),
+                               desc_sw128(aX + kk * 2048, kTileQP, 1024), id_s, 1u);
+                    if (!acc_free(yi)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {  // Y (+)= C . [2^a H_0 | 2^a H_1] over the state dim
+                        const uint32_t off = (kk & 3) * 32 + (kk >> 2) * (kTileQN / 2);
+                        mma_ss(yacc, desc_sw128(aC + off, 16, 1024), desc_sw128(aH + kk * 2048, kTileQP, 1024), id_o,
+                               1u);
+                    }
+                    mma_commit(h_free);
+                    if (!mbar_wait(m_ready, k & 1, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)  // Y += Gc . [X~_0 | X~_1] over the block's tokens
+                        mma_ts(yacc, tmem + kTG + 32 * (kk >> 1) + 8 * (kk & 1),
+                               desc_sw128(aX + kk * 2048, kTileQP, 1024), id_o, 1u);
+                    mma_commit(&y_done[yi]);
+                } else {
+                    const uint32_t oacc = tmem + kTY0 + 128 * (yi ^ 1);
+                    if (!acc_free(yi ^ 1)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {  // Yoff = C . [H_0 | H_1] over the state dim
+                        const uint32_t off = (kk & 3) * 32 + (kk >> 2) * (kTileQN / 2);
+                        mma_ss(oacc, desc_sw128(aC + off, 16, 1024), desc_sw128(aH + kk * 2048, kTileQP, 1024), id_o,
+                               kk > 0);
+                    }
+                    mma_commit(yo_done);
+                    if (!mbar_wait(x_ready, k & 1, abort)) {  // X' written over the state copy
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)  // S += B^T . [X'_0 | X'_1] over the block's tokens
+                        mma_ss(tmem + kTS, desc_sw128(aB + kk * 2048, kTileQN / 2, 1024),
+                               desc_sw128(aH + kk * 2048, kTileQP, 1024), id_s, 1u);
+                    mma_commit(h_free);
+                    if (!mbar_wait(m_ready, k & 1, abort) || !acc_free(yi)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+#pragma unroll
+                    for (int j = 0; j < 2; ++j)
+#pragma unroll
+                        for (int kk = 0; kk < 8; ++kk)  // Y_j (+)= M_j . x_j over the block's tokens
+                            mma_ts(yacc + 64 * j, tmem + kTG + 32 * (kk >> 1) + 16 * j + 8 * (kk & 1),
+                                   desc_sw128(aX + j * kTileQP + kk * 2048, kTileQP, 1024), id_y, 1u);
+                    mma_commit(&y_done[yi]);
                 }
-                if (!mbar_wait(mx_ready, k & 1, abort)) {
-                    raise_timeout(abort, p.status);
-                    break;
-                }
-                tc_fence_after();
-                // Y first, so the epilogue can start while S still runs
-#pragma unroll
-                for (int j = 0; j < 2; ++j)
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)  // Y_j = M_j . X_j over the block's tokens
-                        mma_ts(tmem + kTY + 64 * j, tmem + kTG + 32 * (kk >> 1) + 16 * j + 8 * (kk & 1),
-                               desc_sw128(aX + j * kTileQP + kk * 2048, kTileQP, 1024), id_y, kk > 0);
-                mma_commit(y_done);
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)  // S += B^T . [X'_0 | X'_1] over the block's tokens
-                    mma_ss(tmem + kTS, desc_sw128(aB + kk * 2048, kTileQN / 2, 1024),
-                           desc_sw128(aHX + kk * 2048, kTileQP, 1024), id_s, 1u);
-                mma_commit(ys_full);
             }
-            // every issued load lands before the CTA exits (bounded; only the last two can be pending)
-            for (int j = max(0, loaded - kNStage); j < loaded; ++j) mbar_wait(&full[j % kNStage], (j / kNStage) & 1, abort);
+            if (!ok) raise_timeout(abort, p.status);
             mma_commit(done);
-            mbar_wait(done, 0, nullptr);
+            mbar_wait(done, 0, nullptr);  // every issued MMA is done before TMEM can be released (bounded)
         }
-    } else if (warp < 8) {  // ------------------------------------------------------ M builders
-        const int q = warp & 3, hb = warp >> 2, r = 32 * q + lane;
+    } else if (warp < 8) {  // ------------------------------------------------------------- builders
+        const int q = warp & 3, r = 32 * q + lane;
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-        // causal column blocks of this warp, and the zero blocks it writes
-        // quarter 0: {0} (its second warp is the control warp); 1: {0} {1}; 2: {0,1} {2}; 3: {0,1} {2,3}
-        const int cb_lo = hb == 0 ? 0 : (q >= 2 ? 2 : 1);
-        const int cb_hi = hb == 0 ? (q >= 2 ? 1 : 0) : q;  // inclusive
-        const bool zero_writer = (q <= 1) ? hb == 0 : hb == 1;
-        float A2[2], dn[2] = {0.0f, 0.0f};
+        const bool upper = warp < 4;  // warps 2, 3: the upper column blocks of quarters 2 and 3
+        const int cb_lo = upper ? 2 : 0;
+        const int cb_hi = upper ? q : min(q, 1);  // inclusive
+        const bool zero_writer = upper ? q == 2 : q <= 1;
+        float A2[2];
 #pragma unroll
         for (int j = 0; j < 2; ++j) A2[j] = head0 + j < p.h ? p.A[head0 + j] * kLog2e : 0.0f;
-        if (nch > 0 && c_begin * kQ + r < p.L) {
+        for (int k = 0; k < nch; ++k) {  // every warp runs every iteration (named barrier 4)
+            const bool okm = __all_sync(0xffffffffu, mbar_wait(mode_rdy, k & 1, abort));
+            const bool fast = !okm || tab[kTabMode + (k & 1)] != 0.0f;
+            // steep blocks: cs and dt of both heads for every token of the block (warps 4-7, one row
+            // each), through the per-quarter totals
+            float c2[2] = {0.0f, 0.0f}, dv[2] = {0.0f, 0.0f};
+            if (!fast && !upper) {
+                const int t = (c_begin + k) * kQ + r;
 #pragma unroll
-            for (int j = 0; j < 2; ++j)
-                if (head0 + j < p.h) dn[j] = p.dt[(tok0 + c_begin * kQ + r) * p.sdt + head0 + j];
-        }
-        for (int k = 0; k < nch; ++k) {  // every warp runs every iteration (named barrier 1)
-            const float dv[2] = {dn[0], dn[1]};
-            const int t1 = (c_begin + k + 1) * kQ + r;
-            dn[0] = dn[1] = 0.0f;
-            if (k + 1 < nch && t1 < p.L) {  // prefetch the next block's dt
-#pragma unroll
-                for (int j = 0; j < 2; ++j)
-                    if (head0 + j < p.h) dn[j] = p.dt[(tok0 + t1) * p.sdt + head0 + j];
-            }
-            float* wt = tab + kTabWtotM + 8 * (k & 1);
-            float c2[2];
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {  // inclusive scan of dt A (log2 units) within the warp
-                float sc = dv[j] * A2[j];
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const float v = __shfl_up_sync(0xffffffffu, sc, o);
-                    if (lane >= o) sc += v;
-                }
-                if (lane == 31 && hb == 0) wt[4 * j + q] = sc;
-                c2[j] = sc;
-            }
-            asm volatile("bar.sync 1, 224;" ::: "memory");
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                float pre = 0.0f;
-#pragma unroll
-                for (int i = 0; i < 4; ++i) pre += i < q ? wt[4 * j + i] : 0.0f;
-                c2[j] += pre;
-                if (hb == 0) {  // this row block's anchor (cs at its first row) and the decay across it
-                    const float a = __shfl_sync(0xffffffffu, c2[j], 0);
-                    const float last = __shfl_sync(0xffffffffu, c2[j], 31);
-                    const bool fb = a - last > kDropMax;
-                    tab[kTabG + 128 * j + r] = fb ? dv[j] : ex2(a - c2[j]) * dv[j];
-                    tab[kTabC + 128 * j + r] = c2[j];
-                    if (lane == 0) {
-                        tab[kTabAnch + 4 * j + q] = a;
-                        tab[kTabFlag + 4 * j + q] = fb ? 1.0f : 0.0f;
-                    }
+                for (int j = 0; j < 2; ++j) {
+                    dv[j] = (t < p.L && head0 + j < p.h) ? p.dt[(tok0 + t) * p.sdt + head0 + j] : 0.0f;
+                    c2[j] = warp_incl_scan(dv[j] * A2[j], lane);
+                    if (lane == 31) tab[kTabBPart + 4 * j + q] = c2[j];
                 }
             }
-            asm volatile("bar.sync 1, 224;" ::: "memory");  // tables of block k complete
+            asm volatile("bar.sync 4, 192;" ::: "memory");
+            if (!fast && !upper) {
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    float pre = 0.0f;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) pre += i < q ? tab[kTabBPart + 4 * j + i] : 0.0f;
+                    tab[kTabCs + 128 * j + r] = c2[j] + pre;
+                    tab[kTabDt + 128 * j + r] = dv[j];
+                }
+            }
+            asm volatile("bar.sync 4, 192;" ::: "memory");
 
-            const bool ok = __all_sync(0xffffffffu, mbar_wait(g_done, k & 1, abort));
+            const bool ok = okm && __all_sync(0xffffffffu, mbar_wait(g_done, k & 1, abort));
             if (ok) {
                 tc_fence_after();
-                if (zero_writer) {  // above the diagonal: zeros for both heads
+                if (zero_writer) {  // above the diagonal: zeros (both heads' columns in steep blocks)
                     uint32_t z[32];
 #pragma unroll
                     for (int e = 0; e < 32; ++e) z[e] = 0u;
@@ -363,61 +467,58 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
                     for (int cb = 1; cb < 4; ++cb)
                         if (cb > q) tmem_st32(tmem + lane_base + kTG + 32 * cb, z);
                 }
+                float ct[2] = {0.0f, 0.0f};
+                if (!fast) {
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) ct[j] = tab[kTabCs + 128 * j + r];
+                }
 #pragma unroll 1
                 for (int cb = cb_lo; cb <= cb_hi; ++cb) {  // column block s in [32 cb, 32 cb + 32)
                     uint32_t gv[32];
                     tmem_ld32(tmem + lane_base + kTG + 32 * cb, gv);
                     tmem_ld_wait();
                     const bool diag = cb == q;
-#pragma unroll
-                    for (int j = 0; j < 2; ++j) {
+                    if (fast) {  // Gc: G with the causal mask s <= t, as bf16 pairs
                         uint32_t pk[16];
-                        const float* gt = tab + kTabG + 128 * j + 32 * cb;
-                        if (tab[kTabFlag + 4 * j + cb] == 0.0f) {
-                            const float er = ex2(c2[j] - tab[kTabAnch + 4 * j + cb]);
-                            const float2 er2 = make_float2(er, er);
 #pragma unroll
-                            for (int e = 0; e < 32; e += 4) {
-                                const float4 g4 = *reinterpret_cast<const float4*>(gt + e);
-                                float2 m01 = mul2(mul2(make_float2(__uint_as_float(gv[e]), __uint_as_float(gv[e + 1])), er2),
-                                                  make_float2(g4.x, g4.y));
-                                float2 m23 = mul2(mul2(make_float2(__uint_as_float(gv[e + 2]), __uint_as_float(gv[e + 3])), er2),
-                                                  make_float2(g4.z, g4.w));
-                                if (diag) {  // causal mask inside the diagonal block: s <= t
-                                    m01.x = e <= lane ? m01.x : 0.0f;
-                                    m01.y = e + 1 <= lane ? m01.y : 0.0f;
-                                    m23.x = e + 2 <= lane ? m23.x : 0.0f;
-                                    m23.y = e + 3 <= lane ? m23.y : 0.0f;
-                                }
-                                pk[e >> 1] = pack2(m01);
-                                pk[(e >> 1) + 1] = pack2(m23);
+                        for (int e = 0; e < 32; e += 2) {
+                            float g0 = __uint_as_float(gv[e]), g1 = __uint_as_float(gv[e + 1]);
+                            if (diag) {
+                                g0 = e <= lane ? g0 : 0.0f;
+                                g1 = e + 1 <= lane ? g1 : 0.0f;
                             }
-                        } else {  // steep block: direct exponentials, g holds dt
-                            const float* ct = tab + kTabC + 128 * j + 32 * cb;
+                            pk[e >> 1] = pack_bf16(g0, g1);
+                        }
+                        tmem_st16(tmem + lane_base + kTG + 32 * cb, pk);
+                    } else {  // M_j = G 2^min(cs_t - cs_s, 0) dt_s, s <= t, one head after the other
+#pragma unroll
+                        for (int j = 0; j < 2; ++j) {
+                            uint32_t pk[16];
+                            const float* cs = tab + kTabCs + 128 * j + 32 * cb;
+                            const float* dts = tab + kTabDt + 128 * j + 32 * cb;
 #pragma unroll
                             for (int e = 0; e < 32; e += 2) {
-                                float m0 = __uint_as_float(gv[e]) * ex2(fminf(c2[j] - ct[e], 0.0f)) * gt[e];
-                                float m1 = __uint_as_float(gv[e + 1]) * ex2(fminf(c2[j] - ct[e + 1], 0.0f)) * gt[e + 1];
+                                float m0 = __uint_as_float(gv[e]) * ex2(fminf(ct[j] - cs[e], 0.0f)) * dts[e];
+                                float m1 = __uint_as_float(gv[e + 1]) * ex2(fminf(ct[j] - cs[e + 1], 0.0f)) * dts[e + 1];
                                 if (diag) {
                                     m0 = e <= lane ? m0 : 0.0f;
                                     m1 = e + 1 <= lane ? m1 : 0.0f;
                                 }
                                 pk[e >> 1] = pack_bf16(m0, m1);
                             }
+                            tmem_st16(tmem + lane_base + kTG + 32 * cb + 16 * j, pk);
                         }
-                        // head j's 16 packed columns of this block (the A operand of Y_j)
-                        tmem_st16(tmem + lane_base + kTG + 32 * cb + 16 * j, pk);
                     }
                 }
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(mx_ready);
+                if (lane == 0) mbar_arrive(m_ready);
             } else {
                 raise_timeout(abort, p.status);
             }
         }
-    } else {  // ------------------------------------------------------------------- state warps
+    } else {  // --------------------------------------------------------------------- state warps
         const int cw = warp - 8, q = warp & 3, hf = cw >> 2;
         const int r = 32 * q + lane;
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
@@ -427,14 +528,11 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
         const float Dh = (p.D && head_ok) ? p.D[head] : 0.0f;
         const int64_t bh = (int64_t)b * p.h + head;
         const int PN = kP * kN;
-        uint8_t* myHX = sHX + hf * kTileQP;
-        const uint32_t bar_id = 2 + hf;
+        uint8_t* myH = sH + hf * kTileQP;
+        const uint32_t sacc = tmem + lane_base + kTS + 64 * hf;  // this head's state, row n = r
 
-        // The fp32 state of this head lives in TMEM columns kTS + 64 hf (row n = lane r): each
-        // block, it is read for its bf16 copy (Y_off's operand), 2^tot H_k is written back, and
-        // the S MMA accumulates B^T X' on top, leaving H_{k+1}.  A segment's start state is the
-        // initial state (or zero) carried over the earlier segments:
-        // H <- 2^decay_j H + S_j, S_j being segment j's end state from a zero start.
+        // A segment's start state is the initial state (or zero) carried over the earlier
+        // segments: H <- 2^decay_j H + S_j, S_j being segment j's end state from a zero start.
         {
             if (p.nseg > 1 && (seg > 0 || p.wait_all)) grid_dependency_wait();  // segment end states written
             const float* init = (head_ok && p.init_state)
@@ -454,218 +552,279 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
                 uint32_t u[32];
 #pragma unroll
                 for (int j = 0; j < 32; ++j) u[j] = __float_as_uint(v[j]);
-                tmem_st32(tmem + lane_base + kTS + 64 * hf + 32 * h2, u);
+                tmem_st32(sacc + 32 * h2, u);
             }
             tmem_st_wait();
         }
         float dt_next = 0.0f;
         if (head_ok && nch > 0 && c_begin * kQ + r < p.L) dt_next = p.dt[(tok0 + c_begin * kQ + r) * p.sdt + head];
-        float c2_prev = 0.0f;
+        // the previous block: cs and anchor of this row (log2 units), and its mode
+        float c2_prev = 0.0f, a_prev = 0.0f;
+        bool fast_prev = true;
+        float s_in = 1.0f;  // TMEM state x s_in = the state at the current block's start
+        int nsteep = 0;     // steep blocks so far (phases of yo_done)
         bool ok = __all_sync(0xffffffffu, !*abort);
-        bool pending_release = false;  // the storing warp still owes the previous stage's release
 
-        // Iteration k: decay scan of block k, epilogue of block k-1, read-back and X' of block k.
-        // Every warp runs every iteration (named barrier 2 + hf); a failed wait skips work only.
+        // Epilogue of block kp: y from the output accumulator(s), which already hold the D x term, and
+        // the optional gate (z from the tile the producer loaded into the stage's C region).  y rows go
+        // into the stage's x region in the 128-byte swizzle and leave as one bulk tensor store per head
+        // (rows past L clipped); the stage is released once the store has read them.  Every warp of
+        // the head calls it once per block (named barrier 2 + hf).
+        auto epilogue = [&](int kp) {
+            const int sp = kp & 1;
+            const int tp0 = (c_begin + kp) * kQ;
+            const bool valid = head_ok && tp0 + r < p.L;
+            const int64_t tok = tok0 + tp0 + r;
+            const int col = head * kP;
+            const uint32_t yacc = tmem + lane_base + kTY0 + 128 * sp + 64 * hf;
+            const uint32_t oacc = tmem + lane_base + kTY0 + 128 * (sp ^ 1) + 64 * hf;
+            uint8_t* sX = sm + sp * kStage + kOffX + hf * kTileQP;        // y rows (over X~ or x)
+            const uint8_t* sZ = sm + sp * kStage + kOffC + hf * kTileQP;  // z rows (gated)
+            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&y_done[sp], (kp >> 1) & 1, abort));
+            if (GATED && ok) ok = __all_sync(0xffffffffu, mbar_wait(&zfull[sp], (kp >> 1) & 1, abort));
+            if (ok) {
+                tc_fence_after();
+                // fast: y = 2^(cs - a) Y;  steep: y = Y + 2^cs Yoff
+                const float sy = fast_prev ? ex2(c2_prev - a_prev) : 1.0f;
+                const float so = fast_prev ? 0.0f : ex2(c2_prev);
+                const float2 sy2 = make_float2(sy, sy), so2 = make_float2(so, so);
+                uint4* yrow = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.y) + tok * p.sy + col);
+                float ssq[2] = {0.0f, 0.0f};
+                // 16 output columns from yv (and ov): 16-byte chunks cc and cc + 1 of the row
+                auto out16 = [&](int cc, const uint32_t* yv, const uint32_t* ov) {
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) {
+                        uint4 zq = make_uint4(0, 0, 0, 0), nw4 = make_uint4(0, 0, 0, 0);
+                        if (GATED) {
+                            zq = *reinterpret_cast<const uint4*>(sZ + sw128(r, cc + c));
+                            nw4 = *reinterpret_cast<const uint4*>(p.norm_w + col + 8 * (cc + c));
+                        }
+                        const uint32_t zw[4] = {zq.x, zq.y, zq.z, zq.w};
+                        const uint32_t nw[4] = {nw4.x, nw4.y, nw4.z, nw4.w};
+                        uint32_t o[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int j = 8 * c + 2 * e;
+                            float2 v = mul2(sy2, make_float2(__uint_as_float(yv[j]), __uint_as_float(yv[j + 1])));
+                            if (ov) v = fma2(so2, make_float2(__uint_as_float(ov[j]), __uint_as_float(ov[j + 1])), v);
+                            if (GATED) {
+                                v = mul2(v, make_float2(silu_approx(bf_lo(zw[e])), silu_approx(bf_hi(zw[e]))));
+                                ssq[cc >> 2] = fmaf(v.x, v.x, fmaf(v.y, v.y, ssq[cc >> 2]));
+                                v = mul2(v, bf2(nw[e]));
+                            }
+                            o[e] = pack2(v);
+                        }
+                        const uint4 ow = make_uint4(o[0], o[1], o[2], o[3]);
+                        if (p.y_tma) *reinterpret_cast<uint4*>(sX + sw128(r, cc + c)) = ow;
+                        else if (valid) yrow[cc + c] = ow;
+                    }
+                };
+                auto release = [&]() {  // the accumulators of block kp are read: the MMA lane may reuse them
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) {
+                        mbar_arrive(&yfree[sp]);
+                        if (!fast_prev) mbar_arrive(&yfree[sp ^ 1]);
+                    }
+                };
+                if (fast_prev) {  // 32 columns per TMEM round trip
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        uint32_t yv[32];
+                        tmem_ld32(yacc + 32 * h, yv);
+                        tmem_ld_wait();
+                        if (h == 1) release();
+                        out16(4 * h, yv, nullptr);
+                        out16(4 * h + 2, yv + 16, nullptr);
+                    }
+                } else {  // steep: Y and Yoff, 16 columns of each per round trip
+#pragma unroll
+                    for (int h = 0; h < 4; ++h) {
+                        uint32_t yv[16], ov[16];
+                        tmem_ld16(yacc + 16 * h, yv);
+                        tmem_ld16(oacc + 16 * h, ov);
+                        tmem_ld_wait();
+                        if (h == 3) release();
+                        out16(2 * h, yv, ov);
+                    }
+                }
+                if (GATED && valid) {
+                    p.row_parts[tok * 2 * p.h + 2 * head] = ssq[0];
+                    p.row_parts[tok * 2 * p.h + 2 * head + 1] = ssq[1];
+                }
+            }
+            if (p.y_tma) {  // the head's 128 x 64 tile leaves in one bulk store
+                fence_async_smem();
+                asm volatile("bar.sync %0, 128;" ::"r"(2 + hf) : "memory");
+                if (q == 0) {
+                    ok = __all_sync(0xffffffffu, ok && !*abort);
+                    if (ok && head_ok && lane == 0) {
+                        tma_store_3d(&mapY, sX, head * kP, tp0, b);
+                        bulk_commit();
+                    }
+                    __syncwarp();
+                }
+            }
+            if (ok) {  // stage sp is free once its y tile has been read
+                if (lane == 0) {
+                    if (p.y_tma && q == 0) bulk_wait_read0();
+                    mbar_arrive(&empty[sp]);
+                }
+                __syncwarp();
+            }
+        };
+
+        // X~ (fast blocks, in place over x) or X' (steep blocks, over the state copy once the C.H
+        // MMA has read it) of block k for the state and output MMAs, and the D x term written into
+        // this head's columns of block k's output accumulator, which the output MMAs then add to
+        // (fast blocks: 2^(a - cs) D x, in the accumulator's scale; steep blocks: D x)
+        auto form_x = [&](int k, bool fast, float c2, float a, float tot, float dtv) {
+            const int s = k % kNStage;
+            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&full[s], (k / kNStage) & 1, abort));
+            if (!ok) return;
+            uint8_t* sXk = sm + s * kStage + kOffX + hf * kTileQP;
+            uint8_t* dst = sXk;
+            float wgt, dsc;
+            if (fast) {  // X~[s=r, :] = 2^(a - cs_r) dt_r x[r, :]
+                const float e = ex2(a - c2);
+                wgt = e * dtv;
+                dsc = e * Dh;
+            } else {  // X'[s=r, :] = 2^(tot - cs_r) dt_r x[r, :]
+                ok = __all_sync(0xffffffffu, mbar_wait(yo_done, nsteep & 1, abort));
+                ++nsteep;
+                if (!ok) return;
+                wgt = ex2(tot - c2) * dtv;
+                dsc = Dh;
+                dst = myH;
+            }
+            const float2 w2 = make_float2(wgt, wgt), d2 = make_float2(dsc, dsc);
+            const uint32_t dacc = tmem + lane_base + kTY0 + 128 * (k & 1) + 64 * hf;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {  // 32 columns at a time
+                uint32_t dv[32];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const int cc = 4 * h + c;
+                    const uint4 xv = *reinterpret_cast<const uint4*>(sXk + sw128(r, cc));
+                    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+                    uint32_t o[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 xf = bf2(xw[e]);
+                        o[e] = pack2(mul2(xf, w2));
+                        const float2 dd = mul2(xf, d2);
+                        dv[8 * c + 2 * e] = __float_as_uint(dd.x);
+                        dv[8 * c + 2 * e + 1] = __float_as_uint(dd.y);
+                    }
+                    *reinterpret_cast<uint4*>(dst + sw128(r, cc)) = make_uint4(o[0], o[1], o[2], o[3]);
+                }
+                tmem_st32(dacc + 32 * h, dv);
+            }
+            tmem_st_wait();
+            fence_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(x_ready);
+        };
+
+        // Iteration k: decay scan and mode of block k, read-back of block k, then X~ of block k and
+        // the epilogue of block k-1 (two fast blocks: in that order, so the tensor core gets block k's
+        // operands while block k-1's outputs drain; otherwise the other way round, since a steep block
+        // also uses the other output accumulator).  Every warp runs every iteration (named
+        // barriers 1 and 2 + hf); a failed wait skips work only.
         for (int k = 0; k <= nch; ++k) {
-            float dtv = 0.0f, c2 = 0.0f, tot = 0.0f;
+            float dtv = 0.0f, c2 = 0.0f, a = 0.0f, tot = 0.0f;
+            bool fast = true;
             if (k < nch) {
                 dtv = dt_next;
                 const int t1 = (c_begin + k + 1) * kQ + r;
                 dt_next = (head_ok && k + 1 < nch && t1 < p.L) ? p.dt[(tok0 + t1) * p.sdt + head] : 0.0f;
-                float sc = dtv * A2;
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const float v = __shfl_up_sync(0xffffffffu, sc, o);
-                    if (lane >= o) sc += v;
-                }
-                float* wt = tab + kTabWtotS + 8 * (k & 1) + 4 * hf;
-                if (lane == 31) wt[q] = sc;
-                asm volatile("bar.sync %0, 128;" ::"r"(bar_id) : "memory");
+                const float sc = warp_incl_scan(dtv * A2, lane);
+                float* part = tab + kTabPart + 8 * (k & 1);
+                if (lane == 31) part[4 * hf + q] = sc;
+                asm volatile("bar.sync 1, 256;" ::: "memory");
                 float pre = 0.0f;
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float w = wt[i];
-                    pre += i < q ? w : 0.0f;
-                    tot += w;
-                }
+                for (int i = 0; i < 4; ++i) pre += i < q ? part[4 * hf + i] : 0.0f;
                 c2 = sc + pre;
-            }
+                float a0, t0, a1, t1s;
+                const bool f0 = fast_head(part, &a0, &t0);
+                const bool f1 = fast_head(part + 4, &a1, &t1s);
+                fast = f0 && f1;
+                a = hf ? a1 : a0;
+                tot = hf ? t1s : t0;
+                if (threadIdx.x == 8 * 32) {  // one thread publishes the mode to the builders and the MMA lane
+                    tab[kTabMode + (k & 1)] = fast ? 1.0f : 0.0f;
+                    mbar_arrive(mode_rdy);
+                }
 
-            if (k > 0) {  // ---- epilogue of block k-1 (TMEM loads are warp-collective)
-                if (ok) ok = __all_sync(0xffffffffu, mbar_wait(y_done, (k - 1) & 1, abort));
-                const int sp = (k - 1) % kNStage;
-                const int tp0 = (c_begin + k - 1) * kQ;
-                // x of block k-1 (this head); with bulk stores each thread overwrites its own row of
-                // it with its y row, in the same swizzled layout, once that row's x has been read
-                uint8_t* sX = sm + sp * kStage + kOffX + hf * kTileQP;
+                // ---- read-back: the state at the block's start, as bf16 for the C.H term and back
+                // into TMEM for the state MMA (fast: both scaled by 2^a; steep: 1 and 2^tot)
+                if (ok && k > 0) ok = __all_sync(0xffffffffu, mbar_wait(h_free, (k - 1) & 1, abort));
                 if (ok) {
                     tc_fence_after();
-                    const bool valid = head_ok && tp0 + r < p.L;
-                    const float ey = ex2(c2_prev);
-                    const float2 ey2 = make_float2(ey, ey), dh2 = make_float2(Dh, Dh);
-                    const int64_t tok = tok0 + tp0 + r;
-                    const int col = head * kP;
-                    __nv_bfloat16* yo = static_cast<__nv_bfloat16*>(p.y) + tok * p.sy + col;
-                    float ssq[2] = {0.0f, 0.0f};
-                    // z rows of this warp's 32 tokens, loaded four rows per instruction (coalesced) into
-                    // this warp's 4 KB of block k-1's C tile, which no MMA reads any more
-                    uint8_t* zs = sm + sp * kStage + kOffC + hf * (kTileQN / 2) + 32 * q * 128;
-                    if (p.z) {
+                    const float beta = fast ? ex2(a) : 1.0f;
+                    const float sb = s_in * beta, sg = s_in * (fast ? beta : ex2(tot));
+                    const float2 sb2 = make_float2(sb, sb), sg2 = make_float2(sg, sg);
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const int rr = (lane >> 3) + 4 * i, ch = lane & 7;
-                            uint4 zv = make_uint4(0, 0, 0, 0);
-                            if (head_ok && tp0 + 32 * q + rr < p.L)
-                                zv = *reinterpret_cast<const uint4*>(p.z + (tok0 + tp0 + 32 * q + rr) * p.sz + col + 8 * ch);
-                            *reinterpret_cast<uint4*>(zs + rr * 128 + ((ch ^ (rr & 7)) << 4)) = zv;
-                        }
-                        __syncwarp();
-                    }
-#pragma unroll
-                    for (int h2 = 0; h2 < 4; ++h2) {  // 16 output columns at a time
-                        uint32_t yv[16], ov[16];
-                        tmem_ld16(tmem + lane_base + kTY + 64 * hf + 16 * h2, yv);
-                        tmem_ld16(tmem + lane_base + kTYO + 64 * hf + 16 * h2, ov);
+                    for (int h2 = 0; h2 < 2; ++h2) {  // 32 state columns per TMEM round trip
+                        uint32_t v[32];
+                        tmem_ld32(sacc + 32 * h2, v);
                         tmem_ld_wait();
-                        if (!valid && !p.y_tma) continue;
 #pragma unroll
-                        for (int c = 0; c < 2; ++c) {
-                            const int cc = 2 * h2 + c;
-                            const uint4 xv = *reinterpret_cast<const uint4*>(sX + sw128(r, cc));
-                            const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
-                            uint4 zw4 = make_uint4(0, 0, 0, 0), nw4 = make_uint4(0, 0, 0, 0);
-                            if (p.z && valid) {
-                                zw4 = *reinterpret_cast<const uint4*>(zs + lane * 128 + ((cc ^ (lane & 7)) << 4));
-                                nw4 = *reinterpret_cast<const uint4*>(p.norm_w + col + 8 * cc);
-                            }
-                            const uint32_t zw[4] = {zw4.x, zw4.y, zw4.z, zw4.w};
-                            const uint32_t nw[4] = {nw4.x, nw4.y, nw4.z, nw4.w};
-                            uint32_t o[4];
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const int j = 8 * c + 2 * e;
-                                // y = Y + 2^cs Y_off + D x, two columns at a time
-                                float2 a = fma2(ey2, make_float2(__uint_as_float(ov[j]), __uint_as_float(ov[j + 1])),
-                                                make_float2(__uint_as_float(yv[j]), __uint_as_float(yv[j + 1])));
-                                a = fma2(dh2, bf2(xw[e]), a);
-                                if (p.z) {
-                                    const float z0 = bf_lo(zw[e]), z1 = bf_hi(zw[e]);
-                                    a = mul2(a, make_float2(silu_approx(z0), silu_approx(z1)));
-                                    ssq[h2 >> 1] = fmaf(a.x, a.x, fmaf(a.y, a.y, ssq[h2 >> 1]));
-                                    a = mul2(a, bf2(nw[e]));
-                                }
-                                o[e] = pack2(a);
-                            }
-                            if (p.y_tma) *reinterpret_cast<uint4*>(sX + sw128(r, cc)) = make_uint4(o[0], o[1], o[2], o[3]);
-                            else reinterpret_cast<uint4*>(yo)[cc] = make_uint4(o[0], o[1], o[2], o[3]);
+                        for (int c = 0; c < 4; ++c) {
+                            uint4 w;
+                            w.x = pack2(mul2(sb2, make_float2(__uint_as_float(v[8 * c + 0]), __uint_as_float(v[8 * c + 1]))));
+                            w.y = pack2(mul2(sb2, make_float2(__uint_as_float(v[8 * c + 2]), __uint_as_float(v[8 * c + 3]))));
+                            w.z = pack2(mul2(sb2, make_float2(__uint_as_float(v[8 * c + 4]), __uint_as_float(v[8 * c + 5]))));
+                            w.w = pack2(mul2(sb2, make_float2(__uint_as_float(v[8 * c + 6]), __uint_as_float(v[8 * c + 7]))));
+                            *reinterpret_cast<uint4*>(myH + sw128(r, 4 * h2 + c)) = w;
                         }
+#pragma unroll
+                        for (int j = 0; j < 32; j += 2) {
+                            const float2 d = mul2(sg2, make_float2(__uint_as_float(v[j]), __uint_as_float(v[j + 1])));
+                            v[j] = __float_as_uint(d.x);
+                            v[j + 1] = __float_as_uint(d.y);
+                        }
+                        tmem_st32(sacc + 32 * h2, v);
                     }
-                    if (p.z && valid) {
-                        p.row_parts[tok * 2 * p.h + 2 * head] = ssq[0];
-                        p.row_parts[tok * 2 * p.h + 2 * head + 1] = ssq[1];
-                    }
+                    tmem_st_wait();
+                    fence_async_smem();
                     tc_fence_before();
-                }
-                if (p.y_tma) {  // the head's 128 x 64 tile leaves in one bulk store (rows past L clipped)
-                    fence_async_smem();
-                    asm volatile("bar.sync %0, 128;" ::"r"(bar_id) : "memory");
-                    if (q == 0) {
-                        ok = __all_sync(0xffffffffu, ok && !*abort);
-                        if (ok && head_ok && lane == 0) {
-                            tma_store_3d(&mapY, sX, head * kP, tp0, b);
-                            bulk_commit();
-                        }
-                        __syncwarp();
-                    }
-                }
-                // Block k-1's stage is released after the read-back below, which waits for its S MMA
-                // (S reads B there); the storing warp also waits for its store to read the y tile.
-                pending_release = ok;
-            }
-            if (k == nch) break;
-
-            const int s = k % kNStage;
-            if (ok && k > 0) ok = __all_sync(0xffffffffu, mbar_wait(ys_full, (k - 1) & 1, abort));  // S done
-            if (ok) {  // ---- read-back: H_k as bf16 for Y_off, 2^tot H_k back into TMEM
-                const float dec = ex2(tot);
-                const float2 dec2 = make_float2(dec, dec);
-#pragma unroll
-                for (int h4 = 0; h4 < 4; ++h4) {  // 16 state columns at a time
-                    uint32_t v[16];
-                    tmem_ld16(tmem + lane_base + kTS + 64 * hf + 16 * h4, v);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int c = 0; c < 2; ++c) {
-                        uint4 w;
-                        w.x = pack_bf16(__uint_as_float(v[8 * c + 0]), __uint_as_float(v[8 * c + 1]));
-                        w.y = pack_bf16(__uint_as_float(v[8 * c + 2]), __uint_as_float(v[8 * c + 3]));
-                        w.z = pack_bf16(__uint_as_float(v[8 * c + 4]), __uint_as_float(v[8 * c + 5]));
-                        w.w = pack_bf16(__uint_as_float(v[8 * c + 6]), __uint_as_float(v[8 * c + 7]));
-                        *reinterpret_cast<uint4*>(myHX + sw128(r, 2 * h4 + c)) = w;
-                    }
-#pragma unroll
-                    for (int j = 0; j < 16; j += 2) {
-                        const float2 d = mul2(dec2, make_float2(__uint_as_float(v[j]), __uint_as_float(v[j + 1])));
-                        v[j] = __float_as_uint(d.x);
-                        v[j + 1] = __float_as_uint(d.y);
-                    }
-                    tmem_st16(tmem + lane_base + kTS + 64 * hf + 16 * h4, v);
-                }
-                tmem_st_wait();
-                fence_async_smem();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(h_ready);
-            }
-            if (pending_release) {  // block k-1 is done with its stage: release it
-                if (lane == 0) {
-                    if (p.y_tma && q == 0) bulk_wait_read0();  // the y tile has been read
-                    mbar_arrive(&empty[(k - 1) % kNStage]);
-                }
-                __syncwarp();
-                pending_release = false;
-            }
-            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&full[s], (k / kNStage) & 1, abort));
-            if (ok) {  // ---- X'_j[s=r, :] = 2^(tot - cs_r) dt_r x_j[r, :], formed while Y_off runs
-                const uint8_t* sX = sm + s * kStage + kOffX + hf * kTileQP;
-                const float wgt = ex2(tot - c2) * dtv;
-                const float2 w2 = make_float2(wgt, wgt);
-                uint4 xq[8];
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const uint4 xv = *reinterpret_cast<const uint4*>(sX + sw128(r, c));
-                    xq[c].x = pack2(mul2(bf2(xv.x), w2));
-                    xq[c].y = pack2(mul2(bf2(xv.y), w2));
-                    xq[c].z = pack2(mul2(bf2(xv.z), w2));
-                    xq[c].w = pack2(mul2(bf2(xv.w), w2));
-                }
-                ok = __all_sync(0xffffffffu, mbar_wait(yo_done, k & 1, abort));  // H read: X' may go there
-                if (ok) {
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(myHX + sw128(r, c)) = xq[c];
-                    fence_async_smem();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(mx_ready);
+                    if (lane == 0) mbar_arrive(h_ready);
                 }
+            }
+            // a fast block after a fast block: X~ first (block k-1's outputs use one accumulator only)
+            if (k < nch && fast && fast_prev) {
+                form_x(k, fast, c2, a, tot, dtv);
+                if (k > 0) epilogue(k - 1);
+            } else {
+                if (k > 0) epilogue(k - 1);
+                if (k < nch) form_x(k, fast, c2, a, tot, dtv);
             }
             if (!ok) raise_timeout(abort, p.status);
+            if (k == nch) break;
             c2_prev = c2;
+            a_prev = a;
+            fast_prev = fast;
+            s_in = fast ? ex2(tot - a) : 1.0f;  // state MMA result -> state at the next block's start
         }
 
         if (p.y_tma && q == 0 && lane == 0) bulk_wait0();  // this head's y tiles are in global memory
-        if (seg == p.nseg - 1 && p.final_state) {  // state after the last block: its S MMA is done
-            if (ok && nch > 0) ok = __all_sync(0xffffffffu, mbar_wait(ys_full, (nch - 1) & 1, abort));
+        if (seg == p.nseg - 1 && p.final_state) {  // state after the last block (its MMAs are done)
             ok = __all_sync(0xffffffffu, ok && !*abort);
             if (ok) {
+                tc_fence_after();
                 float* dst = p.final_state + (int64_t)b * p.state_stride + (int64_t)head * PN;
 #pragma unroll
                 for (int h2 = 0; h2 < 2; ++h2) {
                     uint32_t v[32];
-                    tmem_ld32(tmem + lane_base + kTS + 64 * hf + 32 * h2, v);
+                    tmem_ld32(sacc + 32 * h2, v);
                     tmem_ld_wait();
                     if (head_ok) {
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) dst[(32 * h2 + j) * kN + r] = __uint_as_float(v[j]);
+                        for (int j = 0; j < 32; ++j) dst[(32 * h2 + j) * kN + r] = s_in * __uint_as_float(v[j]);
                     }
                 }
             }
@@ -674,7 +833,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == kCtlWarp) tmem_dealloc(tmem, kTCols);
+    if (warp == 1) tmem_dealloc(tmem, kTCols);
 }
 
 // Segment end states from a zero start, for every segment but the last:
@@ -971,17 +1130,20 @@ static cudaError_t launch_scan_tc_impl(const ScanArgs& a, const ScanGate* gate, 
     if (!make_tmap_bf16(&mapC, a.C, (uint64_t)a.G * kN, rows, a.sC * 2, 64, kQ)) return cudaErrorInvalidValue;
 
     // y leaves through bulk tensor stores when it is 16-byte aligned with 16-byte row pitches
-    CUtensorMap mapY;
-    std::memset(&mapY, 0, sizeof(mapY));
-    const bool y_tma = (reinterpret_cast<uintptr_t>(a.y) & 15u) == 0 && (a.sy * 2) % 16 == 0 &&
-                       make_tmap_bf16_3d(&mapY, a.y, (uint64_t)a.h * kP, (uint64_t)a.L, (uint64_t)a.batch,
-                                         (uint64_t)a.sy * 2, (uint64_t)a.sy * 2 * a.L, 64, kQ);
-
     ScanTcParams p{};
     p.L = a.L; p.h = a.h; p.nseg = pl.nseg; p.cps = pl.cps; p.nchunks = pl.nchunks; p.hpg = a.hpg;
     p.c0 = pl.c0;
-    p.y_tma = y_tma ? 1 : 0;
     p.dt = a.dt; p.sdt = a.sdt; p.A = a.A; p.D = a.D; p.y = a.y; p.sy = a.sy;
+    // y leaves through bulk tensor stores when it is 16-byte aligned with 16-byte row pitches
+    CUtensorMap mapY, mapZ;
+    std::memset(&mapY, 0, sizeof(mapY));
+    std::memset(&mapZ, 0, sizeof(mapZ));
+    const bool y_tma = (reinterpret_cast<uintptr_t>(a.y) & 15u) == 0 && (a.sy * 2) % 16 == 0 &&
+                       make_tmap_bf16_3d(&mapY, a.y, (uint64_t)a.h * kP, (uint64_t)a.L, (uint64_t)a.batch,
+                                         (uint64_t)a.sy * 2, (uint64_t)a.sy * 2 * a.L, 64, kQ);
+    p.y_tma = y_tma ? 1 : 0;
+    if (gate && !make_tmap_bf16(&mapZ, gate->z, (uint64_t)a.h * kP, (uint64_t)rows, (uint64_t)gate->sz * 2, 64, kQ))
+        return cudaErrorInvalidValue;
     p.init_state = a.init_state; p.final_state = a.final_state; p.state_stride = a.state_stride;
     p.status = device_status_ptr();
     if (gate) {
@@ -1000,8 +1162,10 @@ static cudaError_t launch_scan_tc_impl(const ScanArgs& a, const ScanGate* gate, 
     cudaGetDevice(&dev);
     static unsigned long long attr_set = 0;
     if (dev < 64 && !(attr_set >> dev & 1ull)) {
-        cudaError_t e = cudaFuncSetAttribute(ssd_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(ssd_chunk_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              kChunkSmem);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(ssd_chunk_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kChunkSmem);
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(ssd_seg_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      kSegSmemBytes);
@@ -1010,7 +1174,8 @@ static cudaError_t launch_scan_tc_impl(const ScanArgs& a, const ScanGate* gate, 
     }
     const dim3 cgrid((a.h + 1) / 2, a.batch, pl.nseg);
     if (pl.nseg == 1) {
-        ssd_chunk_kernel<<<cgrid, kChunkThreads, kChunkSmem, s>>>(mapX, mapB, mapC, mapY, p);
+        if (gate) ssd_chunk_kernel<true><<<cgrid, kChunkThreads, kChunkSmem, s>>>(mapX, mapB, mapC, mapY, mapZ, p);
+        else ssd_chunk_kernel<false><<<cgrid, kChunkThreads, kChunkSmem, s>>>(mapX, mapB, mapC, mapY, mapZ, p);
         return cudaGetLastError();
     }
     // The chunk scan is launched as a programmatic dependent of the segment-state grid: segment
@@ -1042,7 +1207,8 @@ static cudaError_t launch_scan_tc_impl(const ScanArgs& a, const ScanGate* gate, 
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, ssd_chunk_kernel, mapX, mapB, mapC, mapY, p);
+    if (gate) return cudaLaunchKernelEx(&cfg, ssd_chunk_kernel<true>, mapX, mapB, mapC, mapY, mapZ, p);
+    return cudaLaunchKernelEx(&cfg, ssd_chunk_kernel<false>, mapX, mapB, mapC, mapY, mapZ, p);
 }
 
 }  // namespace mm
