@@ -227,7 +227,7 @@ int ssd_scan(int dtype, const void* x, int64_t x_stride, const float* dt, int64_
  * call on a device looks up the array's device address and caches it; make
  * that first call before any stream capture.
  */
-#define MM_SCAN_STATIC_SCRATCH_BYTES ((size_t)16 << 20) /* 16 MiB per device */
+#define MM_SCAN_STATIC_SCRATCH_BYTES ((size_t)32 << 20) /* 32 MiB per device */
 
 int ssd_scan_static(int dtype, const void* x, int64_t x_stride, const float* dt, int64_t dt_stride, const float* A,
                     const void* B, int64_t B_stride, const void* C, int64_t C_stride, const float* D, int batch,

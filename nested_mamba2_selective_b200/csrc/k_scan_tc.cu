@@ -29,6 +29,9 @@
 
 #include <cmath>
 #include <cstring>
+#include <map>
+#include <mutex>
+#include <tuple>
 #include <utility>
 
 #include "mm_internal.cuh"
@@ -64,8 +67,10 @@ struct ScanTcParams {
     const float* D;
     void* y;
     int64_t sy;
-    float* states;     // [b*h][nseg][P*N]: slot k = start state of segment k
-    float* seg_decay;  // [b*h][nseg]: log2 of the decay over segment k (k < nseg - 1)
+    float* states;     // [b*h][nslot][P*N]: slot j + 1 = end state of sub-segment j from a zero start
+    float* seg_decay;  // [b*h][nslot - 1]: log2 of the decay over sub-segment j
+    int nsub;          // segment-state sub-segments per segment but the last
+    int nslot;         // (nseg - 1) * nsub + 1
     const float* init_state;
     float* final_state;
     int64_t state_stride;
@@ -78,7 +83,6 @@ struct ScanTcParams {
     int y_tma;  // 1: y tiles leave through bulk tensor stores (mapY), 0: per-thread stores
 };
 
-__device__ __forceinline__ void named_sync_compute() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
 // Byte offset of 16-byte chunk `c` (0..7) of row `r` in a 128-byte-swizzled panel.
 __device__ __forceinline__ uint32_t sw128(int r, int c) { return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)); }
@@ -146,6 +150,16 @@ __device__ __forceinline__ void seg_range(const ScanTcParams& p, int seg, int* c
     *c_end = min(p.nchunks, seg == 0 ? p.c0 : *c_begin + p.cps);
 }
 
+// Blocks [c_begin, c_end) of segment-state sub-segment j: part j % nsub of segment j / nsub.
+__device__ __forceinline__ void sub_range(const ScanTcParams& p, int j, int* c_begin, int* c_end)
+{
+    int b0, b1;
+    seg_range(p, j / p.nsub, &b0, &b1);
+    const int u = j % p.nsub, len = max(b1 - b0, 0);
+    *c_begin = b0 + (len * u) / p.nsub;
+    *c_end = b0 + (len * (u + 1)) / p.nsub;
+}
+
 // Programmatic dependent launch: let the dependent grid start, and wait for the
 // prerequisite grid's completion (and its memory) before reading what it wrote.
 __device__ __forceinline__ void grid_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
@@ -154,9 +168,10 @@ __device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepco
 constexpr int kChunkThreads = 512;
 constexpr float kFastMax = 64.0f;  // log2 units
 // small tables after the H buffer (floats): state-warp scan totals [2 parity][2 heads][4], block
-// mode [2 parity], builder tables for steep blocks: cs [2 heads][128], dt [2 heads][128], builder
+// mode [2 parity], builder tables for steep blocks: cs [2 heads][128], column factors
+// 2^(m - cs_s) dt_s [2 heads][128] (m: cs at the last row of the 32-row quarter of s), builder
 // scan totals [2 heads][4]
-constexpr int kTabPart = 0, kTabMode = 16, kTabCs = 20, kTabDt = 276, kTabBPart = 532, kTabFloats = 540;
+constexpr int kTabPart = 0, kTabMode = 16, kTabCs = 20, kTabV = 276, kTabBPart = 532, kTabFloats = 540;
 constexpr int kOffH = kNStage * kStage;  // bf16 state copy of two heads (steep blocks: then X')
 constexpr int kOffTab = kOffH + 2 * kTileQP;
 constexpr int kOffBar = kOffTab + kTabFloats * 4;
@@ -431,27 +446,37 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
         for (int k = 0; k < nch; ++k) {  // every warp runs every iteration (named barrier 4)
             const bool okm = __all_sync(0xffffffffu, mbar_wait(mode_rdy, k & 1, abort));
             const bool fast = !okm || tab[kTabMode + (k & 1)] != 0.0f;
-            // steep blocks: cs and dt of both heads for every token of the block (warps 4-7, one row
-            // each), through the per-quarter totals
+            // steep blocks: every builder thread loads dt of its row for both heads; warps 4-7 (one
+            // row each) scan dt A into cs through the per-quarter totals and publish cs and the
+            // column factors V_s = 2^(m - cs_s) dt_s, m = cs at the last row of the quarter of s
             float c2[2] = {0.0f, 0.0f}, dv[2] = {0.0f, 0.0f};
-            if (!fast && !upper) {
+            if (!fast) {
                 const int t = (c_begin + k) * kQ + r;
 #pragma unroll
                 for (int j = 0; j < 2; ++j) {
                     dv[j] = (t < p.L && head0 + j < p.h) ? p.dt[(tok0 + t) * p.sdt + head0 + j] : 0.0f;
-                    c2[j] = warp_incl_scan(dv[j] * A2[j], lane);
-                    if (lane == 31) tab[kTabBPart + 4 * j + q] = c2[j];
+                    if (!upper) {
+                        c2[j] = warp_incl_scan(dv[j] * A2[j], lane);
+                        if (lane == 31) tab[kTabBPart + 4 * j + q] = c2[j];
+                    }
                 }
             }
             asm volatile("bar.sync 4, 192;" ::: "memory");
+            // the diagonal tile may use the factored form when its quarter spans at most 2^64 (read
+            // here: the next block's totals overwrite the table before its first barrier)
+            bool diag_split[2] = {true, true};
+#pragma unroll
+            for (int j = 0; j < 2; ++j) diag_split[j] = fast || -tab[kTabBPart + 4 * j + q] <= kFastMax;
             if (!fast && !upper) {
 #pragma unroll
                 for (int j = 0; j < 2; ++j) {
                     float pre = 0.0f;
 #pragma unroll
                     for (int i = 0; i < 4; ++i) pre += i < q ? tab[kTabBPart + 4 * j + i] : 0.0f;
-                    tab[kTabCs + 128 * j + r] = c2[j] + pre;
-                    tab[kTabDt + 128 * j + r] = dv[j];
+                    const float cs = c2[j] + pre;
+                    const float m = __shfl_sync(0xffffffffu, cs, 31);
+                    tab[kTabCs + 128 * j + r] = cs;
+                    tab[kTabV + 128 * j + r] = ex2(m - cs) * dv[j];
                 }
             }
             asm volatile("bar.sync 4, 192;" ::: "memory");
@@ -490,21 +515,43 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
                             pk[e >> 1] = pack_bf16(g0, g1);
                         }
                         tmem_st16(tmem + lane_base + kTG + 32 * cb, pk);
-                    } else {  // M_j = G 2^min(cs_t - cs_s, 0) dt_s, s <= t, one head after the other
+                    } else {  // M_j = G 2^(cs_t - cs_s) dt_s for s <= t, one head after the other
 #pragma unroll
                         for (int j = 0; j < 2; ++j) {
                             uint32_t pk[16];
-                            const float* cs = tab + kTabCs + 128 * j + 32 * cb;
-                            const float* dts = tab + kTabDt + 128 * j + 32 * cb;
+                            if (!diag || diag_split[j]) {
+                                // 2^(cs_t - cs_s) = 2^(cs_t - m) 2^(m - cs_s), m = cs at the last row of
+                                // the column block: below the diagonal both factors are <= 1 (a factor
+                                // that underflows belongs to an entry below 2^-126); on it the quarter
+                                // spans at most 2^64, so neither overflows
+                                const float u = ex2(ct[j] - tab[kTabCs + 128 * j + 32 * cb + 31]);
+                                const float2 u2 = make_float2(u, u);
+                                const float2* v2 = reinterpret_cast<const float2*>(tab + kTabV + 128 * j + 32 * cb);
 #pragma unroll
-                            for (int e = 0; e < 32; e += 2) {
-                                float m0 = __uint_as_float(gv[e]) * ex2(fminf(ct[j] - cs[e], 0.0f)) * dts[e];
-                                float m1 = __uint_as_float(gv[e + 1]) * ex2(fminf(ct[j] - cs[e + 1], 0.0f)) * dts[e + 1];
-                                if (diag) {
+                                for (int e = 0; e < 32; e += 2) {
+                                    float2 mv = mul2(mul2(make_float2(__uint_as_float(gv[e]), __uint_as_float(gv[e + 1])),
+                                                          v2[e >> 1]), u2);
+                                    if (diag) {
+                                        mv.x = e <= lane ? mv.x : 0.0f;
+                                        mv.y = e + 1 <= lane ? mv.y : 0.0f;
+                                    }
+                                    pk[e >> 1] = pack2(mv);
+                                }
+                            } else {  // a diagonal quarter spanning more than 2^64: one exponent per entry,
+                                      // cs_s and dt_s from the lane that owns row s
+                                const float cs_own = ct[j];
+#pragma unroll
+                                for (int e = 0; e < 32; e += 2) {
+                                    const float cs0 = __shfl_sync(0xffffffffu, cs_own, e);
+                                    const float cs1 = __shfl_sync(0xffffffffu, cs_own, e + 1);
+                                    const float d0 = __shfl_sync(0xffffffffu, dv[j], e);
+                                    const float d1 = __shfl_sync(0xffffffffu, dv[j], e + 1);
+                                    float m0 = __uint_as_float(gv[e]) * ex2(fminf(cs_own - cs0, 0.0f)) * d0;
+                                    float m1 = __uint_as_float(gv[e + 1]) * ex2(fminf(cs_own - cs1, 0.0f)) * d1;
                                     m0 = e <= lane ? m0 : 0.0f;
                                     m1 = e + 1 <= lane ? m1 : 0.0f;
+                                    pk[e >> 1] = pack_bf16(m0, m1);
                                 }
-                                pk[e >> 1] = pack_bf16(m0, m1);
                             }
                             tmem_st16(tmem + lane_base + kTG + 32 * cb + 16 * j, pk);
                         }
@@ -543,9 +590,9 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
                 float v[32];
 #pragma unroll
                 for (int j = 0; j < 32; ++j) v[j] = init ? init[(32 * h2 + j) * kN + r] : 0.0f;
-                for (int sj = 0; head_ok && sj < seg; ++sj) {
-                    const float dec = exp2f(p.seg_decay[bh * p.nseg + sj]);
-                    const float* sp = p.states + (bh * p.nseg + sj + 1) * PN;
+                for (int sj = 0; head_ok && sj < seg * p.nsub; ++sj) {
+                    const float dec = exp2f(p.seg_decay[bh * (p.nslot - 1) + sj]);
+                    const float* sp = p.states + (bh * p.nslot + sj + 1) * PN;
 #pragma unroll
                     for (int j = 0; j < 32; ++j) v[j] = fmaf(dec, v[j], sp[(32 * h2 + j) * kN + r]);
                 }
@@ -841,35 +888,41 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
 // The segment's blocks are visited last to first.  With D the decay of the
 // blocks already visited (those after the current one), token s of the block
 // gets the weight 2^(D + tot - cs_s) <= 1, and every block's B^T X'' is
-// accumulated into one TMEM accumulator: no per-block state update, and the
-// compute warps wait for the tensor core only to reuse one of two X'' buffers.
-// Two heads per CTA as in the chunk scan; S of head j sits in TMEM columns
-// [64 j, 64 j + 64), row n = state dim.
-constexpr int kSegStage = kTileQN + 2 * kTileQP;          // B | x of two heads
-constexpr int kSegOffXP = kNStage * kSegStage;            // two X'' buffers of two heads
-constexpr int kSegOffSmall = kSegOffXP + 2 * 2 * kTileQP;
-constexpr int kSegSmemBytes = kSegOffSmall + 2 * kQ * 4 + 32 + 256;
+// accumulated into one TMEM accumulator: no per-block state update.  X'' is
+// formed in place over x in the stage, which the MMA's commit then frees.
+// A CTA takes HC heads of one group (4 when the group allows: one MMA of N = 256
+// then serves four heads, at about the cost of an N = 128 one); S of head j sits
+// in TMEM columns [64 j, 64 j + 64), row n = state dim.
+template <int HC>
+struct SegCfg {
+    static constexpr int kStageBytes = kTileQN + HC * kTileQP;  // B | x of HC heads
+    static constexpr int kOffSmall = kNStage * kStageBytes;
+    static constexpr int kSmem = kOffSmall + 4 * HC * 4 + 8 * 8 + 16;
+    static constexpr int kThreads = 64 + 128 * HC;
+};
+static_assert(SegCfg<4>::kSmem <= 232448, "segment-state kernel exceeds 227 KB of shared memory");
 
-__global__ void __launch_bounds__(320, 1)
+template <int HC>
+__global__ void __launch_bounds__(SegCfg<HC>::kThreads, 1)
     ssd_seg_state_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CUtensorMap mapB,
                          const ScanTcParams p)
 {
+    using Cfg = SegCfg<HC>;
     extern __shared__ __align__(1024) uint8_t sm[];
-    float* wtot = reinterpret_cast<float*>(sm + kSegOffSmall);  // [2 heads][4]
-    uint64_t* full = reinterpret_cast<uint64_t*>(wtot + 8 + 2 * kQ);
-    uint64_t* empty = full + kNStage;
-    uint64_t* xr = empty + kNStage;   // X'' buffer written (compute -> MMA)
-    uint64_t* xf = xr + 2;            // X'' buffer consumed (MMA -> compute)
-    uint64_t* done = xf + 2;
+    float* wtot = reinterpret_cast<float*>(sm + Cfg::kOffSmall);  // [HC heads][4]
+    uint64_t* full = reinterpret_cast<uint64_t*>(wtot + 4 * HC);
+    uint64_t* empty = full + kNStage;  // stage read by the MMA (commit)
+    uint64_t* xr = empty + kNStage;    // X'' of the stage written (compute warps)
+    uint64_t* done = xr + kNStage;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
     volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
-    const int pair = blockIdx.x, seg = blockIdx.y, b = blockIdx.z;
-    const int head0 = 2 * pair;
+    const int grpc = blockIdx.x, sub = blockIdx.y, b = blockIdx.z;
+    const int head0 = HC * grpc;
     int c_begin, c_end;
-    seg_range(p, seg, &c_begin, &c_end);
+    sub_range(p, sub, &c_begin, &c_end);
     const int nch = max(c_end - c_begin, 0);
-    const int grp = head0 / p.hpg;
+    const int grp = head0 / p.hpg;  // all HC heads read one group
     const int64_t tok0 = (int64_t)b * p.L;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     grid_launch_dependents();  // the chunk scan may start its first segment beside this grid
@@ -878,8 +931,7 @@ __global__ void __launch_bounds__(320, 1)
         for (int i = 0; i < kNStage; ++i) {
             mbar_init(&full[i], 1);
             mbar_init(&empty[i], 1);
-            mbar_init(&xr[i], 8);
-            mbar_init(&xf[i], 1);
+            mbar_init(&xr[i], 4 * HC);
         }
         mbar_init(done, 1);
         *abort = (smem_u32(sm) & 1023u) ? 1 : 0;
@@ -889,7 +941,7 @@ __global__ void __launch_bounds__(320, 1)
         prefetch_tmap(&mapB);
     }
     if (warp == 1) {
-        tmem_alloc(tmem_slot, 128);
+        tmem_alloc(tmem_slot, 64 * HC);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -902,118 +954,115 @@ __global__ void __launch_bounds__(320, 1)
             int k = 0;
             for (; k < nch; ++k) {
                 const int s = k % kNStage;
-                if (!mbar_wait(&empty[s], ((k / kNStage) & 1) ^ 1, abort)) {
+                if (k >= kNStage && !mbar_wait(&empty[s], ((k / kNStage) - 1) & 1, abort)) {
                     raise_timeout(abort, p.status);
                     break;
                 }
                 const int row = (int)(tok0 + (int64_t)(c_end - 1 - k) * kQ);
-                uint8_t* base = sm + s * kSegStage;
-                mbar_arrive_expect_tx(&full[s], kSegStage);
+                uint8_t* base = sm + s * Cfg::kStageBytes;
+                mbar_arrive_expect_tx(&full[s], Cfg::kStageBytes);
                 tma_load_2d(base, &mapB, &full[s], grp * kN, row);
                 tma_load_2d(base + kTileQN / 2, &mapB, &full[s], grp * kN + 64, row);
-                tma_load_2d(base + kTileQN, &mapX, &full[s], head0 * kP, row);
-                tma_load_2d(base + kTileQN + kTileQP, &mapX, &full[s], min(head0 + 1, p.h - 1) * kP, row);
+#pragma unroll
+                for (int j = 0; j < HC; ++j)  // heads past the last one reload it (their dt is zero)
+                    tma_load_2d(base + kTileQN + j * kTileQP, &mapX, &full[s], min(head0 + j, p.h - 1) * kP, row);
             }
-            for (int j = max(0, k - kNStage); j < k; ++j) mbar_wait(&full[j % kNStage], (j / kNStage) & 1, abort);
+            for (int j = max(0, k - kNStage); j < k; ++j) mbar_wait(&full[j % kNStage], (j / kNStage) & 1, nullptr);
         }
     } else if (warp == 1) {
-        if (lane == 0 && !*abort) {  // MMA issuer: S += B^T [X''_0 | X''_1]
-            const uint32_t id_s = idesc_bf16(128, 128, 1, 1);
+        if (lane == 0 && !*abort) {  // MMA issuer: S += B^T [X''_0 | ... | X''_(HC-1)]
+            const uint32_t id_s = idesc_bf16(128, 64 * HC, 1, 1);
             for (int k = 0; k < nch; ++k) {
-                const int s = k % kNStage, xb = k & 1;
-                if (!mbar_wait(&full[s], (k / kNStage) & 1, abort) || !mbar_wait(&xr[xb], (k >> 1) & 1, abort)) {
+                const int s = k % kNStage;
+                if (!mbar_wait(&full[s], (k / kNStage) & 1, abort) || !mbar_wait(&xr[s], (k / kNStage) & 1, abort)) {
                     raise_timeout(abort, p.status);
                     break;
                 }
                 tc_fence_after();
-                const uint32_t aB = smem_u32(sm + s * kSegStage);
-                const uint32_t aXP = smem_u32(sm + kSegOffXP + xb * 2 * kTileQP);
+                const uint32_t aB = smem_u32(sm + s * Cfg::kStageBytes);
+                const uint32_t aXP = aB + kTileQN;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                     mma_ss(tmem, desc_sw128(aB + kk * 2048, kTileQN / 2, 1024), desc_sw128(aXP + kk * 2048, kTileQP, 1024),
                            id_s, (k | kk) != 0);
-                mma_commit(&xf[xb]);
                 mma_commit(&empty[s]);
             }
             mma_commit(done);
             mbar_wait(done, 0, nullptr);  // every issued MMA is done before TMEM can be released (bounded)
         }
-    } else {  // compute warps: thread (quarter q, lane) = token / state row r, head hf of the pair
+    } else {  // compute warps: thread (quarter q, lane) = token / state row r, head hf of the group
         const int cw = warp - 2, q = warp & 3, hf = cw >> 2;
         const int r = q * 32 + lane;
         const int head = head0 + hf;
         const bool head_ok = head < p.h;
         const float A2 = head_ok ? p.A[head] * kLog2e : 0.0f;
+        const uint32_t bar_cnt = 128 * HC;
         float D2 = 0.0f;
         float dt_next = 0.0f;
         if (head_ok && nch > 0) {
             const int t0 = (c_end - 1) * kQ;
             if (t0 + r < p.L) dt_next = p.dt[(tok0 + t0 + r) * p.sdt + head];
         }
-        for (int k = 0; k < nch; ++k) {  // every warp runs every iteration (named barriers)
-            const int s = k % kNStage, xb = k & 1;
+        bool ok = true;
+        for (int k = 0; k < nch; ++k) {  // every warp runs every iteration (named barrier 1)
+            const int s = k % kNStage;
             const int t0 = (c_end - 1 - k) * kQ;
             const float dtv = dt_next;
             if (k + 1 < nch) {
                 const int t1 = t0 - kQ;
                 dt_next = (head_ok && t1 + r < p.L) ? p.dt[(tok0 + t1 + r) * p.sdt + head] : 0.0f;
             }
-            float sc = dtv * A2;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const float v = __shfl_up_sync(0xffffffffu, sc, o);
-                if (lane >= o) sc += v;
-            }
-            if (lane == 31) wtot[hf * 4 + q] = sc;
-            named_sync_compute();
+            const float sc = warp_incl_scan(dtv * A2, lane);
+            float* wt = wtot + 4 * hf;
+            if (lane == 31) wt[q] = sc;
+            asm volatile("bar.sync 1, %0;" ::"r"(bar_cnt) : "memory");
             float pre = 0.0f, tot = 0.0f;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                const float w = wtot[hf * 4 + j];
+                const float w = wt[j];
                 pre += j < q ? w : 0.0f;
                 tot += w;
             }
-            named_sync_compute();
+            asm volatile("bar.sync 1, %0;" ::"r"(bar_cnt) : "memory");
             const float c2 = sc + pre;
-            bool ok = __all_sync(0xffffffffu, mbar_wait(&full[s], (k / kNStage) & 1, abort));
-            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&xf[xb], ((k >> 1) & 1) ^ 1, abort));
-            if (ok) {  // X''[r, :] = 2^(D + tot - cs_r) dt_r x[r, :]
+            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&full[s], (k / kNStage) & 1, abort));
+            if (ok) {  // X''[r, :] = 2^(D + tot - cs_r) dt_r x[r, :], in place
                 const float wgt = ex2(D2 + tot - c2) * dtv;
-                const uint8_t* sX = sm + s * kSegStage + kTileQN + hf * kTileQP;
-                uint8_t* dX = sm + kSegOffXP + xb * 2 * kTileQP + hf * kTileQP;
+                const float2 w2 = make_float2(wgt, wgt);
+                uint8_t* sX = sm + s * Cfg::kStageBytes + kTileQN + hf * kTileQP;
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
                     const uint4 xv = *reinterpret_cast<const uint4*>(sX + sw128(r, c));
                     uint4 o;
-                    o.x = pack_bf16(bf_lo(xv.x) * wgt, bf_hi(xv.x) * wgt);
-                    o.y = pack_bf16(bf_lo(xv.y) * wgt, bf_hi(xv.y) * wgt);
-                    o.z = pack_bf16(bf_lo(xv.z) * wgt, bf_hi(xv.z) * wgt);
-                    o.w = pack_bf16(bf_lo(xv.w) * wgt, bf_hi(xv.w) * wgt);
-                    *reinterpret_cast<uint4*>(dX + sw128(r, c)) = o;
+                    o.x = pack2(mul2(bf2(xv.x), w2));
+                    o.y = pack2(mul2(bf2(xv.y), w2));
+                    o.z = pack2(mul2(bf2(xv.z), w2));
+                    o.w = pack2(mul2(bf2(xv.w), w2));
+                    *reinterpret_cast<uint4*>(sX + sw128(r, c)) = o;
                 }
                 fence_async_smem();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&xr[xb]);
+                if (lane == 0) mbar_arrive(&xr[s]);
             } else {
                 raise_timeout(abort, p.status);
             }
             D2 += tot;
         }
-        const bool ok = __all_sync(0xffffffffu, mbar_wait(done, 0, abort));
+        ok = __all_sync(0xffffffffu, ok && mbar_wait(done, 0, abort));
         if (ok) {
             tc_fence_after();
-            float* dst = p.states + (((int64_t)b * p.h + head) * p.nseg + seg + 1) * (kP * kN);
+            float* dst = p.states + (((int64_t)b * p.h + head) * p.nslot + sub + 1) * (kP * kN);
 #pragma unroll
             for (int h2 = 0; h2 < 2; ++h2) {
                 uint32_t sv[32];
                 tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + 64 * hf + 32 * h2, sv);
                 tmem_ld_wait();
-                if (head_ok && !*abort) {
+                if (head_ok && !*abort) {  // an empty sub-segment contributes a zero state
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) dst[(32 * h2 + j) * kN + r] = __uint_as_float(sv[j]);
+                    for (int j = 0; j < 32; ++j) dst[(32 * h2 + j) * kN + r] = nch > 0 ? __uint_as_float(sv[j]) : 0.0f;
                 }
             }
-            if (head_ok && r == 0 && !*abort) p.seg_decay[((int64_t)b * p.h + head) * p.nseg + seg] = D2;
+            if (head_ok && r == 0 && !*abort) p.seg_decay[((int64_t)b * p.h + head) * (p.nslot - 1) + sub] = D2;
         }
     }
     tc_fence_before();
@@ -1021,59 +1070,139 @@ __global__ void __launch_bounds__(320, 1)
     tc_fence_after();
     if (warp == 1) {
         __syncwarp();
-        tmem_dealloc(tmem, 128);
+        tmem_dealloc(tmem, 64 * HC);
     }
 }
 
 struct Plan {
     int nchunks, nseg, cps;
-    int c0;       // blocks of segment 0 (>= cps when it runs beside the segment-state grid)
-    bool overlap;  // segment 0's CTAs fit beside the segment-state grid
+    int nsub;      // segment-state sub-segments per segment but the last
+    int c0;        // blocks of segment 0
+    double cost;   // modelled makespan, in chunk-scan blocks
 };
 
-Plan plan_for(const ScanArgs& a, int sms)
+// Free times of the SMs as (time, count) pairs, for list-scheduling whole grids of equal CTAs.
+struct SmPool {
+    std::map<double, int64_t> free_at;
+    explicit SmPool(int sms) { free_at[0.0] = sms; }
+    // Dispatch n CTAs in launch order onto the earliest free SMs; a CTA holds its SM from then
+    // on, starts its work no earlier than `floor` and runs `dur`.  Returns the latest end and the
+    // latest dispatch time.
+    std::pair<double, double> take(int64_t n, double floor, double dur)
+    {
+        double last_end = 0.0, last_disp = 0.0;
+        while (n > 0) {
+            auto it = free_at.begin();
+            const double t = it->first;
+            const int64_t k = std::min(n, it->second);
+            if ((it->second -= k) == 0) free_at.erase(it);
+            const double end = std::max(t, floor) + dur;
+            free_at[end] += k;
+            last_end = std::max(last_end, end);
+            last_disp = std::max(last_disp, t);
+            n -= k;
+        }
+        return {last_end, last_disp};
+    }
+};
+
+// Model costs in units of one 128-token block of the chunk scan with every SM busy (about 3.8 us
+// on B200 for a block of two heads whose decay fits the factored form).
+constexpr double kCtaStart = 1.5;    // chunk CTA: TMEM, barriers, state fold, pipeline fill
+constexpr double kSegStart = 1.0;    // segment-state CTA: the same, without a fold
+constexpr double kSegGridEnd = 0.5;  // the segment-state grid's drain before the chunk scan may fold
+constexpr double kSteep = 1.6;       // a block of a head pair that needs the exact decay form
+
+// Makespan of one plan: the segment-state grid is dispatched first, then the chunk scan (a
+// programmatic dependent, so only once every segment-state CTA is resident), segment by segment;
+// CTAs of segments > 0 start their blocks when the segment-state grid has finished.  Heads with a
+// steep decay make some CTAs kSteep times slower, wherever they land; the modelled makespan is
+// the later of the uniform one and the end of such a CTA dispatched last in its segment.
+double plan_cost(int sms, int64_t ctas, int64_t sctas, double seg_block, int nchunks, int ns, int nsub, int c0,
+                 int c1)
 {
-    // Costs in units of one 128-token block of chunk-scan work per CTA.  A CTA also pays a
-    // fixed start (TMEM, barriers, state fold and pipeline fill: about 1.5 blocks).  A block of
-    // the segment-state pass costs about 0.3 of a chunk-scan block.  Segment 0 needs no carried
-    // state: when its CTAs fit on the SMs the segment-state grid leaves free, it starts at once
-    // and may take more blocks than the others, which start after the segment-state grid.
+    SmPool pool(sms);
+    double seg_end = 0.0, seg_disp = 0.0;
+    if (ns > 1) {
+        for (int g = 0; g < 2; ++g) {  // sub-segments of segment 0, then those of the others
+            const int len = g == 0 ? c0 : c1;
+            const int64_t n = sctas * nsub * (g == 0 ? 1 : ns - 2);
+            if (n == 0) continue;
+            const auto r = pool.take(n, 0.0, seg_block * ((len + nsub - 1) / nsub + kSegStart));
+            seg_end = std::max(seg_end, r.first);
+            seg_disp = std::max(seg_disp, r.second);
+        }
+        seg_end += kSegGridEnd;
+    }
+    double cost = 0.0;
+    for (int k = 0; k < ns; ++k) {
+        const int len = k == 0 ? c0 : std::min(c1, nchunks - c0 - (k - 1) * c1);
+        const double floor = k == 0 ? seg_disp : seg_end;
+        const auto r = pool.take(ctas, floor, len + kCtaStart);
+        cost = std::max(cost, std::max(r.first, std::max(r.second, floor) + kSteep * len + kCtaStart));
+    }
+    return cost;
+}
+
+Plan plan_for_uncached(const ScanArgs& a, int sms)
+{
+    // Long sequences are cut into segments whose CTAs run side by side: a segment-state pass
+    // computes each earlier segment's end state from a zero start (split into nsub sub-segments,
+    // one CTA each, to shorten it), and every chunk-scan CTA folds the end states before its
+    // segment.  Segment 0 needs no carried state: it starts at once and may take more blocks.
     Plan pl;
     pl.nchunks = (a.L + kQ - 1) / kQ;
-    const int64_t ctas = (int64_t)a.batch * ((a.h + 1) / 2);  // CTAs per segment: head pairs
-    double best = 1e30;
+    const int64_t ctas = (int64_t)a.batch * ((a.h + 1) / 2);  // chunk CTAs per segment: head pairs
+    const bool quad = a.G == 1 || a.hpg % 4 == 0;
+    const int64_t sctas = (int64_t)a.batch * (quad ? (a.h + 3) / 4 : (a.h + 1) / 2);  // per sub-segment
+    const double seg_block = quad ? 0.43 : 0.34;  // a segment-state block, four (two) heads per CTA
     pl.nseg = 1;
-    pl.cps = pl.nchunks;
-    pl.c0 = pl.nchunks;
-    pl.overlap = false;
-    for (int ns = 1; ns <= pl.nchunks && ns <= 64; ++ns) {
-        const bool overlap = ns > 1 && ctas * ns <= sms;
+    pl.nsub = 1;
+    pl.cps = pl.c0 = pl.nchunks;
+    pl.cost = plan_cost(sms, ctas, sctas, seg_block, pl.nchunks, 1, 1, pl.nchunks, pl.nchunks);
+    // Measured on B200: when two or more segments fit on the SMs at once, plans whose chunk-scan
+    // CTAs and segment-state CTAs all fit in one wave beat every plan that needs a second one;
+    // the model alone does not see that, so such plans are the only ones searched.
+    const bool one_wave = sms / ctas >= 2;
+    for (int ns = 2; ns <= pl.nchunks && ns <= 64; ++ns) {
+        if (one_wave && ctas * ns > sms) break;
         const int even = (pl.nchunks + ns - 1) / ns;
-        // segment 0 of c0 blocks, the others of c1 blocks each (the last one shorter, never empty);
-        // only an overlapped segment 0 may be longer than the even split
-        for (int c0 = even; c0 <= (overlap ? pl.nchunks - (ns - 1) : even); ++c0) {
-            const int rest = pl.nchunks - c0;
-            int c1 = 0;
-            double cost;
-            if (ns == 1) {
-                cost = std::ceil((double)ctas / sms) * (c0 + 1.5);
-            } else {
-                if (rest < ns - 1) continue;
-                c1 = (rest + ns - 2) / (ns - 1);
+        for (int nsub = 1; nsub <= 4; ++nsub) {
+            if (one_wave && ctas + sctas * nsub * (ns - 1) > sms) break;
+            // segment 0 of c0 >= even blocks, the others of c1 blocks each (the last one shorter,
+            // never empty)
+            for (int c0 = even; c0 <= std::min(pl.nchunks - (ns - 1), 2 * even + 2); ++c0) {
+                const int rest = pl.nchunks - c0;
+                const int c1 = (rest + ns - 2) / (ns - 1);
                 if (rest - (ns - 2) * c1 <= 0) continue;
-                const double seg_pass = 0.3 * std::ceil((double)(ctas * (ns - 1)) / sms) * (std::max(c0, c1) + 1.5) + 0.4;
-                cost = overlap ? std::max(c0 + 1.5, seg_pass + (c1 + 1.5))
-                               : seg_pass + std::ceil((double)(ctas * ns) / sms) * (std::max(c0, c1) + 1.5);
-            }
-            if (cost < best - 1e-9) {
-                best = cost;
-                pl.nseg = ns;
-                pl.c0 = c0;
-                pl.cps = ns > 1 ? c1 : c0;
-                pl.overlap = overlap;
+                const double cost = plan_cost(sms, ctas, sctas, seg_block, pl.nchunks, ns, nsub, c0, c1);
+                if (cost < pl.cost - 1e-9) {
+                    pl.cost = cost;
+                    pl.nseg = ns;
+                    pl.nsub = nsub;
+                    pl.c0 = c0;
+                    pl.cps = c1;
+                }
             }
         }
     }
+    return pl;
+}
+
+// Plans depend only on the shape and the SM count; the search is cached per shape.
+Plan plan_for(const ScanArgs& a, int sms)
+{
+    static std::mutex mu;
+    static std::map<std::tuple<int, int, int, int, int, int>, Plan> cache;
+    const auto key = std::make_tuple(a.batch, a.L, a.h, a.G, a.hpg, sms);
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        const auto it = cache.find(key);
+        if (it != cache.end()) return it->second;
+    }
+    const Plan pl = plan_for_uncached(a, sms);
+    std::lock_guard<std::mutex> lock(mu);
+    if (cache.size() < 4096) cache[key] = pl;
     return pl;
 }
 
@@ -1101,7 +1230,8 @@ size_t scan_tc_workspace(const ScanArgs& a)
     const Plan pl = plan_for(a, num_sms());
     if (pl.nseg == 1) return 256;
     const size_t bh = (size_t)a.batch * a.h;
-    return align256(bh * pl.nseg * kP * kN * 4) + align256(bh * pl.nseg * 4);
+    const size_t nslot = (size_t)(pl.nseg - 1) * pl.nsub + 1;
+    return align256(bh * nslot * kP * kN * 4) + align256(bh * (nslot - 1) * 4);
 }
 
 int scan_tc_kernel_count(const ScanArgs& a) { return plan_for(a, num_sms()).nseg > 1 ? 2 : 1; }
@@ -1133,6 +1263,8 @@ static cudaError_t launch_scan_tc_impl(const ScanArgs& a, const ScanGate* gate, 
     ScanTcParams p{};
     p.L = a.L; p.h = a.h; p.nseg = pl.nseg; p.cps = pl.cps; p.nchunks = pl.nchunks; p.hpg = a.hpg;
     p.c0 = pl.c0;
+    p.nsub = pl.nsub;
+    p.nslot = (pl.nseg - 1) * pl.nsub + 1;
     p.dt = a.dt; p.sdt = a.sdt; p.A = a.A; p.D = a.D; p.y = a.y; p.sy = a.sy;
     // y leaves through bulk tensor stores when it is 16-byte aligned with 16-byte row pitches
     CUtensorMap mapY, mapZ;
@@ -1156,7 +1288,7 @@ static cudaError_t launch_scan_tc_impl(const ScanArgs& a, const ScanGate* gate, 
     if (pl.nseg > 1) {
         if (!ws || ws_bytes < scan_tc_workspace(a)) return cudaErrorInvalidValue;
         p.states = static_cast<float*>(ws);
-        p.seg_decay = reinterpret_cast<float*>(static_cast<char*>(ws) + align256(bh * pl.nseg * kP * kN * 4));
+        p.seg_decay = reinterpret_cast<float*>(static_cast<char*>(ws) + align256(bh * p.nslot * kP * kN * 4));
     }
     int dev = 0;
     cudaGetDevice(&dev);
@@ -1167,8 +1299,11 @@ static cudaError_t launch_scan_tc_impl(const ScanArgs& a, const ScanGate* gate, 
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(ssd_chunk_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kChunkSmem);
         if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(ssd_seg_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     kSegSmemBytes);
+            e = cudaFuncSetAttribute(ssd_seg_state_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     SegCfg<4>::kSmem);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(ssd_seg_state_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     SegCfg<2>::kSmem);
         if (e != cudaSuccess) return e;
         attr_set |= 1ull << dev;
     }
@@ -1190,11 +1325,16 @@ static cudaError_t launch_scan_tc_impl(const ScanArgs& a, const ScanGate* gate, 
         const std::pair<uintptr_t, uintptr_t> ins[3] = {span(a.x, ((T - 1) * a.sx + (int64_t)a.h * kP) * esz),
                                                         span(a.B, ((T - 1) * a.sB + (int64_t)a.G * kN) * esz),
                                                         span(a.dt, ((T - 1) * a.sdt + a.h) * 4)};
-        p.wait_all = (pl.overlap ? 0 : 1);
+        p.wait_all = 0;
         for (const auto& in : ins)
             if (ys.first < in.second && in.first < ys.second) p.wait_all = 1;
     }
-    ssd_seg_state_kernel<<<dim3((a.h + 1) / 2, pl.nseg - 1, a.batch), 320, kSegSmemBytes, s>>>(mapX, mapB, p);
+    if (a.G == 1 || a.hpg % 4 == 0)  // four heads of one group per CTA
+        ssd_seg_state_kernel<4><<<dim3((a.h + 3) / 4, p.nslot - 1, a.batch), SegCfg<4>::kThreads, SegCfg<4>::kSmem, s>>>(
+            mapX, mapB, p);
+    else
+        ssd_seg_state_kernel<2><<<dim3((a.h + 1) / 2, p.nslot - 1, a.batch), SegCfg<2>::kThreads, SegCfg<2>::kSmem, s>>>(
+            mapX, mapB, p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};

@@ -60,21 +60,20 @@ def test_static_scratch_matches_workspace_entry_point_on_consecutive_calls():
 
 
 def oversized_shape():
-    """A scan whose segment states need more scratch than the fixed array holds."""
-    for L in (65536, 131072, 262144):
-        for h in (64, 128):
-            if ssd_scan_workspace(torch.bfloat16, 1, L, h, 64, 128, 1, 256) > CAPACITY:
-                return L, h
+    """A scan whose segment states need more scratch than the fixed array holds (smallest first)."""
+    for b, L, h in ((2, 8192, 128), (4, 8192, 128), (8, 16384, 24), (4, 16384, 128), (8, 16384, 128)):
+        if ssd_scan_workspace(torch.bfloat16, b, L, h, 64, 128, 1, 256) > CAPACITY:
+            return b, L, h
     raise AssertionError("no oversized shape found")
 
 
 def test_static_scratch_rejects_sizes_beyond_its_capacity():
-    L, h = oversized_shape()
-    x = torch.zeros((1, L, h, 64), dtype=torch.bfloat16, device="cuda")
-    Bm = torch.zeros((1, L, 1, 128), dtype=torch.bfloat16, device="cuda")
-    dt = torch.full((1, L, h), 1e-3, device="cuda")
+    b, L, h = oversized_shape()
+    x = torch.zeros((b, L, h, 64), dtype=torch.bfloat16, device="cuda")
+    Bm = torch.zeros((b, L, 1, 128), dtype=torch.bfloat16, device="cuda")
+    dt = torch.full((b, L, h), 1e-3, device="cuda")
     A = torch.full((h,), -1.0, device="cuda")
-    y = torch.full((1, L, h, 64), 3.0, dtype=torch.bfloat16, device="cuda")
+    y = torch.full((b, L, h, 64), 3.0, dtype=torch.bfloat16, device="cuda")
     with pytest.raises(MatMambaError) as ei:
         ssd_scan_static(x, dt, A, Bm, Bm, None, chunk=256, y=y)
     assert ei.value.status == 5  # MM_ERR_WORKSPACE: nothing launched
