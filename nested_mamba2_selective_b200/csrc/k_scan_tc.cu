@@ -1108,8 +1108,10 @@ struct SmPool {
 
 // Model costs in units of one 128-token block of the chunk scan with every SM busy (about 3.8 us
 // on B200 for a block of two heads whose decay fits the factored form).
-constexpr double kCtaStart = 1.5;    // chunk CTA: TMEM, barriers, state fold, pipeline fill
-constexpr double kSegStart = 1.0;    // segment-state CTA: the same, without a fold
+// The constants were fitted to plans timed on B200 over the scan and block shapes of 3 to 64 heads.
+constexpr double kCtaStart = 1.0;    // chunk CTA: TMEM, barriers, pipeline fill
+constexpr double kFoldSlot = 0.2;    // chunk CTA: folding one earlier sub-segment state (two heads)
+constexpr double kSegStart = 0.5;    // segment-state CTA: TMEM, barriers, pipeline fill
 constexpr double kSegGridEnd = 0.5;  // the segment-state grid's drain before the chunk scan may fold
 constexpr double kSteep = 1.6;       // a block of a head pair that needs the exact decay form
 
@@ -1138,8 +1140,9 @@ double plan_cost(int sms, int64_t ctas, int64_t sctas, double seg_block, int nch
     for (int k = 0; k < ns; ++k) {
         const int len = k == 0 ? c0 : std::min(c1, nchunks - c0 - (k - 1) * c1);
         const double floor = k == 0 ? seg_disp : seg_end;
-        const auto r = pool.take(ctas, floor, len + kCtaStart);
-        cost = std::max(cost, std::max(r.first, std::max(r.second, floor) + kSteep * len + kCtaStart));
+        const double start = kCtaStart + kFoldSlot * k * nsub;
+        const auto r = pool.take(ctas, floor, len + start);
+        cost = std::max(cost, std::max(r.first, std::max(r.second, floor) + kSteep * len + start));
     }
     return cost;
 }
@@ -1160,9 +1163,11 @@ Plan plan_for_uncached(const ScanArgs& a, int sms)
     pl.nsub = 1;
     pl.cps = pl.c0 = pl.nchunks;
     pl.cost = plan_cost(sms, ctas, sctas, seg_block, pl.nchunks, 1, 1, pl.nchunks, pl.nchunks);
-    // Measured on B200: when two or more segments fit on the SMs at once, plans whose chunk-scan
-    // CTAs and segment-state CTAs all fit in one wave beat every plan that needs a second one;
-    // the model alone does not see that, so such plans are the only ones searched.
+    // Measured on B200, beyond what the model sees: when one segment's CTAs fill three quarters
+    // of the SMs, a single segment is fastest; when two or more segments fit on the SMs at once,
+    // plans whose chunk-scan and segment-state CTAs all fit in one wave beat every plan that
+    // needs a second one, so only those are searched.
+    if (4 * ctas >= 3 * (int64_t)sms) return pl;
     const bool one_wave = sms / ctas >= 2;
     for (int ns = 2; ns <= pl.nchunks && ns <= 64; ++ns) {
         if (one_wave && ctas * ns > sms) break;

@@ -61,7 +61,7 @@ def test_static_scratch_matches_workspace_entry_point_on_consecutive_calls():
 
 def oversized_shape():
     """A scan whose segment states need more scratch than the fixed array holds (smallest first)."""
-    for b, L, h in ((2, 8192, 128), (4, 8192, 128), (8, 16384, 24), (4, 16384, 128), (8, 16384, 128)):
+    for b, L, h in ((8, 32768, 24), (4, 32768, 48), (8, 65536, 24), (4, 65536, 48), (8, 131072, 24)):
         if ssd_scan_workspace(torch.bfloat16, b, L, h, 64, 128, 1, 256) > CAPACITY:
             return b, L, h
     raise AssertionError("no oversized shape found")
