@@ -10,14 +10,16 @@
 //   H_next = 2^(tot - a) [ 2^a H_prev + B^T X~ ],   X~_s = 2^(a - cs_s) dt_s x_s
 // with Gc the causally masked C B^T (log2 units): the decay becomes per-token
 // scales of x and per-row scales of y, and one contraction serves both heads of
-// a CTA.  Blocks whose decay across half a block exceeds 2^64 use exact
-// per-element decay matrices instead (see ssd_chunk_kernel).  Both unroll the
+// a CTA.  Blocks whose decay across half a block exceeds 2^64 use per-head
+// masked decay matrices instead (see ssd_chunk_kernel).  Both unroll the
 // recurrence exactly.  The sequence is cut into segments of whole blocks so
 // that (batch, head pair, segment) CTAs fill the GPU:
-//   1. seg_state  : each segment's end state from a zero start (tcgen05)
+//   1. seg_state  : the end state of each sub-segment of every segment but the
+//                   last, from a zero start (tcgen05, four heads per CTA)
 //   2. chunk_scan : every segment from its true start state (the initial state
-//                   carried over the earlier segments' end states at the CTA's
-//                   start), carrying the state across blocks in TMEM (tcgen05).
+//                   carried over the earlier sub-segments' end states at the
+//                   CTA's start), carrying the state across blocks in TMEM
+//                   (tcgen05).
 //                   It is a programmatic dependent of seg_state: segment 0 needs
 //                   no carried state and may run beside it.
 // Only segment end states touch HBM.
@@ -122,9 +124,12 @@ __device__ __forceinline__ float bf_hi(uint32_t v) { return __uint_as_float(v & 
 // output.  Every exponent stays within the decay across half a block, which fast blocks bound by
 // 2^kFastMax (64 in log2 units) for both heads.
 // Steep blocks (either half of a head decays faster than that) take the direct form instead:
-// per-head masked decay matrices M_j[t,s] = G[t,s] 2^(cs_t - cs_s) dt_s with exact exponentials,
+// per-head masked decay matrices M_j[t,s] = G[t,s] 2^(cs_t - cs_s) dt_s,
 //   y_t = M_j x + 2^(cs_t) C_t H + D x_t,   H_next = 2^tot H + B^T X',  X'_s = 2^(tot - cs_s) dt_s x_s,
-// with the state term in a second output accumulator.
+// with the state term in a second output accumulator.  The builders factor each entry's decay at
+// the last row m of its 32-token column block, 2^(cs_t - m) 2^(m - cs_s), so a tile needs one power
+// of two per row and per column; only a diagonal tile whose quarter decays by more than 2^64 takes
+// one exponential per entry.
 //
 // 512 threads in roles:
 //   warp 0      TMA producer (one lane)
