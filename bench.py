@@ -170,6 +170,10 @@ def decode_work(m, Bt, Dm=2048, E=4096, P=64, N=128, K=4):
         "step_scan": ("hbm", Bt * (h * P * N * 4 * 2 + nconv * 2 + h * 4 + d * 2)),
         "step_gate_rmsnorm": ("hbm", Bt * d * 2 * 3),
         "step_out_proj": ("hbm", Dm * d * 2 + Bt * d * 2 + Bt * Dm * 2),
+        # fused forms: the state update with the gate (state read and written, xBC, dt and z read, the
+        # gated row and its per-half sums of squares written), and out_proj with the 1/RMS row scale
+        "step_scan_gate": ("hbm", Bt * (h * P * N * 4 * 2 + nconv * 2 + h * 4 + d * 2 + d * 2 + 2 * h * 4)),
+        "step_out_proj_norm": ("hbm", Dm * d * 2 + Bt * d * 2 + Bt * 2 * h * 4 + Bt * Dm * 2),
     }
 
 
