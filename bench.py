@@ -122,6 +122,9 @@ def peaks():
 
 # ------------------------------------------------------------------------------------ workload sizes
 
+# device spin before each timed step (about 200 us at B200 clocks), longer than the host needs to enqueue one
+LEAD_CYCLES = 400_000
+
 BLOCK = dict(workload="block_130m_b8_L2048", batch=8, seq_len=2048, d_model=768, d_inner=1536, d_head=64,
              d_state=128, ngroups=1, d_conv=4, chunk=256, widths=[768, 384, 192, 96])
 SCAN = dict(workload="ssd_b4_L8192_h24", batch=4, seq_len=8192, heads=24, d_head=64, d_state=128, chunk=256,
@@ -354,18 +357,22 @@ def run_ours(args):
     clk = ClockSampler(dev).__enter__()  # samples only inside timed regions
 
     def timed(fn, steps, warmup, trace=False):
+        """Device time of each of `steps` calls of fn between CUDA events, L2 flushed before each.  Before
+        every step the device spins for LEAD_CYCLES so that the host has enqueued the whole step when the
+        first event is reached: the events then bracket device work only, not Python and launch latency.
+        With trace, a second pass of the same steps (untimed) collects the library's per-stage device times
+        and its kernel count, so the stage events never sit inside the timed steps."""
         for _ in range(warmup):
             fn()
         torch.cuda.synchronize()
         barrier()
-        if trace:
-            mm.mm_trace_enable(steps * 32)
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
         torch.cuda.synchronize()
         barrier()
         clk.region_begin()
         for e0, e1 in ev:
             flush_buf.zero_()
+            torch.cuda._sleep(LEAD_CYCLES)
             e0.record(stream)
             fn()
             e1.record(stream)
@@ -375,6 +382,12 @@ def run_ours(args):
         ms = [e0.elapsed_time(e1) for e0, e1 in ev]
         tr = None
         if trace:
+            mm.mm_trace_enable(steps * 32)
+            for _ in range(steps):
+                flush_buf.zero_()
+                torch.cuda._sleep(LEAD_CYCLES)
+                fn()
+            torch.cuda.synchronize()
             tr = mm.mm_trace_collect()
             mm.mm_trace_enable(0)
         return ms, tr
@@ -481,7 +494,9 @@ def run_ours(args):
                        "chunk_note": "the chunked scan's result does not depend on chunk; the bf16 kernels "
                                      "evaluate every chunk of 256 as two 128-token blocks",
                        "width": m0, "parallelism": "replicas%d" % world,
-                       "l2": "flushed (256 MiB write) before every timed step"},
+                       "l2": "flushed (256 MiB write) before every timed step",
+                       "timing": "CUDA events around each step after a device spin that lets the host enqueue "
+                                 "the whole step; per-stage times from a separate traced pass"},
             "per_width": per_width,
             "roofline": roof,
             "stages": stage_rows,
