@@ -513,6 +513,10 @@ def run_ours(args):
         if not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(arrays, u_np, m0)
             line["cpu_baseline_scan"] = cpu_baseline_scan()
+            if stack:
+                line["cpu_baseline_stack"] = cpu_baseline_stack()
+            if decode:
+                line["cpu_baseline_decode"] = cpu_baseline_decode()
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
@@ -686,6 +690,55 @@ def cpu_baseline_scan(budget_s=6.0):
     except Exception as e:  # noqa: BLE001 - the 1-core figure is informative only
         res["one_core"] = {"error": str(e)[:200]}
     return res
+
+
+def cpu_baseline_stack(layers=4, tokens=256):
+    """The fp64 oracle's stack forward at full width on a bounded slice of the 48-layer workload: one batch
+    row, a causal prefix of `tokens` tokens (exact for those outputs, by causality and batch independence)
+    through `layers` layers of random weights; the rate for all 48 layers is the measured per-layer rate
+    divided by 48 (layers cost the same)."""
+    import numpy as np
+
+    import oracle
+    from nested_mamba2_selective_b200 import synth
+    S = STACK
+    dims = oracle.Dims(S["d_model"], S["d_inner"], S["d_head"], S["d_state"])
+    params = [{k: v.astype(np.float64) for k, v in synth.block_params(S["d_model"], S["d_inner"], S["d_head"],
+                                                                       S["d_state"], dtype="bf16",
+                                                                       seed=1003 + l).items()} for l in range(layers)]
+    prenorm = np.ones(S["d_model"])
+    u = synth.activations((1, tokens, S["d_model"]), "bf16", seed=1003)
+    t0 = time.perf_counter()
+    oracle.stack_fwd(dims, layers, lambda l: params[l], lambda l: prenorm, u, [S["d_model"]] * layers)
+    el = time.perf_counter() - t0
+    return {"value": tokens / (el * S["nlayers"] / layers), "unit": "tokens/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": "one batch row x %d-token prefix through %d of the 48 layers at width %d, scaled to 48 layers "
+                      "(fp64 oracle, OpenMP)" % (tokens, layers, S["d_model"])}
+
+
+def cpu_baseline_decode(seqs=4, steps=50):
+    """The fp64 oracle's recurrent step at full width on `seqs` of the 256 sequences for `steps` consecutive
+    tokens from an N(0, 1) state (sequences are independent)."""
+    import numpy as np
+
+    import oracle
+    from nested_mamba2_selective_b200 import synth
+    D = DECODE
+    dims = oracle.Dims(D["d_model"], D["d_inner"], D["d_head"], D["d_state"])
+    p = {k: v.astype(np.float64) for k, v in synth.block_params(D["d_model"], D["d_inner"], D["d_head"],
+                                                                  D["d_state"], dtype="bf16", seed=1004).items()}
+    H = D["d_inner"] // D["d_head"]
+    ssm, conv = synth.states(seqs, H, D["d_head"], D["d_state"], D["d_inner"] + 2 * D["d_state"], 4, "bf16", seed=1004)
+    ssm, conv = ssm.astype(np.float64), conv.astype(np.float64)
+    u = synth.activations((steps, seqs, D["d_model"]), "bf16", seed=1004)
+    t0 = time.perf_counter()
+    for i in range(steps):
+        oracle.block_step(dims, p, u[i], D["d_model"], ssm, conv)
+    el = time.perf_counter() - t0
+    return {"value": seqs * steps / el, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": "%d of %d sequences x %d consecutive steps at width %d (fp64 oracle, OpenMP)"
+                      % (seqs, D["batch"], steps, D["d_model"])}
 
 
 def cpu_baseline(arrays, u_np, m, budget_s=10.0):
