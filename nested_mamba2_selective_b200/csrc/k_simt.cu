@@ -456,11 +456,94 @@ __global__ void step_conv_dt_kernel(const T* __restrict__ zxbc, int64_t ld_in, i
     xbc_out[(int64_t)b * nconv + c] = from_f32<T>(silu_f(acc));
 }
 
+// The same for bf16 and a window of 4 taps, four channels per thread: the three stored inputs of
+// four channels are 24 contiguous bytes, their taps 32, so every access is an 8- or 16-byte vector.
+__device__ __forceinline__ float bf16_bits_to_f32(uint32_t v, int hi) { return __uint_as_float(hi ? (v & 0xFFFF0000u) : (v << 16)); }
+
+__global__ void step_conv_dt4_kernel(const __nv_bfloat16* __restrict__ zxbc, int64_t ld_in, int col0,
+                                     const float* __restrict__ dt_raw, const __nv_bfloat16* __restrict__ conv_w,
+                                     const __nv_bfloat16* __restrict__ conv_b, const float* __restrict__ dt_bias, int E,
+                                     int d, int nconv, int h, __nv_bfloat16* __restrict__ conv_state, int conv_rows,
+                                     __nv_bfloat16* __restrict__ xbc_out, float* __restrict__ dt_out)
+{
+    const int t = blockIdx.x * blockDim.x + threadIdx.x;
+    const int b = blockIdx.y;
+    const int ngrp = nconv / 4;
+    if (t >= ngrp + h) return;
+    if (t >= ngrp) {
+        const int i = t - ngrp;
+        dt_out[(int64_t)b * h + i] = softplus_f(dt_raw[(int64_t)b * h + i] + dt_bias[i]);
+        return;
+    }
+    const int c0 = 4 * t;
+    const int row0 = c0 < d ? c0 : E + (c0 - d);  // groups of four never straddle d (a multiple of 4)
+    uint2* st = reinterpret_cast<uint2*>(conv_state + ((int64_t)b * conv_rows + row0) * 3);
+    const uint2 s01 = st[0], s12 = st[1], s23 = st[2];  // channel j's inputs are bf16 [3 j, 3 j + 3) of these 12
+    const uint32_t sw[6] = {s01.x, s01.y, s12.x, s12.y, s23.x, s23.y};
+    const uint2 xn = *reinterpret_cast<const uint2*>(zxbc + (int64_t)b * ld_in + col0 + c0);
+    const uint32_t xw[2] = {xn.x, xn.y};
+    const uint4 w01 = *reinterpret_cast<const uint4*>(conv_w + (int64_t)row0 * 4);
+    const uint4 w23 = *reinterpret_cast<const uint4*>(conv_w + (int64_t)row0 * 4 + 8);
+    const uint32_t ww[8] = {w01.x, w01.y, w01.z, w01.w, w23.x, w23.y, w23.z, w23.w};
+    const uint2 bb = *reinterpret_cast<const uint2*>(conv_b + row0);
+    const uint32_t bw[2] = {bb.x, bb.y};
+    float in[4][4];  // [channel][tap]: three stored inputs, then the new one
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+#pragma unroll
+        for (int k = 0; k < 3; ++k) {
+            const int e = 3 * j + k;  // bf16 element of the 12 stored ones
+            in[j][k] = bf16_bits_to_f32(sw[e >> 1], e & 1);
+        }
+        in[j][3] = bf16_bits_to_f32(xw[j >> 1], j & 1);
+    }
+    float out[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        float acc = bf16_bits_to_f32(bw[j >> 1], j & 1);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) acc = fmaf(bf16_bits_to_f32(ww[(4 * j + k) >> 1], k & 1), in[j][k], acc);
+        out[j] = silu_f(acc);
+    }
+    // the shifted window: channel j keeps inputs 1, 2 and the new one
+    uint32_t nw[6];
+#pragma unroll
+    for (int e2 = 0; e2 < 6; ++e2) {
+        uint32_t v = 0;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            const int e = 2 * e2 + half, j = e / 3, k = e % 3;
+            const __nv_bfloat16 q = __float2bfloat16_rn(in[j][k + 1]);  // exact: a bf16 value moves
+            v |= (uint32_t)__bfloat16_as_ushort(q) << (16 * half);
+        }
+        nw[e2] = v;
+    }
+    st[0] = make_uint2(nw[0], nw[1]);
+    st[1] = make_uint2(nw[2], nw[3]);
+    st[2] = make_uint2(nw[4], nw[5]);
+    uint2 o;
+    o.x = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(out[0])) |
+          ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(out[1])) << 16);
+    o.y = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(out[2])) |
+          ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(out[3])) << 16);
+    *reinterpret_cast<uint2*>(xbc_out + (int64_t)b * nconv + c0) = o;
+}
+
 cudaError_t launch_step_conv_dt(int dtype, const void* zxbc, int64_t ld_in, int col0, const float* dt_raw,
                                 const void* conv_w, const void* conv_b, const float* dt_bias, int E, int d, int nconv,
                                 int h, int K, int batch, void* conv_state, int conv_rows, void* xbc_out, float* dt_out,
                                 cudaStream_t s)
 {
+    auto al = [](const void* q, uintptr_t a) { return (reinterpret_cast<uintptr_t>(q) & (a - 1)) == 0; };
+    if (dtype == MM_BF16 && K == 4 && nconv % 4 == 0 && d % 4 == 0 && E % 4 == 0 && conv_rows % 4 == 0 &&
+        ld_in % 4 == 0 && col0 % 4 == 0 && al(zxbc, 8) && al(conv_w, 16) && al(conv_b, 8) && al(conv_state, 8) &&
+        al(xbc_out, 8)) {
+        dim3 grid((nconv / 4 + h + 127) / 128, batch);
+        step_conv_dt4_kernel<<<grid, 128, 0, s>>>(
+            (const __nv_bfloat16*)zxbc, ld_in, col0, dt_raw, (const __nv_bfloat16*)conv_w, (const __nv_bfloat16*)conv_b,
+            dt_bias, E, d, nconv, h, (__nv_bfloat16*)conv_state, conv_rows, (__nv_bfloat16*)xbc_out, dt_out);
+        return cudaGetLastError();
+    }
     dim3 grid((nconv + h + 127) / 128, batch);
     if (dtype == MM_BF16)
         step_conv_dt_kernel<__nv_bfloat16><<<grid, 128, 0, s>>>(
