@@ -376,11 +376,68 @@ __global__ void rmsnorm_rows_kernel(const float* __restrict__ x, const T* __rest
     for (int c = lane; c < cols; c += 32) out[(int64_t)row * cols + c] = from_f32<T>(xr[c] * rstd * to_f32(w[c]));
 }
 
+// The same for bf16 weights and output with cols = 128 NV: a lane keeps its NV float4 of the row in
+// registers, so the row is read once with 16-byte loads and written with 8-byte stores.
+template <int NV>
+__global__ void rmsnorm_rows_vec_kernel(const float* __restrict__ x, const __nv_bfloat16* __restrict__ w, float eps,
+                                        int rows, __nv_bfloat16* __restrict__ out)
+{
+    constexpr int cols = 128 * NV;
+    const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= rows) return;
+    const float4* xr = reinterpret_cast<const float4*>(x + (int64_t)row * cols);
+    float4 v[NV];
+    float ss = 0.0f;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+        v[i] = xr[lane + 32 * i];
+        ss = fmaf(v[i].x, v[i].x, ss);
+        ss = fmaf(v[i].y, v[i].y, ss);
+        ss = fmaf(v[i].z, v[i].z, ss);
+        ss = fmaf(v[i].w, v[i].w, ss);
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    const float rstd = rsqrtf(ss / cols + eps);
+    const uint2* wr = reinterpret_cast<const uint2*>(w);
+    uint2* orow = reinterpret_cast<uint2*>(out + (int64_t)row * cols);
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+        const uint2 wv = wr[lane + 32 * i];
+        const float w0 = __uint_as_float(wv.x << 16), w1 = __uint_as_float(wv.x & 0xFFFF0000u);
+        const float w2 = __uint_as_float(wv.y << 16), w3 = __uint_as_float(wv.y & 0xFFFF0000u);
+        uint2 o;
+        o.x = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v[i].x * rstd * w0)) |
+              ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v[i].y * rstd * w1)) << 16);
+        o.y = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v[i].z * rstd * w2)) |
+              ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v[i].w * rstd * w3)) << 16);
+        orow[lane + 32 * i] = o;
+    }
+}
+
 cudaError_t launch_rmsnorm_rows_f32in(int dtype, const float* x, const void* w, float eps, int cols, int rows, void* out,
                                       cudaStream_t s)
 {
     if (rows == 0) return cudaSuccess;
     dim3 grid((rows + 7) / 8);
+    const bool vec = dtype == MM_BF16 && cols % 128 == 0 && cols <= 2048 &&
+                     (reinterpret_cast<uintptr_t>(x) & 15u) == 0 && (reinterpret_cast<uintptr_t>(w) & 7u) == 0 &&
+                     (reinterpret_cast<uintptr_t>(out) & 7u) == 0;
+    if (vec) {
+        const __nv_bfloat16* wb = (const __nv_bfloat16*)w;
+        __nv_bfloat16* ob = (__nv_bfloat16*)out;
+        switch (cols / 128) {
+            case 1: rmsnorm_rows_vec_kernel<1><<<grid, 256, 0, s>>>(x, wb, eps, rows, ob); return cudaGetLastError();
+            case 2: rmsnorm_rows_vec_kernel<2><<<grid, 256, 0, s>>>(x, wb, eps, rows, ob); return cudaGetLastError();
+            case 4: rmsnorm_rows_vec_kernel<4><<<grid, 256, 0, s>>>(x, wb, eps, rows, ob); return cudaGetLastError();
+            case 6: rmsnorm_rows_vec_kernel<6><<<grid, 256, 0, s>>>(x, wb, eps, rows, ob); return cudaGetLastError();
+            case 8: rmsnorm_rows_vec_kernel<8><<<grid, 256, 0, s>>>(x, wb, eps, rows, ob); return cudaGetLastError();
+            case 12: rmsnorm_rows_vec_kernel<12><<<grid, 256, 0, s>>>(x, wb, eps, rows, ob); return cudaGetLastError();
+            case 16: rmsnorm_rows_vec_kernel<16><<<grid, 256, 0, s>>>(x, wb, eps, rows, ob); return cudaGetLastError();
+            default: break;
+        }
+    }
     if (dtype == MM_BF16)
         rmsnorm_rows_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(x, (const __nv_bfloat16*)w, eps, cols, rows,
                                                                   (__nv_bfloat16*)out);
@@ -413,9 +470,30 @@ cudaError_t launch_to_f32(int dtype, const void* in, float* out, int64_t n, cuda
     return cudaGetLastError();
 }
 
+// fp32 -> bf16, four elements per thread (16-byte loads, 8-byte stores)
+__global__ void from_f32_bf16x4_kernel(const float4* __restrict__ in, uint2* __restrict__ out, int64_t n4)
+{
+    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n4; e += (int64_t)gridDim.x * blockDim.x) {
+        const float4 v = in[e];
+        uint2 o;
+        o.x = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v.x)) |
+              ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v.y)) << 16);
+        o.y = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v.z)) |
+              ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v.w)) << 16);
+        out[e] = o;
+    }
+}
+
 cudaError_t launch_from_f32(int dtype, const float* in, void* out, int64_t n, cudaStream_t s)
 {
     if (n == 0) return cudaSuccess;
+    if (dtype == MM_BF16 && n % 4 == 0 && (reinterpret_cast<uintptr_t>(in) & 15u) == 0 &&
+        (reinterpret_cast<uintptr_t>(out) & 7u) == 0) {
+        const int64_t blocks = (n / 4 + 255) / 256;
+        const int grid = (int)(blocks < 148 * 8 ? blocks : 148 * 8);
+        from_f32_bf16x4_kernel<<<grid, 256, 0, s>>>(reinterpret_cast<const float4*>(in), static_cast<uint2*>(out), n / 4);
+        return cudaGetLastError();
+    }
     const int64_t blocks = (n + 255) / 256;
     const int grid = (int)(blocks < 148 * 16 ? blocks : 148 * 16);
     if (dtype == MM_BF16) from_f32_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(in, (__nv_bfloat16*)out, n);
