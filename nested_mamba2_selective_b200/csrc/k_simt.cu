@@ -460,9 +460,26 @@ __global__ void from_f32_kernel(const float* __restrict__ in, T* __restrict__ ou
         out[e] = from_f32<T>(in[e]);
 }
 
+// bf16 -> fp32, four elements per thread (8-byte loads, 16-byte stores)
+__global__ void to_f32_bf16x4_kernel(const uint2* __restrict__ in, float4* __restrict__ out, int64_t n4)
+{
+    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n4; e += (int64_t)gridDim.x * blockDim.x) {
+        const uint2 v = in[e];
+        out[e] = make_float4(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xFFFF0000u), __uint_as_float(v.y << 16),
+                             __uint_as_float(v.y & 0xFFFF0000u));
+    }
+}
+
 cudaError_t launch_to_f32(int dtype, const void* in, float* out, int64_t n, cudaStream_t s)
 {
     if (n == 0) return cudaSuccess;
+    if (dtype == MM_BF16 && n % 4 == 0 && (reinterpret_cast<uintptr_t>(in) & 7u) == 0 &&
+        (reinterpret_cast<uintptr_t>(out) & 15u) == 0) {
+        const int64_t blocks = (n / 4 + 255) / 256;
+        const int grid = (int)(blocks < 148 * 8 ? blocks : 148 * 8);
+        to_f32_bf16x4_kernel<<<grid, 256, 0, s>>>(static_cast<const uint2*>(in), reinterpret_cast<float4*>(out), n / 4);
+        return cudaGetLastError();
+    }
     const int64_t blocks = (n + 255) / 256;
     const int grid = (int)(blocks < 148 * 16 ? blocks : 148 * 16);
     if (dtype == MM_BF16) to_f32_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>((const __nv_bfloat16*)in, out, n);
