@@ -107,3 +107,34 @@ def test_prefill_then_step_equals_longer_prefill(block, m):
     full = matmamba_block_fwd(wt, u, m, 256)
     torch.cuda.synchronize()
     assert max_abs_rel(to_np(step), to_np(full[:, 200])) <= TOL["bf16"]
+
+
+def test_unaligned_conv_state_gives_the_same_steps(orc, block):
+    """A conv state that starts 2 bytes past an 8-byte boundary takes the one-channel-per-thread roll
+    instead of the vector one.  Both do the same arithmetic in the same order, so the conv and SSM
+    states agree bit for bit; the outputs (summed over K slices in arrival order) both match the
+    oracle."""
+    wt, p64 = block
+    dims = dims_of(W)
+    m = 1024
+    s_np, c_np = states(4, seed=377)
+    runs = []
+    for offset in (0, 1):
+        buf = torch.zeros(c_np.size + 4, dtype=torch.bfloat16, device="cuda")
+        c_gpu = buf[offset:offset + c_np.size].view(c_np.shape)
+        c_gpu.copy_(to_device(c_np, "bf16"))
+        s_gpu = torch.from_numpy(s_np).cuda()
+        outs = []
+        for step in range(3):
+            u = synth.activations((4, W.d_model), "bf16", seed=380 + step)
+            outs.append(ssd_step(wt, s_gpu, c_gpu, to_device(u, "bf16"), m))
+        torch.cuda.synchronize()
+        runs.append((torch.stack(outs), s_gpu, c_gpu.clone()))
+    assert torch.equal(runs[0][1], runs[1][1])
+    assert torch.equal(runs[0][2], runs[1][2])
+    s_ref, c_ref = s_np.astype(np.float64), c_np.astype(np.float64)
+    for step in range(3):
+        u = synth.activations((4, W.d_model), "bf16", seed=380 + step)
+        ref = orc.block_step(dims, p64, u, m, s_ref, c_ref)
+        for run in runs:
+            assert max_abs_rel(to_np(run[0][step]), ref) <= TOL["bf16"]

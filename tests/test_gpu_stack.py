@@ -79,3 +79,20 @@ def test_stack48_full_size_sampled():
             xs[m] = oracle.stack_fwd(DIMS, 1, lambda _: p64, lambda _: w64, xs[m], [m])
     for m in widths:
         assert max_abs_rel(outs[m], xs[m]) <= TOL["bf16"], m
+
+
+def test_stack_with_unaligned_prenorm_weights():
+    """Pre-norm weights that start 2 bytes past an 8-byte boundary take the one-row-per-warp scalar
+    pre-norm instead of the vector one; two layers still match the oracle."""
+    layers, pw = gpu_layers(2)
+    shifted = []
+    for w in pw:
+        buf = torch.zeros(w.numel() + 4, dtype=torch.bfloat16, device="cuda")
+        v = buf[1:1 + w.numel()]
+        v.copy_(w)
+        assert v.data_ptr() % 8 != 0
+        shifted.append(v)
+    u = synth.activations((1, 200, W.d_model), "bf16", seed=411)
+    out = matmamba_stack_fwd(layers, shifted, to_device(u, "bf16"), [2048, 1024], chunk=256)
+    torch.cuda.synchronize()
+    assert max_abs_rel(to_np(out), oracle_stack(2, u, [2048, 1024])) <= TOL["bf16"]
