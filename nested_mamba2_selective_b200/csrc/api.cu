@@ -296,6 +296,7 @@ int block_impl_fused(const mm_block_params* p, const View& v, const void* u, int
     go.ex.nparts = 2 * v.h;
     go.ex.rs_inv_n = 1.0f / (float)v.d;
     go.ex.rs_eps = p->norm_eps;
+    go.pdl = 1;  // out_proj may set up during the chunk scan's tail, then waits for it
     MM_TRY(stage("out_proj_norm", 1, s, [&] { return launch_gemm_tc(go, s); }));
     return MM_OK;
 }

@@ -73,6 +73,7 @@ struct TcParams {
     TcSeg seg[kMaxSeg];
     GemmExtra ex;
     int* status;
+    int pdl;  // launched as a programmatic dependent: wait for the previous kernel before reading
 };
 
 template <int BN>
@@ -198,6 +199,11 @@ __global__ void __launch_bounds__(320, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // Programmatic dependent launch: the set-up above may overlap the previous kernel's tail; nothing
+    // that kernel writes is read before it has completed.  A following dependent may start its own
+    // set-up once every CTA of this grid has started.
+    if (p.pdl) asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     // tiles: (K slice, row block, N tile), K slices slowest
     const int total = p.mtiles * p.ntiles * p.ksplit;
     auto release_acc = [&](int b) { mbar_arrive(&tempty[b]); };  // this drain warp is done with accumulator b
@@ -885,8 +891,21 @@ static cudaError_t launch_bn(const GemmDesc& g, const TcParams& p0, cudaStream_t
         attr_set |= 1ull << dev;
     }
     // one CTA per tile: the CTAs that start first take over the others' tiles as they go
-    kernel<<<p.mtiles * p.ntiles * p.ksplit, 320, smem, s>>>(mapA, mapB, mapB2, om, p);
-    return cudaGetLastError();
+    if (!p.pdl) {
+        kernel<<<p.mtiles * p.ntiles * p.ksplit, 320, smem, s>>>(mapA, mapB, mapB2, om, p);
+        return cudaGetLastError();
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.mtiles * p.ntiles * p.ksplit);
+    cfg.blockDim = dim3(320);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, mapA, mapB, mapB2, om, p);
 }
 
 cudaError_t launch_gemm_tc(const GemmDesc& g, cudaStream_t s)
@@ -897,6 +916,7 @@ cudaError_t launch_gemm_tc(const GemmDesc& g, cudaStream_t s)
     p.ktiles = (g.K + kBK - 1) / kBK;
     p.nseg = g.nseg;
     p.ex = g.ex;
+    p.pdl = g.pdl;
     p.shift = 0;
     for (int i = 0; i < g.nseg; ++i)
         if (g.seg[i].kind == kEpiConv) p.shift = g.ex.K - 1;

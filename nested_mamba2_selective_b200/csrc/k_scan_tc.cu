@@ -282,6 +282,9 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     uint8_t* sH = sm + kOffH;
+    // a following programmatic dependent (the output projection) may start its set-up once every CTA
+    // of this grid has started; it reads nothing of ours before this grid has completed
+    grid_launch_dependents();
 
     if (warp == 0) {
         if (lane == 0 && !*abort) {  // ------------------------------------------------ TMA producer

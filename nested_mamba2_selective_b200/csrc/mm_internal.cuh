@@ -75,6 +75,9 @@ struct GemmDesc {
     int nseg;
     GemmSeg seg[kMaxSeg];
     GemmExtra ex;
+    // launch as a programmatic dependent of the stream's previous kernel: the CTAs may become resident
+    // while it finishes, and wait for its completion before reading anything
+    int pdl = 0;
 };
 
 // ------------------------------------------------------------------ scan arguments
