@@ -145,6 +145,9 @@ __device__ __forceinline__ float bf_hi(uint32_t v) { return __uint_as_float(v & 
 // fast blocks S += B^T X~, Y = C . [2^a H_0 | 2^a H_1] and Y += Gc . [X~_0 | X~_1]; for steep
 // blocks Yoff = C . [H_0 | H_1], S += B^T X', Y_j = M_j x_j.  The two output accumulators
 // alternate between blocks, so block k-1's epilogue runs under block k's tensor work.
+// A stage's B and x regions are free once the block's MMAs are done (a commit), so the next
+// block but one starts loading them at once; its C region (where the gated form's z tile then
+// lands) holds the block's y tile until the bulk store has read it, and only C waits for that.
 // Element-wise products use the paired fp32 instructions (mul/fma .f32x2, rounded per lane
 // exactly like their scalar forms).
 
@@ -180,7 +183,7 @@ constexpr int kTabPart = 0, kTabMode = 16, kTabCs = 20, kTabV = 276, kTabBPart =
 constexpr int kOffH = kNStage * kStage;  // bf16 state copy of two heads (steep blocks: then X')
 constexpr int kOffTab = kOffH + 2 * kTileQP;
 constexpr int kOffBar = kOffTab + kTabFloats * 4;
-constexpr int kNumBars = 18;
+constexpr int kNumBars = 22;
 constexpr int kChunkSmem = kOffBar + kNumBars * 8 + 16;
 static_assert(kChunkSmem <= 232448, "chunk scan exceeds the 227 KB of shared memory a CTA can have");
 static_assert(kOffBar % 8 == 0, "mbarriers need 8-byte alignment");
@@ -220,9 +223,11 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
 {
     extern __shared__ __align__(1024) uint8_t sm[];
     float* tab = reinterpret_cast<float*>(sm + kOffTab);
-    uint64_t* full = reinterpret_cast<uint64_t*>(sm + kOffBar);  // [2] stage loaded (TMA transaction)
-    uint64_t* empty = full + 2;                                   // [2] stage free: its y tile stored (8 warps)
-    uint64_t* g_done = empty + 2;                                 // G of the block done (commit)
+    uint64_t* full = reinterpret_cast<uint64_t*>(sm + kOffBar);  // [2] B and x of the stage loaded (TMA)
+    uint64_t* full_c = full + 2;                                  // [2] C of the stage loaded (TMA)
+    uint64_t* empty = full_c + 2;                                 // [2] B and x free: the block's MMAs done (commit)
+    uint64_t* empty_c = empty + 2;                                // [2] C region free: its y tile stored (8 warps)
+    uint64_t* g_done = empty_c + 2;                               // G of the block done (commit)
     uint64_t* m_ready = g_done + 1;                               // Gc or M built (6 builder warps)
     uint64_t* mode_rdy = m_ready + 1;                             // block mode written (1 state thread)
     uint64_t* h_ready = mode_rdy + 1;                             // read-back done (8 state warps)
@@ -251,7 +256,9 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < kNStage; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 8);
+            mbar_init(&full_c[s], 1);
+            mbar_init(&empty[s], 1);
+            mbar_init(&empty_c[s], 8);
             mbar_init(&yfree[s], 8);
             mbar_init(&y_done[s], 1);
             mbar_init(&zfull[s], 1);
@@ -301,24 +308,32 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
                 ++zk;
                 return true;
             };
-            int k = 0;
+            int k = 0, kbx = 0, kc = 0;  // blocks whose B and x / C loads are issued
             for (; k < nch; ++k) {
                 const int s = k % kNStage;
-                // block k goes into the stage block k-2 used, once its epilogue released it
+                // block k goes into the stage block k-2 used: B and x once that block's MMAs are
+                // done, C once its y tile (staged in the C region) has been stored
                 if (k >= kNStage && !mbar_wait(&empty[s], ((k / kNStage) - 1) & 1, abort)) {
                     raise_timeout(abort, p.status);
                     break;
                 }
                 const int row = (int)(tok0 + (int64_t)(c_begin + k) * kQ);
                 uint8_t* base = sm + s * kStage;
-                mbar_arrive_expect_tx(&full[s], kStage);
-                tma_load_2d(base + kOffC, &mapC, &full[s], grp * kN, row);
-                tma_load_2d(base + kOffC + kTileQN / 2, &mapC, &full[s], grp * kN + 64, row);
+                mbar_arrive_expect_tx(&full[s], kStage - kOffB);
                 tma_load_2d(base + kOffB, &mapB, &full[s], grp * kN, row);
                 tma_load_2d(base + kOffB + kTileQN / 2, &mapB, &full[s], grp * kN + 64, row);
                 tma_load_2d(base + kOffX, &mapX, &full[s], head0 * kP, row);
                 // a pair's second head past the last head reloads the last head (its dt is zero)
                 tma_load_2d(base + kOffX + kTileQP, &mapX, &full[s], min(head0 + 1, p.h - 1) * kP, row);
+                kbx = k + 1;
+                if (k >= kNStage && !mbar_wait(&empty_c[s], ((k / kNStage) - 1) & 1, abort)) {
+                    raise_timeout(abort, p.status);
+                    break;
+                }
+                mbar_arrive_expect_tx(&full_c[s], kTileQN);
+                tma_load_2d(base + kOffC, &mapC, &full_c[s], grp * kN, row);
+                tma_load_2d(base + kOffC + kTileQN / 2, &mapC, &full_c[s], grp * kN + 64, row);
+                kc = k + 1;
                 if (GATED && k > 0 && !load_z(k - 1)) {  // block k-1's z, once its C.H MMA is done
                     raise_timeout(abort, p.status);
                     break;
@@ -326,7 +341,8 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
             }
             if (GATED && k == nch && nch > 0 && !load_z(nch - 1)) raise_timeout(abort, p.status);
             // every issued load lands before the CTA can exit (bounded; only the last two can be pending)
-            for (int j = max(0, k - kNStage); j < k; ++j) mbar_wait(&full[j % kNStage], (j / kNStage) & 1, nullptr);
+            for (int j = max(0, kbx - kNStage); j < kbx; ++j) mbar_wait(&full[j % kNStage], (j / kNStage) & 1, nullptr);
+            for (int j = max(0, kc - kNStage); j < kc; ++j) mbar_wait(&full_c[j % kNStage], (j / kNStage) & 1, nullptr);
             for (int j = max(0, zk - kNStage); j < zk; ++j) mbar_wait(&zfull[j % kNStage], (j / kNStage) & 1, nullptr);
         }
     } else if (warp == 1) {
@@ -346,7 +362,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
             for (int k = 0; ok && k < nch; ++k) {
                 const int s = k % kNStage, yi = k & 1;
                 // stage k is loaded, and block k-1's output MMAs (the last readers of the G columns) are done
-                if (!mbar_wait(&full[s], (k / kNStage) & 1, abort) ||
+                if (!mbar_wait(&full[s], (k / kNStage) & 1, abort) || !mbar_wait(&full_c[s], (k / kNStage) & 1, abort) ||
                     (k > 0 && !mbar_wait(&y_done[(k - 1) & 1], ((k - 1) >> 1) & 1, abort))) {
                     ok = false;
                     break;
@@ -399,6 +415,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
                         mma_ts(yacc, tmem + kTG + 32 * (kk >> 1) + 8 * (kk & 1),
                                desc_sw128(aX + kk * 2048, kTileQP, 1024), id_o, 1u);
                     mma_commit(&y_done[yi]);
+                    mma_commit(&empty[s]);  // B and x of the stage are read
                 } else {
                     const uint32_t oacc = tmem + kTY0 + 128 * (yi ^ 1);
                     if (!acc_free(yi ^ 1)) {
@@ -435,6 +452,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
                             mma_ts(yacc + 64 * j, tmem + kTG + 32 * (kk >> 1) + 16 * j + 8 * (kk & 1),
                                    desc_sw128(aX + j * kTileQP + kk * 2048, kTileQP, 1024), id_y, 1u);
                     mma_commit(&y_done[yi]);
+                    mma_commit(&empty[s]);  // B and x of the stage are read
                 }
             }
             if (!ok) raise_timeout(abort, p.status);
@@ -622,9 +640,10 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
 
         // Epilogue of block kp: y from the output accumulator(s), which already hold the D x term, and
         // the optional gate (z from the tile the producer loaded into the stage's C region).  y rows go
-        // into the stage's x region in the 128-byte swizzle and leave as one bulk tensor store per head
-        // (rows past L clipped); the stage is released once the store has read them.  Every warp of
-        // the head calls it once per block (named barrier 2 + hf).
+        // into the stage's C region (over z: each thread reads its row's z chunk before writing the
+        // y chunk there) in the 128-byte swizzle and leave as one bulk tensor store per head (rows
+        // past L clipped); the C region is released once the store has read them.  Every warp of the
+        // head calls it once per block (named barrier 2 + hf).
         auto epilogue = [&](int kp) {
             const int sp = kp & 1;
             const int tp0 = (c_begin + kp) * kQ;
@@ -633,7 +652,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
             const int col = head * kP;
             const uint32_t yacc = tmem + lane_base + kTY0 + 128 * sp + 64 * hf;
             const uint32_t oacc = tmem + lane_base + kTY0 + 128 * (sp ^ 1) + 64 * hf;
-            uint8_t* sX = sm + sp * kStage + kOffX + hf * kTileQP;        // y rows (over X~ or x)
+            uint8_t* sX = sm + sp * kStage + kOffC + hf * kTileQP;        // y rows (over C, or z)
             const uint8_t* sZ = sm + sp * kStage + kOffC + hf * kTileQP;  // z rows (gated)
             if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&y_done[sp], (kp >> 1) & 1, abort));
             if (GATED && ok) ok = __all_sync(0xffffffffu, mbar_wait(&zfull[sp], (kp >> 1) & 1, abort));
@@ -720,10 +739,10 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
                     __syncwarp();
                 }
             }
-            if (ok) {  // stage sp is free once its y tile has been read
+            if (ok) {  // the C region of stage sp is free once its y tile has been read
                 if (lane == 0) {
                     if (p.y_tma && q == 0) bulk_wait_read0();
-                    mbar_arrive(&empty[sp]);
+                    mbar_arrive(&empty_c[sp]);
                 }
                 __syncwarp();
             }
