@@ -183,7 +183,7 @@ constexpr int kTabPart = 0, kTabMode = 16, kTabCs = 20, kTabV = 276, kTabBPart =
 constexpr int kOffH = kNStage * kStage;  // bf16 state copy of two heads (steep blocks: then X')
 constexpr int kOffTab = kOffH + 2 * kTileQP;
 constexpr int kOffBar = kOffTab + kTabFloats * 4;
-constexpr int kNumBars = 22;
+constexpr int kNumBars = 24;
 constexpr int kChunkSmem = kOffBar + kNumBars * 8 + 16;
 static_assert(kChunkSmem <= 232448, "chunk scan exceeds the 227 KB of shared memory a CTA can have");
 static_assert(kOffBar % 8 == 0, "mbarriers need 8-byte alignment");
@@ -229,12 +229,13 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
     uint64_t* empty_c = empty + 2;                                // [2] C region free: its y tile stored (8 warps)
     uint64_t* g_done = empty_c + 2;                               // G of the block done (commit)
     uint64_t* m_ready = g_done + 1;                               // Gc or M built (6 builder warps)
-    uint64_t* mode_rdy = m_ready + 1;                             // block mode written (1 state thread)
-    uint64_t* h_ready = mode_rdy + 1;                             // read-back done (8 state warps)
+    uint64_t* mode_rdy = m_ready + 1;                             // [2] block mode written (1 state thread)
+    uint64_t* h_ready = mode_rdy + 2;                             // read-back done (8 state warps)
     uint64_t* h_free = h_ready + 1;                               // state MMA and H copy consumed (commit)
     uint64_t* yo_done = h_free + 1;                               // steep blocks: C.H done (commit)
-    uint64_t* x_ready = yo_done + 1;                              // X~ or X' written (8 state warps)
-    uint64_t* y_done = x_ready + 1;                               // [2] every MMA of a block using output
+    uint64_t* x_ready = yo_done + 1;                              // [2] X~ or X' written (8 state warps);
+                                                                  // a fast block's X~ may come one block early
+    uint64_t* y_done = x_ready + 2;                               // [2] every MMA of a block using output
                                                                   // accumulator i done (commit)
     uint64_t* yfree = y_done + 2;                                 // [2] output accumulator read (8 warps)
     uint64_t* zfull = yfree + 2;                                  // [2] gated: z tile in the C region (TMA)
@@ -265,11 +266,13 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
         }
         mbar_init(g_done, 1);
         mbar_init(m_ready, 6);
-        mbar_init(mode_rdy, 1);
+        mbar_init(&mode_rdy[0], 1);
+        mbar_init(&mode_rdy[1], 1);
         mbar_init(h_ready, 8);
         mbar_init(h_free, 1);
         mbar_init(yo_done, 1);
-        mbar_init(x_ready, 8);
+        mbar_init(&x_ready[0], 8);
+        mbar_init(&x_ready[1], 8);
         mbar_init(done, 1);
         *abort = (smem_u32(sm) & 1023u) ? 1 : 0;  // tiles need 1024-byte alignment; never fault on it
         if (*abort) raise_timeout(abort, p.status);
@@ -384,7 +387,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
                 const bool fast = tab[kTabMode + (k & 1)] != 0.0f;
                 const uint32_t yacc = tmem + kTY0 + 128 * yi;
                 if (fast) {
-                    if (!mbar_wait(x_ready, k & 1, abort)) {
+                    if (!mbar_wait(&x_ready[k & 1], (k >> 1) & 1, abort)) {
                         ok = false;
                         break;
                     }
@@ -430,7 +433,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
                                kk > 0);
                     }
                     mma_commit(yo_done);
-                    if (!mbar_wait(x_ready, k & 1, abort)) {  // X' written over the state copy
+                    if (!mbar_wait(&x_ready[k & 1], (k >> 1) & 1, abort)) {  // X' written over the state copy
                         ok = false;
                         break;
                     }
@@ -470,7 +473,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
 #pragma unroll
         for (int j = 0; j < 2; ++j) A2[j] = head0 + j < p.h ? p.A[head0 + j] * kLog2e : 0.0f;
         for (int k = 0; k < nch; ++k) {  // every warp runs every iteration (named barrier 4)
-            const bool okm = __all_sync(0xffffffffu, mbar_wait(mode_rdy, k & 1, abort));
+            const bool okm = __all_sync(0xffffffffu, mbar_wait(&mode_rdy[k & 1], (k >> 1) & 1, abort));
             const bool fast = !okm || tab[kTabMode + (k & 1)] != 0.0f;
             // steep blocks: every builder thread loads dt of its row for both heads; warps 4-7 (one
             // row each) scan dt A into cs through the per-quarter totals and publish cs and the
@@ -798,14 +801,14 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
             fence_async_smem();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(x_ready);
+            if (lane == 0) mbar_arrive(&x_ready[k & 1]);
         };
 
-        // Iteration k: decay scan and mode of block k, read-back of block k, then X~ of block k and
-        // the epilogue of block k-1 (two fast blocks: in that order, so the tensor core gets block k's
-        // operands while block k-1's outputs drain; otherwise the other way round, since a steep block
-        // also uses the other output accumulator).  Every warp runs every iteration (named
-        // barriers 1 and 2 + hf); a failed wait skips work only.
+        // Iteration k: decay scan and mode of block k; after a fast block, a fast block k then forms
+        // X~, reads the state back and runs block k-1's epilogue, in the order their inputs arrive;
+        // otherwise the read-back, block k-1's epilogue (a steep block also uses the other output
+        // accumulator), then X~ or X' of block k.  Every warp runs every iteration (named barriers
+        // 1 and 2 + hf); a failed wait skips work only.
         for (int k = 0; k <= nch; ++k) {
             float dtv = 0.0f, c2 = 0.0f, a = 0.0f, tot = 0.0f;
             bool fast = true;
@@ -829,8 +832,12 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
                 tot = hf ? t1s : t0;
                 if (threadIdx.x == 8 * 32) {  // one thread publishes the mode to the builders and the MMA lane
                     tab[kTabMode + (k & 1)] = fast ? 1.0f : 0.0f;
-                    mbar_arrive(mode_rdy);
+                    mbar_arrive(&mode_rdy[k & 1]);
                 }
+                // a fast block after a fast block forms X~ before the read-back: it needs only its
+                // stage's x and the output accumulator whose epilogue (block k-2) this loop has run,
+                // so the state MMA may start as soon as the read-back is done
+                if (fast && fast_prev) form_x(k, fast, c2, a, tot, dtv);
 
                 // ---- read-back: the state at the block's start, as bf16 for the C.H term and back
                 // into TMEM for the state MMA (fast: both scaled by 2^a; steep: 1 and 2^tot)
@@ -869,9 +876,9 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
                     if (lane == 0) mbar_arrive(h_ready);
                 }
             }
-            // a fast block after a fast block: X~ first (block k-1's outputs use one accumulator only)
+            // otherwise block k-1's epilogue comes first (a steep block uses both output accumulators,
+            // and a steep block's X' goes over the state copy once the C.H MMA has read it)
             if (k < nch && fast && fast_prev) {
-                form_x(k, fast, c2, a, tot, dtv);
                 if (k > 0) epilogue(k - 1);
             } else {
                 if (k > 0) epilogue(k - 1);
