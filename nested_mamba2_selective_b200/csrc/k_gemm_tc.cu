@@ -942,10 +942,10 @@ cudaError_t launch_gemm_tc(const GemmDesc& g, cudaStream_t s)
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    // One tcgen05.mma of N = 128 columns costs about as much as one of N = 256 (measured on B200:
-    // about 170-190 cycles each from one CTA), so a tile's MMA time depends on K alone and wide tiles
-    // do twice the work per instruction.  Narrow tiles only when they take no more waves over the
-    // SMs than wide ones (each SM then drains half as many columns).
+    // A 128 x 256 tile and a 128 x 128 one keep the tensor core equally busy per flop (an MMA of
+    // N = 256 takes twice the cycles of one of N = 128), but the wide tile loads each A row once for
+    // twice the columns.  Narrow tiles only when they take no more waves over the SMs than wide ones
+    // (each SM then drains half as many columns).
     const int tiles256 = p.mtiles * ((n_total + 255) / 256);
     const int tiles128 = p.mtiles * ((n_total + 127) / 128);
     auto waves = [&](int t) { return (t + sms - 1) / sms; };

@@ -925,7 +925,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
 // accumulated into one TMEM accumulator: no per-block state update.  X'' is
 // formed in place over x in the stage, which the MMA's commit then frees.
 // A CTA takes HC heads of one group (4 when the group allows: one MMA of N = 256
-// then serves four heads, at about the cost of an N = 128 one); S of head j sits
+// then serves four heads and reads B^T once for all four); S of head j sits
 // in TMEM columns [64 j, 64 j + 64), row n = state dim.
 template <int HC>
 struct SegCfg {
