@@ -35,6 +35,7 @@ __device__ __forceinline__ float bf_hi_u(uint32_t v) { return __uint_as_float(v 
 constexpr int kBM = 128;  // rows of a tile = TMEM lanes
 constexpr int kBK = 64;   // one 128-byte swizzle atom of bf16 along K
 constexpr int kStageLd = 36;  // fp32 row pitch of the conv walks' staging rows (32 columns + pad)
+constexpr int kUsePairs = 1;  // plain wide tiles on CTA pairs (cta_group::2)
 constexpr int kTileRing = 6;  // launch-control answers in flight (producer leads the drain by <= 4 tiles)
 
 struct TcSeg {
@@ -83,19 +84,15 @@ struct TileInfo {
     int k0, k1;        // k-tiles [k0, k1) of this tile's K slice
 };
 
+// Tile j of row block mt (mt may be one past the last row block: a pair's odd CTA then has a tile
+// of rows past M, which load as zeros and store nothing).
 template <int BN>
-__device__ __forceinline__ TileInfo<BN> tile_info(const TcParams& p, int tile)
+__device__ __forceinline__ TileInfo<BN> tile_info_mj(const TcParams& p, int mt, int j)
 {
     TileInfo<BN> t;
-    const int per_slice = p.mtiles * p.ntiles;
-    const int ks = tile / per_slice;
-    tile -= ks * per_slice;
-    t.k0 = ks * p.kper;
-    t.k1 = min(p.ktiles, t.k0 + p.kper);
-    // row-block major: the N tiles of a row block are consecutive, so CTAs working at the same
-    // time share its A rows in L2
-    t.mt = tile / p.ntiles;
-    int j = tile % p.ntiles;
+    t.k0 = 0;
+    t.k1 = p.ktiles;
+    t.mt = mt;
     t.seg2 = -1;
     t.b_row2 = 0;
     if (j < p.pair_tiles) {
@@ -114,6 +111,20 @@ __device__ __forceinline__ TileInfo<BN> tile_info(const TcParams& p, int tile)
     t.n0 = j * BN;
     t.nvalid = min(BN, p.seg[s].n - t.n0);
     t.b_row = p.seg[s].b_row0 + t.n0;
+    return t;
+}
+
+// Tile index -> (K slice, row block, N tile), K slices slowest.  Row-block major: the N tiles of a
+// row block are consecutive, so CTAs working at the same time share its A rows in L2.
+template <int BN>
+__device__ __forceinline__ TileInfo<BN> tile_info(const TcParams& p, int tile)
+{
+    const int per_slice = p.mtiles * p.ntiles;
+    const int ks = tile / per_slice;
+    tile -= ks * per_slice;
+    TileInfo<BN> t = tile_info_mj<BN>(p, tile / p.ntiles, tile % p.ntiles);
+    t.k0 = ks * p.kper;
+    t.k1 = min(p.ktiles, t.k0 + p.kper);
     return t;
 }
 
@@ -141,14 +152,22 @@ __device__ __forceinline__ void store_bf16_chunk(__nv_bfloat16* o, int ncols, bo
     }
 }
 
-template <int BN, int STAGES, bool CONV>
+// PAIR: the kernel runs as clusters of two CTAs sharing each MMA (M = 256 over the pair).  CTA r
+// of a cluster takes row block 2 m + r of tile pair (m, j): it loads its own A rows and half of the
+// tile's B rows (the store rows of a paired tile in the even CTA and its conv rows in the odd one;
+// otherwise the first and second halves of the N columns the MMA uses), and drains its own
+// accumulator rows.  The even CTA issues the MMAs; both CTAs' loads complete its stage barriers,
+// its commits reach both CTAs, and the odd CTA's drain warps release the accumulator with remote
+// arrives.  Per SM, a pair tile loads 128 A rows and 128 B rows per K step for the work that one
+// CTA alone loads 128 and 256 for.  The walk over tile pairs is static.
+template <int BN, int STAGES, bool CONV, bool PAIR>
 __global__ void __launch_bounds__(320, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
                    const __grid_constant__ CUtensorMap mapB2, const __grid_constant__ OutMaps omaps, const TcParams p)
 {
     constexpr int A_BYTES = kBM * kBK * 2;
     constexpr int B_BYTES = BN * kBK * 2;
-    constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    constexpr int STAGE_BYTES = A_BYTES + (PAIR ? B_BYTES / 2 : B_BYTES);  // this CTA's bytes of a stage
     constexpr uint32_t TMEM_COLS = 2 * BN;
 
     extern __shared__ uint8_t smem_raw[];
@@ -171,14 +190,15 @@ __global__ void __launch_bounds__(320, 1)
     volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = PAIR ? cluster_ctarank() : 0;  // the pair's even CTA (0) issues its MMAs
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&full[s], 1);
+            mbar_init(&full[s], 1);  // the pair: the even CTA's arrive; both CTAs' loads complete it
             mbar_init(&empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&tfull[b], 1);
-            mbar_init(&tempty[b], 8);
+            mbar_init(&tempty[b], PAIR ? 16 : 8);  // the pair: both CTAs' drain warps
         }
         for (int j = 0; j < kTileRing; ++j) {
             mbar_init(&cfull[j], 1);
@@ -192,11 +212,17 @@ __global__ void __launch_bounds__(320, 1)
         if (p.pair_tiles) prefetch_tmap(&mapB2);
     }
     if (warp == 1) {
-        tmem_alloc(tmem_slot, TMEM_COLS);
-        tmem_relinquish();
+        if (PAIR) {
+            tmem_alloc_pair(tmem_slot, TMEM_COLS);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(tmem_slot, TMEM_COLS);
+            tmem_relinquish();
+        }
     }
     tc_fence_before();
     __syncthreads();
+    if (PAIR) cluster_sync();  // both CTAs' barriers are initialised before any arrives on them
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     // Programmatic dependent launch: the set-up above may overlap the previous kernel's tail; nothing
@@ -206,7 +232,25 @@ __global__ void __launch_bounds__(320, 1)
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     // tiles: (K slice, row block, N tile), K slices slowest
     const int total = p.mtiles * p.ntiles * p.ksplit;
-    auto release_acc = [&](int b) { mbar_arrive(&tempty[b]); };  // this drain warp is done with accumulator b
+    // the pair's static walk: tile pair tp = (row-block pair tp / ntiles, N tile tp % ntiles); CTA r
+    // takes tile (2 (tp / ntiles) + r) ntiles + tp % ntiles
+    const int total_pairs = ((p.mtiles + 1) / 2) * p.ntiles;
+    const int ncl = (int)gridDim.x / 2, cl = (int)blockIdx.x / 2;
+    auto pair_info = [&](int tp) -> TileInfo<BN> {
+        return tile_info_mj<BN>(p, (tp / p.ntiles) * 2 + (int)rank, tp % p.ntiles);
+    };
+    const uint32_t tempty_even = PAIR ? cluster_addr(tempty, 0) : 0;  // the even CTA's barriers
+    const uint32_t full_even = PAIR ? cluster_addr(full, 0) : 0;
+    auto release_acc = [&](int b) {  // this drain warp is done with accumulator b
+        if (PAIR) mbar_arrive_remote(tempty_even + 8u * b);
+        else mbar_arrive(&tempty[b]);
+    };
+    // the MMA's N for a tile: a paired tile's BN; otherwise its columns rounded up to 16 (32 for a pair)
+    auto mma_n = [&](const TileInfo<BN>& t) -> int {
+        if (t.seg2 >= 0) return BN;
+        const int n = (t.nvalid + 15) & ~15;
+        return PAIR ? max(n, 32) : n;
+    };
     // The tile of position j + 1 (`total` once the walk is over) from the scheduler's answer j;
     // each reader then releases the answer's slot (the MMA lane alone, or a drain warp once all
     // its lanes have read).  The wait ignores the abort flag, so every reader of an answer that
@@ -222,7 +266,31 @@ __global__ void __launch_bounds__(320, 1)
     };
 
     if (warp == 0) {
-        if (lane == 0) {  // ---------------- tile scheduler and TMA producer
+        if (PAIR && lane == 0) {  // ---------------- TMA producer of a pair CTA
+            int it = 0;
+            for (int j = 0; cl + j * ncl < total_pairs && !*abort; ++j) {
+                const TileInfo<BN> t = pair_info(cl + j * ncl);
+                const int arow = t.mt * p.rows - p.shift;  // rows outside [0, M) load as zeros
+                const int brow = t.seg2 >= 0 ? (rank ? t.b_row2 : t.b_row) : t.b_row + (int)rank * (mma_n(t) / 2);
+                for (int kt = 0; kt < p.ktiles; ++kt, ++it) {
+                    const int s = it % STAGES;
+                    if (!mbar_wait(&empty[s], ((it / STAGES) & 1) ^ 1, abort)) {
+                        raise_timeout(abort, p.status);
+                        break;
+                    }
+                    uint8_t* sa = smem + s * STAGE_BYTES;
+                    // the even CTA expects both CTAs' bytes; the odd CTA's loads can only land after
+                    // the previous phase completed (its stage was freed by an MMA that waited for it)
+                    if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * STAGE_BYTES);
+                    tma_load_2d_pair(sa, &mapA, full_even + 8u * s, kt * kBK, arow);
+                    tma_load_2d_pair(sa + A_BYTES, &mapB2, full_even + 8u * s, kt * kBK, brow);
+                }
+            }
+            // the even CTA sees every load of both CTAs land (bounded); the odd CTA's loads have
+            // landed before the even CTA reaches the closing cluster barrier
+            if (rank == 0)
+                for (int i = max(0, it - STAGES); i < it; ++i) mbar_wait(&full[i % STAGES], (i / STAGES) & 1, nullptr);
+        } else if (!PAIR && lane == 0) {  // ---------------- tile scheduler and TMA producer
             // Tile position 0 is this CTA's own index; the tile of position j + 1 is the index of a
             // CTA that had not started yet, cancelled by a launch-control request made while tile j
             // loads.  An answer that cancelled nothing ends the walk (the grid has one CTA per tile).
@@ -269,7 +337,39 @@ __global__ void __launch_bounds__(320, 1)
             for (int i = max(0, it - STAGES); i < it; ++i) mbar_wait(&full[i % STAGES], (i / STAGES) & 1, nullptr);
         }
     } else if (warp == 1) {
-        if (lane == 0) {  // ---------------- MMA issuer
+        if (PAIR && lane == 0 && rank == 0) {  // ---------------- MMA issuer of the pair
+            int it = 0;
+            for (int j = 0; cl + j * ncl < total_pairs && !*abort; ++j) {
+                const TileInfo<BN> t = pair_info(cl + j * ncl);
+                const int buf = j & 1;
+                if (!mbar_wait(&tempty[buf], ((j >> 1) & 1) ^ 1, abort)) {
+                    raise_timeout(abort, p.status);
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem + buf * BN;
+                const uint32_t idesc = idesc_bf16(2 * kBM, mma_n(t), 0, 0);
+                for (int kt = 0; kt < p.ktiles; ++kt, ++it) {
+                    const int s = it % STAGES;
+                    if (!mbar_wait(&full[s], (it / STAGES) & 1, abort)) {
+                        raise_timeout(abort, p.status);
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a0 = smem_u32(smem + s * STAGE_BYTES);
+                    const uint32_t b0 = a0 + A_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < kBK / 16; ++kk)
+                        mma_ss_pair(d_tmem, desc_sw128(a0 + kk * 32, 16, 1024), desc_sw128(b0 + kk * 32, 16, 1024),
+                                    idesc, (kt != 0 || kk != 0) ? 1u : 0u);
+                    mma_commit_pair(&empty[s]);
+                }
+                mma_commit_pair(&tfull[buf]);
+            }
+            // every issued MMA has finished before TMEM can be released (bounded)
+            mma_commit_pair(done);
+            mbar_wait(done, 0, nullptr);
+        } else if (!PAIR && lane == 0) {  // ---------------- MMA issuer
             int it = 0, tc = 0;
             for (int tile = blockIdx.x; tile < total && !*abort; ++tc) {
                 const TileInfo<BN> t = tile_info<BN>(p, tile);
@@ -280,8 +380,7 @@ __global__ void __launch_bounds__(320, 1)
                 }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem + buf * BN;
-                const int nmma = t.seg2 >= 0 ? BN : (t.nvalid + 15) & ~15;
-                const uint32_t idesc = idesc_bf16(kBM, nmma, 0, 0);
+                const uint32_t idesc = idesc_bf16(kBM, mma_n(t), 0, 0);
                 for (int kt = t.k0; kt < t.k1; ++kt, ++it) {
                     const int s = it % STAGES;
                     if (!mbar_wait(&full[s], (it / STAGES) & 1, abort)) {
@@ -310,9 +409,11 @@ __global__ void __launch_bounds__(320, 1)
         const int r = q * 32 + lane;  // tile row = TMEM lane
         const GemmExtra& ex = p.ex;
         int tc = 0;
-        // the walk: this CTA's own tile, then the scheduler's answers
-        for (int tile = (int)blockIdx.x; tile < total; tile = next_tile(tc++, false)) {
-            const TileInfo<BN> t = tile_info<BN>(p, tile);
+        // the walk: the pair's static one over tile pairs, else this CTA's own tile, then the
+        // scheduler's answers
+        for (int tile = PAIR ? cl : (int)blockIdx.x; PAIR ? tile < total_pairs : tile < total;
+             tile = PAIR ? tile + ncl : next_tile(tc, false), ++tc) {
+            const TileInfo<BN> t = PAIR ? pair_info(tile) : tile_info<BN>(p, tile);
             const int buf = tc & 1;
             const TcSeg& sg = p.seg[t.seg];
             const bool paired = t.seg2 >= 0;
@@ -730,8 +831,12 @@ __global__ void __launch_bounds__(320, 1)
     if (warp >= 2 && (warp & 3) == 2 && lane == 0) bulk_wait0();  // this group's bulk stores are complete
     tc_fence_before();
     __syncthreads();
+    if (PAIR) cluster_sync();  // the pair's MMAs, loads and arrives are all done
     tc_fence_after();
-    if (warp == 1) tmem_dealloc(tmem, TMEM_COLS);
+    if (warp == 1) {
+        if (PAIR) tmem_dealloc_pair(tmem, TMEM_COLS);
+        else tmem_dealloc(tmem, TMEM_COLS);
+    }
 }
 
 // --------------------------------------------------------------------------- host side
@@ -826,7 +931,7 @@ static bool tc_shape_ok(const GemmDesc& g)
 
 bool gemm_tc_supported(const GemmDesc& g) { return tc_shape_ok(g) && encode_fn() != nullptr; }
 
-template <int BN, int STAGES, bool CONV>
+template <int BN, int STAGES, bool CONV, bool PAIR>
 static cudaError_t launch_bn(const GemmDesc& g, const TcParams& p0, cudaStream_t s, int* status)
 {
     TcParams p = p0;
@@ -877,10 +982,11 @@ static cudaError_t launch_bn(const GemmDesc& g, const TcParams& p0, cudaStream_t
         p.ksplit = 1;
         p.kper = p.ktiles;
     }
-    constexpr int smem = STAGES * (kBM + BN) * kBK * 2 +
+    constexpr int smem = STAGES * (kBM + (PAIR ? BN / 2 : BN)) * kBK * 2 +
                          (CONV ? 2 * kBM * kStageLd * 4 : 2 * kBM * 128) + 1024 + 512;
     static_assert(smem <= 232448, "GEMM configuration exceeds 227 KB of shared memory");
-    auto kernel = gemm_tc_kernel<BN, STAGES, CONV>;
+    static_assert(!PAIR || BN == 256, "pairs run 256 x 256 MMAs");
+    auto kernel = gemm_tc_kernel<BN, STAGES, CONV, PAIR>;
     int dev = 0;
     cudaGetDevice(&dev);
     static unsigned long long attr_set = 0;  // one bit per device
@@ -890,21 +996,40 @@ static cudaError_t launch_bn(const GemmDesc& g, const TcParams& p0, cudaStream_t
         if (e != cudaSuccess) return e;
         attr_set |= 1ull << dev;
     }
-    // one CTA per tile: the CTAs that start first take over the others' tiles as they go
-    if (!p.pdl) {
-        kernel<<<p.mtiles * p.ntiles * p.ksplit, 320, smem, s>>>(mapA, mapB, mapB2, om, p);
+    // one CTA per tile: the CTAs that start first take over the others' tiles as they go.  Pairs:
+    // one cluster of two per pair of SMs, walking the tile pairs statically.
+    int grid = p.mtiles * p.ntiles * p.ksplit;
+    if (PAIR) {
+        int sms = 148;
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        const int pairs = ((p.mtiles + 1) / 2) * p.ntiles;
+        grid = 2 * (pairs < sms / 2 ? pairs : sms / 2);
+    }
+    if (!p.pdl && !PAIR) {
+        kernel<<<grid, 320, smem, s>>>(mapA, mapB, mapB2, om, p);
         return cudaGetLastError();
     }
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(p.mtiles * p.ntiles * p.ksplit);
+    cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(320);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchAttribute attr[2];
+    int na = 0;
+    if (p.pdl) {
+        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[na].val.programmaticStreamSerializationAllowed = 1;
+        ++na;
+    }
+    if (PAIR) {
+        attr[na].id = cudaLaunchAttributeClusterDimension;
+        attr[na].val.clusterDim.x = 2;
+        attr[na].val.clusterDim.y = 1;
+        attr[na].val.clusterDim.z = 1;
+        ++na;
+    }
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = na;
     return cudaLaunchKernelEx(&cfg, kernel, mapA, mapB, mapB2, om, p);
 }
 
@@ -962,9 +1087,16 @@ cudaError_t launch_gemm_tc(const GemmDesc& g, cudaStream_t s)
         p.kper = (p.ktiles + ks - 1) / ks;
         p.ksplit = (p.ktiles + p.kper - 1) / p.kper;
     }
+    // Plain wide tiles with a long enough K run on CTA pairs (measured on B200 for the block's
+    // out_proj, K = 1536: 39.3 -> 37.3 us; with K = 192 the pair was slower).  The conv tiles of
+    // in_proj stay on single CTAs: their drains differ from tile to tile, and the pairs' static walk
+    // lost to the dynamic one (105 -> 113 us).
+    if (wide && kUsePairs && !conv && p.ksplit == 1 && p.mtiles >= 2 && p.ktiles >= 8)
+        return launch_bn<256, 6, false, true>(g, p, s, status);
     if (wide)
-        return conv ? launch_bn<256, 3, true>(g, p, s, status) : launch_bn<256, 4, false>(g, p, s, status);
-    return conv ? launch_bn<128, 5, true>(g, p, s, status) : launch_bn<128, 6, false>(g, p, s, status);
+        return conv ? launch_bn<256, 3, true, false>(g, p, s, status)
+                    : launch_bn<256, 4, false, false>(g, p, s, status);
+    return conv ? launch_bn<128, 5, true, false>(g, p, s, status) : launch_bn<128, 6, false, false>(g, p, s, status);
 }
 
 }  // namespace mm
