@@ -1087,12 +1087,12 @@ cudaError_t launch_gemm_tc(const GemmDesc& g, cudaStream_t s)
         p.kper = (p.ktiles + ks - 1) / ks;
         p.ksplit = (p.ktiles + p.kper - 1) / p.kper;
     }
-    // Plain wide tiles with a long enough K run on CTA pairs (measured on B200 for the block's
-    // out_proj, K = 1536: 39.3 -> 37.3 us; with K = 192 the pair was slower).  The conv tiles of
-    // in_proj stay on single CTAs: their drains differ from tile to tile, and the pairs' static walk
-    // lost to the dynamic one (105 -> 113 us).
-    if (wide && kUsePairs && !conv && p.ksplit == 1 && p.mtiles >= 2 && p.ktiles >= 8)
-        return launch_bn<256, 6, false, true>(g, p, s, status);
+    // Wide tiles with a long enough K run on CTA pairs (measured on B200: the block's out_proj,
+    // K = 1536, 40.1 -> 38.9 us, but slower with K = 192; in_proj with its conv drain, K = 2048,
+    // 457 -> 420 us, but 105 -> 113 us with K = 768, where the pairs' static walk loses more to the
+    // uneven drains than the halved B loads gain).
+    if (wide && kUsePairs && p.ksplit == 1 && p.mtiles >= 2 && p.ktiles >= (conv ? 32 : 8))
+        return conv ? launch_bn<256, 5, true, true>(g, p, s, status) : launch_bn<256, 6, false, true>(g, p, s, status);
     if (wide)
         return conv ? launch_bn<256, 3, true, false>(g, p, s, status)
                     : launch_bn<256, 4, false, false>(g, p, s, status);
