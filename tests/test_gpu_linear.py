@@ -68,3 +68,23 @@ def test_linear_many_tiles_writes_every_tile_once(out_f32):
     assert not torch.isnan(out).any()
     ref = a.astype(np.float64) @ w.astype(np.float64).T
     assert max_abs_rel(to_np(out), ref) <= (1e-5 if out_f32 else 5e-3)
+
+
+@pytest.mark.parametrize("out_f32", [False, True])
+def test_linear_cta_pairs_odd_row_blocks(out_f32):
+    """Wide tiles with K >= 512 run on CTA pairs, each pair taking two 128-row blocks.  With 9 row
+    blocks the last pair's second CTA gets rows past M: they must load as zeros and store nothing.
+    The output sits inside a NaN-filled buffer: every row of it is written, and the 64 rows after
+    it stay untouched."""
+    M, K, N = 128 * 8 + 50, 768, 3352
+    a = synth.activations((M, K), "bf16", seed=21)
+    w = synth.activations((N, K), "bf16", seed=22, std=0.05)
+    A, W = torch.from_numpy(a).cuda().bfloat16(), torch.from_numpy(w).cuda().bfloat16()
+    full = torch.full((M + 64, N), float("nan"), dtype=torch.float32 if out_f32 else torch.bfloat16, device="cuda")
+    mm_linear(A, W, out=full[:M], out_f32=out_f32)
+    torch.cuda.synchronize()
+    assert mm_device_status() == 0
+    assert not torch.isnan(full[:M]).any()
+    assert torch.isnan(full[M:]).all()
+    ref = a.astype(np.float64) @ w.astype(np.float64).T
+    assert max_abs_rel(to_np(full[:M]), ref) <= (1e-5 if out_f32 else 5e-3)
