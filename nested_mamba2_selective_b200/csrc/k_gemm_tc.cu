@@ -35,7 +35,7 @@ __device__ __forceinline__ float bf_hi_u(uint32_t v) { return __uint_as_float(v 
 constexpr int kBM = 128;  // rows of a tile = TMEM lanes
 constexpr int kBK = 64;   // one 128-byte swizzle atom of bf16 along K
 constexpr int kStageLd = 36;  // fp32 row pitch of the conv walks' staging rows (32 columns + pad)
-constexpr int kUsePairs = 1;  // plain wide tiles on CTA pairs (cta_group::2)
+constexpr int kUsePairs = 1;  // wide tiles on CTA pairs (cta_group::2) where launch_gemm_tc selects them
 constexpr int kTileRing = 6;  // launch-control answers in flight (producer leads the drain by <= 4 tiles)
 
 struct TcSeg {
