@@ -23,6 +23,11 @@
  *  - dtype MM_BF16 runs the tensor-core path (bf16 storage, fp32
  *    accumulation and fp32 scan state); MM_F32 runs an fp32 CUDA-core path
  *    (fp32 storage and arithmetic throughout).
+ *  - Host threads: entry points may be called from several host threads at
+ *    once.  Calls that share a buffer (a workspace, a state, an output) must
+ *    be ordered by the caller, as for any two kernels; matmamba_block_fwd_host
+ *    calls on one device take turns by themselves; tracing (mm_trace_*) is
+ *    for one host thread.
  *  - Symbols: d_model = D_m, E = d_inner, P = d_head, N = d_state,
  *    G = ngroups, GN = G*N, H = E/P heads, K = d_conv.  At width m:
  *    d = E*m/D_m channels, h = d/P heads, nconv = d + 2*GN conv channels.
@@ -104,7 +109,8 @@ typedef struct mm_block_params {
 /* Human-readable name of a status code (static string, never NULL). */
 const char* mm_status_string(int status);
 
-/* Name of the most recent CUDA error behind an MM_ERR_CUDA ("cudaSuccess" if none). */
+/* Name of the most recent CUDA error behind an MM_ERR_CUDA returned to the
+ * calling host thread ("cudaSuccess" if none). */
 const char* mm_last_cuda_error(void);
 
 /* Library version: major*10000 + minor*100 + patch. */
@@ -167,7 +173,8 @@ int matmamba_block_fwd(const mm_block_params* p, const void* u, int batch, int L
  * copy streams the library creates once per device, so with pinned host
  * buffers the transfers in both directions overlap the compute.  The call
  * orders itself after earlier work on `stream` and returns once out_host
- * holds the result.
+ * holds the result.  Calls on one device from several host threads take
+ * turns (they share that device's copy streams).
  */
 int matmamba_block_fwd_host(const mm_block_params* p, const void* u_host, int batch, int L, int m_i, int chunk,
                             void* out_host, void* u_dev, void* out_dev, void* workspace, size_t ws_bytes,

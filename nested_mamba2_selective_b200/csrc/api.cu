@@ -1,7 +1,9 @@
 // C-ABI entry points: host-side validation, width views, workspace carving and
 // launch sequences.  Every step of the computation runs in this library's
 // kernels; nothing here computes on the host.
+#include <atomic>
 #include <cstring>
+#include <mutex>
 
 #include "mm_internal.cuh"
 
@@ -13,15 +15,17 @@ __device__ int g_mm_device_status;
 namespace mm {
 int* device_status_ptr()
 {
-    static int* ptrs[64] = {};
+    static std::atomic<int*> ptrs[64] = {};  // host threads may look it up at the same time
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return nullptr;
-    if (!ptrs[dev]) {
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    int* ptr = ptrs[dev].load(std::memory_order_acquire);
+    if (!ptr) {
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_mm_device_status) != cudaSuccess) return nullptr;
-        ptrs[dev] = static_cast<int*>(p);
+        ptr = static_cast<int*>(p);
+        ptrs[dev].store(ptr, std::memory_order_release);
     }
-    return ptrs[dev];
+    return ptr;
 }
 }  // namespace mm
 
@@ -97,7 +101,7 @@ int resolve(const mm_block_params* p, int m, View& v)
     return MM_OK;
 }
 
-cudaError_t g_last_cuda_error = cudaSuccess;  // most recent CUDA error a call reported
+thread_local cudaError_t g_last_cuda_error = cudaSuccess;  // most recent CUDA error a call of this thread reported
 
 inline int cuda_status(cudaError_t e)
 {
@@ -457,6 +461,8 @@ struct HostPipe {
     bool ready = false;
 };
 HostPipe g_pipes[64];
+// Calls on one device take turns: they share that device's copy streams and events.
+std::mutex g_pipe_mu[64];
 
 cudaError_t host_pipe(HostPipe** out)
 {
@@ -502,6 +508,10 @@ int matmamba_block_fwd_host(const mm_block_params* p, const void* u_host, int ba
         size_t sub_need;
         if (!matmamba_block_workspace(p, per, L, m_i, chunk, &sub_need) && sub_need <= ws_bytes) break;
     }
+    int dev = 0;
+    MM_TRY(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= 64) return cuda_status(cudaErrorInvalidDevice);
+    std::lock_guard<std::mutex> turn(g_pipe_mu[dev]);
     HostPipe* hp;
     MM_TRY(host_pipe(&hp));
     MM_TRY(cudaEventRecord(hp->start, s));  // earlier work on s (users of u_dev / out_dev) comes first

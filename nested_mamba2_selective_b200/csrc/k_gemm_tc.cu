@@ -18,6 +18,7 @@
 // that drain their tiles faster take more of them and all finish together.
 #include <cuda.h>
 
+#include <atomic>
 #include <cstring>
 
 #include "mm_internal.cuh"
@@ -847,14 +848,15 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
 
 EncodeTiledFn encode_fn()
 {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
+    // resolved once (the initialisation of a function-local static is thread-safe)
+    static const EncodeTiledFn fn = [] {
         void* p = nullptr;
         cudaDriverEntryPointQueryResult q;
         if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
             q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    }
+            return reinterpret_cast<EncodeTiledFn>(p);
+        return static_cast<EncodeTiledFn>(nullptr);
+    }();
     return fn;
 }
 
@@ -989,12 +991,12 @@ static cudaError_t launch_bn(const GemmDesc& g, const TcParams& p0, cudaStream_t
     auto kernel = gemm_tc_kernel<BN, STAGES, CONV, PAIR>;
     int dev = 0;
     cudaGetDevice(&dev);
-    static unsigned long long attr_set = 0;  // one bit per device
+    static std::atomic<unsigned long long> attr_set{0};  // one bit per device
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    if (!(attr_set >> dev & 1ull)) {
+    if (!(attr_set.load() >> dev & 1ull)) {
         cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
-        attr_set |= 1ull << dev;
+        attr_set.fetch_or(1ull << dev);
     }
     // one CTA per tile: the CTAs that start first take over the others' tiles as they go.  Pairs:
     // one cluster of two per pair of SMs, walking the tile pairs statically.

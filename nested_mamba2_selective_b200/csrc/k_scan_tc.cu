@@ -30,6 +30,7 @@
 #include <cuda.h>
 
 #include <cmath>
+#include <atomic>
 #include <cstring>
 #include <map>
 #include <mutex>
@@ -1331,8 +1332,8 @@ static cudaError_t launch_scan_tc_impl(const ScanArgs& a, const ScanGate* gate, 
     }
     int dev = 0;
     cudaGetDevice(&dev);
-    static unsigned long long attr_set = 0;
-    if (dev < 64 && !(attr_set >> dev & 1ull)) {
+    static std::atomic<unsigned long long> attr_set{0};  // one bit per device
+    if (dev >= 0 && dev < 64 && !(attr_set.load() >> dev & 1ull)) {
         cudaError_t e = cudaFuncSetAttribute(ssd_chunk_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              kChunkSmem);
         if (e == cudaSuccess)
@@ -1344,7 +1345,7 @@ static cudaError_t launch_scan_tc_impl(const ScanArgs& a, const ScanGate* gate, 
             e = cudaFuncSetAttribute(ssd_seg_state_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      SegCfg<2>::kSmem);
         if (e != cudaSuccess) return e;
-        attr_set |= 1ull << dev;
+        attr_set.fetch_or(1ull << dev);
     }
     const dim3 cgrid((a.h + 1) / 2, a.batch, pl.nseg);
     if (pl.nseg == 1) {

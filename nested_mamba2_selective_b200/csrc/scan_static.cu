@@ -22,6 +22,8 @@
 //  - The first call on a device looks up the array's device address
 //    (cudaGetSymbolAddress, with that device current) and caches it; make
 //    that first call before any stream capture.
+#include <atomic>
+
 #include "mm_internal.cuh"
 
 namespace {
@@ -36,15 +38,15 @@ static __device__ __align__(256) unsigned char g_scan_scratch[kScanScratchBytes]
 // device); nullptr if the runtime cannot resolve it.
 void* scratch_address()
 {
-    static void* addr[64] = {};
+    static std::atomic<void*> addr[64] = {};  // host threads may look it up at the same time
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-    if (!addr[dev]) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_scan_scratch) != cudaSuccess) return nullptr;
-        addr[dev] = p;
+    void* a = addr[dev].load(std::memory_order_acquire);
+    if (!a) {
+        if (cudaGetSymbolAddress(&a, g_scan_scratch) != cudaSuccess) return nullptr;
+        addr[dev].store(a, std::memory_order_release);
     }
-    return addr[dev];
+    return a;
 }
 
 }  // namespace

@@ -151,6 +151,53 @@ def test_host_buffer_entry_point_matches_oracle(orc, batch, L):
     assert max_abs_rel(got, to_np(ref)) <= TOL["bf16"]
 
 
+def test_host_entry_point_from_two_threads():
+    """Two host threads calling matmamba_block_fwd_host on one device, each with its own buffers and
+    stream, get bit for bit what one thread gets: calls on one device take turns on its copy streams
+    and events instead of interleaving their records and waits."""
+    import threading
+
+    w = synth.WORKLOADS["block_130m_b8_L2048"]
+    wt, _ = make_block(w)
+    batch, L, m = 4, 384, 384
+    jobs = []
+    for k in range(2):
+        u = to_device(synth.activations((batch, L, w.d_model), "bf16", seed=70 + k), "bf16")
+        job = dict(u_host=u.cpu().pin_memory(), out_host=torch.empty_like(u.cpu()).pin_memory(),
+                   u_dev=torch.empty_like(u), out_dev=torch.empty_like(u), results=[], errors=[],
+                   ws=torch.empty(matmamba_block_workspace(wt, batch, L, m, 256), dtype=torch.uint8,
+                                  device="cuda"))
+        matmamba_block_fwd_host(wt, job["u_host"], m, 256, job["out_host"], job["u_dev"], job["out_dev"], job["ws"])
+        job["ref"] = job["out_host"].clone()
+        jobs.append(job)
+    assert not torch.equal(jobs[0]["ref"], jobs[1]["ref"])
+
+    def worker(job):
+        try:
+            torch.cuda.set_device(0)
+            with torch.cuda.stream(torch.cuda.Stream()):
+                for _ in range(6):
+                    job["out_host"].fill_(0.0)
+                    matmamba_block_fwd_host(wt, job["u_host"], m, 256, job["out_host"], job["u_dev"],
+                                            job["out_dev"], job["ws"])
+                    job["results"].append(job["out_host"].clone())
+        except Exception as e:  # reported by the main thread
+            job["errors"].append(repr(e))
+
+    threads = [threading.Thread(target=worker, args=(job,)) for job in jobs]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join(timeout=120)
+    assert not any(t.is_alive() for t in threads)
+    torch.cuda.synchronize()
+    for job in jobs:
+        assert job["errors"] == []
+        assert len(job["results"]) == 6
+        for got in job["results"]:
+            assert torch.equal(got, job["ref"])
+
+
 def test_invalid_width_raises_and_launches_nothing():
     w = synth.WORKLOADS["block_130m_b8_L2048"]
     wt, _ = make_block(w)
