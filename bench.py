@@ -473,6 +473,7 @@ def run_ours(args):
         e2e_fn()
     e2e_s = slowest(time.perf_counter() - t0)
     io_bytes = T * B["d_model"] * 2
+    link = copy_rates(torch, u_host, out_host, u_dev, out_dev)
     del ws, u_dev, out_dev
 
     stack = decode = None
@@ -502,7 +503,12 @@ def run_ours(args):
             "stages": stage_rows,
             "ssd_scan": {"workload": S["workload"], "by_heads": scan},
             "e2e": {"value": whole_job_rate(T, args.steps, world, e2e_s), "unit": "tokens/s",
-                    "h2d_bytes_per_step": io_bytes, "d2h_bytes_per_step": io_bytes},
+                    "h2d_bytes_per_step": io_bytes, "d2h_bytes_per_step": io_bytes,
+                    "h2d_gbs": link["h2d_gbs"], "d2h_gbs": link["d2h_gbs"],
+                    "both_directions_ms": link["both_ms"],
+                    "copy_bound": whole_job_rate(T, 1, world, link["both_ms"] / 1e3),
+                    "note": "copy_bound = tokens per step / the time of one step's upload and download "
+                            "running at once (pinned buffers, no compute)"},
             "gpu_launches": kernels,
             "clocks": clocks,
         }
@@ -521,6 +527,42 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def copy_rates(torch, u_host, out_host, u_dev, out_dev, reps=5):
+    """PCIe rates of one step's copies between pinned host buffers and the device: the upload alone,
+    the download alone (GB/s, CUDA events on the copy's stream) and both at once on two streams (ms
+    between events on a third stream that waits for both)."""
+    s_in, s_out, s_main = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.current_stream()
+    nbytes = u_host.numel() * u_host.element_size()
+
+    def one(dst, src, stream):
+        with torch.cuda.stream(stream):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            dst.copy_(src, non_blocking=True)
+            e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1)
+
+    h2d = min(one(u_dev, u_host, s_in) for _ in range(reps))
+    d2h = min(one(out_host, out_dev, s_out) for _ in range(reps))
+    both = []
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(s_main)
+        s_in.wait_event(e0)
+        s_out.wait_event(e0)
+        with torch.cuda.stream(s_in):
+            u_dev.copy_(u_host, non_blocking=True)
+        with torch.cuda.stream(s_out):
+            out_host.copy_(out_dev, non_blocking=True)
+        s_main.wait_stream(s_in)
+        s_main.wait_stream(s_out)
+        e1.record(s_main)
+        torch.cuda.synchronize()
+        both.append(e0.elapsed_time(e1))
+    return {"h2d_gbs": nbytes / (h2d / 1e3) / 1e9, "d2h_gbs": nbytes / (d2h / 1e3) / 1e9, "both_ms": min(both)}
 
 
 def device_block_weights(mm, torch, gen, Dm, E, P, N, dev, K=4):
