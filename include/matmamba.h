@@ -16,6 +16,8 @@
  *  - Calls are asynchronous on the given CUDA stream (a cudaStream_t passed
  *    as void*, NULL = legacy default stream).  Output buffers must not alias
  *    inputs unless a parameter says so.
+ *  - Limits per call: at most 65535 sequences (batch) and fewer than 2^31
+ *    tokens (batch * L); larger calls return MM_ERR_SHAPE.
  *  - Every call returns an mm_status.  Shapes, widths, dtypes, alignment and
  *    workspace size are checked on the host before anything is launched; a
  *    rejected call launches nothing and leaves every buffer untouched.

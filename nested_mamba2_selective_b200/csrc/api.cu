@@ -34,6 +34,14 @@ namespace {
 constexpr size_t kAlign = 256;
 
 size_t esize(int dtype) { return dtype == MM_BF16 ? 2 : 4; }
+
+// Shape limits of the launches: sequences go on a grid's y or z dimension (at most 65535 of them per
+// call), and the projections and scans index tokens (batch * L) with 32-bit rows.
+constexpr int kMaxBatch = 65535;
+bool batch_ok(int batch, int L)
+{
+    return batch > 0 && L > 0 && batch <= kMaxBatch && (int64_t)batch * L < (1ll << 31);
+}
 bool dtype_ok(int dtype) { return dtype == MM_F32 || dtype == MM_BF16; }
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 size_t round_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
@@ -417,7 +425,7 @@ int matmamba_block_workspace(const mm_block_params* p, int batch, int L, int m_i
     int rc = resolve(p, m_i, v);
     if (rc) return rc;
     if (!bytes) return MM_ERR_NULL;
-    if (batch <= 0 || L <= 0) return MM_ERR_SHAPE;
+    if (!batch_ok(batch, L)) return MM_ERR_SHAPE;
     if ((rc = check_chunk(chunk))) return rc;
     *bytes = block_ws_bytes(p, v, batch, L, chunk);
     return MM_OK;
@@ -431,7 +439,7 @@ int matmamba_block_fwd(const mm_block_params* p, const void* u, int batch, int L
     int rc = resolve(p, m_i, v);
     if (rc) return rc;
     if (!u || !out) return MM_ERR_NULL;
-    if (batch <= 0 || L <= 0) return MM_ERR_SHAPE;
+    if (!batch_ok(batch, L)) return MM_ERR_SHAPE;
     if ((rc = check_chunk(chunk))) return rc;
     if (p->dtype == MM_BF16 && (!aligned16(u) || !aligned16(out))) return MM_ERR_ALIGN;
     // a state output may not share a byte with its input: CTAs write one sequence's output while
@@ -495,7 +503,7 @@ int matmamba_block_fwd_host(const mm_block_params* p, const void* u_host, int ba
     View v;
     int rc = resolve(p, m_i, v);
     if (rc) return rc;
-    if (batch <= 0 || L <= 0) return MM_ERR_SHAPE;
+    if (!batch_ok(batch, L)) return MM_ERR_SHAPE;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const size_t row_bytes = (size_t)L * v.Dm * esize(p->dtype);  // one sequence of u or out
     size_t need;
@@ -551,7 +559,7 @@ static int scan_args_check(int dtype, const void* x, int64_t x_stride, const flo
 {
     if (!dtype_ok(dtype)) return MM_ERR_DTYPE;
     if (!x || !dt || !A || !B || !C || !y) return MM_ERR_NULL;
-    if (batch <= 0 || L <= 0 || h <= 0 || P <= 0 || N <= 0 || G <= 0 || hpg <= 0) return MM_ERR_SHAPE;
+    if (!batch_ok(batch, L) || h <= 0 || P <= 0 || N <= 0 || G <= 0 || hpg <= 0) return MM_ERR_SHAPE;
     if (N > 256) return MM_ERR_SHAPE;
     if ((h - 1) / hpg >= G) return MM_ERR_SHAPE;
     if (x_stride < (int64_t)h * P || y_stride < (int64_t)h * P || dt_stride < h || B_stride < (int64_t)G * N ||
@@ -584,7 +592,7 @@ int ssd_scan_workspace(int dtype, int batch, int L, int h, int P, int N, int G, 
 {
     if (!bytes) return MM_ERR_NULL;
     if (!dtype_ok(dtype)) return MM_ERR_DTYPE;
-    if (batch <= 0 || L <= 0 || h <= 0 || P <= 0 || N <= 0 || G <= 0 || chunk <= 0) return MM_ERR_SHAPE;
+    if (!batch_ok(batch, L) || h <= 0 || P <= 0 || N <= 0 || G <= 0 || chunk <= 0) return MM_ERR_SHAPE;
     const int hpg = (h + G - 1) / G;
     ScanArgs a = make_scan_args(nullptr, (int64_t)h * P, nullptr, h, nullptr, nullptr, (int64_t)G * N, nullptr,
                                 (int64_t)G * N, nullptr, batch, L, h, P, N, G, hpg, chunk, nullptr, (int64_t)h * P * N,
@@ -676,7 +684,7 @@ int ssd_step_workspace(const mm_block_params* p, int batch, int m_i, size_t* byt
     int rc = resolve(p, m_i, v);
     if (rc) return rc;
     if (!bytes) return MM_ERR_NULL;
-    if (batch <= 0) return MM_ERR_SHAPE;
+    if (!batch_ok(batch, 1)) return MM_ERR_SHAPE;
     *bytes = step_ws(v, p, batch);
     return MM_OK;
 }
@@ -688,7 +696,7 @@ int ssd_step(const mm_block_params* p, float* ssm_state, void* conv_state, const
     int rc = resolve(p, m_i, v);
     if (rc) return rc;
     if (!ssm_state || !conv_state || !u_t || !out_t) return MM_ERR_NULL;
-    if (batch <= 0) return MM_ERR_SHAPE;
+    if (!batch_ok(batch, 1)) return MM_ERR_SHAPE;
     if (p->dtype == MM_BF16 && (!aligned16(u_t) || !aligned16(out_t))) return MM_ERR_ALIGN;
     if (!workspace || ws_bytes < step_ws(v, p, batch)) return MM_ERR_WORKSPACE;
     if (reinterpret_cast<uintptr_t>(workspace) % kAlign) return MM_ERR_ALIGN;
@@ -736,7 +744,7 @@ static int stack_check(const mm_block_params* layers, int nlayers, const int* m_
                        size_t* need)
 {
     if (!layers || !m_per_layer) return MM_ERR_NULL;
-    if (nlayers <= 0 || batch <= 0 || L <= 0) return MM_ERR_SHAPE;
+    if (nlayers <= 0 || !batch_ok(batch, L)) return MM_ERR_SHAPE;
     int rc;
     if ((rc = check_chunk(chunk))) return rc;
     size_t block_max = 0;

@@ -31,7 +31,7 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(GemmDesc g, int n_total)
     __shared__ float As[BK][BM + 4];
     __shared__ float Bs[BK][BN + 4];
     const int tid = threadIdx.x;
-    const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
+    const int m0 = blockIdx.x * BM, n0 = blockIdx.y * BN;  // row blocks on x: up to 2^31 - 1 of them
     const T* A = static_cast<const T*>(g.A);
 
     // loader role: one A row and one B row, 8 consecutive k each
@@ -93,7 +93,8 @@ cudaError_t launch_gemm_simt(int dtype, const GemmDesc& g, cudaStream_t s)
     int n_total = 0;
     for (int i = 0; i < g.nseg; ++i) n_total += g.seg[i].n;
     if (g.M == 0 || n_total == 0) return cudaSuccess;
-    dim3 grid((n_total + 63) / 64, (g.M + 63) / 64);
+    if ((n_total + 63) / 64 > 65535) return cudaErrorInvalidValue;
+    dim3 grid((g.M + 63) / 64, (n_total + 63) / 64);
     if (dtype == MM_BF16) gemm_simt_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(g, n_total);
     else gemm_simt_kernel<float><<<grid, 256, 0, s>>>(g, n_total);
     return cudaGetLastError();

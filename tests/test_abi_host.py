@@ -90,6 +90,26 @@ def test_rejected_calls_launch_nothing(lib):
                         128, 1, 1, 256, None, 0, fake, 64, None, None, 0, None) == 4
 
 
+def test_batch_and_token_limits_are_checked_on_the_host(lib):
+    """At most 65535 sequences (they go on a grid's y or z dimension) and fewer than 2^31 tokens per
+    call: queries and calls beyond that return MM_ERR_SHAPE before anything is launched."""
+    p = params()
+    n = ctypes.c_size_t()
+    assert lib.matmamba_block_workspace(ctypes.byref(p), 65535, 16, 768, 256, ctypes.byref(n)) == 0
+    assert lib.matmamba_block_workspace(ctypes.byref(p), 65536, 16, 768, 256, ctypes.byref(n)) == 2
+    assert lib.matmamba_block_workspace(ctypes.byref(p), 1024, 1 << 21, 768, 256, ctypes.byref(n)) == 2
+    assert lib.ssd_scan_workspace(1, 65535, 64, 24, 64, 128, 1, 256, ctypes.byref(n)) == 0
+    assert lib.ssd_scan_workspace(1, 65536, 64, 24, 64, 128, 1, 256, ctypes.byref(n)) == 2
+    assert lib.ssd_step_workspace(ctypes.byref(p), 65535, 768, ctypes.byref(n)) == 0
+    assert lib.ssd_step_workspace(ctypes.byref(p), 65536, 768, ctypes.byref(n)) == 2
+    fake = ctypes.c_void_p(1 << 20)
+    assert lib.matmamba_block_fwd(ctypes.byref(p), fake, 65536, 1, 768, 256, fake, None, None, None, None, fake,
+                                  1 << 40, None) == 2
+    assert lib.ssd_scan(1, fake, 64, fake, 1, fake, fake, 128, fake, 128, None, 65536, 1, 1, 64, 128, 1, 1, 256,
+                        None, 0, fake, 64, None, fake, 1 << 40, None) == 2
+    assert lib.ssd_step(ctypes.byref(p), fake, fake, fake, 65536, 768, fake, fake, 1 << 40, None) == 2
+
+
 def test_overlapping_state_buffers_are_rejected(lib):
     """A final state that shares bytes with the initial state is refused before any launch; disjoint
     buffers pass validation (and would launch, so they are not called here)."""
