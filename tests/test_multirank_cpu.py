@@ -74,3 +74,17 @@ def test_single_gpu_runs_in_process():
     rc, lines, err = _bench(["--stub", "--steps", "2", "--warmup", "1"])
     assert rc == 0, err[-2000:]
     assert lines[0]["n_gpus"] == 1
+
+
+def test_reference_arm_prints_on_rank_zero_only():
+    """The reference arm under N ranks: rank 0 times the oracle and prints the one line (counting N
+    GPUs); any other rank exits 0 at once without work or output."""
+    rc, lines, err = _bench(["--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "1"])
+    assert rc == 0, err[-2000:]
+    assert len(lines) == 1
+    line = lines[0]
+    assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["e2e"]["h2d_bytes_per_step"] == 0
+    rc, lines, err = _bench(["--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "1"],
+                            {"WORLD_SIZE": "2", "RANK": "1", "LOCAL_RANK": "1"})
+    assert rc == 0 and not lines, err[-2000:]
