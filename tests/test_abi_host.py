@@ -108,6 +108,8 @@ def test_batch_and_token_limits_are_checked_on_the_host(lib):
     assert lib.ssd_scan(1, fake, 64, fake, 1, fake, fake, 128, fake, 128, None, 65536, 1, 1, 64, 128, 1, 1, 256,
                         None, 0, fake, 64, None, fake, 1 << 40, None) == 2
     assert lib.ssd_step(ctypes.byref(p), fake, fake, fake, 65536, 768, fake, fake, 1 << 40, None) == 2
+    assert lib.matmamba_block_fwd_host(ctypes.byref(p), fake, 65536, 1, 768, 256, fake, fake, fake, fake, 1 << 40,
+                                       None) == 2
 
 
 def test_overlapping_state_buffers_are_rejected(lib):

@@ -66,3 +66,18 @@ def test_decode_state_traffic_is_the_active_state(lib, m):
     rest = Bt * ((d + 2 * N) * 2 + h * 4 + d * 2 + d * 2 + 2 * h * 4)  # xBC, dt, z read; row and sums written
     assert kind == "hbm" and nbytes == 2 * state_bytes + rest
     assert conv.shape[1] == E + 2 * N
+
+
+def test_stage_table_fraction_is_work_over_time_over_peak():
+    """A stage's fraction is its algorithmic work per launch over its mean launch time, against the
+    peak of its bound (bf16 tensor FLOP/s or HBM GB/s)."""
+    pk = {"bf16_tflops": 1000.0, "hbm_gbs": 5000.0}
+    stages = {"in_proj_conv": (4, 12, 0.4), "ssd_scan_gate": (2, 4, 0.2)}  # launches, kernels, total ms
+    work = {"in_proj_conv": ("tensor", 50e9), "ssd_scan_gate": ("hbm", 250e6)}
+    rows = bench.stage_table(stages, work, pk)
+    assert rows["in_proj_conv"]["ms_per_launch"] == pytest.approx(0.1)
+    assert rows["in_proj_conv"]["achieved"] == pytest.approx(500.0)  # 50 GFLOP in 0.1 ms
+    assert rows["in_proj_conv"]["frac"] == pytest.approx(0.5)
+    assert rows["ssd_scan_gate"]["achieved"] == pytest.approx(2500.0)  # 250 MB in 0.1 ms
+    assert rows["ssd_scan_gate"]["frac"] == pytest.approx(0.5)
+    assert rows["in_proj_conv"]["share"] == pytest.approx(2 / 3)
